@@ -1,0 +1,224 @@
+/*
+ * nvfp4_moe.h — C ABI of the B200 (sm_100a) NVFP4 Mixture-of-Experts expert-FFN library.
+ *
+ * The operation is the MoE expert FFN of the nvfp4-megamoe-kernel pages:
+ *   route -> quantize activations (NVFP4, global scale from amax on the GPU) ->
+ *   L1 2D x 3D block-scaled grouped GEMM with SwiGLU and FP4 re-quantization in its epilogue ->
+ *   L2 grouped GEMM with the routing weight and scatter-add in its epilogue.
+ * ("NVFP4 MegaMoE Kernel Rewrite — CuTeDSL", sections "Our Adaptation" and "Phase 3: Full MoE
+ *  pipeline"; "May 24, 2026 — Session Start Plan", section 5 "NVFP4-1.1: Fuse FP4 into SwiGLU
+ *  Epilogue".)
+ *
+ * Data formats
+ *   NVFP4 tensor (rows x cols): E2M1 codes packed two per byte, row-major, element 2j in the low
+ *   nibble of byte j (uint8 [rows][cols/2]); one E4M3 block scale per 16 consecutive elements of a
+ *   row; one FP32 global scale gs.  Value = E2M1(code) * E4M3(scale) / gs.
+ *   Block scales are stored TILED: the (rows x cols/16) scale matrix is cut into atoms of
+ *   128 rows x 4 scale columns (512 bytes), atoms row-major over (rows/128, cols/64); inside an
+ *   atom scale (r, c) is at byte (r%32)*16 + ((r/32)%4)*4 + c%4.  A scale buffer for R rows holds
+ *   ceil(R/128)*128 * cols/16 bytes.
+ *   Grouped ("2D x 3D") operands: activations A (R rows x K) whose rows are bucketed by expert,
+ *   expert e owning rows [offs[e], offs[e+1]) (every offs a multiple of 128); weights B
+ *   (E x N x K) as one NVFP4 tensor of E*N rows with a global scale per expert gs_b[e].
+ *
+ * Conventions (every call)
+ *   - All pointers not marked "host" are device pointers, 16-byte aligned; the caller owns and
+ *     allocates every buffer.  The library never allocates, never synchronizes the host (except
+ *     nvfp4_read_status, which exists to do so) and never throws.
+ *   - Work is enqueued on `stream`; arguments are checked on the host first and nothing is
+ *     launched when a check fails.
+ *   - dev_status (nullable): device int32 that kernels OR error bits into (NVFP4_DEVERR_*).
+ *     Every wait inside a kernel is bounded; a wait that runs out sets NVFP4_DEVERR_TIMEOUT and
+ *     the kernel returns instead of hanging.  Out-of-range routing ids set NVFP4_DEVERR_BAD_INDEX
+ *     and are skipped.
+ *   - Launch failures return NVFP4_ERR_CUDA; nvfp4_last_error() gives the CUDA error string.
+ */
+#ifndef NVFP4_MOE_H
+#define NVFP4_MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define NVFP4_API __attribute__((visibility("default")))
+#else
+#define NVFP4_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* nvfp4_stream_t; /* same handle as cudaStream_t */
+
+typedef enum {
+  NVFP4_OK = 0,
+  NVFP4_ERR_INVALID_ARG = 1,
+  NVFP4_ERR_UNSUPPORTED_SHAPE = 2,
+  NVFP4_ERR_MISALIGNED = 3,
+  NVFP4_ERR_WORKSPACE_TOO_SMALL = 4,
+  NVFP4_ERR_CUDA = 5,
+  NVFP4_ERR_TIMEOUT = 6,
+  NVFP4_ERR_BAD_INDEX = 7
+} nvfp4_status_t;
+
+/* Bits a kernel ORs into *dev_status. */
+#define NVFP4_DEVERR_TIMEOUT 1
+#define NVFP4_DEVERR_BAD_INDEX 2
+#define NVFP4_DEVERR_BAD_OFFSETS 4
+
+/* ---------------------------------------------------------------------------------------------
+ * nvfp4_quantize — BF16 -> NVFP4 with the FP8-round-tripped block scale.
+ *
+ * Follows the commit log of dsv4/kernels/cuda (nvfp4-megamoe-kernel): the global scale "gsa" is
+ * computed from amax on the GPU into a GPU buffer with no host sync ("Two-kernel approach":
+ * amax kernel, then a quantize kernel that reads gsa from the buffer), and the element codes are
+ * computed against the decoded FP8 block scale ("quantize must use the FP8-round-tripped block
+ * scale").  NVFP4 itself: "May 24, 2026 — Session Start Plan", section 1 "NVFP4-0".
+ *
+ *   gs = 2688 / max|x| (1.0 if that is not finite and positive)            [compute_gs = 1]
+ *   per 16-element block: s = (amax_b / 6) * gs ; scale = E4M3_rn_satfinite(s) ; d = decode(scale)
+ *   code_i = E2M1_rn_satfinite(x_i * (gs / d))   (all-zero codes when d == 0)
+ *
+ *   x        bf16 [rows][ld] (ld >= cols, ld % 8 == 0)
+ *   dst_row  NULL: row i goes to output row i (out_rows >= rows).  Otherwise int32 [rows*k]: row i
+ *            is written to output rows dst_row[i*k + j], j < k; entries < 0 are skipped; entries
+ *            >= out_rows set NVFP4_DEVERR_BAD_INDEX and are skipped.  (The permuted write of the
+ *            MoE path: each token's codes go straight to its k expert rows.)
+ *   codes    uint8 [out_rows][cols/2];  sf: tiled scales for out_rows rows (see top).
+ *   gs       device float[1]: written when compute_gs = 1, read when compute_gs = 0.
+ *   ws       device scratch of nvfp4_quantize_workspace_size() bytes (the amax word).
+ *   Constraints: cols % 64 == 0, rows >= 0, k in [1, 64] when dst_row != NULL.
+ * ------------------------------------------------------------------------------------------- */
+NVFP4_API size_t nvfp4_quantize_workspace_size(void);
+NVFP4_API nvfp4_status_t nvfp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t ld,
+                              const int32_t* dst_row, int k, int64_t out_rows,
+                              uint8_t* codes, uint8_t* sf, float* gs, int compute_gs,
+                              void* ws, size_t ws_bytes, int32_t* dev_status,
+                              nvfp4_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------------
+ * moe_permute — top-k softmax routing and the expert-bucketed row map.
+ *
+ * The pages list "the MoE routing logic (top-k selection, slot mapping)" as work outside the
+ * grouped GEMM ("NVFP4 MegaMoE Kernel Rewrite — CuTeDSL", section "Our Adaptation").  Reading:
+ * the k largest logits of a token (ties to the lower expert id; a -inf logit is a dropped slot),
+ * weights softmax(logits)[e], renormalized over the k when renormalize != 0.  Rows: experts in
+ * ascending id, each segment padded to a multiple of 128 rows, slots inside a segment in
+ * ascending (token, j).
+ *
+ *   logits    float [T][E], or NULL: topk_ids/topk_w are then INPUTS (ids < 0 = dropped slot)
+ *   topk_ids  int32 [T][k] (output when logits != NULL); topk_w float [T][k] likewise
+ *   offs      int32 [E+1]: start row of each expert's segment, offs[E] = rows used
+ *   dst_row   int32 [T*k]: row of slot (t, j), -1 when dropped
+ *   row_token int32 [R_max]: token of each row, -1 for padding and unused rows
+ *   row_w     float [R_max]: routing weight of each row, 0 for padding and unused rows
+ *   R_max     = moe_rows_max(T, E, k)
+ *   Constraints: 1 <= k <= E <= 256, k <= 32, T >= 0.
+ * ------------------------------------------------------------------------------------------- */
+NVFP4_API int64_t moe_rows_max(int T, int E, int k);
+NVFP4_API size_t moe_permute_workspace_size(int T, int E, int k);
+NVFP4_API nvfp4_status_t moe_permute(const float* logits, int T, int E, int k, int renormalize,
+                           int32_t* topk_ids, float* topk_w, int32_t* offs, int32_t* dst_row,
+                           int32_t* row_token, float* row_w, void* ws, size_t ws_bytes,
+                           int32_t* dev_status, nvfp4_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------------
+ * nvfp4_grouped_gemm — plain 2D x 3D block-scaled grouped GEMM, C = A_e * B_e^T per expert.
+ *
+ * The grouped GEMM of "NVFP4 MegaMoE Kernel Rewrite — CuTeDSL", section "The Reference Kernel:
+ * ScaledGroupedGemmKernel" (NVFP4: E2M1 + E4M3 per 16, 2D x 3D A(tokens,K) x B(experts,K,N)).
+ * FP32 accumulation in tensor memory; C[r][n] = acc * 1/(gs_a * gs_b[e]).
+ *
+ *   a, sfa    NVFP4 [R_max][K] (tiled scales), gs_a device float[1]
+ *   b, sfb    NVFP4 [E*N][K], gs_b device float[E]
+ *   offs      device int32 [E+1], multiples of 128, offs[E] <= R_max
+ *   out       [R_max][N], out_dtype 0 = float32, 1 = bf16; every row of every segment is written
+ *             (rows of a segment beyond its real tokens hold whatever A's padding rows give)
+ *   Constraints: K % 64 == 0, N % 256 == 0, R_max % 128 == 0, 1 <= E <= 256.
+ * ------------------------------------------------------------------------------------------- */
+NVFP4_API nvfp4_status_t nvfp4_grouped_gemm(const uint8_t* a, const uint8_t* sfa, const float* gs_a,
+                                  const uint8_t* b, const uint8_t* sfb, const float* gs_b,
+                                  const int32_t* offs, int E, int N, int K, int64_t R_max,
+                                  void* out, int out_dtype, int32_t* dev_status,
+                                  nvfp4_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------------
+ * moe_grouped_gemm_l1_swiglu_q — L1 grouped GEMM with SwiGLU and NVFP4 re-quantization fused in
+ * the epilogue ("May 24, 2026 — Session Start Plan", section 5 "NVFP4-1.1": L1 GEMM -> SwiGLU ->
+ * FP4 pack in registers -> FP4 GMEM).
+ *
+ *   W1 of expert e is [2I][H]: rows [0, I) gate, rows [I, 2I) up.
+ *   g = acc_gate / (gs_a*gs_w1[e]), u = acc_up / (gs_a*gs_w1[e]), h = silu(g) * u (FP32),
+ *   h quantized with the static global scale *gs_h exactly like nvfp4_quantize.
+ *
+ *   a, sfa, gs_a    activations NVFP4 [R_max][H]
+ *   w1, sfw1, gs_w1 NVFP4 [E*2I][H], gs_w1 float[E]
+ *   offs            int32 [E+1] (from moe_permute)
+ *   gs_h            device float[1]
+ *   h, sfh          output NVFP4 [R_max][I] (tiled scales); rows of every segment are written
+ *   Constraints: H % 64 == 0, I % 128 == 0, R_max % 128 == 0, 1 <= E <= 256.
+ * ------------------------------------------------------------------------------------------- */
+NVFP4_API nvfp4_status_t moe_grouped_gemm_l1_swiglu_q(const uint8_t* a, const uint8_t* sfa, const float* gs_a,
+                                            const uint8_t* w1, const uint8_t* sfw1,
+                                            const float* gs_w1, const int32_t* offs, int E, int H,
+                                            int I, int64_t R_max, const float* gs_h, uint8_t* h,
+                                            uint8_t* sfh, int32_t* dev_status,
+                                            nvfp4_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------------
+ * moe_grouped_gemm_l2_scatter — L2 grouped GEMM with the routing weight and the scatter-add in
+ * its epilogue ("NVFP4 MegaMoE Kernel Rewrite — CuTeDSL", section "Our Adaptation": "Scatter
+ * with routing weights"; section "Phase 3").
+ *
+ *   acc_ws[t][n] = sum over rows r of token t of  row_w[r] * (h_r . W2_e[n]) / (gs_h*gs_w2[e]),
+ *   computed with FP32 reductions into acc_ws (zeroed by this call), then out = bf16_rn(acc_ws)
+ *   when out_bf16 != NULL.  Padding rows (row_token < 0) contribute nothing.
+ *
+ *   h, sfh, gs_h     NVFP4 [R_max][I]
+ *   w2, sfw2, gs_w2  NVFP4 [E*H][I], gs_w2 float[E]
+ *   offs, row_token, row_w  from moe_permute
+ *   acc_ws           float [T][H] scratch/output;  out_bf16  bf16 [T][H] or NULL
+ *   Constraints: H % 256 == 0, I % 64 == 0, R_max % 128 == 0, 1 <= E <= 256, T >= 0.
+ * ------------------------------------------------------------------------------------------- */
+NVFP4_API nvfp4_status_t moe_grouped_gemm_l2_scatter(const uint8_t* h, const uint8_t* sfh, const float* gs_h,
+                                           const uint8_t* w2, const uint8_t* sfw2,
+                                           const float* gs_w2, const int32_t* offs,
+                                           const int32_t* row_token, const float* row_w, int E,
+                                           int H, int I, int T, int64_t R_max, float* acc_ws,
+                                           void* out_bf16, int32_t* dev_status,
+                                           nvfp4_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------------
+ * moe_ffn_forward — the whole expert FFN in one stream-ordered call:
+ *   moe_permute -> nvfp4_quantize (amax -> gs on the GPU, permuted write) ->
+ *   moe_grouped_gemm_l1_swiglu_q -> moe_grouped_gemm_l2_scatter -> bf16 out.
+ *
+ *   x_bf16   bf16 [T][H];  logits float [T][E] (softmax top-k routing, renormalized)
+ *   w1.. / w2..  expert weights as above; gs_h device float[1] (static intermediate scale)
+ *   out_bf16 bf16 [T][H]; tokens whose slots are all dropped get exact zeros.
+ *   ws       device scratch of moe_ffn_workspace_size(T, H, I, E, k) bytes (256-byte aligned)
+ *   Constraints: those of the four calls above.
+ * ------------------------------------------------------------------------------------------- */
+NVFP4_API size_t moe_ffn_workspace_size(int T, int H, int I, int E, int k);
+NVFP4_API nvfp4_status_t moe_ffn_forward(const void* x_bf16, const float* logits, int T, int H, int I, int E,
+                               int k, const uint8_t* w1, const uint8_t* sfw1, const float* gs_w1,
+                               const uint8_t* w2, const uint8_t* sfw2, const float* gs_w2,
+                               const float* gs_h, void* out_bf16, void* ws, size_t ws_bytes,
+                               int32_t* dev_status, nvfp4_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------------
+ * Status helpers.
+ *   nvfp4_read_status: copies *dev_status to *host_code (host pointer) on `stream` and waits for
+ *   the stream; returns NVFP4_ERR_TIMEOUT / NVFP4_ERR_BAD_INDEX when the matching bit is set.
+ *   nvfp4_last_error: the last CUDA error string seen by this library on this thread.
+ * ------------------------------------------------------------------------------------------- */
+NVFP4_API nvfp4_status_t nvfp4_read_status(const int32_t* dev_status, int32_t* host_code,
+                                 nvfp4_stream_t stream);
+NVFP4_API const char* nvfp4_last_error(void);
+NVFP4_API int nvfp4_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* NVFP4_MOE_H */

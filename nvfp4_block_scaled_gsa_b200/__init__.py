@@ -1,0 +1,22 @@
+"""B200-native (sm_100a) NVFP4 Mixture-of-Experts expert-FFN.
+
+The compute path is the C-ABI library ``_lib/libnvfp4moe.so`` (hand-written CUDA, declared in
+``include/nvfp4_moe.h``); this package only builds it, loads it with ctypes and marshals torch
+tensors and the current CUDA stream into its calls.
+"""
+
+from .api import (  # noqa: F401
+    NVFP4Weights,
+    ffn_workspace_bytes,
+    grouped_gemm,
+    l1_swiglu_q,
+    l2_scatter,
+    moe_ffn_forward,
+    permute,
+    quantize,
+    quantize_weights,
+    read_status,
+    rows_max,
+    sf_bytes,
+)
+from ._native import Nvfp4Error, lib  # noqa: F401

@@ -1,0 +1,167 @@
+"""Torch-facing wrappers over the C ABI: allocate outputs with torch, pass pointers and the
+current CUDA stream, check the status.  No arithmetic of the method happens here.
+"""
+
+from dataclasses import dataclass
+
+import torch
+
+from ._native import call, lib
+
+U8, I32, F32, BF16 = torch.uint8, torch.int32, torch.float32, torch.bfloat16
+
+
+def _p(t):
+    return None if t is None else t.data_ptr()
+
+
+def _stream():
+    return torch.cuda.current_stream().cuda_stream
+
+
+def round_up(v, m):
+    return (v + m - 1) // m * m
+
+
+def sf_bytes(rows, cols):
+    """Bytes of a tiled block-scale buffer for `rows` rows of `cols` elements."""
+    return round_up(rows, 128) * cols // 16
+
+
+@dataclass
+class NVFP4Weights:
+    """Expert weights (E, N, K) as one NVFP4 tensor of E*N rows: codes (E*N, K/2) uint8, tiled
+    scales, global scale per expert (E,) float32."""
+    codes: torch.Tensor
+    sf: torch.Tensor
+    gs: torch.Tensor
+    E: int
+    N: int
+    K: int
+
+
+def quantize(x, gs=None, dst_row=None, k=1, out_rows=None, status=None):
+    """NVFP4-quantize bf16 x (rows, cols).  gs=None: the global scale is computed on the GPU from
+    amax (returned as a device tensor); otherwise gs (device float[1]) is used as given.
+    dst_row/k/out_rows: permuted write (see nvfp4_quantize in the header)."""
+    assert x.dtype == BF16 and x.dim() == 2 and x.stride(1) == 1
+    rows, cols = x.shape
+    if out_rows is None:
+        out_rows = rows
+    dev = x.device
+    codes = torch.empty(out_rows, cols // 2, dtype=U8, device=dev)
+    sf = torch.empty(sf_bytes(out_rows, cols), dtype=U8, device=dev)
+    compute = gs is None
+    if compute:
+        gs = torch.empty(1, dtype=F32, device=dev)
+    ws = torch.empty(int(lib().nvfp4_quantize_workspace_size()), dtype=U8, device=dev)
+    call("nvfp4_quantize", _p(x), rows, cols, x.stride(0), _p(dst_row), k, out_rows, _p(codes),
+         _p(sf), _p(gs), int(compute), _p(ws), ws.numel(), _p(status), _stream())
+    return codes, sf, gs
+
+
+def quantize_weights(get_expert, E, N, K, device="cuda"):
+    """Pre-pack expert weights: get_expert(e) -> bf16 (N, K) on the device; each expert gets its
+    own global scale from its amax."""
+    codes = torch.empty(E * N, K // 2, dtype=U8, device=device)
+    sf = torch.empty(E * N * K // 16, dtype=U8, device=device)
+    gs = torch.empty(E, dtype=F32, device=device)
+    ws = torch.empty(int(lib().nvfp4_quantize_workspace_size()), dtype=U8, device=device)
+    per_sf = N * K // 16
+    for e in range(E):
+        w = get_expert(e)
+        assert w.dtype == BF16 and tuple(w.shape) == (N, K)
+        w = w.contiguous()
+        call("nvfp4_quantize", _p(w), N, K, K, None, 1, N, _p(codes[e * N:(e + 1) * N]),
+             sf.data_ptr() + e * per_sf, gs.data_ptr() + 4 * e, 1, _p(ws), ws.numel(), None,
+             _stream())
+    return NVFP4Weights(codes, sf, gs, E, N, K)
+
+
+def rows_max(T, E, k):
+    return int(lib().moe_rows_max(T, E, k))
+
+
+def permute(logits, k, renormalize=True, ids=None, weights=None, E=None, status=None):
+    """Top-k routing + expert-bucketed row map.  With logits=None, ids/weights (T, k) are the
+    routing (ids < 0 dropped) and E must be given."""
+    if logits is not None:
+        T, E = logits.shape
+        dev = logits.device
+        ids = torch.empty(T, k, dtype=I32, device=dev)
+        weights = torch.empty(T, k, dtype=F32, device=dev)
+    else:
+        T = ids.shape[0]
+        dev = ids.device
+    R = rows_max(T, E, k)
+    offs = torch.empty(E + 1, dtype=I32, device=dev)
+    dst_row = torch.empty(T * k, dtype=I32, device=dev)
+    row_token = torch.empty(max(R, 1), dtype=I32, device=dev)
+    row_w = torch.empty(max(R, 1), dtype=F32, device=dev)
+    call("moe_permute", _p(logits), T, E, k, int(renormalize), _p(ids), _p(weights), _p(offs),
+         _p(dst_row), _p(row_token), _p(row_w), None, 0, _p(status), _stream())
+    return dict(ids=ids, weights=weights, offs=offs, dst_row=dst_row, row_token=row_token,
+                row_w=row_w, R_max=R, E=E, T=T, k=k)
+
+
+def grouped_gemm(a_codes, a_sf, gs_a, w: NVFP4Weights, offs, out_dtype=F32, status=None):
+    """Plain 2D x 3D grouped GEMM: out[r] = A[r] . W_e^T / (gs_a * gs_w[e])."""
+    R = a_codes.shape[0]
+    out = torch.empty(R, w.N, dtype=out_dtype, device=a_codes.device)
+    call("nvfp4_grouped_gemm", _p(a_codes), _p(a_sf), _p(gs_a), _p(w.codes), _p(w.sf), _p(w.gs),
+         _p(offs), w.E, w.N, w.K, R, _p(out), 0 if out_dtype == F32 else 1, _p(status), _stream())
+    return out
+
+
+def l1_swiglu_q(a_codes, a_sf, gs_a, w1: NVFP4Weights, offs, gs_h, status=None):
+    """L1 GEMM + SwiGLU + NVFP4 re-quantization -> (h codes (R, I/2), h tiled scales)."""
+    R = a_codes.shape[0]
+    I = w1.N // 2
+    h = torch.empty(R, I // 2, dtype=U8, device=a_codes.device)
+    sfh = torch.empty(sf_bytes(R, I), dtype=U8, device=a_codes.device)
+    call("moe_grouped_gemm_l1_swiglu_q", _p(a_codes), _p(a_sf), _p(gs_a), _p(w1.codes),
+         _p(w1.sf), _p(w1.gs), _p(offs), w1.E, w1.K, I, R, _p(gs_h), _p(h), _p(sfh), _p(status),
+         _stream())
+    return h, sfh
+
+
+def l2_scatter(h, sfh, gs_h, w2: NVFP4Weights, offs, row_token, row_w, T, out_bf16=True,
+               status=None):
+    """L2 GEMM + routing weight + scatter-add -> (acc fp32 (T, H), out bf16 (T, H) or None)."""
+    R = h.shape[0]
+    H = w2.N
+    I = w2.K
+    acc = torch.empty(T, H, dtype=F32, device=h.device)
+    out = torch.empty(T, H, dtype=BF16, device=h.device) if out_bf16 else None
+    call("moe_grouped_gemm_l2_scatter", _p(h), _p(sfh), _p(gs_h), _p(w2.codes), _p(w2.sf),
+         _p(w2.gs), _p(offs), _p(row_token), _p(row_w), w2.E, H, I, T, R, _p(acc), _p(out),
+         _p(status), _stream())
+    return acc, out
+
+
+def ffn_workspace_bytes(T, H, I, E, k):
+    return int(lib().moe_ffn_workspace_size(T, H, I, E, k))
+
+
+def moe_ffn_forward(x, logits, k, w1: NVFP4Weights, w2: NVFP4Weights, gs_h, out=None, ws=None,
+                    status=None):
+    """The whole expert FFN: bf16 x (T, H), float logits (T, E) -> bf16 out (T, H)."""
+    T, H = x.shape
+    E = logits.shape[1]
+    I = w1.N // 2
+    if out is None:
+        out = torch.empty(T, H, dtype=BF16, device=x.device)
+    need = ffn_workspace_bytes(T, H, I, E, k)
+    if ws is None:
+        ws = torch.empty(max(need, 256), dtype=U8, device=x.device)
+    call("moe_ffn_forward", _p(x), _p(logits), T, H, I, E, k, _p(w1.codes), _p(w1.sf), _p(w1.gs),
+         _p(w2.codes), _p(w2.sf), _p(w2.gs), _p(gs_h), _p(out), _p(ws), ws.numel(), _p(status),
+         _stream())
+    return out
+
+
+def read_status(status):
+    """Host copy of a device status word (synchronizes the current stream)."""
+    host = torch.zeros(1, dtype=torch.int32)
+    rc = lib().nvfp4_read_status(_p(status), host.data_ptr(), _stream())
+    return int(host.item()), rc

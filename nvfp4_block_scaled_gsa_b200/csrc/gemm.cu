@@ -1,0 +1,587 @@
+// gemm.cu — persistent 2D x 3D NVFP4 block-scaled grouped GEMM for sm_100a (tcgen05 + TMEM).
+//
+// The operation is the grouped GEMM of "NVFP4 MegaMoE Kernel Rewrite — CuTeDSL" (section "The
+// Reference Kernel: ScaledGroupedGemmKernel"): A(tokens, K) x B(experts, N, K) -> C(tokens, N),
+// tokens bucketed per expert, E2M1 operands with one E4M3 scale per 16 elements, FP32
+// accumulation.  The pages' kernel is a 7-warp CuTeDSL design; this one is written directly in
+// PTX for sm_100a:
+//
+//   warp 0      TMA producer: A and B tiles (cp.async.bulk.tensor, 128-byte swizzle) and the
+//               pre-tiled scale atoms (cp.async.bulk) into a 4-stage shared-memory ring
+//   warp 1      MMA issuer: tcgen05.cp moves the stage's scales into tensor memory, then
+//               tcgen05.mma.kind::mxf4nvf4.block_scale (M=128, N=256, K=64) accumulates in TMEM
+//   warp 2      owns the tensor-memory allocation (512 columns)
+//   warps 4..7  epilogue: tcgen05.ld of the accumulator (warp w reads lanes 32*(w%4)..+31),
+//               then one of the fused epilogues below
+//
+// Epilogues (the MODE template parameter):
+//   PLAIN_F32 / PLAIN_BF16  C = acc / (gs_a * gs_b[e])
+//   L1  SwiGLU + NVFP4 re-quantization in registers ("May 24, 2026 — Session Start Plan",
+//       section 5 "NVFP4-1.1"): the B tile stacks gate rows n0..n0+127 over up rows
+//       I+n0..I+n0+127, so each epilogue thread holds matching gate and up columns of its row.
+//   L2  routing weight + scatter-add: red.global.add.v4.f32 into an FP32 [T][H] buffer.
+//
+// Tile scheduler: each expert's 128-padded row segment gives (rows/128) M-tiles; tiles are
+// numbered expert by expert with the N-tile outer and the M-tile inner, so CTAs running at the
+// same time share B (weight) tiles through L2.  CTAs take tiles with a static stride.  The
+// segment offsets are read on the device: no host sync between routing and the GEMM.
+//
+// Every mbarrier wait is bounded (NVFP4_WAIT_TIMEOUT_NS).  A wait that runs out raises a CTA-wide
+// abort flag: the producer waits (bounded) for its copies in flight, the MMA warp drains its
+// MMAs, the tensor memory is freed and the kernel reports NVFP4_DEVERR_TIMEOUT.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "common.cuh"
+
+namespace nvfp4 {
+namespace {
+
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int BK_BYTES = 128;  // 256 FP4 elements per stage along K
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * BK_BYTES;                // 16 KB
+constexpr int B_BYTES = BN * BK_BYTES;                // 32 KB
+constexpr int SFA_BYTES = 4 * 512;                    // 128 rows x 16 scales
+constexpr int SFB_BYTES = 2 * 4 * 512;                // 256 rows x 16 scales
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024;
+static_assert(STAGE_BYTES % 1024 == 0, "stages must keep 1024-byte alignment (128B swizzle)");
+
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t TM_ACC = 0;                       // 256 FP32 columns
+constexpr uint32_t TM_SFA = 256;                     // 16 columns per stage
+constexpr uint32_t TM_SFB = TM_SFA + STAGES * 16;    // 32 columns per stage
+static_assert(TM_SFB + STAGES * 32 <= TMEM_COLS, "tensor memory budget");
+
+constexpr uint32_t IDESC = idesc_nvf4(BN);
+constexpr int NUM_THREADS = 256;
+constexpr int EPI_WARP0 = 4;
+constexpr int MAX_E = 256;
+
+enum Mode { PLAIN_F32 = 0, PLAIN_BF16 = 1, L1_SWIGLU = 2, L2_SCATTER = 3 };
+
+struct GemmArgs {
+  const uint8_t* sfa;
+  const uint8_t* sfb;
+  const float* gs_a;
+  const float* gs_b;
+  const int32_t* offs;
+  int E;
+  int N;         // rows per expert in B (2I for L1)
+  int K;         // reduction length (elements)
+  int n_tiles;   // N-tiles per expert
+  int64_t R_max;
+  void* out;     // PLAIN: [R_max][N]
+  const float* gs_h;  // L1
+  uint8_t* h;         // L1: [R_max][I/2]
+  uint8_t* sfh;       // L1
+  int I;              // L1
+  const int32_t* row_token;  // L2
+  const float* row_w;        // L2
+  float* acc;                // L2: [T][H]
+  int T;                     // L2
+  int32_t* status;
+};
+
+__device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c),
+               "f"(d)
+               : "memory");
+}
+
+struct Tile {
+  int e, m0, nt;
+};
+
+__device__ __forceinline__ Tile decode_tile(int t, const int* tile_start, const int* seg, int E,
+                                            int n_tiles) {
+  int lo = 0, hi = E;  // tile_start[lo] <= t < tile_start[hi]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (tile_start[mid] <= t) lo = mid;
+    else hi = mid;
+  }
+  const int local = t - tile_start[lo];
+  const int mt_cnt = (seg[lo + 1] - seg[lo]) >> 7;
+  Tile r;
+  r.e = lo;
+  r.nt = local / mt_cnt;
+  r.m0 = seg[lo] + (local - r.nt * mt_cnt) * BM;
+  return r;
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_a,
+                        const __grid_constant__ CUtensorMap tm_b, const GemmArgs args) {
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t bar_full[STAGES];
+  __shared__ __align__(8) uint64_t bar_empty[STAGES];
+  __shared__ __align__(8) uint64_t bar_acc_full;
+  __shared__ __align__(8) uint64_t bar_acc_empty;
+  __shared__ __align__(8) uint64_t bar_drain;
+  __shared__ uint32_t tmem_slot;
+  __shared__ int seg[MAX_E + 1];
+  __shared__ int tile_start[MAX_E + 1];
+  __shared__ int warp_sums[NUM_THREADS / 32];
+  __shared__ int bad_offsets;
+  __shared__ volatile int abort_flag;
+
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int E = args.E;
+
+  // ---- scheduler table: tiles per expert, exclusive scan over experts
+  if (tid == 0) {
+    bad_offsets = 0;
+    abort_flag = 0;
+  }
+  if (tid <= E) seg[tid] = __ldg(args.offs + tid);
+  __syncthreads();
+  int my_tiles = 0;
+  if (tid < E) {
+    const int lo = seg[tid], hi = seg[tid + 1];
+    if (lo < 0 || hi < lo || (lo & 127) || (hi & 127) || hi > args.R_max) bad_offsets = 1;
+    else my_tiles = ((hi - lo) >> 7) * args.n_tiles;
+  }
+  int incl = my_tiles;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  if (lane == 31) warp_sums[warp] = incl;
+  __syncthreads();
+  if (tid == 0) {
+    int run = 0;
+    for (int w = 0; w < NUM_THREADS / 32; ++w) {
+      const int c = warp_sums[w];
+      warp_sums[w] = run;
+      run += c;
+    }
+  }
+  __syncthreads();
+  const int excl = warp_sums[warp] + incl - my_tiles;
+  if (tid < E) tile_start[tid] = excl;
+  if (tid == E - 1) tile_start[E] = excl + my_tiles;
+
+  // ---- barriers and tensor memory
+  if (tid == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(smem_u32(&bar_full[s]), 1);
+      mbar_init(smem_u32(&bar_empty[s]), 1);
+    }
+    mbar_init(smem_u32(&bar_acc_full), 1);
+    mbar_init(smem_u32(&bar_acc_empty), 4);
+    mbar_init(smem_u32(&bar_drain), 1);
+    fence_mbar_init();
+  }
+  if (warp == 2) {
+    tmem_alloc(smem_u32(&tmem_slot), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_slot;
+  const int total = bad_offsets ? 0 : tile_start[E];
+  if (tid == 0 && bad_offsets && blockIdx.x == 0) report(args.status, NVFP4_DEVERR_BAD_OFFSETS);
+
+  const int K = args.K;
+  const int nk = (K + 255) / 256;  // stages along K
+  const int atoms_k = K / 64;      // 64-element scale atoms along K
+
+  if (warp == 0) {
+    // =========================== TMA producer ===========================
+    if (lane == 0) {
+      prefetch_tmap(&tm_a);
+      prefetch_tmap(&tm_b);
+      uint32_t it = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        const Tile tl = decode_tile(t, tile_start, seg, E, args.n_tiles);
+        int b_row0, b_row1;
+        if (MODE == L1_SWIGLU) {
+          b_row0 = tl.e * args.N + tl.nt * 128;
+          b_row1 = b_row0 + args.I;
+        } else {
+          b_row0 = tl.e * args.N + tl.nt * BN;
+          b_row1 = b_row0 + 128;
+        }
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1u;
+          if (!mbar_wait_bounded(smem_u32(&bar_empty[s]), ph ^ 1u, &abort_flag)) {
+            ok = false;
+            break;
+          }
+          const int natoms = min(4, atoms_k - kb * 4);
+          const uint32_t full = smem_u32(&bar_full[s]);
+          uint8_t* st = smem + s * STAGE_BYTES;
+          const uint32_t sA = smem_u32(st), sB = sA + A_BYTES, sSFA = sB + B_BYTES,
+                         sSFB = sSFA + SFA_BYTES;
+          mbar_arrive_expect_tx(full, A_BYTES + B_BYTES + natoms * 512 * 3);
+          tma_load_2d(sA, &tm_a, full, kb * BK_BYTES, tl.m0);
+          tma_load_2d(sB, &tm_b, full, kb * BK_BYTES, b_row0);
+          tma_load_2d(sB + B_BYTES / 2, &tm_b, full, kb * BK_BYTES, b_row1);
+          const int64_t a_atom = (int64_t)(tl.m0 >> 7) * atoms_k + kb * 4;
+          const int64_t b_atom0 = (int64_t)(b_row0 >> 7) * atoms_k + kb * 4;
+          const int64_t b_atom1 = (int64_t)(b_row1 >> 7) * atoms_k + kb * 4;
+          bulk_load(sSFA, args.sfa + a_atom * 512, natoms * 512, full);
+          bulk_load(sSFB, args.sfb + b_atom0 * 512, natoms * 512, full);
+          bulk_load(sSFB + SFB_BYTES / 2, args.sfb + b_atom1 * 512, natoms * 512, full);
+        }
+      }
+      if (!ok) {
+        // let the copies already issued land before the CTA can exit
+        volatile int never = 0;
+        const uint32_t first = it > (uint32_t)STAGES ? it - STAGES : 0u;
+        for (uint32_t j = first; j < it; ++j)
+          mbar_wait_bounded(smem_u32(&bar_full[j % STAGES]), (j / STAGES) & 1u, &never,
+                            NVFP4_WAIT_TIMEOUT_NS / 4);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // =========================== MMA issuer ===========================
+    if (lane == 0) {
+      uint32_t it = 0, tile_it = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++tile_it) {
+        if (!mbar_wait_bounded(smem_u32(&bar_acc_empty), (tile_it & 1u) ^ 1u, &abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1u;
+          if (!mbar_wait_bounded(smem_u32(&bar_full[s]), ph, &abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const int natoms = min(4, atoms_k - kb * 4);
+          uint8_t* st = smem + s * STAGE_BYTES;
+          const uint32_t sA = smem_u32(st), sB = sA + A_BYTES, sSFA = sB + B_BYTES,
+                         sSFB = sSFA + SFA_BYTES;
+          const uint32_t t_sfa = tmem + TM_SFA + s * 16;
+          const uint32_t t_sfb = tmem + TM_SFB + s * 32;
+          for (int a = 0; a < natoms; ++a) {
+            tc_cp_sf(t_sfa + a * 4, smem_desc(sSFA + a * 512, 0, 128, 0));
+            tc_cp_sf(t_sfb + a * 8, smem_desc(sSFB + a * 512, 0, 128, 0));
+            tc_cp_sf(t_sfb + a * 8 + 4, smem_desc(sSFB + SFB_BYTES / 2 + a * 512, 0, 128, 0));
+          }
+          for (int a = 0; a < natoms; ++a) {
+            const uint64_t ad = smem_desc(sA + a * 32, 16, 1024, 2);
+            const uint64_t bd = smem_desc(sB + a * 32, 16, 1024, 2);
+            tc_mma_nvf4(tmem + TM_ACC, ad, bd, IDESC, t_sfa + a * 4, t_sfb + a * 8,
+                        (kb | a) != 0 ? 1u : 0u);
+          }
+          tc_commit(smem_u32(&bar_empty[s]));
+        }
+        if (!ok) break;
+        tc_commit(smem_u32(&bar_acc_full));
+      }
+      // all MMAs issued by this thread complete before the CTA frees tensor memory
+      tc_commit(smem_u32(&bar_drain));
+      volatile int never = 0;
+      mbar_wait_bounded(smem_u32(&bar_drain), 0, &never);
+    }
+    __syncwarp();
+  } else if (warp >= EPI_WARP0) {
+    // =========================== epilogue ===========================
+    const int q = warp - EPI_WARP0;  // lane quadrant of tensor memory
+    const uint32_t t_row = tmem + TM_ACC + (static_cast<uint32_t>(q * 32) << 16);
+    uint32_t tile_it = 0;
+    for (int t = blockIdx.x; t < total; t += gridDim.x, ++tile_it) {
+      const Tile tl = decode_tile(t, tile_start, seg, E, args.n_tiles);
+      if (!mbar_wait_bounded(smem_u32(&bar_acc_full), tile_it & 1u, &abort_flag)) break;
+      tc_fence_after();
+      const float alpha = 1.0f / (__ldg(args.gs_a) * __ldg(args.gs_b + tl.e));
+      const int64_t row = tl.m0 + q * 32 + lane;
+
+      if (MODE == L1_SWIGLU) {
+        const float gs_h = __ldg(args.gs_h);
+        const int I = args.I;
+        uint8_t* hrow = args.h + row * (I / 2) + tl.nt * 64;
+        uint32_t sfw[2] = {0u, 0u};
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t g[32], u[32];
+          tmem_ld32(t_row + 32 * c, g);
+          tmem_ld32(t_row + 128 + 32 * c, u);
+          tmem_wait_ld();
+          float hv[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float gg = __uint_as_float(g[i]) * alpha;
+            const float uu = __uint_as_float(u[i]) * alpha;
+            hv[i] = gg / (1.0f + expf(-gg)) * uu;
+          }
+          uint32_t packed[4];
+#pragma unroll
+          for (int b = 0; b < 2; ++b) {
+            float amax = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(hv[16 * b + i]));
+            float rcp;
+            const uint32_t sb = nvfp4_block_scale(amax, gs_h, rcp);
+            packed[2 * b] = nvfp4_pack8(hv + 16 * b, rcp);
+            packed[2 * b + 1] = nvfp4_pack8(hv + 16 * b + 8, rcp);
+            const int sc = 2 * c + b;  // scale column inside the tile (0..7)
+            sfw[sc >> 2] |= sb << (8 * (sc & 3));
+          }
+          *reinterpret_cast<uint4*>(hrow + 16 * c) =
+              make_uint4(packed[0], packed[1], packed[2], packed[3]);
+        }
+        const int n_sf = I / 16;
+#pragma unroll
+        for (int a = 0; a < 2; ++a)
+          *reinterpret_cast<uint32_t*>(args.sfh + sf_offset(row, tl.nt * 8 + 4 * a, n_sf)) = sfw[a];
+      } else if (MODE == L2_SCATTER) {
+        int tok = __ldg(args.row_token + row);
+        if (tok >= args.T) {
+          report(args.status, NVFP4_DEVERR_BAD_INDEX);
+          tok = -1;
+        }
+        const float scale = alpha * (tok >= 0 ? __ldg(args.row_w + row) : 0.0f);
+        const int H = args.N;
+        float* dst = args.acc + (int64_t)(tok >= 0 ? tok : 0) * H + tl.nt * BN;
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(t_row + 32 * c, v);
+          tmem_wait_ld();
+          if (tok >= 0) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              red_add_v4(dst + 32 * c + 4 * i, __uint_as_float(v[4 * i]) * scale,
+                         __uint_as_float(v[4 * i + 1]) * scale,
+                         __uint_as_float(v[4 * i + 2]) * scale,
+                         __uint_as_float(v[4 * i + 3]) * scale);
+          }
+        }
+      } else {
+        const int N = args.N;
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(t_row + 32 * c, v);
+          tmem_wait_ld();
+          const int64_t col = (int64_t)tl.nt * BN + 32 * c;
+          if (MODE == PLAIN_F32) {
+            float4* o = reinterpret_cast<float4*>(static_cast<float*>(args.out) + row * N + col);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              o[i] = make_float4(__uint_as_float(v[4 * i]) * alpha,
+                                 __uint_as_float(v[4 * i + 1]) * alpha,
+                                 __uint_as_float(v[4 * i + 2]) * alpha,
+                                 __uint_as_float(v[4 * i + 3]) * alpha);
+          } else {
+            uint4* o = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(args.out) + row * N + col);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              uint32_t wds[4];
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                const __nv_bfloat162 p = __floats2bfloat162_rn(
+                    __uint_as_float(v[8 * i + 2 * j]) * alpha,
+                    __uint_as_float(v[8 * i + 2 * j + 1]) * alpha);
+                wds[j] = *reinterpret_cast<const uint32_t*>(&p);
+              }
+              o[i] = make_uint4(wds[0], wds[1], wds[2], wds[3]);
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bar_acc_empty));
+    }
+  }
+
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 2) tmem_dealloc(tmem, TMEM_COLS);
+  if (tid == 0 && abort_flag) report(args.status, NVFP4_DEVERR_TIMEOUT);
+}
+
+// ------------------------------------------------------------------------------ host side
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2D byte tensor [rows][row_bytes], box 128 bytes x 128 rows, 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* base, uint64_t row_bytes, uint64_t rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {row_bytes, rows};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {128, 128};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int num_sms() {
+  int dev = 0, n = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+template <int MODE>
+nvfp4_status_t launch(const uint8_t* a, const uint8_t* b, int64_t b_rows, GemmArgs args,
+                      cudaStream_t s) {
+  CUtensorMap ma, mb;
+  if (!make_map(&ma, a, args.K / 2, args.R_max) || !make_map(&mb, b, args.K / 2, b_rows)) {
+    set_last_error("cuTensorMapEncodeTiled failed");
+    return NVFP4_ERR_CUDA;
+  }
+  static bool attr_set = false;  // per instantiation; idempotent, so a race is harmless
+  if (!attr_set) {
+    if (cudaFuncSetAttribute(grouped_gemm_kernel<MODE>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             SMEM_BYTES) != cudaSuccess)
+      return check_launch("cudaFuncSetAttribute");
+    attr_set = true;
+  }
+  grouped_gemm_kernel<MODE><<<num_sms(), NUM_THREADS, SMEM_BYTES, s>>>(ma, mb, args);
+  return check_launch("grouped_gemm_kernel");
+}
+
+__global__ void cast_bf16_kernel(const float* __restrict__ acc, __nv_bfloat16* __restrict__ out,
+                                 int64_t n8) {
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n8;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const float4 a = reinterpret_cast<const float4*>(acc)[2 * i];
+    const float4 b = reinterpret_cast<const float4*>(acc)[2 * i + 1];
+    const __nv_bfloat162 p0 = __floats2bfloat162_rn(a.x, a.y), p1 = __floats2bfloat162_rn(a.z, a.w),
+                         p2 = __floats2bfloat162_rn(b.x, b.y), p3 = __floats2bfloat162_rn(b.z, b.w);
+    uint4 o;
+    o.x = *reinterpret_cast<const uint32_t*>(&p0);
+    o.y = *reinterpret_cast<const uint32_t*>(&p1);
+    o.z = *reinterpret_cast<const uint32_t*>(&p2);
+    o.w = *reinterpret_cast<const uint32_t*>(&p3);
+    reinterpret_cast<uint4*>(out)[i] = o;
+  }
+}
+
+bool ok_ptr(const void* p) { return p != nullptr && aligned16(p); }
+
+}  // namespace
+
+nvfp4_status_t gemm_plain(const uint8_t* a, const uint8_t* sfa, const float* gs_a, const uint8_t* b,
+                          const uint8_t* sfb, const float* gs_b, const int32_t* offs, int E, int N,
+                          int K, int64_t R_max, void* out, int out_dtype, int32_t* status,
+                          cudaStream_t s) {
+  GemmArgs g{};
+  g.sfa = sfa; g.sfb = sfb; g.gs_a = gs_a; g.gs_b = gs_b; g.offs = offs;
+  g.E = E; g.N = N; g.K = K; g.n_tiles = N / BN; g.R_max = R_max; g.out = out; g.status = status;
+  const int64_t b_rows = (int64_t)E * N;
+  return out_dtype == 0 ? launch<PLAIN_F32>(a, b, b_rows, g, s) : launch<PLAIN_BF16>(a, b, b_rows, g, s);
+}
+
+nvfp4_status_t gemm_l1(const uint8_t* a, const uint8_t* sfa, const float* gs_a, const uint8_t* w1,
+                       const uint8_t* sfw1, const float* gs_w1, const int32_t* offs, int E, int H,
+                       int I, int64_t R_max, const float* gs_h, uint8_t* h, uint8_t* sfh,
+                       int32_t* status, cudaStream_t s) {
+  GemmArgs g{};
+  g.sfa = sfa; g.sfb = sfw1; g.gs_a = gs_a; g.gs_b = gs_w1; g.offs = offs;
+  g.E = E; g.N = 2 * I; g.K = H; g.n_tiles = I / 128; g.R_max = R_max;
+  g.gs_h = gs_h; g.h = h; g.sfh = sfh; g.I = I; g.status = status;
+  return launch<L1_SWIGLU>(a, w1, (int64_t)E * 2 * I, g, s);
+}
+
+nvfp4_status_t gemm_l2(const uint8_t* h, const uint8_t* sfh, const float* gs_h, const uint8_t* w2,
+                       const uint8_t* sfw2, const float* gs_w2, const int32_t* offs,
+                       const int32_t* row_token, const float* row_w, int E, int H, int I, int T,
+                       int64_t R_max, float* acc, void* out_bf16, int32_t* status,
+                       cudaStream_t s) {
+  if (T == 0) return NVFP4_OK;
+  if (cudaMemsetAsync(acc, 0, (size_t)T * H * sizeof(float), s) != cudaSuccess)
+    return check_launch("memset acc");
+  GemmArgs g{};
+  g.sfa = sfh; g.sfb = sfw2; g.gs_a = gs_h; g.gs_b = gs_w2; g.offs = offs;
+  g.E = E; g.N = H; g.K = I; g.n_tiles = H / BN; g.R_max = R_max;
+  g.row_token = row_token; g.row_w = row_w; g.acc = acc; g.T = T; g.status = status;
+  nvfp4_status_t st = launch<L2_SCATTER>(h, w2, (int64_t)E * H, g, s);
+  if (st != NVFP4_OK || out_bf16 == nullptr) return st;
+  const int64_t n8 = (int64_t)T * H / 8;
+  const int64_t want = (n8 + 255) / 256;
+  cast_bf16_kernel<<<(unsigned)(want < 148 * 16 ? want : 148 * 16), 256, 0, s>>>(
+      acc, static_cast<__nv_bfloat16*>(out_bf16), n8);
+  return check_launch("cast_bf16_kernel");
+}
+
+}  // namespace nvfp4
+
+using namespace nvfp4;
+
+extern "C" nvfp4_status_t nvfp4_grouped_gemm(const uint8_t* a, const uint8_t* sfa,
+                                             const float* gs_a, const uint8_t* b,
+                                             const uint8_t* sfb, const float* gs_b,
+                                             const int32_t* offs, int E, int N, int K,
+                                             int64_t R_max, void* out, int out_dtype,
+                                             int32_t* dev_status, nvfp4_stream_t stream) {
+  if (E < 1 || E > MAX_E || N <= 0 || K <= 0 || R_max < 0) return NVFP4_ERR_INVALID_ARG;
+  if (K % 64 || N % BN || R_max % 128) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (out_dtype != 0 && out_dtype != 1) return NVFP4_ERR_INVALID_ARG;
+  if (!gs_a || !gs_b || !offs) return NVFP4_ERR_INVALID_ARG;
+  if (R_max == 0) return NVFP4_OK;
+  if (!ok_ptr(a) || !ok_ptr(sfa) || !ok_ptr(b) || !ok_ptr(sfb) || !ok_ptr(out))
+    return (a && sfa && b && sfb && out) ? NVFP4_ERR_MISALIGNED : NVFP4_ERR_INVALID_ARG;
+  return gemm_plain(a, sfa, gs_a, b, sfb, gs_b, offs, E, N, K, R_max, out, out_dtype, dev_status,
+                    reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" nvfp4_status_t moe_grouped_gemm_l1_swiglu_q(
+    const uint8_t* a, const uint8_t* sfa, const float* gs_a, const uint8_t* w1,
+    const uint8_t* sfw1, const float* gs_w1, const int32_t* offs, int E, int H, int I,
+    int64_t R_max, const float* gs_h, uint8_t* h, uint8_t* sfh, int32_t* dev_status,
+    nvfp4_stream_t stream) {
+  if (E < 1 || E > MAX_E || H <= 0 || I <= 0 || R_max < 0) return NVFP4_ERR_INVALID_ARG;
+  if (H % 64 || I % 128 || R_max % 128) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (!gs_a || !gs_w1 || !offs || !gs_h) return NVFP4_ERR_INVALID_ARG;
+  if (R_max == 0) return NVFP4_OK;
+  if (!ok_ptr(a) || !ok_ptr(sfa) || !ok_ptr(w1) || !ok_ptr(sfw1) || !ok_ptr(h) || !ok_ptr(sfh))
+    return (a && sfa && w1 && sfw1 && h && sfh) ? NVFP4_ERR_MISALIGNED : NVFP4_ERR_INVALID_ARG;
+  return gemm_l1(a, sfa, gs_a, w1, sfw1, gs_w1, offs, E, H, I, R_max, gs_h, h, sfh, dev_status,
+                 reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" nvfp4_status_t moe_grouped_gemm_l2_scatter(
+    const uint8_t* h, const uint8_t* sfh, const float* gs_h, const uint8_t* w2,
+    const uint8_t* sfw2, const float* gs_w2, const int32_t* offs, const int32_t* row_token,
+    const float* row_w, int E, int H, int I, int T, int64_t R_max, float* acc_ws, void* out_bf16,
+    int32_t* dev_status, nvfp4_stream_t stream) {
+  if (E < 1 || E > MAX_E || H <= 0 || I <= 0 || T < 0 || R_max < 0) return NVFP4_ERR_INVALID_ARG;
+  if (H % BN || I % 64 || R_max % 128) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (!gs_h || !gs_w2 || !offs || !row_token || !row_w) return NVFP4_ERR_INVALID_ARG;
+  if (T == 0 || R_max == 0) return NVFP4_OK;
+  if (!ok_ptr(h) || !ok_ptr(sfh) || !ok_ptr(w2) || !ok_ptr(sfw2) || !ok_ptr(acc_ws) ||
+      (out_bf16 && !aligned16(out_bf16)))
+    return (h && sfh && w2 && sfw2 && acc_ws) ? NVFP4_ERR_MISALIGNED : NVFP4_ERR_INVALID_ARG;
+  return gemm_l2(h, sfh, gs_h, w2, sfw2, gs_w2, offs, row_token, row_w, E, H, I, T, R_max, acc_ws,
+                 out_bf16, dev_status, reinterpret_cast<cudaStream_t>(stream));
+}

@@ -1,0 +1,157 @@
+// quantize.cu — BF16 -> NVFP4 quantization (amax -> global scale on the GPU, then codes).
+//
+// Two stream-ordered kernels, as the commit log of dsv4/kernels/cuda (nvfp4-megamoe-kernel)
+// settles on after a single-launch version raced across CTAs: an amax kernel reduces max|x| into
+// one device word, and the quantize kernel derives gs = 2688 / amax from that word itself (no
+// host sync, no .item()).  Codes are computed against the decoded FP8 block scale (the commit
+// log's "quantize must use the FP8-round-tripped block scale").
+#include "common.cuh"
+
+namespace nvfp4 {
+namespace {
+
+constexpr int kThreads = 256;
+
+// max|x| over the (rows x cols) bf16 matrix with row stride ld -> atomicMax on the float bits
+// (non-negative floats order like their bit patterns).
+__global__ void __launch_bounds__(kThreads) amax_kernel(const __nv_bfloat16* __restrict__ x,
+                                                        int64_t rows, int64_t cols, int64_t ld,
+                                                        uint32_t* __restrict__ amax_bits) {
+  const int64_t vec_per_row = cols / 8;
+  const int64_t nvec = rows * vec_per_row;
+  uint32_t m = 0;  // max of |bf16| bit patterns (sign cleared)
+  for (int64_t v = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; v < nvec;
+       v += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t r = v / vec_per_row, c = (v - r * vec_per_row) * 8;
+    const uint4 q = __ldg(reinterpret_cast<const uint4*>(x + r * ld + c));
+    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      m = max(m, w[i] & 0x7FFFu);
+      m = max(m, (w[i] >> 16) & 0x7FFFu);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+  __shared__ uint32_t red[kThreads / 32];
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    uint32_t b = 0;
+    for (int i = 0; i < kThreads / 32; ++i) b = max(b, red[i]);
+    atomicMax(amax_bits, b << 16);  // bf16 bits -> float bits
+  }
+}
+
+// One thread per 16-element block.  gs comes from the amax word (compute mode, and thread 0
+// publishes it to *gs) or is read from *gs.  Codes and the scale byte go to output row i
+// (dst_row == nullptr) or to the k rows dst_row[i*k + j].
+__global__ void __launch_bounds__(kThreads) quantize_kernel(
+    const __nv_bfloat16* __restrict__ x, int64_t rows, int64_t cols, int64_t ld,
+    const int32_t* __restrict__ dst_row, int k, int64_t out_rows, uint8_t* __restrict__ codes,
+    uint8_t* __restrict__ sf, float* __restrict__ gs_io, const uint32_t* __restrict__ amax_bits,
+    int32_t* __restrict__ dev_status) {
+  const int64_t nblk_row = cols / 16;
+  const int64_t nblk = rows * nblk_row;
+  const int64_t gid = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  float gs;
+  if (amax_bits != nullptr) {
+    gs = gs_from_amax(__uint_as_float(__ldg(amax_bits)));
+    if (gid == 0) *gs_io = gs;
+  } else {
+    gs = __ldg(gs_io);
+  }
+  if (gid >= nblk) return;
+  const int64_t r = gid / nblk_row, c = gid - r * nblk_row;
+  const uint4* src = reinterpret_cast<const uint4*>(x + r * ld + c * 16);
+  const uint4 q0 = __ldg(src), q1 = __ldg(src + 1);
+  const uint32_t w[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+  float v[16];
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    v[2 * i] = __uint_as_float(w[i] << 16);
+    v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    amax = fmaxf(amax, fmaxf(fabsf(v[2 * i]), fabsf(v[2 * i + 1])));
+  }
+  float rcp;
+  const uint32_t sbyte = nvfp4_block_scale(amax, gs, rcp);
+  uint2 packed;
+  packed.x = nvfp4_pack8(v, rcp);
+  packed.y = nvfp4_pack8(v + 8, rcp);
+  const int64_t row_bytes = cols / 2;
+  if (dst_row == nullptr) {
+    *reinterpret_cast<uint2*>(codes + r * row_bytes + c * 8) = packed;
+    sf[sf_offset(r, c, nblk_row)] = static_cast<uint8_t>(sbyte);
+    return;
+  }
+  for (int j = 0; j < k; ++j) {
+    const int64_t d = __ldg(dst_row + r * k + j);
+    if (d < 0) continue;
+    if (d >= out_rows) {
+      report(dev_status, NVFP4_DEVERR_BAD_INDEX);
+      continue;
+    }
+    *reinterpret_cast<uint2*>(codes + d * row_bytes + c * 8) = packed;
+    sf[sf_offset(d, c, nblk_row)] = static_cast<uint8_t>(sbyte);
+  }
+}
+
+}  // namespace
+
+nvfp4_status_t quantize_launch(const void* x, int64_t rows, int64_t cols, int64_t ld,
+                               const int32_t* dst_row, int k, int64_t out_rows, uint8_t* codes,
+                               uint8_t* sf, float* gs, int compute_gs, void* ws,
+                               int32_t* dev_status, cudaStream_t s) {
+  uint32_t* amax = nullptr;
+  if (compute_gs) {
+    amax = static_cast<uint32_t*>(ws);
+    if (cudaMemsetAsync(amax, 0, sizeof(uint32_t), s) != cudaSuccess)
+      return check_launch("memset amax");
+    const int64_t nvec = rows * (cols / 8);
+    if (nvec > 0) {
+      const int64_t want = (nvec + kThreads - 1) / kThreads;
+      const int grid = static_cast<int>(want < 148 * 8 ? want : 148 * 8);
+      amax_kernel<<<grid, kThreads, 0, s>>>(static_cast<const __nv_bfloat16*>(x), rows, cols, ld,
+                                            amax);
+      nvfp4_status_t st = check_launch("amax_kernel");
+      if (st != NVFP4_OK) return st;
+    }
+  }
+  const int64_t nblk = rows * (cols / 16);
+  const int64_t grid = nblk > 0 ? (nblk + kThreads - 1) / kThreads : 1;
+  quantize_kernel<<<static_cast<unsigned>(grid), kThreads, 0, s>>>(
+      static_cast<const __nv_bfloat16*>(x), rows, cols, ld, dst_row, k, out_rows, codes, sf, gs,
+      amax, dev_status);
+  return check_launch("quantize_kernel");
+}
+
+}  // namespace nvfp4
+
+extern "C" size_t nvfp4_quantize_workspace_size(void) { return 256; }
+
+extern "C" nvfp4_status_t nvfp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t ld,
+                                         const int32_t* dst_row, int k, int64_t out_rows,
+                                         uint8_t* codes, uint8_t* sf, float* gs, int compute_gs,
+                                         void* ws, size_t ws_bytes, int32_t* dev_status,
+                                         nvfp4_stream_t stream) {
+  using namespace nvfp4;
+  if (rows < 0 || out_rows < 0 || cols <= 0 || ld < cols) return NVFP4_ERR_INVALID_ARG;
+  if (cols % 64 != 0 || ld % 8 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (gs == nullptr) return NVFP4_ERR_INVALID_ARG;
+  if (rows > 0 && (x == nullptr || codes == nullptr || sf == nullptr)) return NVFP4_ERR_INVALID_ARG;
+  if (dst_row == nullptr) {
+    if (out_rows < rows) return NVFP4_ERR_INVALID_ARG;
+  } else if (k < 1 || k > 64) {
+    return NVFP4_ERR_INVALID_ARG;
+  }
+  if (compute_gs) {
+    if (ws == nullptr) return NVFP4_ERR_INVALID_ARG;
+    if (ws_bytes < nvfp4_quantize_workspace_size()) return NVFP4_ERR_WORKSPACE_TOO_SMALL;
+  }
+  if (!aligned16(x) || !aligned16(codes) || !aligned16(sf) || !aligned16(ws) ||
+      (reinterpret_cast<uintptr_t>(gs) & 3u) || (reinterpret_cast<uintptr_t>(dst_row) & 3u))
+    return NVFP4_ERR_MISALIGNED;
+  return quantize_launch(x, rows, cols, ld, dst_row, k, out_rows, codes, sf, gs, compute_gs, ws,
+                         dev_status, reinterpret_cast<cudaStream_t>(stream));
+}

@@ -6,7 +6,7 @@ top-8), matching the pages' model (DSV4 NVFP4 MegaMoE); no trained weights are u
 Seeds and order (torch generators):
   logits : seed                    (CPU)
   x      : seed + 1                (CPU), drawn in float32 then rounded to bf16
-  W1[e]  : 1000 * seed + e         (N(0, 0.02), float32, on the requested device)
+  W1[e]  : 1000 * seed + e         (N(0, 0.02) in float32, rounded to bf16, on the requested device)
   W2[e]  : 1000 * seed + 500 + e
 For the E=256 workloads the weights are drawn on the GPU (6+ GB of float32 would take minutes
 on the host); a check that needs an expert's floats on the host copies them back.
@@ -29,6 +29,7 @@ class MoEConfig:
     x_outliers: bool = False
     seed: int = 0
     renormalize: bool = True
+    gs_h: float = 1.0    # static global scale of the intermediate h (calibrated per shape)
 
     @property
     def slots(self):
@@ -50,7 +51,7 @@ class SweepConfig:
 
 
 CONFIGS = {
-    "tiny": MoEConfig("tiny", T=64, H=256, I=128, E=8, k=2, logits="normal"),
+    "tiny": MoEConfig("tiny", T=64, H=256, I=128, E=8, k=2, logits="normal", gs_h=64.0),
     "decode": MoEConfig("decode", T=16, H=7168, I=2048, E=256, k=8, logits="uniform"),
     "mid": MoEConfig("mid", T=512, H=7168, I=2048, E=256, k=8, logits="zipf_gumbel", x_outliers=True),
     "prefill": MoEConfig("prefill", T=8192, H=7168, I=2048, E=256, k=8, logits="uniform"),
@@ -101,10 +102,12 @@ def gen_x(cfg, T=None, H=None):
 
 
 def gen_weight_expert(seed, which, e, N, K, device="cpu", std=0.02):
-    """Float32 (N, K) weight of expert e: which=1 for W1 (2I x H), 2 for W2 (H x I)."""
+    """bf16 (N, K) weight of expert e (drawn in float32, rounded to bf16 like model weights):
+    which=1 for W1 (2I x H, gate rows then up rows), 2 for W2 (H x I)."""
     s = 1000 * seed + (0 if which == 1 else 500) + e
     g = torch.Generator(device=device).manual_seed(s)
-    return torch.randn(N, K, generator=g, dtype=torch.float32, device=device) * std
+    w = torch.randn(N, K, generator=g, dtype=torch.float32, device=device) * std
+    return w.to(torch.bfloat16)
 
 
 def gen_sweep(cfg, device="cpu"):

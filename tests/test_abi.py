@@ -1,0 +1,106 @@
+"""CPU checks of the C ABI: the library builds, loads, exports every entry point the header
+declares, and rejects bad arguments on the host before touching the GPU."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from nvfp4_block_scaled_gsa_b200 import build as B
+from nvfp4_block_scaled_gsa_b200 import _native as N
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include",
+                      "nvfp4_moe.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    B.build()
+    return N.lib()
+
+
+def declared_names():
+    text = open(HEADER).read()
+    return re.findall(r"NVFP4_API\s+[\w\s\*]+?\b(\w+)\s*\(", text)
+
+
+def test_header_declares_the_entry_points():
+    names = set(declared_names())
+    for must in ["nvfp4_quantize", "moe_permute", "moe_grouped_gemm_l1_swiglu_q",
+                 "moe_grouped_gemm_l2_scatter", "moe_ffn_forward", "nvfp4_grouped_gemm"]:
+        assert must in names
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = declared_names()
+    assert len(names) >= 13
+    for n in names:
+        assert hasattr(L, n), n
+    assert set(names) == set(N.SIGNATURES), "binding signatures out of sync with the header"
+
+
+def test_host_only_queries(L):
+    assert L.nvfp4_abi_version() == 1
+    assert L.nvfp4_quantize_workspace_size() == 256
+    assert L.moe_rows_max(16, 256, 8) == 128 + 127 * 128  # 128 slots, at most 128 busy experts
+    assert L.moe_rows_max(8192, 256, 8) == 65536 + 127 * 256
+    assert L.moe_rows_max(0, 8, 2) == 0
+    assert L.moe_rows_max(64, 8, 2) == 128 + 127 * 8 + 8  # rounded up to 128
+    big = L.moe_ffn_workspace_size(8192, 7168, 2048, 256, 8)
+    R = L.moe_rows_max(8192, 256, 8)
+    assert big >= R * (7168 // 2 + 7168 // 16 + 2048 // 2 + 2048 // 16) + 8192 * 7168 * 4
+    assert L.moe_ffn_workspace_size(0, 7168, 2048, 256, 8) > 0
+    assert L.moe_ffn_workspace_size(-1, 7168, 2048, 256, 8) == 0
+
+
+FAKE = ctypes.c_void_p(1 << 20)  # never dereferenced: every call below fails host validation
+
+
+@pytest.mark.parametrize("args,code", [
+    # rows, cols, ld, dst, k, out_rows, compute_gs
+    ((4, 65, 65, None, 1, 4, 1), 2),     # cols % 64
+    ((4, 64, 60, None, 1, 4, 1), 1),     # ld < cols
+    ((4, 64, 66, None, 1, 4, 1), 2),     # ld % 8
+    ((4, 64, 64, None, 1, 2, 1), 1),     # out_rows < rows without a row map
+    ((4, 64, 64, FAKE, 0, 4, 1), 1),     # k = 0
+    ((-1, 64, 64, None, 1, 4, 1), 1),    # negative rows
+])
+def test_quantize_rejects_bad_arguments(L, args, code):
+    rows, cols, ld, dst, k, out_rows, comp = args
+    rc = L.nvfp4_quantize(FAKE, rows, cols, ld, dst, k, out_rows, FAKE, FAKE, FAKE, comp, FAKE,
+                          256, None, None)
+    assert rc == code
+
+
+def test_quantize_rejects_misaligned_and_small_workspace(L):
+    odd = ctypes.c_void_p((1 << 20) + 8)
+    assert L.nvfp4_quantize(odd, 4, 64, 64, None, 1, 4, FAKE, FAKE, FAKE, 1, FAKE, 256, None,
+                            None) == 3
+    assert L.nvfp4_quantize(FAKE, 4, 64, 64, None, 1, 4, FAKE, FAKE, FAKE, 1, FAKE, 4, None,
+                            None) == 4
+
+
+def test_permute_rejects_bad_shapes(L):
+    f = FAKE
+    assert L.moe_permute(f, 4, 0, 1, 1, f, f, f, f, f, f, None, 0, None, None) == 2     # E = 0
+    assert L.moe_permute(f, 4, 300, 8, 1, f, f, f, f, f, f, None, 0, None, None) == 2   # E > 256
+    assert L.moe_permute(f, 4, 8, 9, 1, f, f, f, f, f, f, None, 0, None, None) == 2     # k > E
+    assert L.moe_permute(f, 4, 64, 33, 1, f, f, f, f, f, f, None, 0, None, None) == 2   # k > 32
+    assert L.moe_permute(f, 4, 8, 2, 1, f, f, None, f, f, f, None, 0, None, None) == 1  # offs
+
+
+def test_gemms_reject_bad_shapes(L):
+    f = FAKE
+    assert L.nvfp4_grouped_gemm(f, f, f, f, f, f, f, 2, 200, 64, 128, f, 0, None, None) == 2
+    assert L.nvfp4_grouped_gemm(f, f, f, f, f, f, f, 2, 256, 96, 128, f, 0, None, None) == 2
+    assert L.nvfp4_grouped_gemm(f, f, f, f, f, f, f, 2, 256, 64, 100, f, 0, None, None) == 2
+    assert L.nvfp4_grouped_gemm(f, f, f, f, f, f, f, 2, 256, 64, 128, f, 7, None, None) == 1
+    assert L.moe_grouped_gemm_l1_swiglu_q(f, f, f, f, f, f, f, 8, 256, 96, 128, f, f, f, None,
+                                          None) == 2  # I % 128
+    assert L.moe_grouped_gemm_l2_scatter(f, f, f, f, f, f, f, f, f, 8, 200, 128, 4, 128, f, f,
+                                         None, None) == 2  # H % 256
+    assert L.moe_ffn_forward(f, f, 4, 256, 128, 8, 2, f, f, f, f, f, f, f, f, f, 10, None,
+                             None) == 4  # workspace too small
+    assert L.moe_ffn_forward(f, f, 4, 256, 128, 8, 2, f, f, f, f, f, f, f, f, None, 1 << 30, None,
+                             None) == 1

@@ -1,0 +1,86 @@
+"""GPU parity of the whole expert FFN (moe_ffn_forward) and of the weight pre-pack, against the
+oracle: final bf16 output within relative Frobenius 1e-3 and cosine >= 0.9999."""
+
+import numpy as np
+import pytest
+import torch
+
+import nvfp4_block_scaled_gsa_b200 as nv
+from oracle import formats as F
+from oracle import moe as M
+from oracle import quant as Q
+from synth import CONFIGS, gen_logits, gen_weight_expert, gen_x
+from tests._gpu_util import DEV, cosine, rel_fro
+
+pytestmark = pytest.mark.gpu
+
+
+def _prepack_both(cfg, which, N, K):
+    wf = [gen_weight_expert(cfg.seed, which, e, N, K) for e in range(cfg.E)]
+    wd = nv.quantize_weights(lambda e: wf[e].to(DEV), cfg.E, N, K)
+    wo = M.QuantWeights.from_float(np.stack([w.float().numpy() for w in wf]))
+    return wd, wo
+
+
+def test_weight_prepack_bit_exact():
+    cfg = CONFIGS["tiny"]
+    wd, wo = _prepack_both(cfg, 1, 2 * cfg.I, cfg.H)
+    torch.cuda.synchronize()
+    E, N, K = cfg.E, 2 * cfg.I, cfg.H
+    assert np.array_equal(wd.gs.cpu().numpy(), wo.gs)
+    assert np.array_equal(wd.codes.cpu().numpy(), wo.codes.reshape(E * N, K // 2))
+    assert np.array_equal(Q.untile_sf(wd.sf.cpu().numpy(), E * N, K // 16), wo.sf.reshape(E * N, -1))
+
+
+def _ffn_check(cfg, x, lg):
+    w1d, w1o = _prepack_both(cfg, 1, 2 * cfg.I, cfg.H)
+    w2d, w2o = _prepack_both(cfg, 2, cfg.H, cfg.I)
+    gs_h = torch.tensor([cfg.gs_h], dtype=torch.float32, device=DEV)
+    out = nv.moe_ffn_forward(x.to(DEV), lg.to(DEV), cfg.k, w1d, w2d, gs_h)
+    torch.cuda.synchronize()
+    ref = M.moe_ffn(x.float().numpy(), lg.numpy(), cfg.k, w1o, w2o, np.float32(cfg.gs_h))
+    got = out.float().cpu().numpy()
+    return got, ref
+
+
+def test_ffn_tiny_end_to_end():
+    cfg = CONFIGS["tiny"]
+    got, ref = _ffn_check(cfg, gen_x(cfg), gen_logits(cfg))
+    assert rel_fro(got, ref["out"]) <= 1e-3
+    assert cosine(got, ref["out"]) >= 0.9999
+
+
+def test_ffn_tokens_with_all_slots_dropped_are_zero():
+    cfg = CONFIGS["tiny"]
+    lg = gen_logits(cfg)
+    lg[5] = float("-inf")
+    lg[17] = float("-inf")
+    got, ref = _ffn_check(cfg, gen_x(cfg), lg)
+    assert np.all(got[5] == 0) and np.all(got[17] == 0)
+    assert rel_fro(got, ref["out"]) <= 1e-3
+
+
+def test_ffn_repeatable_and_workspace_reuse():
+    cfg = CONFIGS["tiny"]
+    x, lg = gen_x(cfg).to(DEV), gen_logits(cfg).to(DEV)
+    w1d, _ = _prepack_both(cfg, 1, 2 * cfg.I, cfg.H)
+    w2d, _ = _prepack_both(cfg, 2, cfg.H, cfg.I)
+    gs_h = torch.tensor([cfg.gs_h], dtype=torch.float32, device=DEV)
+    ws = torch.empty(nv.ffn_workspace_bytes(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k), dtype=torch.uint8,
+                     device=DEV)
+    a = nv.moe_ffn_forward(x, lg, cfg.k, w1d, w2d, gs_h, ws=ws).clone()
+    b = nv.moe_ffn_forward(x, lg, cfg.k, w1d, w2d, gs_h, ws=ws)
+    torch.cuda.synchronize()
+    # FP32 reduction order may differ between runs; the bf16 results agree to rounding
+    assert rel_fro(a.float().cpu().numpy(), b.float().cpu().numpy()) <= 1e-3
+
+
+def test_ffn_rejects_small_workspace():
+    cfg = CONFIGS["tiny"]
+    x, lg = gen_x(cfg).to(DEV), gen_logits(cfg).to(DEV)
+    w1d, _ = _prepack_both(cfg, 1, 2 * cfg.I, cfg.H)
+    w2d, _ = _prepack_both(cfg, 2, cfg.H, cfg.I)
+    ws = torch.empty(1024, dtype=torch.uint8, device=DEV)
+    with pytest.raises(nv.Nvfp4Error) as ei:
+        nv.moe_ffn_forward(x, lg, cfg.k, w1d, w2d, torch.ones(1, device=DEV), ws=ws)
+    assert ei.value.code == 4

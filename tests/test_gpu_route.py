@@ -1,0 +1,66 @@
+"""GPU parity: moe_permute (top-k softmax routing + expert-bucketed rows) against the oracle.
+Ids, offsets and the row map are compared exactly; weights to float32 accuracy."""
+
+import numpy as np
+import pytest
+import torch
+
+import nvfp4_block_scaled_gsa_b200 as nv
+from oracle import routing as R
+from synth import CONFIGS, gen_logits
+from tests._gpu_util import DEV, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+def _compare(p, ids_ref, w_ref, E, k):
+    torch.cuda.synchronize()
+    T = ids_ref.shape[0]
+    pr = R.permute(ids_ref, w_ref, E)
+    assert np.array_equal(p["ids"].cpu().numpy(), ids_ref)
+    assert np.allclose(p["weights"].cpu().numpy(), w_ref, rtol=2e-6, atol=1e-7)
+    assert np.array_equal(p["offs"].cpu().numpy(), pr["offs"])
+    assert np.array_equal(p["dst_row"].cpu().numpy().reshape(T, k), pr["dst_row"])
+    Rm = p["R_max"]
+    rt = p["row_token"].cpu().numpy()[:Rm]
+    rw = p["row_w"].cpu().numpy()[:Rm]
+    n = pr["R"]
+    assert np.array_equal(rt[:n], pr["row_token"])
+    assert np.all(rt[n:] == -1) and np.all(rw[n:] == 0)
+    assert np.allclose(rw[:n], pr["row_w"], rtol=2e-6, atol=1e-7)
+
+
+@pytest.mark.parametrize("name", ["tiny", "decode", "mid", "prefill"])
+def test_route_configs(name):
+    cfg = CONFIGS[name]
+    lg = gen_logits(cfg)
+    p = nv.permute(lg.to(DEV), cfg.k)
+    ids_ref, w_ref = R.route_topk(lg.numpy(), cfg.k)
+    _compare(p, ids_ref, w_ref, cfg.E, cfg.k)
+    if name == "mid":  # the masked experts are empty
+        assert (np.diff(p["offs"].cpu().numpy()) == 0).sum() >= 8
+
+
+def test_route_no_renormalize_and_ties():
+    lg = torch.tensor([[1.0, 3.0, 3.0, 0.0, 3.0], [0.0] * 5, [-np.inf, 2.0, -np.inf, -np.inf, 1.0]],
+                      dtype=torch.float32)
+    p = nv.permute(lg.to(DEV), 3, renormalize=False)
+    ids_ref, w_ref = R.route_topk(lg.numpy(), 3, renormalize=False)
+    _compare(p, ids_ref, w_ref, 5, 3)
+
+
+def test_route_given_ids_with_dropped_slots():
+    rng = np.random.default_rng(0)
+    T, E, k = 300, 16, 4
+    ids = rng.integers(0, E, size=(T, k)).astype(np.int32)
+    ids[rng.random((T, k)) < 0.2] = -1
+    w = rng.random((T, k)).astype(np.float32)
+    p = nv.permute(None, k, ids=to_dev(ids), weights=to_dev(w), E=E)
+    _compare(p, ids, w, E, k)
+
+
+def test_route_empty_batch():
+    lg = torch.zeros(0, 8, dtype=torch.float32, device=DEV)
+    p = nv.permute(lg, 2)
+    torch.cuda.synchronize()
+    assert p["offs"].cpu().tolist() == [0] * 9 and p["R_max"] == 0

@@ -122,8 +122,8 @@ def _tiny_inputs(E=8, T=64, H=256, I=128, k=2, seed=0):
     cfg = CONFIGS["tiny"]
     x = gen_x(cfg).float().numpy()[:T, :H]
     lg = gen_logits(cfg).numpy()[:T, :E]
-    w1 = M.QuantWeights.from_float(np.stack([gen_weight_expert(seed, 1, e, 2 * I, H).numpy() for e in range(E)]))
-    w2 = M.QuantWeights.from_float(np.stack([gen_weight_expert(seed, 2, e, H, I).numpy() for e in range(E)]))
+    w1 = M.QuantWeights.from_float(np.stack([gen_weight_expert(seed, 1, e, 2 * I, H).float().numpy() for e in range(E)]))
+    w2 = M.QuantWeights.from_float(np.stack([gen_weight_expert(seed, 2, e, H, I).float().numpy() for e in range(E)]))
     return x, lg, w1, w2
 
 
