@@ -1,0 +1,453 @@
+"""Throughput of the NVFP4 MoE expert-FFN hot path on B200 (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config decode|mid|prefill|tiny]
+                    [--impl ours|reference] [--no-cpu-baseline] [--experts E]
+
+A step is one pass of the whole path over one batch: routing (top-k + expert buckets), amax ->
+global scale -> NVFP4 quantization of the activations, L1 grouped GEMM with SwiGLU + FP4
+re-quantization, L2 grouped GEMM with routing weight + scatter-add, bf16 output.  Inputs are
+resident in HBM when the timed region starts; the same work through moe_ffn_forward with
+host<->device copies inside the timed region gives `e2e`.
+
+The default workload is the decode configuration (T=16 tokens, hidden 7168, intermediate 2048,
+256 experts, top-8 over uniform random logits): weight-bandwidth bound, so `value` is the
+algorithmic HBM traffic per second (GB/s) and `tflops` rides along.  Multi-GPU runs are
+independent replicas (the path has no exchange step on one node's data-parallel batch), so the
+scaling is weak and `value` sums the ranks' bytes over the slowest rank's time.
+
+--impl reference times the CPU oracle (numpy, float64) on a bounded sample of the same workload.
+"""
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE FFN TFLOPS & HBM GB/s on 1 B200, % of NVFP4 tensor/HBM roofline"
+FP4_ELEM_BYTES = 0.5 + 1.0 / 16.0  # E2M1 code + one E4M3 scale per 16 elements
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--config", default="decode")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--experts", type=int, default=0,
+                    help="override E (smaller weight set for profiling captures)")
+    ap.add_argument("--soak", type=float, default=1.0,
+                    help="seconds of extra warm-up load so clock samples cover the timed region")
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------------------- accounting
+
+def algorithmic(cfg, counts):
+    """FLOPs and bytes of one step, and per-kernel bytes of the two GEMM launches.
+
+    Weights of the experts that received tokens (codes + scales), x read as bf16, x codes written
+    and read once per token, h codes written and read once per slot, bf16 output written, logits
+    read.  Padding rows and the FP32 scatter buffer are implementation overhead, not counted."""
+    T, H, I, E, k = cfg.T, cfg.H, cfg.I, cfg.E, cfg.k
+    active = sum(1 for c in counts if c > 0)
+    slots = sum(counts)
+    w1 = 2 * I * H * FP4_ELEM_BYTES
+    w2 = H * I * FP4_ELEM_BYTES
+    x_q = T * H * FP4_ELEM_BYTES
+    h_q = slots * I * FP4_ELEM_BYTES
+    total = active * (w1 + w2) + T * H * 2 + 2 * x_q + 2 * h_q + T * H * 2 + T * E * 4
+    flops = 2 * slots * (H * 2 * I + I * H)
+    l1 = active * w1 + slots * H * FP4_ELEM_BYTES + h_q
+    l2 = active * w2 + h_q + T * H * 4
+    return dict(flops=flops, bytes=total, active=active, slots=slots, l1_bytes=l1, l2_bytes=l2,
+                l1_flops=2 * slots * H * 2 * I, l2_flops=2 * slots * I * H)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm=float(d["hbm_gbs"]), bf16=float(d["bf16_tflops"]),
+                    bf16_sust=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), src="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sust=1400.0, src="fallback")
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.p = None
+        try:
+            self.p = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-i", str(gpu_index)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.p = None
+
+    def stop(self):
+        if self.p is None:
+            return dict(sm_mhz=None, sm_max_mhz=None, reasons=["nvidia-smi unavailable"], samples=0)
+        self.p.terminate()
+        out, _ = self.p.communicate(timeout=10)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return dict(sm_mhz=statistics.median(sm) if sm else None,
+                    sm_max_mhz=max(smax) if smax else None, reasons=sorted(reasons),
+                    samples=len(sm))
+
+
+# ----------------------------------------------------------------------------- our arm
+
+class Plan:
+    """Pre-allocated buffers for the staged path (same kernels as moe_ffn_forward)."""
+
+    def __init__(self, nv, cfg, x, logits, w1, w2, gs_h):
+        import torch
+        self.nv, self.cfg = nv, cfg
+        T, H, I, E, k = cfg.T, cfg.H, cfg.I, cfg.E, cfg.k
+        dev = x.device
+        self.x, self.logits, self.w1, self.w2, self.gs_h = x, logits, w1, w2, gs_h
+        self.R = nv.rows_max(T, E, k)
+        u8, i32, f32 = torch.uint8, torch.int32, torch.float32
+        e = lambda n, t: torch.empty(max(int(n), 1), dtype=t, device=dev)  # noqa: E731
+        self.ids, self.w = e(T * k, i32), e(T * k, f32)
+        self.offs, self.dst = e(E + 1, i32), e(T * k, i32)
+        self.row_token, self.row_w = e(self.R, i32), e(self.R, f32)
+        self.xq, self.xsf = e(self.R * H // 2, u8), e(self.R * H // 16, u8)
+        self.gs_x, self.qws = e(1, f32), e(256, u8)
+        self.hq, self.hsf = e(self.R * I // 2, u8), e(self.R * I // 16, u8)
+        self.acc = e(T * H, f32)
+        self.out = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+        self.status = torch.zeros(1, dtype=i32, device=dev)
+
+    def step(self, ev=None):
+        from nvfp4_block_scaled_gsa_b200._native import call
+        import torch
+        nv, c = self.nv, self.cfg
+        T, H, I, E, k = c.T, c.H, c.I, c.E, c.k
+        s = torch.cuda.current_stream().cuda_stream
+        p = lambda t: t.data_ptr()  # noqa: E731
+        if ev:
+            ev[0].record()
+        call("moe_permute", p(self.logits), T, E, k, 1, p(self.ids), p(self.w), p(self.offs),
+             p(self.dst), p(self.row_token), p(self.row_w), None, 0, p(self.status), s)
+        if ev:
+            ev[1].record()
+        call("nvfp4_quantize", p(self.x), T, H, H, p(self.dst), k, self.R, p(self.xq), p(self.xsf),
+             p(self.gs_x), 1, p(self.qws), 256, p(self.status), s)
+        if ev:
+            ev[2].record()
+        call("moe_grouped_gemm_l1_swiglu_q", p(self.xq), p(self.xsf), p(self.gs_x),
+             p(self.w1.codes), p(self.w1.sf), p(self.w1.gs), p(self.offs), E, H, I, self.R,
+             p(self.gs_h), p(self.hq), p(self.hsf), p(self.status), s)
+        if ev:
+            ev[3].record()
+        call("moe_grouped_gemm_l2_scatter", p(self.hq), p(self.hsf), p(self.gs_h),
+             p(self.w2.codes), p(self.w2.sf), p(self.w2.gs), p(self.offs), p(self.row_token),
+             p(self.row_w), E, H, I, T, self.R, p(self.acc), p(self.out), p(self.status), s)
+        if ev:
+            ev[4].record()
+
+
+KERNELS_PER_STEP = 7  # topk, permute, amax, quantize, L1 GEMM, L2 GEMM, bf16 cast
+
+
+def make_config(args):
+    from dataclasses import replace
+
+    from synth import CONFIGS
+    cfg = CONFIGS[args.config]
+    if args.experts:
+        cfg = replace(cfg, E=args.experts, name=f"{cfg.name}-E{args.experts}")
+    return cfg
+
+
+def setup_inputs(cfg, dev):
+    import torch
+
+    import nvfp4_block_scaled_gsa_b200 as nv
+    from synth import gen_logits, gen_weight_expert, gen_x
+    logits = gen_logits(cfg)
+    x = gen_x(cfg)
+    w1 = nv.quantize_weights(lambda e: gen_weight_expert(cfg.seed, 1, e, 2 * cfg.I, cfg.H, device=dev),
+                             cfg.E, 2 * cfg.I, cfg.H, device=dev)
+    w2 = nv.quantize_weights(lambda e: gen_weight_expert(cfg.seed, 2, e, cfg.H, cfg.I, device=dev),
+                             cfg.E, cfg.H, cfg.I, device=dev)
+    gs_h = torch.tensor([cfg.gs_h], dtype=torch.float32, device=dev)
+    return logits, x, w1, w2, gs_h
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import nvfp4_block_scaled_gsa_b200 as nv
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local = int(os.environ.get("LOCAL_RANK", 0))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    cfg = make_config(args)
+    logits_cpu, x_cpu, w1, w2, gs_h = setup_inputs(cfg, dev)
+    logits, x = logits_cpu.to(dev), x_cpu.to(dev)
+    plan = Plan(nv, cfg, x, logits, w1, w2, gs_h)
+
+    for _ in range(max(args.warmup, 3)):
+        plan.step()
+    torch.cuda.synchronize()
+    ids = plan.ids[: cfg.T * cfg.k].cpu()  # tokens per expert, for the byte count
+    real = torch.bincount(ids[ids >= 0].long(), minlength=cfg.E).tolist()
+    acc = algorithmic(cfg, real)
+
+    # clock soak: keep the GPU under the same load so samples cover the timed region
+    sampler = ClockSampler(local) if rank == 0 else None
+    t_end = time.time() + args.soak
+    while time.time() < t_end:
+        for _ in range(8):
+            plan.step()
+        torch.cuda.synchronize()
+
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    start.record()
+    for i in range(K):
+        plan.step(evs[i])
+    stop.record()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop() if sampler else None
+    total_ms = start.elapsed_time(stop)
+    stage = [[evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(K)] for j in range(4)]
+    l1_ms = statistics.mean(stage[2])
+    l2_ms = statistics.mean(stage[3])
+    code, rc = nv.read_status(plan.status)
+    if code != 0:
+        raise RuntimeError(f"device status {code} after the timed region")
+
+    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms = float(t.item())
+    ms_step = total_ms / K
+    value = world * acc["bytes"] * K / (total_ms * 1e-3) / 1e9
+    tflops = world * acc["flops"] * K / (total_ms * 1e-3) / 1e12
+
+    # ---- end to end through moe_ffn_forward with host buffers (pinned), copies timed
+    x_h = x_cpu.pin_memory()
+    lg_h = logits_cpu.pin_memory()
+    out_h = torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16).pin_memory()
+    x_d, lg_d = torch.empty_like(x), torch.empty_like(logits)
+    out_d = torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(nv.ffn_workspace_bytes(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k), dtype=torch.uint8,
+                     device=dev)
+
+    def e2e_step():
+        x_d.copy_(x_h, non_blocking=True)
+        lg_d.copy_(lg_h, non_blocking=True)
+        nv.moe_ffn_forward(x_d, lg_d, cfg.k, w1, w2, gs_h, out=out_d, ws=ws, status=plan.status)
+        out_h.copy_(out_d, non_blocking=True)
+
+    for _ in range(max(args.warmup, 3)):
+        e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s2.record()
+    for _ in range(K):
+        e2e_step()
+    e2.record()
+    torch.cuda.synchronize()
+    t2 = torch.tensor([s2.elapsed_time(e2)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.barrier()
+        dist.all_reduce(t2, op=dist.ReduceOp.MAX)
+    e2e_ms = float(t2.item())
+    e2e_value = world * acc["bytes"] * K / (e2e_ms * 1e-3) / 1e9
+    h2d = x_h.numel() * x_h.element_size() + lg_h.numel() * lg_h.element_size()
+    d2h = out_h.numel() * out_h.element_size()
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(cfg, logits_cpu, x_cpu, dev)
+
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    peaks = load_peaks()
+    l1_gbs = acc["l1_bytes"] / (l1_ms * 1e-3) / 1e9
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4 (e2m1 + e4m3/16), fp32 accumulate",
+        "data": "synthetic (seeded N(0,1) bf16 activations, N(0,0.02) bf16 weights quantized "
+                "to NVFP4 on the GPU; no trained weights)",
+        "config": {"workload": f"{cfg.name} MoE FFN: T={cfg.T}, H={cfg.H}, I={cfg.I}, E={cfg.E}, "
+                               f"top-{cfg.k} ({cfg.logits} logits)",
+                   "parallelism": f"replicas x{world}",
+                   "l2": f"no flush: each step streams {acc['active']} experts' weights "
+                         f"({acc['active'] * (3 * cfg.I * cfg.H) * FP4_ELEM_BYTES / 1e9:.2f} GB) "
+                         "> 126 MB L2"},
+        "tflops": round(tflops, 3),
+        "algorithmic": {"bytes_per_step": int(acc["bytes"]), "flops_per_step": int(acc["flops"]),
+                        "active_experts": acc["active"], "slots": acc["slots"]},
+        "roofline": {"bound": "hbm", "kernel": "grouped_gemm_kernel<L1_SWIGLU>",
+                     "achieved": round(l1_gbs, 1), "peak": peaks["hbm"], "unit": "GB/s",
+                     "frac": round(l1_gbs / peaks["hbm"], 4), "traffic": None,
+                     "peak_source": peaks["src"],
+                     "step_frac": round(value / world / peaks["hbm"], 4)},
+        "stages_ms": {"route": round(statistics.mean(stage[0]), 4),
+                      "quantize": round(statistics.mean(stage[1]), 4),
+                      "l1_gemm_swiglu_q": round(l1_ms, 4), "l2_gemm_scatter": round(l2_ms, 4)},
+        "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms / K, 4)},
+        "gpu_launches": KERNELS_PER_STEP * K,
+        "clocks": clocks,
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- oracle
+
+class _SparseWeights:
+    """Quantized weights of a few experts, for the oracle's sampled run."""
+
+    def __init__(self, E, N, parts):
+        self.E, self.N, self.parts = E, N, parts
+
+    def dequant(self, e):
+        return self.parts[e].dequant(0)
+
+
+def _oracle_sample(cfg, logits_cpu, x_cpu, dev, n_tokens=1):
+    """Bounded oracle sample: the first n_tokens tokens and the experts they route to.  Weight
+    pre-packing (quantizing the float weights with the oracle) is done here, untimed."""
+    import numpy as np
+
+    from oracle import moe as M
+    from oracle import routing as R
+    from synth import gen_weight_expert
+    lg = logits_cpu[:n_tokens].numpy()
+    x = x_cpu[:n_tokens].float().numpy()
+    ids, _ = R.route_topk(lg, cfg.k)
+    experts = sorted(set(int(e) for e in ids.ravel() if e >= 0))
+    p1, p2 = {}, {}
+    for e in experts:
+        w1 = gen_weight_expert(cfg.seed, 1, e, 2 * cfg.I, cfg.H, device=dev).float().cpu().numpy()
+        w2 = gen_weight_expert(cfg.seed, 2, e, cfg.H, cfg.I, device=dev).float().cpu().numpy()
+        p1[e] = M.QuantWeights.from_float(w1[None])
+        p2[e] = M.QuantWeights.from_float(w2[None])
+    W1 = _SparseWeights(cfg.E, 2 * cfg.I, p1)
+    W2 = _SparseWeights(cfg.E, cfg.H, p2)
+
+    def run():
+        return M.moe_ffn(x, lg, cfg.k, W1, W2, np.float32(cfg.gs_h))
+
+    counts = [0] * cfg.E
+    for e in ids.ravel():
+        if e >= 0:
+            counts[int(e)] += 1
+    from dataclasses import replace
+    return run, algorithmic(replace(cfg, T=n_tokens), counts), experts
+
+
+def _threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = max((d.get("num_threads", 1) for d in threadpool_info()), default=1)
+    except Exception:
+        n = 1
+    return n
+
+
+def cpu_baseline(cfg, logits_cpu, x_cpu, dev):
+    run, acc, experts = _oracle_sample(cfg, logits_cpu, x_cpu, dev)
+    t0 = time.perf_counter()
+    run()
+    dt = time.perf_counter() - t0
+    return {"value": round(acc["bytes"] / dt / 1e9, 4), "unit": "GB/s", "cores": _threads(),
+            "kind": "oracle",
+            "sample": f"1 of {cfg.T} tokens of the {cfg.name} workload ({len(experts)} experts, "
+                      f"{acc['bytes'] / 1e6:.0f} MB algorithmic) in {dt:.1f} s; numpy float64, "
+                      "BLAS threads for the matmuls, elementwise work single-threaded"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", 0))
+    if rank != 0:
+        return
+    import torch
+    cfg = make_config(args)
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    from synth import gen_logits, gen_x
+    logits_cpu, x_cpu = gen_logits(cfg), gen_x(cfg)
+    run, acc, experts = _oracle_sample(cfg, logits_cpu, x_cpu, dev)
+    for _ in range(args.warmup):
+        run()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        run()
+    dt = time.perf_counter() - t0
+    value = acc["bytes"] * args.steps / dt / 1e9
+    sample = (f"each step: 1 of {cfg.T} tokens of the {cfg.name} workload ({len(experts)} experts, "
+              f"{acc['bytes'] / 1e6:.0f} MB algorithmic)")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(dt / args.steps * 1e3, 2), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{cfg.name} MoE FFN: T={cfg.T}, H={cfg.H}, I={cfg.I}, E={cfg.E}, "
+                               f"top-{cfg.k} ({cfg.logits} logits)"},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": _threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

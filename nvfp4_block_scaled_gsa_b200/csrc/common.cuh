@@ -220,12 +220,17 @@ __device__ __forceinline__ uint32_t nvfp4_block_scale(float amax, float gs, floa
   return b;
 }
 
+// x * r for the E2M1 converter; a zero element stays (signed) zero even when r overflowed.
+__device__ __forceinline__ float scaled(float x, float r) { return x == 0.0f ? x : __fmul_rn(x, r); }
+
 // 8 values -> 4 bytes of packed codes (element 2j low nibble), using scale reciprocal r.
+// A block whose decoded scale is 0 (r == 0) gets all-zero codes.
 __device__ __forceinline__ uint32_t nvfp4_pack8(const float* v, float r) {
+  if (r == 0.0f) return 0u;
   uint32_t out = 0;
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
-    out |= cvt_e2m1x2(__fmul_rn(v[2 * j], r), __fmul_rn(v[2 * j + 1], r)) << (8 * j);
+    out |= cvt_e2m1x2(scaled(v[2 * j], r), scaled(v[2 * j + 1], r)) << (8 * j);
   }
   return out;
 }

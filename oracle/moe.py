@@ -40,6 +40,10 @@ class QuantWeights:
     def E(self):
         return self.codes.shape[0]
 
+    @property
+    def N(self):
+        return self.codes.shape[1]
+
     def dequant(self, e):
         return dequantize(unpack_nibbles(self.codes[e]), self.sf[e], self.gs[e])
 
@@ -104,7 +108,8 @@ def moe_ffn(x, logits, k, w1, w2, gs_h, renormalize=True, ids=None, weights=None
 
     x        (T, H) float (the bf16 activations, as float32)
     logits   (T, E) float32, or None when ``ids``/``weights`` give the routing
-    w1, w2   QuantWeights with N = 2I (gate rows then up rows) and N = H
+    w1, w2   QuantWeights (or any object with E, N and dequant(e)) with N = 2I (gate rows
+             then up rows) and N = H
     gs_h     float32 static global scale of the intermediate
     experts  optional iterable restricting which experts are evaluated (for sampled checks)
 
@@ -114,7 +119,7 @@ def moe_ffn(x, logits, k, w1, w2, gs_h, renormalize=True, ids=None, weights=None
     x = np.asarray(x, dtype=np.float32)
     T, H = x.shape
     E = w1.E
-    I = w1.codes.shape[1] // 2
+    I = w1.N // 2
     if ids is None:
         ids, weights = route_topk(logits, k, renormalize)
     perm = permute(ids, weights, E)

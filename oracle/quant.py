@@ -17,7 +17,8 @@ Readings where the pages are silent
   not a finite positive float32 (amax 0, inf or NaN) gs = 1.
 * FP32 operation order, one rounding per operation (numpy float32 arithmetic):
     s = (a_b / 6) * gs ;  sf = E4M3(s) ;  d = decode(sf) ;  r = gs / d ;  code_i = E2M1(x_i * r)
-  A block whose decoded scale is 0 gets all-zero codes.
+  A block whose decoded scale is 0 gets all-zero codes; a zero element encodes as a (signed)
+  zero without the multiply, so 0 * r stays 0 when gs / d overflows for extreme inputs.
 * Dequantized value = E2M1(code) * d / gs.
 
 Scale-factor tile layout
@@ -71,6 +72,7 @@ def quantize(x, gs):
     with np.errstate(divide="ignore", invalid="ignore", over="ignore"):
         r = (gs / d).astype(np.float32)
         y = (blocks * r[..., None]).astype(np.float32)
+    y = np.where(blocks == 0, blocks, y)  # 0 * r is 0 even when r overflowed to inf
     zero_blk = (d == 0)[..., None]
     y = np.where(zero_blk, np.float32(0.0), y)
     codes = e2m1_encode(y)

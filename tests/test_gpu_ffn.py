@@ -1,5 +1,7 @@
 """GPU parity of the whole expert FFN (moe_ffn_forward) and of the weight pre-pack, against the
-oracle: final bf16 output within relative Frobenius 1e-3 and cosine >= 0.9999."""
+oracle: final bf16 output within relative Frobenius 1e-3 and cosine >= 0.9999 of the oracle's
+float64 result rounded once to bf16 (the output type; bf16 rounding alone is ~1e-3 relative, so
+the comparison is made in the output's own precision)."""
 
 import numpy as np
 import pytest
@@ -46,8 +48,10 @@ def _ffn_check(cfg, x, lg):
 def test_ffn_tiny_end_to_end():
     cfg = CONFIGS["tiny"]
     got, ref = _ffn_check(cfg, gen_x(cfg), gen_logits(cfg))
-    assert rel_fro(got, ref["out"]) <= 1e-3
-    assert cosine(got, ref["out"]) >= 0.9999
+    want = M.bf16_round(ref["out"])
+    assert rel_fro(got, want) <= 1e-3
+    assert cosine(got, want) >= 0.9999
+    assert rel_fro(got, ref["out"]) <= 3e-3  # unrounded: bf16 rounding dominates
 
 
 def test_ffn_tokens_with_all_slots_dropped_are_zero():
@@ -57,7 +61,7 @@ def test_ffn_tokens_with_all_slots_dropped_are_zero():
     lg[17] = float("-inf")
     got, ref = _ffn_check(cfg, gen_x(cfg), lg)
     assert np.all(got[5] == 0) and np.all(got[17] == 0)
-    assert rel_fro(got, ref["out"]) <= 1e-3
+    assert rel_fro(got, M.bf16_round(ref["out"])) <= 1e-3
 
 
 def test_ffn_repeatable_and_workspace_reuse():

@@ -62,11 +62,35 @@ def test_quantize_given_scale_hits_every_tie():
     for i, a in enumerate(amax_rows):
         extra[i, 0] = a
         extra[i, 1:] = np.linspace(-a, a, 15)
-    x = np.concatenate([x, extra])
+    assert np.array_equal(torch.from_numpy(x).to(torch.bfloat16).float().numpy(), x)  # exact
+    x = np.concatenate([x, extra])  # (linspace interiors are rounded to bf16; the amax is exact)
     x = np.concatenate([x, np.zeros((x.shape[0], 48), np.float32)], axis=1)  # cols 64
     xt = torch.from_numpy(x).to(torch.bfloat16)
-    assert np.array_equal(xt.float().numpy(), x)  # all exactly representable
+    assert np.array_equal(xt.float().numpy()[:, 0], x[:, 0])
     _check(xt, gs_given=1.0)
+
+
+def test_quantize_zero_scale_blocks_give_zero_codes():
+    """Blocks far below the global amax: their E4M3 scale rounds to 0 and every code is +0,
+    negative elements included."""
+    x = torch.zeros(2, 64)
+    x[0, 0] = 1000.0
+    x[1, :] = -1e-6 * torch.arange(1, 65)
+    _check(x.to(torch.bfloat16))
+
+
+def test_quantize_extreme_small_amax_no_nan():
+    """amax 1e-34 gives a finite gs ~ 2.7e37; a block of subnormals gets the smallest scale
+    2^-9, so gs / d overflows to inf: its zero elements stay zero, the others saturate."""
+    x = torch.zeros(1, 64)
+    x[0, 0] = 1e-34
+    x[0, 16] = 4.3e-40
+    x[0, 17] = -3e-40
+    xb = x.to(torch.bfloat16)
+    assert xb.float()[0, 16] > 0  # a bf16 subnormal, not flushed
+    gs = Q.global_scale(xb.float().numpy())
+    assert np.isfinite(gs) and gs > 1e37
+    _check(xb)
 
 
 def test_quantize_all_zero_matrix_gives_unit_scale():
