@@ -140,7 +140,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     bad_offsets = 0;
     abort_flag = 0;
   }
-  if (tid <= E) seg[tid] = __ldg(args.offs + tid);
+  for (int i = tid; i <= E; i += NUM_THREADS) seg[i] = __ldg(args.offs + i);  // E + 1 entries
   __syncthreads();
   int my_tiles = 0;
   if (tid < E) {

@@ -42,7 +42,7 @@ def _setup(T, H, I, E, k, seed=0, drop=0.0):
 
 
 @pytest.mark.parametrize("T,H,I,E,k", [(64, 256, 128, 8, 2), (200, 512, 256, 6, 3),
-                                       (33, 7168, 2048, 2, 2)])
+                                       (33, 7168, 2048, 2, 2), (96, 256, 128, 256, 8)])
 def test_l1_and_l2_match_oracle(T, H, I, E, k):
     x, ids, w32, w1, w1d, w2, w2d = _setup(T, H, I, E, k, drop=0.1)
     gs_h = np.float32(64.0 if H <= 512 else 1.0)
