@@ -43,6 +43,7 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--experts", type=int, default=0,
                     help="override E (smaller weight set for profiling captures)")
+    ap.add_argument("--tokens", type=int, default=0, help="override T (profiling captures)")
     ap.add_argument("--soak", type=float, default=1.0,
                     help="seconds of extra warm-up load so clock samples cover the timed region")
     return ap.parse_args()
@@ -163,7 +164,8 @@ class Plan:
         if ev:
             ev[2].record()
         call("moe_grouped_gemm_l1_swiglu_q", p(self.xq), p(self.xsf), p(self.gs_x),
-             p(self.w1.codes), p(self.w1.sf), p(self.w1.gs), p(self.offs), E, H, I, self.R,
+             p(self.w1.codes), p(self.w1.sf), p(self.w1.gs), p(self.offs), p(self.row_token),
+             E, H, I, self.R,
              p(self.gs_h), p(self.hq), p(self.hsf), p(self.status), s)
         if ev:
             ev[3].record()
@@ -184,6 +186,8 @@ def make_config(args):
     cfg = CONFIGS[args.config]
     if args.experts:
         cfg = replace(cfg, E=args.experts, name=f"{cfg.name}-E{args.experts}")
+    if args.tokens:
+        cfg = replace(cfg, T=args.tokens, name=f"{cfg.name}-T{args.tokens}")
     return cfg
 
 

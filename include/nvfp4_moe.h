@@ -149,20 +149,25 @@ NVFP4_API nvfp4_status_t nvfp4_grouped_gemm(const uint8_t* a, const uint8_t* sfa
  * FP4 pack in registers -> FP4 GMEM).
  *
  *   W1 of expert e is [2I][H]: rows [0, I) gate, rows [I, 2I) up.
- *   g = acc_gate / (gs_a*gs_w1[e]), u = acc_up / (gs_a*gs_w1[e]), h = silu(g) * u (FP32),
- *   h quantized with the static global scale *gs_h exactly like nvfp4_quantize.
+ *   g = acc_gate / (gs_a*gs_w1[e]), u = acc_up / (gs_a*gs_w1[e]), h = g*u / (1 + exp(-g)) in
+ *   FP32 (hardware exp2 and reciprocal: a few ulp), then quantized with the static global scale
+ *   *gs_h by the same rule as nvfp4_quantize.
  *
  *   a, sfa, gs_a    activations NVFP4 [R_max][H]
  *   w1, sfw1, gs_w1 NVFP4 [E*2I][H], gs_w1 float[E]
  *   offs            int32 [E+1] (from moe_permute)
+ *   row_token       optional int32 [R_max] (from moe_permute).  NULL: every row of every segment
+ *                   is written.  Given: groups of 32 rows that are all padding (row_token < 0)
+ *                   are skipped and their h rows left unwritten.
  *   gs_h            device float[1]
- *   h, sfh          output NVFP4 [R_max][I] (tiled scales); rows of every segment are written
+ *   h, sfh          output NVFP4 [R_max][I] (tiled scales)
  *   Constraints: H % 64 == 0, I % 128 == 0, R_max % 128 == 0, 1 <= E <= 256.
  * ------------------------------------------------------------------------------------------- */
 NVFP4_API nvfp4_status_t moe_grouped_gemm_l1_swiglu_q(const uint8_t* a, const uint8_t* sfa, const float* gs_a,
                                             const uint8_t* w1, const uint8_t* sfw1,
-                                            const float* gs_w1, const int32_t* offs, int E, int H,
-                                            int I, int64_t R_max, const float* gs_h, uint8_t* h,
+                                            const float* gs_w1, const int32_t* offs,
+                                            const int32_t* row_token, int E, int H, int I,
+                                            int64_t R_max, const float* gs_h, uint8_t* h,
                                             uint8_t* sfh, int32_t* dev_status,
                                             nvfp4_stream_t stream);
 

@@ -57,8 +57,9 @@ constexpr uint32_t TM_SFB = TM_SFA + STAGES * 16;    // 32 columns per stage
 static_assert(TM_SFB + STAGES * 32 <= TMEM_COLS, "tensor memory budget");
 
 constexpr uint32_t IDESC = idesc_nvf4(BN);
-constexpr int NUM_THREADS = 256;
+constexpr int NUM_THREADS = 384;  // 4 role warps + 8 epilogue warps
 constexpr int EPI_WARP0 = 4;
+constexpr int EPI_WARPS = 8;
 constexpr int MAX_E = 256;
 
 enum Mode { PLAIN_F32 = 0, PLAIN_BF16 = 1, L1_SWIGLU = 2, L2_SCATTER = 3 };
@@ -79,7 +80,7 @@ struct GemmArgs {
   uint8_t* h;         // L1: [R_max][I/2]
   uint8_t* sfh;       // L1
   int I;              // L1
-  const int32_t* row_token;  // L2
+  const int32_t* row_token;  // L2 (required), L1 (optional: skip padding rows)
   const float* row_w;        // L2
   float* acc;                // L2: [T][H]
   int T;                     // L2
@@ -176,7 +177,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(smem_u32(&bar_empty[s]), 1);
     }
     mbar_init(smem_u32(&bar_acc_full), 1);
-    mbar_init(smem_u32(&bar_acc_empty), 4);
+    mbar_init(smem_u32(&bar_acc_empty), EPI_WARPS);
     mbar_init(smem_u32(&bar_drain), 1);
     fence_mbar_init();
   }
@@ -295,7 +296,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     __syncwarp();
   } else if (warp >= EPI_WARP0) {
     // =========================== epilogue ===========================
-    const int q = warp - EPI_WARP0;  // lane quadrant of tensor memory
+    // Two warps per tensor-memory lane quadrant (a warp may only read lanes 32*(warp%4)..+31);
+    // `half` splits the tile's columns between them.
+    const int q = warp & 3;
+    const int half = (warp - EPI_WARP0) >> 2;
     const uint32_t t_row = tmem + TM_ACC + (static_cast<uint32_t>(q * 32) << 16);
     uint32_t tile_it = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x, ++tile_it) {
@@ -304,72 +308,81 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_after();
       const float alpha = 1.0f / (__ldg(args.gs_a) * __ldg(args.gs_b + tl.e));
       const int64_t row = tl.m0 + q * 32 + lane;
+      // rows of the row map that are padding produce nothing; skip groups of 32 of them
+      int tok = 0;
+      if (MODE == L1_SWIGLU || MODE == L2_SCATTER) {
+        if (args.row_token != nullptr) tok = __ldg(args.row_token + row);
+      }
+      const bool live = __any_sync(0xffffffffu, tok >= 0);
 
       if (MODE == L1_SWIGLU) {
-        const float gs_h = __ldg(args.gs_h);
-        const int I = args.I;
-        uint8_t* hrow = args.h + row * (I / 2) + tl.nt * 64;
-        uint32_t sfw[2] = {0u, 0u};
+        if (live) {
+          const float gs_h = __ldg(args.gs_h);
+          const int I = args.I;
+          uint8_t* hrow = args.h + row * (I / 2) + tl.nt * 64;
+          uint32_t sfw = 0u;
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t g[32], u[32];
-          tmem_ld32(t_row + 32 * c, g);
-          tmem_ld32(t_row + 128 + 32 * c, u);
-          tmem_wait_ld();
-          float hv[32];
+          for (int c = 2 * half; c < 2 * half + 2; ++c) {
+            uint32_t g[32], u[32];
+            tmem_ld32(t_row + 32 * c, g);
+            tmem_ld32(t_row + 128 + 32 * c, u);
+            tmem_wait_ld();
+            float hv[32];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float gg = __uint_as_float(g[i]) * alpha;
-            const float uu = __uint_as_float(u[i]) * alpha;
-            hv[i] = gg / (1.0f + expf(-gg)) * uu;
+            for (int i = 0; i < 32; ++i) {
+              // h = silu(g) * u = g * u / (1 + e^-g), g and u de-scaled by alpha
+              const float gg = __uint_as_float(g[i]) * alpha;
+              const float uu = __uint_as_float(u[i]) * alpha;
+              hv[i] = __fdividef(gg * uu, 1.0f + __expf(-gg));
+            }
+            uint32_t packed[4];
+#pragma unroll
+            for (int b = 0; b < 2; ++b) {
+              float amax = 0.0f;
+#pragma unroll
+              for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(hv[16 * b + i]));
+              float rcp;
+              const uint32_t sb = nvfp4_block_scale(amax, gs_h, rcp);
+              packed[2 * b] = nvfp4_pack8(hv + 16 * b, rcp);
+              packed[2 * b + 1] = nvfp4_pack8(hv + 16 * b + 8, rcp);
+              const int sc = 2 * c + b;  // scale column inside the tile (0..7)
+              sfw |= sb << (8 * (sc & 3));
+            }
+            *reinterpret_cast<uint4*>(hrow + 16 * c) =
+                make_uint4(packed[0], packed[1], packed[2], packed[3]);
           }
-          uint32_t packed[4];
-#pragma unroll
-          for (int b = 0; b < 2; ++b) {
-            float amax = 0.0f;
-#pragma unroll
-            for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(hv[16 * b + i]));
-            float rcp;
-            const uint32_t sb = nvfp4_block_scale(amax, gs_h, rcp);
-            packed[2 * b] = nvfp4_pack8(hv + 16 * b, rcp);
-            packed[2 * b + 1] = nvfp4_pack8(hv + 16 * b + 8, rcp);
-            const int sc = 2 * c + b;  // scale column inside the tile (0..7)
-            sfw[sc >> 2] |= sb << (8 * (sc & 3));
-          }
-          *reinterpret_cast<uint4*>(hrow + 16 * c) =
-              make_uint4(packed[0], packed[1], packed[2], packed[3]);
+          // this half's 4 scale columns are one 4-byte group of the tiled layout
+          *reinterpret_cast<uint32_t*>(args.sfh + sf_offset(row, tl.nt * 8 + 4 * half, I / 16)) =
+              sfw;
         }
-        const int n_sf = I / 16;
-#pragma unroll
-        for (int a = 0; a < 2; ++a)
-          *reinterpret_cast<uint32_t*>(args.sfh + sf_offset(row, tl.nt * 8 + 4 * a, n_sf)) = sfw[a];
       } else if (MODE == L2_SCATTER) {
-        int tok = __ldg(args.row_token + row);
-        if (tok >= args.T) {
-          report(args.status, NVFP4_DEVERR_BAD_INDEX);
-          tok = -1;
-        }
-        const float scale = alpha * (tok >= 0 ? __ldg(args.row_w + row) : 0.0f);
-        const int H = args.N;
-        float* dst = args.acc + (int64_t)(tok >= 0 ? tok : 0) * H + tl.nt * BN;
+        if (live) {
+          if (tok >= args.T) {
+            report(args.status, NVFP4_DEVERR_BAD_INDEX);
+            tok = -1;
+          }
+          const float scale = alpha * (tok >= 0 ? __ldg(args.row_w + row) : 0.0f);
+          const int H = args.N;
+          float* dst = args.acc + (int64_t)(tok >= 0 ? tok : 0) * H + tl.nt * BN;
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
-          uint32_t v[32];
-          tmem_ld32(t_row + 32 * c, v);
-          tmem_wait_ld();
-          if (tok >= 0) {
+          for (int c = 4 * half; c < 4 * half + 4; ++c) {
+            uint32_t v[32];
+            tmem_ld32(t_row + 32 * c, v);
+            tmem_wait_ld();
+            if (tok >= 0) {
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-              red_add_v4(dst + 32 * c + 4 * i, __uint_as_float(v[4 * i]) * scale,
-                         __uint_as_float(v[4 * i + 1]) * scale,
-                         __uint_as_float(v[4 * i + 2]) * scale,
-                         __uint_as_float(v[4 * i + 3]) * scale);
+              for (int i = 0; i < 8; ++i)
+                red_add_v4(dst + 32 * c + 4 * i, __uint_as_float(v[4 * i]) * scale,
+                           __uint_as_float(v[4 * i + 1]) * scale,
+                           __uint_as_float(v[4 * i + 2]) * scale,
+                           __uint_as_float(v[4 * i + 3]) * scale);
+            }
           }
         }
       } else {
         const int N = args.N;
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
+        for (int c = 4 * half; c < 4 * half + 4; ++c) {
           uint32_t v[32];
           tmem_ld32(t_row + 32 * c, v);
           tmem_wait_ld();
@@ -503,13 +516,14 @@ nvfp4_status_t gemm_plain(const uint8_t* a, const uint8_t* sfa, const float* gs_
 }
 
 nvfp4_status_t gemm_l1(const uint8_t* a, const uint8_t* sfa, const float* gs_a, const uint8_t* w1,
-                       const uint8_t* sfw1, const float* gs_w1, const int32_t* offs, int E, int H,
-                       int I, int64_t R_max, const float* gs_h, uint8_t* h, uint8_t* sfh,
-                       int32_t* status, cudaStream_t s) {
+                       const uint8_t* sfw1, const float* gs_w1, const int32_t* offs,
+                       const int32_t* row_token, int E, int H, int I, int64_t R_max,
+                       const float* gs_h, uint8_t* h, uint8_t* sfh, int32_t* status,
+                       cudaStream_t s) {
   GemmArgs g{};
   g.sfa = sfa; g.sfb = sfw1; g.gs_a = gs_a; g.gs_b = gs_w1; g.offs = offs;
   g.E = E; g.N = 2 * I; g.K = H; g.n_tiles = I / 128; g.R_max = R_max;
-  g.gs_h = gs_h; g.h = h; g.sfh = sfh; g.I = I; g.status = status;
+  g.gs_h = gs_h; g.h = h; g.sfh = sfh; g.I = I; g.row_token = row_token; g.status = status;
   return launch<L1_SWIGLU>(a, w1, (int64_t)E * 2 * I, g, s);
 }
 
@@ -557,8 +571,8 @@ extern "C" nvfp4_status_t nvfp4_grouped_gemm(const uint8_t* a, const uint8_t* sf
 
 extern "C" nvfp4_status_t moe_grouped_gemm_l1_swiglu_q(
     const uint8_t* a, const uint8_t* sfa, const float* gs_a, const uint8_t* w1,
-    const uint8_t* sfw1, const float* gs_w1, const int32_t* offs, int E, int H, int I,
-    int64_t R_max, const float* gs_h, uint8_t* h, uint8_t* sfh, int32_t* dev_status,
+    const uint8_t* sfw1, const float* gs_w1, const int32_t* offs, const int32_t* row_token, int E,
+    int H, int I, int64_t R_max, const float* gs_h, uint8_t* h, uint8_t* sfh, int32_t* dev_status,
     nvfp4_stream_t stream) {
   if (E < 1 || E > MAX_E || H <= 0 || I <= 0 || R_max < 0) return NVFP4_ERR_INVALID_ARG;
   if (H % 64 || I % 128 || R_max % 128) return NVFP4_ERR_UNSUPPORTED_SHAPE;
@@ -566,8 +580,9 @@ extern "C" nvfp4_status_t moe_grouped_gemm_l1_swiglu_q(
   if (R_max == 0) return NVFP4_OK;
   if (!ok_ptr(a) || !ok_ptr(sfa) || !ok_ptr(w1) || !ok_ptr(sfw1) || !ok_ptr(h) || !ok_ptr(sfh))
     return (a && sfa && w1 && sfw1 && h && sfh) ? NVFP4_ERR_MISALIGNED : NVFP4_ERR_INVALID_ARG;
-  return gemm_l1(a, sfa, gs_a, w1, sfw1, gs_w1, offs, E, H, I, R_max, gs_h, h, sfh, dev_status,
-                 reinterpret_cast<cudaStream_t>(stream));
+  if (reinterpret_cast<uintptr_t>(row_token) & 3u) return NVFP4_ERR_MISALIGNED;
+  return gemm_l1(a, sfa, gs_a, w1, sfw1, gs_w1, offs, row_token, E, H, I, R_max, gs_h, h, sfh,
+                 dev_status, reinterpret_cast<cudaStream_t>(stream));
 }
 
 extern "C" nvfp4_status_t moe_grouped_gemm_l2_scatter(

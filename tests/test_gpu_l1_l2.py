@@ -62,14 +62,19 @@ def test_l1_and_l2_match_oracle(T, H, I, E, k):
 
     # ---- L1 GEMM stage on its own (plain epilogue, FP32) within 1e-5
     c1 = nv.grouped_gemm(a, asf, gs_x, w1d, offs, out_dtype=torch.float32)
-    # ---- L1 fused SwiGLU + re-quantization
+    # ---- L1 fused SwiGLU + re-quantization (every row; and with the row map, which skips
+    # all-padding row groups but must give the same bytes on real rows)
     h, sfh = nv.l1_swiglu_q(a, asf, gs_x, w1d, offs, gs_h_d)
+    row_token_d = to_dev(perm["row_token"].astype(np.int32))
+    h2, sfh2 = nv.l1_swiglu_q(a, asf, gs_x, w1d, offs, gs_h_d, row_token=row_token_d)
     torch.cuda.synchronize()
+    hc2, hs2 = download_nvfp4(h2, sfh2, Rr, I)
     assert rel_fro(c1.cpu().numpy()[valid], ref["c1"][valid]) <= 1e-5
     hc, hs = download_nvfp4(h, sfh, Rr, I)
     frac, far = compare_requant(hc[valid], hs[valid], ref["h_codes"][valid], ref["h_sf"][valid], gs_h)
     assert far == 0
     assert frac <= 1e-3
+    assert np.array_equal(hc2[valid], hc[valid]) and np.array_equal(hs2[valid], hs[valid])
 
     # ---- L2 + scatter on the oracle's h codes (identical operands)
     h_o, sfh_o = upload_nvfp4(ref["h_codes"], ref["h_sf"])
