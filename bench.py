@@ -72,6 +72,34 @@ def algorithmic(cfg, counts):
                 l1_flops=2 * slots * H * 2 * I, l2_flops=2 * slots * I * H)
 
 
+def kernel_sources_sha16():
+    import hashlib
+    h = hashlib.sha256()
+    for f in ("gemm.cu", "common.cuh"):
+        with open(os.path.join(ROOT, "nvfp4_block_scaled_gsa_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def captured_traffic(cfg):
+    """DRAM bytes per L1 launch from the committed ncu summary, or None when the kernel sources
+    changed since that capture (or the workload is not the one it covers)."""
+    if cfg.name != "decode":
+        return None
+    path = os.path.join(ROOT, "profiles", "grouped_gemm_l1_decode.md")
+    if not os.path.exists(path):
+        return None
+    fields = {}
+    for line in open(path):
+        if ":" in line:
+            k, _, v = line.strip().partition(":")
+            fields[k.strip()] = v.strip()
+    if fields.get("kernel_sources_sha256_16") != kernel_sources_sha16():
+        return None
+    v = fields.get("decode_l1_traffic_bytes_per_launch")
+    return int(v) if v else None
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -331,7 +359,8 @@ def run_ours(args):
                         "active_experts": acc["active"], "slots": acc["slots"]},
         "roofline": {"bound": "hbm", "kernel": "grouped_gemm_kernel<L1_SWIGLU>",
                      "achieved": round(l1_gbs, 1), "peak": peaks["hbm"], "unit": "GB/s",
-                     "frac": round(l1_gbs / peaks["hbm"], 4), "traffic": None,
+                     "frac": round(l1_gbs / peaks["hbm"], 4), "traffic": captured_traffic(cfg),
+                     "algorithmic_bytes_per_launch": int(acc["l1_bytes"]),
                      "peak_source": peaks["src"],
                      "step_frac": round(value / world / peaks["hbm"], 4)},
         "stages_ms": {"route": round(statistics.mean(stage[0]), 4),
