@@ -195,6 +195,31 @@ NVFP4_API nvfp4_status_t moe_grouped_gemm_l2_scatter(const uint8_t* h, const uin
                                            nvfp4_stream_t stream);
 
 /* ---------------------------------------------------------------------------------------------
+ * moe_grouped_gemm_l2_scatter_noalloc — moe_grouped_gemm_l2_scatter without a caller-provided
+ * FP32 accumulation buffer.  The pages have no counterpart to this call; it exists for callers
+ * that cannot allocate device memory for scratch: runtimes that reserve all device memory up front
+ * (weights, KV cache, a fixed activation pool) and forbid later cudaMalloc, or foreign-language
+ * callers that are handed input and output buffers but have no device allocator of their own.
+ *
+ *   Same arguments and result as moe_grouped_gemm_l2_scatter, minus acc_ws; out_bf16 is required.
+ *   The FP32 accumulator lives in a static device array inside this library of
+ *   NVFP4_L2_NOALLOC_MAX_ELEMS floats (4 MiB), which every GPU that loads the library holds until
+ *   the process exits.  T*H beyond that returns NVFP4_ERR_WORKSPACE_TOO_SMALL (nothing launched;
+ *   nvfp4_last_error() says why).
+ *   The array's device address is looked up once per device (cudaGetSymbolAddress) by the first
+ *   call made with that device current; make that first call before any stream capture.
+ *   No cudaMalloc / cudaFree or allocating library routine is called.  All calls share the one
+ *   array: each call zeroes it on its stream before use, and calls that overlap on the GPU (other
+ *   streams, other threads) race on it.
+ * ------------------------------------------------------------------------------------------- */
+#define NVFP4_L2_NOALLOC_MAX_ELEMS (1 << 20)
+NVFP4_API nvfp4_status_t moe_grouped_gemm_l2_scatter_noalloc(
+    const uint8_t* h, const uint8_t* sfh, const float* gs_h, const uint8_t* w2,
+    const uint8_t* sfw2, const float* gs_w2, const int32_t* offs, const int32_t* row_token,
+    const float* row_w, int E, int H, int I, int T, int64_t R_max, void* out_bf16,
+    int32_t* dev_status, nvfp4_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------------
  * moe_ffn_forward — the whole expert FFN in one stream-ordered call:
  *   moe_permute -> nvfp4_quantize (amax -> gs on the GPU, permuted write) ->
  *   moe_grouped_gemm_l1_swiglu_q -> moe_grouped_gemm_l2_scatter -> bf16 out.

@@ -600,3 +600,56 @@ extern "C" nvfp4_status_t moe_grouped_gemm_l2_scatter(
   return gemm_l2(h, sfh, gs_h, w2, sfw2, gs_w2, offs, row_token, row_w, E, H, I, T, R_max, acc_ws,
                  out_bf16, dev_status, reinterpret_cast<cudaStream_t>(stream));
 }
+
+// ------------------------------------------------------------------------------ no-alloc variant
+// The FP32 accumulator of moe_grouped_gemm_l2_scatter_noalloc: one static array per device that
+// loads the library.  Host code must not pass its name to a kernel (on the host it is only a
+// stand-in symbol); its device address comes from cudaGetSymbolAddress, looked up once per device.
+static __device__ __align__(256) float g_l2_noalloc_acc[NVFP4_L2_NOALLOC_MAX_ELEMS];
+
+namespace {
+constexpr int kMaxDevices = 64;
+
+float* l2_noalloc_scratch() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    set_last_error("moe_grouped_gemm_l2_scatter_noalloc: no usable current device");
+    return nullptr;
+  }
+  static std::mutex mu;
+  static float* addr[kMaxDevices] = {};
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_l2_noalloc_acc);
+    if (e != cudaSuccess || p == nullptr) {
+      check_launch("cudaGetSymbolAddress(g_l2_noalloc_acc)");
+      return nullptr;
+    }
+    addr[dev] = static_cast<float*>(p);
+  }
+  return addr[dev];
+}
+}  // namespace
+
+extern "C" nvfp4_status_t moe_grouped_gemm_l2_scatter_noalloc(
+    const uint8_t* h, const uint8_t* sfh, const float* gs_h, const uint8_t* w2,
+    const uint8_t* sfw2, const float* gs_w2, const int32_t* offs, const int32_t* row_token,
+    const float* row_w, int E, int H, int I, int T, int64_t R_max, void* out_bf16,
+    int32_t* dev_status, nvfp4_stream_t stream) {
+  if (E < 1 || E > MAX_E || H <= 0 || I <= 0 || T < 0 || R_max < 0) return NVFP4_ERR_INVALID_ARG;
+  if (H % BN || I % 64 || R_max % 128) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (!gs_h || !gs_w2 || !offs || !row_token || !row_w || !out_bf16) return NVFP4_ERR_INVALID_ARG;
+  if ((int64_t)T * H > NVFP4_L2_NOALLOC_MAX_ELEMS) {
+    set_last_error("moe_grouped_gemm_l2_scatter_noalloc: T*H exceeds the static FP32 scratch "
+                   "(NVFP4_L2_NOALLOC_MAX_ELEMS floats)");
+    return NVFP4_ERR_WORKSPACE_TOO_SMALL;
+  }
+  if (T == 0 || R_max == 0) return NVFP4_OK;
+  if (!ok_ptr(h) || !ok_ptr(sfh) || !ok_ptr(w2) || !ok_ptr(sfw2) || !aligned16(out_bf16))
+    return (h && sfh && w2 && sfw2) ? NVFP4_ERR_MISALIGNED : NVFP4_ERR_INVALID_ARG;
+  float* acc = l2_noalloc_scratch();
+  if (acc == nullptr) return NVFP4_ERR_CUDA;
+  return gemm_l2(h, sfh, gs_h, w2, sfw2, gs_w2, offs, row_token, row_w, E, H, I, T, R_max, acc,
+                 out_bf16, dev_status, reinterpret_cast<cudaStream_t>(stream));
+}
