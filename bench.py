@@ -193,7 +193,7 @@ class Plan:
             ev[2].record()
         call("moe_grouped_gemm_l1_swiglu_q", p(self.xq), p(self.xsf), p(self.gs_x),
              p(self.w1.codes), p(self.w1.sf), p(self.w1.gs), p(self.offs), p(self.row_token),
-             E, H, I, self.R,
+             T, E, H, I, self.R,
              p(self.gs_h), p(self.hq), p(self.hsf), p(self.status), s)
         if ev:
             ev[3].record()
@@ -226,8 +226,8 @@ def setup_inputs(cfg, dev):
     from synth import gen_logits, gen_weight_expert, gen_x
     logits = gen_logits(cfg)
     x = gen_x(cfg)
-    w1 = nv.quantize_weights(lambda e: gen_weight_expert(cfg.seed, 1, e, 2 * cfg.I, cfg.H, device=dev),
-                             cfg.E, 2 * cfg.I, cfg.H, device=dev)
+    w1 = nv.quantize_w1(lambda e: gen_weight_expert(cfg.seed, 1, e, 2 * cfg.I, cfg.H, device=dev),
+                        cfg.E, cfg.I, cfg.H, device=dev)
     w2 = nv.quantize_weights(lambda e: gen_weight_expert(cfg.seed, 2, e, cfg.H, cfg.I, device=dev),
                              cfg.E, cfg.H, cfg.I, device=dev)
     gs_h = torch.tensor([cfg.gs_h], dtype=torch.float32, device=dev)

@@ -148,7 +148,9 @@ NVFP4_API nvfp4_status_t nvfp4_grouped_gemm(const uint8_t* a, const uint8_t* sfa
  * the epilogue ("May 24, 2026 — Session Start Plan", section 5 "NVFP4-1.1": L1 GEMM -> SwiGLU ->
  * FP4 pack in registers -> FP4 GMEM).
  *
- *   W1 of expert e is [2I][H]: rows [0, I) gate, rows [I, 2I) up.
+ *   W1 of expert e is [2I][H] with gate and up rows interleaved in blocks of 16: stored row
+ *   32*j + i (i < 16) is gate row 16*j + i, stored row 32*j + 16 + i is up row 16*j + i
+ *   (moe_w1_row_map gives the map; nvfp4_quantize applies it through dst_row at pre-pack).
  *   g = acc_gate / (gs_a*gs_w1[e]), u = acc_up / (gs_a*gs_w1[e]), h = g*u / (1 + exp(-g)) in
  *   FP32 (hardware exp2 and reciprocal: a few ulp), then quantized with the static global scale
  *   *gs_h by the same rule as nvfp4_quantize.
@@ -159,6 +161,11 @@ NVFP4_API nvfp4_status_t nvfp4_grouped_gemm(const uint8_t* a, const uint8_t* sfa
  *   row_token       optional int32 [R_max] (from moe_permute).  NULL: every row of every segment
  *                   is written.  Given: groups of 32 rows that are all padding (row_token < 0)
  *                   are skipped and their h rows left unwritten.
+ *   T               number of tokens routed (0 = unknown).  With row_token given and T <= 32 the
+ *                   small-batch kernel runs (weights as the 128-row operand, an expert's tokens as
+ *                   a 32-column tile); it requires each token to reach an expert at most once
+ *                   (as moe_permute's routing does) and flags a longer segment with
+ *                   NVFP4_DEVERR_BAD_OFFSETS.
  *   gs_h            device float[1]
  *   h, sfh          output NVFP4 [R_max][I] (tiled scales)
  *   Constraints: H % 64 == 0, I % 128 == 0, R_max % 128 == 0, 1 <= E <= 256.
@@ -166,10 +173,18 @@ NVFP4_API nvfp4_status_t nvfp4_grouped_gemm(const uint8_t* a, const uint8_t* sfa
 NVFP4_API nvfp4_status_t moe_grouped_gemm_l1_swiglu_q(const uint8_t* a, const uint8_t* sfa, const float* gs_a,
                                             const uint8_t* w1, const uint8_t* sfw1,
                                             const float* gs_w1, const int32_t* offs,
-                                            const int32_t* row_token, int E, int H, int I,
+                                            const int32_t* row_token, int T, int E, int H, int I,
                                             int64_t R_max, const float* gs_h, uint8_t* h,
                                             uint8_t* sfh, int32_t* dev_status,
                                             nvfp4_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------------
+ * moe_w1_row_map — host helper: the stored row of each logical W1 row (gate rows [0, I), up rows
+ * [I, 2I)) in the 16-row interleaved layout above.  map: host int32 [2I].  I % 16 == 0.
+ * Pure host computation, no CUDA call.  Pass the map (copied to the device) as dst_row with k = 1
+ * to nvfp4_quantize when pre-packing an expert's W1.
+ * ------------------------------------------------------------------------------------------- */
+NVFP4_API nvfp4_status_t moe_w1_row_map(int I, int32_t* map);
 
 /* ---------------------------------------------------------------------------------------------
  * moe_grouped_gemm_l2_scatter — L2 grouped GEMM with the routing weight and the scatter-add in
@@ -184,6 +199,7 @@ NVFP4_API nvfp4_status_t moe_grouped_gemm_l1_swiglu_q(const uint8_t* a, const ui
  *   w2, sfw2, gs_w2  NVFP4 [E*H][I], gs_w2 float[E]
  *   offs, row_token, row_w  from moe_permute
  *   acc_ws           float [T][H] scratch/output;  out_bf16  bf16 [T][H] or NULL
+ *   With T <= 32 the small-batch kernel runs (same condition on the routing as for L1).
  *   Constraints: H % 256 == 0, I % 64 == 0, R_max % 128 == 0, 1 <= E <= 256, T >= 0.
  * ------------------------------------------------------------------------------------------- */
 NVFP4_API nvfp4_status_t moe_grouped_gemm_l2_scatter(const uint8_t* h, const uint8_t* sfh, const float* gs_h,

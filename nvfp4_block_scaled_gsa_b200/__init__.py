@@ -14,7 +14,9 @@ from .api import (  # noqa: F401
     moe_ffn_forward,
     permute,
     quantize,
+    quantize_w1,
     quantize_weights,
+    w1_row_map,
     read_status,
     rows_max,
     sf_bytes,

@@ -60,9 +60,9 @@ def quantize(x, gs=None, dst_row=None, k=1, out_rows=None, status=None):
     return codes, sf, gs
 
 
-def quantize_weights(get_expert, E, N, K, device="cuda"):
+def quantize_weights(get_expert, E, N, K, device="cuda", row_map=None):
     """Pre-pack expert weights: get_expert(e) -> bf16 (N, K) on the device; each expert gets its
-    own global scale from its amax."""
+    own global scale from its amax.  row_map (device int32 [N]): stored row of each row."""
     codes = torch.empty(E * N, K // 2, dtype=U8, device=device)
     sf = torch.empty(E * N * K // 16, dtype=U8, device=device)
     gs = torch.empty(E, dtype=F32, device=device)
@@ -72,10 +72,24 @@ def quantize_weights(get_expert, E, N, K, device="cuda"):
         w = get_expert(e)
         assert w.dtype == BF16 and tuple(w.shape) == (N, K)
         w = w.contiguous()
-        call("nvfp4_quantize", _p(w), N, K, K, None, 1, N, _p(codes[e * N:(e + 1) * N]),
+        call("nvfp4_quantize", _p(w), N, K, K, _p(row_map), 1, N, _p(codes[e * N:(e + 1) * N]),
              sf.data_ptr() + e * per_sf, gs.data_ptr() + 4 * e, 1, _p(ws), ws.numel(), None,
              _stream())
     return NVFP4Weights(codes, sf, gs, E, N, K)
+
+
+def w1_row_map(I):
+    """Host int32 [2I]: stored row of each logical W1 row (gate rows, then up rows)."""
+    m = torch.empty(2 * I, dtype=I32)
+    call("moe_w1_row_map", I, m.data_ptr())
+    return m
+
+
+def quantize_w1(get_expert, E, I, H, device="cuda"):
+    """Pre-pack W1 (E experts of [2I][H]: gate rows then up rows) into the kernels' 64-row
+    gate/up interleaved layout."""
+    row_map = w1_row_map(I).to(device)
+    return quantize_weights(get_expert, E, 2 * I, H, device=device, row_map=row_map)
 
 
 def rows_max(T, E, k):
@@ -113,15 +127,17 @@ def grouped_gemm(a_codes, a_sf, gs_a, w: NVFP4Weights, offs, out_dtype=F32, stat
     return out
 
 
-def l1_swiglu_q(a_codes, a_sf, gs_a, w1: NVFP4Weights, offs, gs_h, row_token=None, status=None):
+def l1_swiglu_q(a_codes, a_sf, gs_a, w1: NVFP4Weights, offs, gs_h, row_token=None, T=0,
+                status=None):
     """L1 GEMM + SwiGLU + NVFP4 re-quantization -> (h codes (R, I/2), h tiled scales).
-    With row_token, all-padding groups of 32 rows are skipped (left unwritten)."""
+    With row_token, all-padding groups of 32 rows are skipped (left unwritten); with row_token
+    and 0 < T <= 32 the small-batch kernel runs."""
     R = a_codes.shape[0]
     I = w1.N // 2
     h = torch.empty(R, I // 2, dtype=U8, device=a_codes.device)
     sfh = torch.empty(sf_bytes(R, I), dtype=U8, device=a_codes.device)
     call("moe_grouped_gemm_l1_swiglu_q", _p(a_codes), _p(a_sf), _p(gs_a), _p(w1.codes),
-         _p(w1.sf), _p(w1.gs), _p(offs), _p(row_token), w1.E, w1.K, I, R, _p(gs_h), _p(h),
+         _p(w1.sf), _p(w1.gs), _p(offs), _p(row_token), T, w1.E, w1.K, I, R, _p(gs_h), _p(h),
          _p(sfh), _p(status), _stream())
     return h, sfh
 

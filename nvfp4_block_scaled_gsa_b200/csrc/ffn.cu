@@ -35,7 +35,7 @@ nvfp4_status_t permute_launch(const float* logits, int T, int E, int k, int reno
                               int32_t* dev_status, cudaStream_t s);
 nvfp4_status_t gemm_l1(const uint8_t* a, const uint8_t* sfa, const float* gs_a, const uint8_t* w1,
                        const uint8_t* sfw1, const float* gs_w1, const int32_t* offs,
-                       const int32_t* row_token, int E, int H, int I, int64_t R_max,
+                       const int32_t* row_token, int T, int E, int H, int I, int64_t R_max,
                        const float* gs_h, uint8_t* h, uint8_t* sfh, int32_t* status,
                        cudaStream_t s);
 nvfp4_status_t gemm_l2(const uint8_t* h, const uint8_t* sfh, const float* gs_h, const uint8_t* w2,
@@ -121,7 +121,8 @@ extern "C" nvfp4_status_t moe_ffn_forward(const void* x_bf16, const float* logit
                        f32(L.gs_x), 1, base + L.amax, dev_status, s);
   if (st != NVFP4_OK) return st;
   st = gemm_l1(base + L.xq, base + L.xsf, f32(L.gs_x), w1, sfw1, gs_w1, i32(L.offs),
-               i32(L.row_token), E, H, I, L.R_max, gs_h, base + L.hq, base + L.hsf, dev_status, s);
+               i32(L.row_token), T, E, H, I, L.R_max, gs_h, base + L.hq, base + L.hsf, dev_status,
+               s);
   if (st != NVFP4_OK) return st;
   return gemm_l2(base + L.hq, base + L.hsf, gs_h, w2, sfw2, gs_w2, i32(L.offs), i32(L.row_token),
                  f32(L.row_w), E, H, I, T, L.R_max, f32(L.acc), out_bf16, dev_status, s);
@@ -143,3 +144,12 @@ extern "C" nvfp4_status_t nvfp4_read_status(const int32_t* dev_status, int32_t* 
 extern "C" const char* nvfp4_last_error(void) { return g_last_error; }
 
 extern "C" int nvfp4_abi_version(void) { return 1; }
+
+extern "C" nvfp4_status_t moe_w1_row_map(int I, int32_t* map) {
+  if (I <= 0 || I % 16 != 0 || map == nullptr) return NVFP4_ERR_INVALID_ARG;
+  for (int p = 0; p < 2 * I; ++p) {
+    const int up = p >= I, r = up ? p - I : p;  // logical gate or up row r
+    map[p] = 32 * (r / 16) + 16 * up + (r % 16);
+  }
+  return NVFP4_OK;
+}

@@ -17,8 +17,9 @@
 // Epilogues (the MODE template parameter):
 //   PLAIN_F32 / PLAIN_BF16  C = acc / (gs_a * gs_b[e])
 //   L1  SwiGLU + NVFP4 re-quantization in registers ("May 24, 2026 — Session Start Plan",
-//       section 5 "NVFP4-1.1"): the B tile stacks gate rows n0..n0+127 over up rows
-//       I+n0..I+n0+127, so each epilogue thread holds matching gate and up columns of its row.
+//       section 5 "NVFP4-1.1"): W1 is stored gate/up interleaved in 16-row blocks, so the
+//       256-row B tile holds gate and up rows of the same 128 h features and each epilogue
+//       thread finds matching gate and up values 16 accumulator columns apart.
 //   L2  routing weight + scatter-add: red.global.add.v4.f32 into an FP32 [T][H] buffer.
 //
 // Tile scheduler: each expert's 128-padded row segment gives (rows/128) M-tiles; tiles are
@@ -205,14 +206,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       bool ok = true;
       for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
         const Tile tl = decode_tile(t, tile_start, seg, E, args.n_tiles);
-        int b_row0, b_row1;
-        if (MODE == L1_SWIGLU) {
-          b_row0 = tl.e * args.N + tl.nt * 128;
-          b_row1 = b_row0 + args.I;
-        } else {
-          b_row0 = tl.e * args.N + tl.nt * BN;
-          b_row1 = b_row0 + 128;
-        }
+        // B rows of this N-tile: 256 consecutive rows (for L1: 8 blocks of 16 gate rows followed
+        // by the 16 matching up rows)
+        const int b_row0 = tl.e * args.N + tl.nt * BN;
+        const int b_row1 = b_row0 + 128;
         for (int kb = 0; kb < nk; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1u;
@@ -250,6 +247,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else if (warp == 1) {
     // =========================== MMA issuer ===========================
     if (lane == 0) {
+      // Descriptors of stage 0; stage s adds s * STAGE_BYTES / 16 to the start-address field
+      // (bits [0,14) hold address >> 4, and every stage address fits, so the add never carries).
+      const uint32_t s0 = smem_u32(smem);
+      const uint64_t a_desc0 = smem_desc(s0, 16, 1024, 2);
+      const uint64_t b_desc0 = smem_desc(s0 + A_BYTES, 16, 1024, 2);
+      const uint64_t sfa_desc0 = smem_desc(s0 + A_BYTES + B_BYTES, 0, 128, 0);
+      const uint64_t sfb_desc0 = smem_desc(s0 + A_BYTES + B_BYTES + SFA_BYTES, 0, 128, 0);
+      constexpr uint64_t kSfbHalf = (SFB_BYTES / 2) >> 4;  // second 128 rows of the B scales
       uint32_t it = 0, tile_it = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++tile_it) {
@@ -266,22 +271,30 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             break;
           }
           tc_fence_after();
-          const int natoms = min(4, atoms_k - kb * 4);
-          uint8_t* st = smem + s * STAGE_BYTES;
-          const uint32_t sA = smem_u32(st), sB = sA + A_BYTES, sSFA = sB + B_BYTES,
-                         sSFB = sSFA + SFA_BYTES;
+          const uint64_t so = static_cast<uint64_t>(s) * (STAGE_BYTES >> 4);
           const uint32_t t_sfa = tmem + TM_SFA + s * 16;
           const uint32_t t_sfb = tmem + TM_SFB + s * 32;
-          for (int a = 0; a < natoms; ++a) {
-            tc_cp_sf(t_sfa + a * 4, smem_desc(sSFA + a * 512, 0, 128, 0));
-            tc_cp_sf(t_sfb + a * 8, smem_desc(sSFB + a * 512, 0, 128, 0));
-            tc_cp_sf(t_sfb + a * 8 + 4, smem_desc(sSFB + SFB_BYTES / 2 + a * 512, 0, 128, 0));
-          }
-          for (int a = 0; a < natoms; ++a) {
-            const uint64_t ad = smem_desc(sA + a * 32, 16, 1024, 2);
-            const uint64_t bd = smem_desc(sB + a * 32, 16, 1024, 2);
-            tc_mma_nvf4(tmem + TM_ACC, ad, bd, IDESC, t_sfa + a * 4, t_sfb + a * 8,
-                        (kb | a) != 0 ? 1u : 0u);
+          const uint32_t first = kb == 0 ? 0u : 1u;
+          // per 64-element K step: its three scale copies, then its MMA, so the MMA of step a
+          // runs while the copies of step a+1 are in flight
+          if (atoms_k - kb * 4 >= 4) {
+#pragma unroll
+            for (int a = 0; a < 4; ++a) {
+              tc_cp_sf(t_sfa + a * 4, sfa_desc0 + so + 32 * a);
+              tc_cp_sf(t_sfb + a * 8, sfb_desc0 + so + 32 * a);
+              tc_cp_sf(t_sfb + a * 8 + 4, sfb_desc0 + so + kSfbHalf + 32 * a);
+              tc_mma_nvf4(tmem + TM_ACC, a_desc0 + so + 2 * a, b_desc0 + so + 2 * a, IDESC,
+                          t_sfa + a * 4, t_sfb + a * 8, a == 0 ? first : 1u);
+            }
+          } else {
+            const int natoms = atoms_k - kb * 4;
+            for (int a = 0; a < natoms; ++a) {
+              tc_cp_sf(t_sfa + a * 4, sfa_desc0 + so + 32 * a);
+              tc_cp_sf(t_sfb + a * 8, sfb_desc0 + so + 32 * a);
+              tc_cp_sf(t_sfb + a * 8 + 4, sfb_desc0 + so + kSfbHalf + 32 * a);
+              tc_mma_nvf4(tmem + TM_ACC, a_desc0 + so + 2 * a, b_desc0 + so + 2 * a, IDESC,
+                          t_sfa + a * 4, t_sfb + a * 8, a == 0 ? first : 1u);
+            }
           }
           tc_commit(smem_u32(&bar_empty[s]));
         }
@@ -323,17 +336,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           uint32_t sfw = 0u;
 #pragma unroll 1
           for (int c = 2 * half; c < 2 * half + 2; ++c) {
-            uint32_t g[32], u[32];
-            tmem_ld32(t_row + 32 * c, g);
-            tmem_ld32(t_row + 128 + 32 * c, u);
+            // h features 32c..32c+31 of the tile live in accumulator columns 64c..64c+63 as two
+            // 32-column blocks, each 16 gate columns followed by the 16 matching up columns
+            uint32_t v0[32], v1[32];
+            tmem_ld32(t_row + 64 * c, v0);
+            tmem_ld32(t_row + 64 * c + 32, v1);
             tmem_wait_ld();
             float hv[32];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
+            for (int i = 0; i < 16; ++i) {
               // h = silu(g) * u = g * u / (1 + e^-g), g and u de-scaled by alpha
-              const float gg = __uint_as_float(g[i]) * alpha;
-              const float uu = __uint_as_float(u[i]) * alpha;
-              hv[i] = __fdividef(gg * uu, 1.0f + __expf(-gg));
+              const float g0 = __uint_as_float(v0[i]) * alpha, u0 = __uint_as_float(v0[16 + i]) * alpha;
+              const float g1 = __uint_as_float(v1[i]) * alpha, u1 = __uint_as_float(v1[16 + i]) * alpha;
+              hv[i] = __fdividef(g0 * u0, 1.0f + __expf(-g0));
+              hv[16 + i] = __fdividef(g1 * u1, 1.0f + __expf(-g1));
             }
             uint32_t packed[4];
 #pragma unroll
@@ -426,6 +442,281 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (tid == 0 && abort_flag) report(args.status, NVFP4_DEVERR_TIMEOUT);
 }
 
+// ------------------------------------------------------------------------------ small batch
+// Swap-AB variant for batches of at most 32 tokens (so every expert has at most 32 rows): the
+// weights are the 128-row M operand and the expert's (at most 32) token rows the N operand, so no
+// tensor-core work and no shared memory goes to padding rows, and a 24 KB stage lets 9 stages
+// (144 KB of weights) stream per SM.  Accumulators are 32 TMEM columns, double buffered, so the
+// epilogue of one tile overlaps the main loop of the next.  A tile covers 128 weight rows of one
+// expert: 64 h features for L1 (16-row gate/up blocks: lane i and lane i+16 of a quadrant hold the
+// gate and up value of one feature), 128 output features for L2.
+constexpr int SB_N = 32;
+constexpr int SB_STAGES = 9;
+constexpr int SB_W_BYTES = 128 * BK_BYTES;
+constexpr int SB_X_BYTES = SB_N * BK_BYTES;
+constexpr int SB_SF_BYTES = 4 * 512;
+constexpr int SB_STAGE_BYTES = SB_W_BYTES + SB_X_BYTES + 2 * SB_SF_BYTES;
+constexpr int SB_SMEM_BYTES = SB_STAGES * SB_STAGE_BYTES + 1024;
+static_assert(SB_STAGE_BYTES % 1024 == 0, "stages must keep 1024-byte alignment (128B swizzle)");
+constexpr uint32_t SB_TM_ACC = 0;                           // 2 x 32 FP32 columns
+constexpr uint32_t SB_TM_SFW = 64;                          // 16 columns per stage
+constexpr uint32_t SB_TM_SFX = SB_TM_SFW + SB_STAGES * 16;  // 16 columns per stage
+static_assert(SB_TM_SFX + SB_STAGES * 16 <= TMEM_COLS, "tensor memory budget");
+constexpr uint32_t SB_IDESC = idesc_nvf4(SB_N);
+constexpr int SB_THREADS = 256;  // 4 role warps + 4 epilogue warps
+
+template <int MODE>
+__global__ void __launch_bounds__(SB_THREADS, 1)
+    grouped_gemm_small_kernel(const __grid_constant__ CUtensorMap tm_x,
+                              const __grid_constant__ CUtensorMap tm_w, const GemmArgs args) {
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t bar_full[SB_STAGES];
+  __shared__ __align__(8) uint64_t bar_empty[SB_STAGES];
+  __shared__ __align__(8) uint64_t bar_acc_full[2];
+  __shared__ __align__(8) uint64_t bar_acc_empty[2];
+  __shared__ __align__(8) uint64_t bar_drain;
+  __shared__ uint32_t tmem_slot;
+  __shared__ int seg[MAX_E + 1];
+  __shared__ int tile_start[MAX_E + 1];
+  __shared__ int warp_sums[SB_THREADS / 32];
+  __shared__ int bad_offsets;
+  __shared__ volatile int abort_flag;
+
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int E = args.E;
+
+  // ---- scheduler table: every non-empty expert segment is one 128-row block holding at most
+  // 32 tokens; it owns n_tiles weight tiles
+  if (tid == 0) {
+    bad_offsets = 0;
+    abort_flag = 0;
+  }
+  for (int i = tid; i <= E; i += SB_THREADS) seg[i] = __ldg(args.offs + i);
+  __syncthreads();
+  int my_tiles = 0;
+  if (tid < E) {
+    const int lo = seg[tid], hi = seg[tid + 1];
+    if (lo < 0 || hi < lo || (lo & 127) || hi > args.R_max || hi - lo > 128 ||
+        (hi > lo && __ldg(args.row_token + lo + SB_N) >= 0))
+      bad_offsets = 1;
+    else
+      my_tiles = ((hi - lo) >> 7) * args.n_tiles;
+  }
+  int incl = my_tiles;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  if (lane == 31) warp_sums[warp] = incl;
+  __syncthreads();
+  if (tid == 0) {
+    int run = 0;
+    for (int w = 0; w < SB_THREADS / 32; ++w) {
+      const int c = warp_sums[w];
+      warp_sums[w] = run;
+      run += c;
+    }
+  }
+  __syncthreads();
+  const int excl = warp_sums[warp] + incl - my_tiles;
+  if (tid < E) tile_start[tid] = excl;
+  if (tid == E - 1) tile_start[E] = excl + my_tiles;
+
+  if (tid == 0) {
+    for (int s = 0; s < SB_STAGES; ++s) {
+      mbar_init(smem_u32(&bar_full[s]), 1);
+      mbar_init(smem_u32(&bar_empty[s]), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(smem_u32(&bar_acc_full[b]), 1);
+      mbar_init(smem_u32(&bar_acc_empty[b]), 4);
+    }
+    mbar_init(smem_u32(&bar_drain), 1);
+    fence_mbar_init();
+  }
+  if (warp == 2) {
+    tmem_alloc(smem_u32(&tmem_slot), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_slot;
+  const int total = bad_offsets ? 0 : tile_start[E];
+  if (tid == 0 && bad_offsets && blockIdx.x == 0) report(args.status, NVFP4_DEVERR_BAD_OFFSETS);
+
+  const int K = args.K;
+  const int nk = (K + 255) / 256;
+  const int atoms_k = K / 64;
+
+  if (warp == 0) {
+    // =========================== TMA producer ===========================
+    if (lane == 0) {
+      prefetch_tmap(&tm_x);
+      prefetch_tmap(&tm_w);
+      uint32_t it = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        const Tile tl = decode_tile(t, tile_start, seg, E, args.n_tiles);
+        const int w_row = tl.e * args.N + tl.nt * 128;
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const int s = it % SB_STAGES;
+          const uint32_t ph = (it / SB_STAGES) & 1u;
+          if (!mbar_wait_bounded(smem_u32(&bar_empty[s]), ph ^ 1u, &abort_flag)) {
+            ok = false;
+            break;
+          }
+          const int natoms = min(4, atoms_k - kb * 4);
+          const uint32_t full = smem_u32(&bar_full[s]);
+          const uint32_t sW = smem_u32(smem + s * SB_STAGE_BYTES), sX = sW + SB_W_BYTES,
+                         sSFW = sX + SB_X_BYTES, sSFX = sSFW + SB_SF_BYTES;
+          mbar_arrive_expect_tx(full, SB_W_BYTES + SB_X_BYTES + natoms * 512 * 2);
+          tma_load_2d(sW, &tm_w, full, kb * BK_BYTES, w_row);
+          tma_load_2d(sX, &tm_x, full, kb * BK_BYTES, tl.m0);
+          const int64_t w_atom = (int64_t)(w_row >> 7) * atoms_k + kb * 4;
+          const int64_t x_atom = (int64_t)(tl.m0 >> 7) * atoms_k + kb * 4;
+          bulk_load(sSFW, args.sfb + w_atom * 512, natoms * 512, full);
+          bulk_load(sSFX, args.sfa + x_atom * 512, natoms * 512, full);
+        }
+      }
+      if (!ok) {
+        volatile int never = 0;
+        const uint32_t first = it > (uint32_t)SB_STAGES ? it - SB_STAGES : 0u;
+        for (uint32_t j = first; j < it; ++j)
+          mbar_wait_bounded(smem_u32(&bar_full[j % SB_STAGES]), (j / SB_STAGES) & 1u, &never,
+                            NVFP4_WAIT_TIMEOUT_NS / 4);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // =========================== MMA issuer ===========================
+    if (lane == 0) {
+      const uint32_t s0 = smem_u32(smem);
+      const uint64_t w_desc0 = smem_desc(s0, 16, 1024, 2);
+      const uint64_t x_desc0 = smem_desc(s0 + SB_W_BYTES, 16, 1024, 2);
+      const uint64_t sfw_desc0 = smem_desc(s0 + SB_W_BYTES + SB_X_BYTES, 0, 128, 0);
+      const uint64_t sfx_desc0 = smem_desc(s0 + SB_W_BYTES + SB_X_BYTES + SB_SF_BYTES, 0, 128, 0);
+      uint32_t it = 0, tile_it = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++tile_it) {
+        const int b = tile_it & 1;
+        if (!mbar_wait_bounded(smem_u32(&bar_acc_empty[b]), ((tile_it >> 1) & 1u) ^ 1u,
+                               &abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem + SB_TM_ACC + b * SB_N;
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const int s = it % SB_STAGES;
+          const uint32_t ph = (it / SB_STAGES) & 1u;
+          if (!mbar_wait_bounded(smem_u32(&bar_full[s]), ph, &abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t so = static_cast<uint64_t>(s) * (SB_STAGE_BYTES >> 4);
+          const uint32_t t_sfw = tmem + SB_TM_SFW + s * 16;
+          const uint32_t t_sfx = tmem + SB_TM_SFX + s * 16;
+          const uint32_t first = kb == 0 ? 0u : 1u;
+          const int natoms = min(4, atoms_k - kb * 4);
+          for (int a = 0; a < natoms; ++a) {
+            tc_cp_sf(t_sfw + a * 4, sfw_desc0 + so + 32 * a);
+            tc_cp_sf(t_sfx + a * 4, sfx_desc0 + so + 32 * a);
+            tc_mma_nvf4(d_tmem, w_desc0 + so + 2 * a, x_desc0 + so + 2 * a, SB_IDESC,
+                        t_sfw + a * 4, t_sfx + a * 4, a == 0 ? first : 1u);
+          }
+          tc_commit(smem_u32(&bar_empty[s]));
+        }
+        if (!ok) break;
+        tc_commit(smem_u32(&bar_acc_full[b]));
+      }
+      tc_commit(smem_u32(&bar_drain));
+      volatile int never = 0;
+      mbar_wait_bounded(smem_u32(&bar_drain), 0, &never);
+    }
+    __syncwarp();
+  } else if (warp >= EPI_WARP0) {
+    // =========================== epilogue ===========================
+    // warp q reads weight rows 32q..32q+31 of the tile (its TMEM lane quadrant) for the 32 token
+    // columns; column j is token row m0 + j, and the real rows of a segment come first
+    const int q = warp & 3;
+    uint32_t tile_it = 0;
+    for (int t = blockIdx.x; t < total; t += gridDim.x, ++tile_it) {
+      const int b = tile_it & 1;
+      const Tile tl = decode_tile(t, tile_start, seg, E, args.n_tiles);
+      if (!mbar_wait_bounded(smem_u32(&bar_acc_full[b]), (tile_it >> 1) & 1u, &abort_flag)) break;
+      tc_fence_after();
+      uint32_t v[32];
+      tmem_ld32(tmem + SB_TM_ACC + b * SB_N + (static_cast<uint32_t>(q * 32) << 16), v);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bar_acc_empty[b]));
+
+      const float alpha = 1.0f / (__ldg(args.gs_a) * __ldg(args.gs_b + tl.e));
+      const int my_tok = __ldg(args.row_token + tl.m0 + lane);
+      const int count = __popc(__ballot_sync(0xffffffffu, my_tok >= 0));
+      if (MODE == L2_SCATTER) {
+        const float my_w = __ldg(args.row_w + tl.m0 + lane);
+        const int H = args.N;
+        const int n = tl.nt * 128 + q * 32 + lane;  // output feature of this thread
+#pragma unroll
+        for (int j = 0; j < SB_N; ++j) {  // unrolled so v[j] stays in registers
+          if (j < count) {
+            const int tok = __shfl_sync(0xffffffffu, my_tok, j);
+            const float w = __shfl_sync(0xffffffffu, my_w, j);
+            if (tok < args.T) {
+              atomicAdd(args.acc + (int64_t)tok * H + n, __uint_as_float(v[j]) * (alpha * w));
+            } else if (lane == 0) {
+              report(args.status, NVFP4_DEVERR_BAD_INDEX);
+            }
+          }
+        }
+      } else {
+        // lanes 0..15: gate rows of h features f0..f0+15, lanes 16..31: the matching up rows
+        const float gs_h = __ldg(args.gs_h);
+        const int I = args.I;
+        const int f0 = tl.nt * 64 + q * 16;
+#pragma unroll
+        for (int j = 0; j < SB_N; ++j) {  // unrolled so v[j] stays in registers
+          if (j >= count) break;
+          const float x = __uint_as_float(v[j]) * alpha;
+          const float other = __shfl_xor_sync(0xffffffffu, x, 16);
+          const float h = lane < 16 ? __fdividef(x * other, 1.0f + __expf(-x)) : 0.0f;
+          float amax = fabsf(h);
+#pragma unroll
+          for (int o = 8; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+          float rcp;
+          const uint32_t sb = nvfp4_block_scale(amax, gs_h, rcp);
+          const uint32_t code = rcp == 0.0f ? 0u : (cvt_e2m1x2(scaled(h, rcp), 0.0f) & 0xFu);
+          // pack: byte of features (2i, 2i+1) in lane 2i, then bytes 0..7 into lanes 0 and 4
+          const uint32_t byte = code | (__shfl_down_sync(0xffffffffu, code, 1) << 4);
+          const uint32_t bb = __shfl_sync(0xffffffffu, byte, (2 * lane) & 31);
+          const uint32_t w2 = bb | (__shfl_down_sync(0xffffffffu, bb, 1) << 8);
+          const uint32_t w4 = w2 | (__shfl_down_sync(0xffffffffu, w2, 2) << 16);
+          const uint32_t hi = __shfl_sync(0xffffffffu, w4, 4);
+          if (lane == 0) {
+            const int64_t row = tl.m0 + j;
+            *reinterpret_cast<uint2*>(args.h + row * (I / 2) + f0 / 2) = make_uint2(w4, hi);
+            args.sfh[sf_offset(row, f0 / 16, I / 16)] = static_cast<uint8_t>(sb);
+          }
+        }
+      }
+    }
+  }
+
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 2) tmem_dealloc(tmem, TMEM_COLS);
+  if (tid == 0 && abort_flag) report(args.status, NVFP4_DEVERR_TIMEOUT);
+}
+
 // ------------------------------------------------------------------------------ host side
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -442,13 +733,14 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 2D byte tensor [rows][row_bytes], box 128 bytes x 128 rows, 128-byte swizzle.
-bool make_map(CUtensorMap* m, const void* base, uint64_t row_bytes, uint64_t rows) {
+// 2D byte tensor [rows][row_bytes], box 128 bytes x box_rows rows, 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* base, uint64_t row_bytes, uint64_t rows,
+              uint32_t box_rows = 128) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {row_bytes, rows};
   cuuint64_t strides[1] = {row_bytes};
-  cuuint32_t box[2] = {128, 128};
+  cuuint32_t box[2] = {128, box_rows};
   cuuint32_t estr[2] = {1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -481,6 +773,22 @@ nvfp4_status_t launch(const uint8_t* a, const uint8_t* b, int64_t b_rows, GemmAr
   }
   grouped_gemm_kernel<MODE><<<num_sms(), NUM_THREADS, SMEM_BYTES, s>>>(ma, mb, args);
   return check_launch("grouped_gemm_kernel");
+}
+
+template <int MODE>
+nvfp4_status_t launch_small(const uint8_t* x, const uint8_t* w, int64_t w_rows, GemmArgs args,
+                            cudaStream_t s) {
+  CUtensorMap mx, mw;
+  if (!make_map(&mx, x, args.K / 2, args.R_max, SB_N) || !make_map(&mw, w, args.K / 2, w_rows)) {
+    set_last_error("cuTensorMapEncodeTiled failed");
+    return NVFP4_ERR_CUDA;
+  }
+  if (cudaFuncSetAttribute(grouped_gemm_small_kernel<MODE>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, SB_SMEM_BYTES) !=
+      cudaSuccess)
+    return check_launch("cudaFuncSetAttribute");
+  grouped_gemm_small_kernel<MODE><<<num_sms(), SB_THREADS, SB_SMEM_BYTES, s>>>(mx, mw, args);
+  return check_launch("grouped_gemm_small_kernel");
 }
 
 __global__ void cast_bf16_kernel(const float* __restrict__ acc, __nv_bfloat16* __restrict__ out,
@@ -517,13 +825,18 @@ nvfp4_status_t gemm_plain(const uint8_t* a, const uint8_t* sfa, const float* gs_
 
 nvfp4_status_t gemm_l1(const uint8_t* a, const uint8_t* sfa, const float* gs_a, const uint8_t* w1,
                        const uint8_t* sfw1, const float* gs_w1, const int32_t* offs,
-                       const int32_t* row_token, int E, int H, int I, int64_t R_max,
+                       const int32_t* row_token, int T, int E, int H, int I, int64_t R_max,
                        const float* gs_h, uint8_t* h, uint8_t* sfh, int32_t* status,
                        cudaStream_t s) {
   GemmArgs g{};
   g.sfa = sfa; g.sfb = sfw1; g.gs_a = gs_a; g.gs_b = gs_w1; g.offs = offs;
-  g.E = E; g.N = 2 * I; g.K = H; g.n_tiles = I / 128; g.R_max = R_max;
+  g.E = E; g.N = 2 * I; g.K = H; g.R_max = R_max;
   g.gs_h = gs_h; g.h = h; g.sfh = sfh; g.I = I; g.row_token = row_token; g.status = status;
+  if (row_token != nullptr && T > 0 && T <= SB_N) {
+    g.n_tiles = 2 * I / 128;  // 128 weight rows (64 h features) per tile
+    return launch_small<L1_SWIGLU>(a, w1, (int64_t)E * 2 * I, g, s);
+  }
+  g.n_tiles = I / 128;
   return launch<L1_SWIGLU>(a, w1, (int64_t)E * 2 * I, g, s);
 }
 
@@ -537,9 +850,16 @@ nvfp4_status_t gemm_l2(const uint8_t* h, const uint8_t* sfh, const float* gs_h, 
     return check_launch("memset acc");
   GemmArgs g{};
   g.sfa = sfh; g.sfb = sfw2; g.gs_a = gs_h; g.gs_b = gs_w2; g.offs = offs;
-  g.E = E; g.N = H; g.K = I; g.n_tiles = H / BN; g.R_max = R_max;
+  g.E = E; g.N = H; g.K = I; g.R_max = R_max;
   g.row_token = row_token; g.row_w = row_w; g.acc = acc; g.T = T; g.status = status;
-  nvfp4_status_t st = launch<L2_SCATTER>(h, w2, (int64_t)E * H, g, s);
+  nvfp4_status_t st;
+  if (T <= SB_N) {
+    g.n_tiles = H / 128;  // 128 output features per tile
+    st = launch_small<L2_SCATTER>(h, w2, (int64_t)E * H, g, s);
+  } else {
+    g.n_tiles = H / BN;
+    st = launch<L2_SCATTER>(h, w2, (int64_t)E * H, g, s);
+  }
   if (st != NVFP4_OK || out_bf16 == nullptr) return st;
   const int64_t n8 = (int64_t)T * H / 8;
   const int64_t want = (n8 + 255) / 256;
@@ -571,17 +891,17 @@ extern "C" nvfp4_status_t nvfp4_grouped_gemm(const uint8_t* a, const uint8_t* sf
 
 extern "C" nvfp4_status_t moe_grouped_gemm_l1_swiglu_q(
     const uint8_t* a, const uint8_t* sfa, const float* gs_a, const uint8_t* w1,
-    const uint8_t* sfw1, const float* gs_w1, const int32_t* offs, const int32_t* row_token, int E,
-    int H, int I, int64_t R_max, const float* gs_h, uint8_t* h, uint8_t* sfh, int32_t* dev_status,
-    nvfp4_stream_t stream) {
-  if (E < 1 || E > MAX_E || H <= 0 || I <= 0 || R_max < 0) return NVFP4_ERR_INVALID_ARG;
+    const uint8_t* sfw1, const float* gs_w1, const int32_t* offs, const int32_t* row_token, int T,
+    int E, int H, int I, int64_t R_max, const float* gs_h, uint8_t* h, uint8_t* sfh,
+    int32_t* dev_status, nvfp4_stream_t stream) {
+  if (E < 1 || E > MAX_E || H <= 0 || I <= 0 || R_max < 0 || T < 0) return NVFP4_ERR_INVALID_ARG;
   if (H % 64 || I % 128 || R_max % 128) return NVFP4_ERR_UNSUPPORTED_SHAPE;
   if (!gs_a || !gs_w1 || !offs || !gs_h) return NVFP4_ERR_INVALID_ARG;
   if (R_max == 0) return NVFP4_OK;
   if (!ok_ptr(a) || !ok_ptr(sfa) || !ok_ptr(w1) || !ok_ptr(sfw1) || !ok_ptr(h) || !ok_ptr(sfh))
     return (a && sfa && w1 && sfw1 && h && sfh) ? NVFP4_ERR_MISALIGNED : NVFP4_ERR_INVALID_ARG;
   if (reinterpret_cast<uintptr_t>(row_token) & 3u) return NVFP4_ERR_MISALIGNED;
-  return gemm_l1(a, sfa, gs_a, w1, sfw1, gs_w1, offs, row_token, E, H, I, R_max, gs_h, h, sfh,
+  return gemm_l1(a, sfa, gs_a, w1, sfw1, gs_w1, offs, row_token, T, E, H, I, R_max, gs_h, h, sfh,
                  dev_status, reinterpret_cast<cudaStream_t>(stream));
 }
 

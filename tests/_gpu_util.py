@@ -63,3 +63,20 @@ def compare_requant(c_gpu, s_gpu, c_ref, s_ref, gs):
     step = np.maximum(e2m1_step(mag), e2m1_step(np.abs(F.e2m1_decode(c_gpu)))) * d
     far = np.abs(d_gpu - d_ref) > step * (1 + 1e-9) + 1e-30
     return float(mism.mean()), int(far.sum())
+
+
+def upload_weights(qw, w1=False):
+    """Oracle QuantWeights -> device NVFP4Weights.  With w1=True the rows are stored in the
+    kernels' 64-row gate/up interleaved layout (moe_w1_row_map)."""
+    import nvfp4_block_scaled_gsa_b200 as nv
+    E, N, K2 = qw.codes.shape
+    K = 2 * K2
+    codes, sf = qw.codes, qw.sf
+    if w1:
+        m = nv.w1_row_map(N // 2).numpy()
+        codes = np.empty_like(qw.codes)
+        sf = np.empty_like(qw.sf)
+        codes[:, m] = qw.codes
+        sf[:, m] = qw.sf
+    return nv.NVFP4Weights(to_dev(codes.reshape(E * N, K // 2)),
+                           to_dev(Q.tile_sf(sf.reshape(E * N, K // 16))), to_dev(qw.gs), E, N, K)

@@ -96,7 +96,7 @@ def test_gemms_reject_bad_shapes(L):
     assert L.nvfp4_grouped_gemm(f, f, f, f, f, f, f, 2, 256, 96, 128, f, 0, None, None) == 2
     assert L.nvfp4_grouped_gemm(f, f, f, f, f, f, f, 2, 256, 64, 100, f, 0, None, None) == 2
     assert L.nvfp4_grouped_gemm(f, f, f, f, f, f, f, 2, 256, 64, 128, f, 7, None, None) == 1
-    assert L.moe_grouped_gemm_l1_swiglu_q(f, f, f, f, f, f, f, None, 8, 256, 96, 128, f, f, f,
+    assert L.moe_grouped_gemm_l1_swiglu_q(f, f, f, f, f, f, f, None, 0, 8, 256, 96, 128, f, f, f,
                                           None, None) == 2  # I % 128
     assert L.moe_grouped_gemm_l2_scatter(f, f, f, f, f, f, f, f, f, 8, 200, 128, 4, 128, f, f,
                                          None, None) == 2  # H % 256
@@ -104,3 +104,16 @@ def test_gemms_reject_bad_shapes(L):
                              None) == 4  # workspace too small
     assert L.moe_ffn_forward(f, f, 4, 256, 128, 8, 2, f, f, f, f, f, f, f, f, None, 1 << 30, None,
                              None) == 1
+
+
+def test_w1_row_map_is_the_documented_interleave(L):
+    I = 192
+    buf = (ctypes.c_int32 * (2 * I))()
+    assert L.moe_w1_row_map(I, ctypes.cast(buf, ctypes.c_void_p)) == 0
+    m = list(buf)
+    assert sorted(m) == list(range(2 * I))
+    for r in (0, 1, 15, 16, 63, 64, 100, 191):
+        assert m[r] == 32 * (r // 16) + r % 16            # gate row r
+        assert m[I + r] == 32 * (r // 16) + 16 + r % 16   # up row r
+    assert m[:3] == [0, 1, 2] and m[16] == 32 and m[I] == 16
+    assert L.moe_w1_row_map(100, ctypes.cast(buf, ctypes.c_void_p)) == 1  # I % 16

@@ -19,19 +19,29 @@ pytestmark = pytest.mark.gpu
 
 def _prepack_both(cfg, which, N, K):
     wf = [gen_weight_expert(cfg.seed, which, e, N, K) for e in range(cfg.E)]
-    wd = nv.quantize_weights(lambda e: wf[e].to(DEV), cfg.E, N, K)
+    if which == 1:
+        wd = nv.quantize_w1(lambda e: wf[e].to(DEV), cfg.E, N // 2, K)
+    else:
+        wd = nv.quantize_weights(lambda e: wf[e].to(DEV), cfg.E, N, K)
     wo = M.QuantWeights.from_float(np.stack([w.float().numpy() for w in wf]))
     return wd, wo
 
 
-def test_weight_prepack_bit_exact():
+@pytest.mark.parametrize("which", [1, 2])
+def test_weight_prepack_bit_exact(which):
     cfg = CONFIGS["tiny"]
-    wd, wo = _prepack_both(cfg, 1, 2 * cfg.I, cfg.H)
+    N, K = (2 * cfg.I, cfg.H) if which == 1 else (cfg.H, cfg.I)
+    wd, wo = _prepack_both(cfg, which, N, K)
     torch.cuda.synchronize()
-    E, N, K = cfg.E, 2 * cfg.I, cfg.H
+    E = cfg.E
+    codes = wd.codes.cpu().numpy().reshape(E, N, K // 2)
+    sf = Q.untile_sf(wd.sf.cpu().numpy(), E * N, K // 16).reshape(E, N, K // 16)
+    if which == 1:  # stored rows are gate/up interleaved; bring them back to logical order
+        m = nv.w1_row_map(cfg.I).numpy()
+        codes, sf = codes[:, m], sf[:, m]
     assert np.array_equal(wd.gs.cpu().numpy(), wo.gs)
-    assert np.array_equal(wd.codes.cpu().numpy(), wo.codes.reshape(E * N, K // 2))
-    assert np.array_equal(Q.untile_sf(wd.sf.cpu().numpy(), E * N, K // 16), wo.sf.reshape(E * N, -1))
+    assert np.array_equal(codes, wo.codes)
+    assert np.array_equal(sf, wo.sf)
 
 
 def _ffn_check(cfg, x, lg):
@@ -88,3 +98,14 @@ def test_ffn_rejects_small_workspace():
     with pytest.raises(nv.Nvfp4Error) as ei:
         nv.moe_ffn_forward(x, lg, cfg.k, w1d, w2d, torch.ones(1, device=DEV), ws=ws)
     assert ei.value.code == 4
+
+
+@pytest.mark.parametrize("T", [16, 32, 3])
+def test_ffn_small_batch_end_to_end(T):
+    """T <= 32 runs the small-batch GEMM kernels inside moe_ffn_forward."""
+    from dataclasses import replace
+    cfg = replace(CONFIGS["tiny"], T=T)
+    got, ref = _ffn_check(cfg, gen_x(cfg), gen_logits(cfg))
+    want = M.bf16_round(ref["out"])
+    assert rel_fro(got, want) <= 1e-3
+    assert cosine(got, want) >= 0.9999

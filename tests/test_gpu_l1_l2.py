@@ -14,7 +14,8 @@ from oracle import moe as M
 from oracle import quant as Q
 from oracle import routing as R
 from synth import CONFIGS, gen_logits, gen_weight_expert, gen_x
-from tests._gpu_util import DEV, compare_requant, download_nvfp4, rel_fro, to_dev, upload_nvfp4
+from tests._gpu_util import (DEV, compare_requant, download_nvfp4, rel_fro, to_dev, upload_nvfp4,
+                             upload_weights)
 
 pytestmark = pytest.mark.gpu
 
@@ -22,9 +23,7 @@ pytestmark = pytest.mark.gpu
 def _weights(seed, which, E, N, K):
     wf = np.stack([gen_weight_expert(seed, which, e, N, K).float().numpy() for e in range(E)])
     w = M.QuantWeights.from_float(wf)
-    wd = nv.NVFP4Weights(to_dev(w.codes.reshape(E * N, K // 2)),
-                         to_dev(Q.tile_sf(w.sf.reshape(E * N, K // 16))), to_dev(w.gs), E, N, K)
-    return w, wd
+    return w, upload_weights(w, w1=(which == 1))
 
 
 def _setup(T, H, I, E, k, seed=0, drop=0.0):
@@ -41,8 +40,11 @@ def _setup(T, H, I, E, k, seed=0, drop=0.0):
     return x, ids, w32, w1, w1d, w2, w2d
 
 
-@pytest.mark.parametrize("T,H,I,E,k", [(64, 256, 128, 8, 2), (200, 512, 256, 6, 3),
-                                       (33, 7168, 2048, 2, 2), (96, 256, 128, 256, 8)])
+@pytest.mark.parametrize("T,H,I,E,k", [
+    (64, 256, 128, 8, 2), (200, 512, 256, 6, 3), (33, 7168, 2048, 2, 2), (96, 256, 128, 256, 8),
+    # T <= 32: the small-batch (weights-as-M) kernels
+    (16, 256, 128, 8, 2), (32, 512, 256, 6, 3), (20, 7168, 2048, 3, 2), (16, 256, 128, 256, 8),
+    (1, 256, 128, 4, 1)])
 def test_l1_and_l2_match_oracle(T, H, I, E, k):
     x, ids, w32, w1, w1d, w2, w2d = _setup(T, H, I, E, k, drop=0.1)
     gs_h = np.float32(64.0 if H <= 512 else 1.0)
@@ -66,22 +68,32 @@ def test_l1_and_l2_match_oracle(T, H, I, E, k):
     # all-padding row groups but must give the same bytes on real rows)
     h, sfh = nv.l1_swiglu_q(a, asf, gs_x, w1d, offs, gs_h_d)
     row_token_d = to_dev(perm["row_token"].astype(np.int32))
-    h2, sfh2 = nv.l1_swiglu_q(a, asf, gs_x, w1d, offs, gs_h_d, row_token=row_token_d)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    h2, sfh2 = nv.l1_swiglu_q(a, asf, gs_x, w1d, offs, gs_h_d, row_token=row_token_d, T=T,
+                              status=status)
     torch.cuda.synchronize()
     hc2, hs2 = download_nvfp4(h2, sfh2, Rr, I)
-    assert rel_fro(c1.cpu().numpy()[valid], ref["c1"][valid]) <= 1e-5
+    c1_logical = c1.cpu().numpy()[:, nv.w1_row_map(I).numpy()]  # stored -> logical columns
+    assert rel_fro(c1_logical[valid], ref["c1"][valid]) <= 1e-5
     hc, hs = download_nvfp4(h, sfh, Rr, I)
     frac, far = compare_requant(hc[valid], hs[valid], ref["h_codes"][valid], ref["h_sf"][valid], gs_h)
     assert far == 0
     assert frac <= 1e-3
-    assert np.array_equal(hc2[valid], hc[valid]) and np.array_equal(hs2[valid], hs[valid])
+    # the row-map call (small-batch kernel when T <= 32) against the oracle too
+    frac2, far2 = compare_requant(hc2[valid], hs2[valid], ref["h_codes"][valid], ref["h_sf"][valid],
+                                  gs_h)
+    assert far2 == 0 and frac2 <= 1e-3
+    if T > 32:  # same kernel, same accumulation order: identical bytes
+        assert np.array_equal(hc2[valid], hc[valid]) and np.array_equal(hs2[valid], hs[valid])
 
     # ---- L2 + scatter on the oracle's h codes (identical operands)
     h_o, sfh_o = upload_nvfp4(ref["h_codes"], ref["h_sf"])
     row_token = to_dev(perm["row_token"].astype(np.int32))
     row_w = to_dev(perm["row_w"].astype(np.float32))
-    acc, out = nv.l2_scatter(h_o, sfh_o, gs_h_d, w2d, offs, row_token, row_w, T)
+    acc, out = nv.l2_scatter(h_o, sfh_o, gs_h_d, w2d, offs, row_token, row_w, T, status=status)
     torch.cuda.synchronize()
+    code, rc = nv.read_status(status)
+    assert code == 0 and rc == 0
     assert rel_fro(acc.cpu().numpy(), ref["out"]) <= 1e-5
     assert torch.equal(out.cpu(), acc.cpu().to(torch.bfloat16))
     dropped = np.all(ids < 0, axis=1)
