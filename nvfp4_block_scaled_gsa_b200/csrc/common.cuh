@@ -183,6 +183,64 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
+// 32 lanes x 16 / 32 consecutive 32-bit columns into tensor memory (one value per column per lane).
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]),
+      "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]),
+      "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]),
+      "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// Scale factors of one stage from shared memory into tensor memory, for the calling warp's lane
+// quadrant.  The tensor-core layout for a 128-row operand (and for each 128-row half of a 256-row
+// one) puts, for K step a, the 4 scales of row i + 32*m at lane i of every quadrant, column
+// 4a + m; in the shared-memory atom those 16 bytes (m = 0..3) are line i, bytes 16i..16i+15.
+// So lane i writes, per 128-row atom, one 16-byte line of its own index as 4 columns.
+__device__ __forceinline__ void sf_rows128_to_tmem(uint32_t taddr, const uint8_t* atoms, int lane) {
+  uint32_t r[16];
+#pragma unroll
+  for (int a = 0; a < 4; ++a) {
+    const uint4 v = *reinterpret_cast<const uint4*>(atoms + a * 512 + lane * 16);
+    r[4 * a] = v.x;
+    r[4 * a + 1] = v.y;
+    r[4 * a + 2] = v.z;
+    r[4 * a + 3] = v.w;
+  }
+  tmem_st16(taddr, r);
+}
+// 256-row operand: columns 8a + 4h + m, h = which 128-row half (atoms of half h at +h*2048).
+__device__ __forceinline__ void sf_rows256_to_tmem(uint32_t taddr, const uint8_t* atoms, int lane) {
+  uint32_t r[32];
+#pragma unroll
+  for (int a = 0; a < 4; ++a) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const uint4 v = *reinterpret_cast<const uint4*>(atoms + h * 2048 + a * 512 + lane * 16);
+      r[8 * a + 4 * h] = v.x;
+      r[8 * a + 4 * h + 1] = v.y;
+      r[8 * a + 4 * h + 2] = v.z;
+      r[8 * a + 4 * h + 3] = v.w;
+    }
+  }
+  tmem_st32(taddr, r);
+}
 
 // ------------------------------------------------------------------------------ conversions
 // E4M3 (round to nearest even, saturate to +-448) of one float; result in the low byte.

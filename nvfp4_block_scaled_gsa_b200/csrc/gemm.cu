@@ -8,11 +8,16 @@
 //
 //   warp 0      TMA producer: A and B tiles (cp.async.bulk.tensor, 128-byte swizzle) and the
 //               pre-tiled scale atoms (cp.async.bulk) into a 4-stage shared-memory ring
-//   warp 1      MMA issuer: tcgen05.cp moves the stage's scales into tensor memory, then
-//               tcgen05.mma.kind::mxf4nvf4.block_scale (M=128, N=256, K=64) accumulates in TMEM
+//   warp 1      MMA issuer: tcgen05.mma.kind::mxf4nvf4.block_scale (M=128, N=256, K=64) into a
+//               TMEM accumulator; it issues nothing else, because the tensor pipe runs its
+//               instructions one after another and scale copies in that stream cost as much as
+//               the MMAs themselves
 //   warp 2      owns the tensor-memory allocation (512 columns)
-//   warps 4..7  epilogue: tcgen05.ld of the accumulator (warp w reads lanes 32*(w%4)..+31),
+//   warps 4..11 epilogue: tcgen05.ld of the accumulator (warp w reads lanes 32*(w%4)..+31),
 //               then one of the fused epilogues below
+//   warps 12..15 scale-factor warps: each stage's scale atoms go from shared memory to the
+//               tensor-memory layout the MMA reads, by ld.shared + tcgen05.st, one warp per
+//               lane quadrant
 //
 // Epilogues (the MODE template parameter):
 //   PLAIN_F32 / PLAIN_BF16  C = acc / (gs_a * gs_b[e])
@@ -58,9 +63,10 @@ constexpr uint32_t TM_SFB = TM_SFA + STAGES * 16;    // 32 columns per stage
 static_assert(TM_SFB + STAGES * 32 <= TMEM_COLS, "tensor memory budget");
 
 constexpr uint32_t IDESC = idesc_nvf4(BN);
-constexpr int NUM_THREADS = 384;  // 4 role warps + 8 epilogue warps
+constexpr int NUM_THREADS = 512;  // 4 role warps + 8 epilogue warps + 4 scale-factor warps
 constexpr int EPI_WARP0 = 4;
 constexpr int EPI_WARPS = 8;
+constexpr int SF_WARP0 = EPI_WARP0 + EPI_WARPS;
 constexpr int MAX_E = 256;
 
 enum Mode { PLAIN_F32 = 0, PLAIN_BF16 = 1, L1_SWIGLU = 2, L2_SCATTER = 3 };
@@ -122,6 +128,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t bar_full[STAGES];
   __shared__ __align__(8) uint64_t bar_empty[STAGES];
+  __shared__ __align__(8) uint64_t bar_sf[STAGES];
   __shared__ __align__(8) uint64_t bar_acc_full;
   __shared__ __align__(8) uint64_t bar_acc_empty;
   __shared__ __align__(8) uint64_t bar_drain;
@@ -176,6 +183,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(smem_u32(&bar_full[s]), 1);
       mbar_init(smem_u32(&bar_empty[s]), 1);
+      mbar_init(smem_u32(&bar_sf[s]), 4);
     }
     mbar_init(smem_u32(&bar_acc_full), 1);
     mbar_init(smem_u32(&bar_acc_empty), EPI_WARPS);
@@ -252,9 +260,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const uint32_t s0 = smem_u32(smem);
       const uint64_t a_desc0 = smem_desc(s0, 16, 1024, 2);
       const uint64_t b_desc0 = smem_desc(s0 + A_BYTES, 16, 1024, 2);
-      const uint64_t sfa_desc0 = smem_desc(s0 + A_BYTES + B_BYTES, 0, 128, 0);
-      const uint64_t sfb_desc0 = smem_desc(s0 + A_BYTES + B_BYTES + SFA_BYTES, 0, 128, 0);
-      constexpr uint64_t kSfbHalf = (SFB_BYTES / 2) >> 4;  // second 128 rows of the B scales
       uint32_t it = 0, tile_it = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++tile_it) {
@@ -266,7 +271,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int kb = 0; kb < nk; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1u;
-          if (!mbar_wait_bounded(smem_u32(&bar_full[s]), ph, &abort_flag)) {
+          if (!mbar_wait_bounded(smem_u32(&bar_full[s]), ph, &abort_flag) ||
+              !mbar_wait_bounded(smem_u32(&bar_sf[s]), ph, &abort_flag)) {
             ok = false;
             break;
           }
@@ -275,26 +281,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const uint32_t t_sfa = tmem + TM_SFA + s * 16;
           const uint32_t t_sfb = tmem + TM_SFB + s * 32;
           const uint32_t first = kb == 0 ? 0u : 1u;
-          // per 64-element K step: its three scale copies, then its MMA, so the MMA of step a
-          // runs while the copies of step a+1 are in flight
-          if (atoms_k - kb * 4 >= 4) {
+          // scales of this stage are already in tensor memory (scale-factor warps)
+          const int natoms = min(4, atoms_k - kb * 4);
+          if (natoms == 4) {
 #pragma unroll
-            for (int a = 0; a < 4; ++a) {
-              tc_cp_sf(t_sfa + a * 4, sfa_desc0 + so + 32 * a);
-              tc_cp_sf(t_sfb + a * 8, sfb_desc0 + so + 32 * a);
-              tc_cp_sf(t_sfb + a * 8 + 4, sfb_desc0 + so + kSfbHalf + 32 * a);
+            for (int a = 0; a < 4; ++a)
               tc_mma_nvf4(tmem + TM_ACC, a_desc0 + so + 2 * a, b_desc0 + so + 2 * a, IDESC,
                           t_sfa + a * 4, t_sfb + a * 8, a == 0 ? first : 1u);
-            }
           } else {
-            const int natoms = atoms_k - kb * 4;
-            for (int a = 0; a < natoms; ++a) {
-              tc_cp_sf(t_sfa + a * 4, sfa_desc0 + so + 32 * a);
-              tc_cp_sf(t_sfb + a * 8, sfb_desc0 + so + 32 * a);
-              tc_cp_sf(t_sfb + a * 8 + 4, sfb_desc0 + so + kSfbHalf + 32 * a);
+            for (int a = 0; a < natoms; ++a)
               tc_mma_nvf4(tmem + TM_ACC, a_desc0 + so + 2 * a, b_desc0 + so + 2 * a, IDESC,
                           t_sfa + a * 4, t_sfb + a * 8, a == 0 ? first : 1u);
-            }
           }
           tc_commit(smem_u32(&bar_empty[s]));
         }
@@ -307,6 +304,30 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_wait_bounded(smem_u32(&bar_drain), 0, &never);
     }
     __syncwarp();
+  } else if (warp >= SF_WARP0) {
+    // =========================== scale-factor warps ===========================
+    // warp (SF_WARP0 + q) writes lane quadrant q of each stage's scale-factor columns
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    uint32_t it = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+      for (int kb = 0; kb < nk; ++kb, ++it) {
+        const int s = it % STAGES;
+        const uint32_t ph = (it / STAGES) & 1u;
+        if (!mbar_wait_bounded(smem_u32(&bar_full[s]), ph, &abort_flag)) {
+          ok = false;
+          break;
+        }
+        const uint8_t* st = smem + s * STAGE_BYTES;
+        sf_rows128_to_tmem(tmem + lane_base + TM_SFA + s * 16, st + A_BYTES + B_BYTES, lane);
+        sf_rows256_to_tmem(tmem + lane_base + TM_SFB + s * 32, st + A_BYTES + B_BYTES + SFA_BYTES,
+                           lane);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&bar_sf[s]));
+      }
+    }
   } else if (warp >= EPI_WARP0) {
     // =========================== epilogue ===========================
     // Two warps per tensor-memory lane quadrant (a warp may only read lanes 32*(warp%4)..+31);
@@ -463,7 +484,8 @@ constexpr uint32_t SB_TM_SFW = 64;                          // 16 columns per st
 constexpr uint32_t SB_TM_SFX = SB_TM_SFW + SB_STAGES * 16;  // 16 columns per stage
 static_assert(SB_TM_SFX + SB_STAGES * 16 <= TMEM_COLS, "tensor memory budget");
 constexpr uint32_t SB_IDESC = idesc_nvf4(SB_N);
-constexpr int SB_THREADS = 256;  // 4 role warps + 4 epilogue warps
+constexpr int SB_THREADS = 384;  // 4 role warps + 4 epilogue warps + 4 scale-factor warps
+constexpr int SB_SF_WARP0 = 8;
 
 template <int MODE>
 __global__ void __launch_bounds__(SB_THREADS, 1)
@@ -472,6 +494,7 @@ __global__ void __launch_bounds__(SB_THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t bar_full[SB_STAGES];
   __shared__ __align__(8) uint64_t bar_empty[SB_STAGES];
+  __shared__ __align__(8) uint64_t bar_sf[SB_STAGES];
   __shared__ __align__(8) uint64_t bar_acc_full[2];
   __shared__ __align__(8) uint64_t bar_acc_empty[2];
   __shared__ __align__(8) uint64_t bar_drain;
@@ -529,6 +552,7 @@ __global__ void __launch_bounds__(SB_THREADS, 1)
     for (int s = 0; s < SB_STAGES; ++s) {
       mbar_init(smem_u32(&bar_full[s]), 1);
       mbar_init(smem_u32(&bar_empty[s]), 1);
+      mbar_init(smem_u32(&bar_sf[s]), 4);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(smem_u32(&bar_acc_full[b]), 1);
@@ -597,8 +621,6 @@ __global__ void __launch_bounds__(SB_THREADS, 1)
       const uint32_t s0 = smem_u32(smem);
       const uint64_t w_desc0 = smem_desc(s0, 16, 1024, 2);
       const uint64_t x_desc0 = smem_desc(s0 + SB_W_BYTES, 16, 1024, 2);
-      const uint64_t sfw_desc0 = smem_desc(s0 + SB_W_BYTES + SB_X_BYTES, 0, 128, 0);
-      const uint64_t sfx_desc0 = smem_desc(s0 + SB_W_BYTES + SB_X_BYTES + SB_SF_BYTES, 0, 128, 0);
       uint32_t it = 0, tile_it = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++tile_it) {
@@ -613,7 +635,8 @@ __global__ void __launch_bounds__(SB_THREADS, 1)
         for (int kb = 0; kb < nk; ++kb, ++it) {
           const int s = it % SB_STAGES;
           const uint32_t ph = (it / SB_STAGES) & 1u;
-          if (!mbar_wait_bounded(smem_u32(&bar_full[s]), ph, &abort_flag)) {
+          if (!mbar_wait_bounded(smem_u32(&bar_full[s]), ph, &abort_flag) ||
+              !mbar_wait_bounded(smem_u32(&bar_sf[s]), ph, &abort_flag)) {
             ok = false;
             break;
           }
@@ -623,12 +646,9 @@ __global__ void __launch_bounds__(SB_THREADS, 1)
           const uint32_t t_sfx = tmem + SB_TM_SFX + s * 16;
           const uint32_t first = kb == 0 ? 0u : 1u;
           const int natoms = min(4, atoms_k - kb * 4);
-          for (int a = 0; a < natoms; ++a) {
-            tc_cp_sf(t_sfw + a * 4, sfw_desc0 + so + 32 * a);
-            tc_cp_sf(t_sfx + a * 4, sfx_desc0 + so + 32 * a);
+          for (int a = 0; a < natoms; ++a)
             tc_mma_nvf4(d_tmem, w_desc0 + so + 2 * a, x_desc0 + so + 2 * a, SB_IDESC,
                         t_sfw + a * 4, t_sfx + a * 4, a == 0 ? first : 1u);
-          }
           tc_commit(smem_u32(&bar_empty[s]));
         }
         if (!ok) break;
@@ -639,6 +659,28 @@ __global__ void __launch_bounds__(SB_THREADS, 1)
       mbar_wait_bounded(smem_u32(&bar_drain), 0, &never);
     }
     __syncwarp();
+  } else if (warp >= SB_SF_WARP0) {
+    // =========================== scale-factor warps ===========================
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    uint32_t it = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+      for (int kb = 0; kb < nk; ++kb, ++it) {
+        const int s = it % SB_STAGES;
+        const uint32_t ph = (it / SB_STAGES) & 1u;
+        if (!mbar_wait_bounded(smem_u32(&bar_full[s]), ph, &abort_flag)) {
+          ok = false;
+          break;
+        }
+        const uint8_t* st = smem + s * SB_STAGE_BYTES + SB_W_BYTES + SB_X_BYTES;
+        sf_rows128_to_tmem(tmem + lane_base + SB_TM_SFW + s * 16, st, lane);
+        sf_rows128_to_tmem(tmem + lane_base + SB_TM_SFX + s * 16, st + SB_SF_BYTES, lane);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&bar_sf[s]));
+      }
+    }
   } else if (warp >= EPI_WARP0) {
     // =========================== epilogue ===========================
     // warp q reads weight rows 32q..32q+31 of the tile (its TMEM lane quadrant) for the 32 token
