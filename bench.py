@@ -193,7 +193,7 @@ class Plan:
             ev[2].record()
         call("moe_grouped_gemm_l1_swiglu_q", p(self.xq), p(self.xsf), p(self.gs_x),
              p(self.w1.codes), p(self.w1.sf), p(self.w1.gs), p(self.offs), p(self.row_token),
-             T, E, H, I, self.R,
+             E, H, I, self.R,
              p(self.gs_h), p(self.hq), p(self.hsf), p(self.status), s)
         if ev:
             ev[3].record()

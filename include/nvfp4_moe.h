@@ -161,11 +161,6 @@ NVFP4_API nvfp4_status_t nvfp4_grouped_gemm(const uint8_t* a, const uint8_t* sfa
  *   row_token       optional int32 [R_max] (from moe_permute).  NULL: every row of every segment
  *                   is written.  Given: groups of 32 rows that are all padding (row_token < 0)
  *                   are skipped and their h rows left unwritten.
- *   T               number of tokens routed (0 = unknown).  With row_token given and T <= 32 the
- *                   small-batch kernel runs (weights as the 128-row operand, an expert's tokens as
- *                   a 32-column tile); it requires each token to reach an expert at most once
- *                   (as moe_permute's routing does) and flags a longer segment with
- *                   NVFP4_DEVERR_BAD_OFFSETS.
  *   gs_h            device float[1]
  *   h, sfh          output NVFP4 [R_max][I] (tiled scales)
  *   Constraints: H % 64 == 0, I % 128 == 0, R_max % 128 == 0, 1 <= E <= 256.
@@ -173,7 +168,7 @@ NVFP4_API nvfp4_status_t nvfp4_grouped_gemm(const uint8_t* a, const uint8_t* sfa
 NVFP4_API nvfp4_status_t moe_grouped_gemm_l1_swiglu_q(const uint8_t* a, const uint8_t* sfa, const float* gs_a,
                                             const uint8_t* w1, const uint8_t* sfw1,
                                             const float* gs_w1, const int32_t* offs,
-                                            const int32_t* row_token, int T, int E, int H, int I,
+                                            const int32_t* row_token, int E, int H, int I,
                                             int64_t R_max, const float* gs_h, uint8_t* h,
                                             uint8_t* sfh, int32_t* dev_status,
                                             nvfp4_stream_t stream);
@@ -199,8 +194,7 @@ NVFP4_API nvfp4_status_t moe_w1_row_map(int I, int32_t* map);
  *   w2, sfw2, gs_w2  NVFP4 [E*H][I], gs_w2 float[E]
  *   offs, row_token, row_w  from moe_permute
  *   acc_ws           float [T][H] scratch/output;  out_bf16  bf16 [T][H] or NULL
- *   With T <= 32 the small-batch kernel runs (same condition on the routing as for L1).
- *   Constraints: H % 256 == 0, I % 64 == 0, R_max % 128 == 0, 1 <= E <= 256, T >= 0.
+ *   Constraints: H % 128 == 0, I % 64 == 0, R_max % 128 == 0, 1 <= E <= 256, T >= 0.
  * ------------------------------------------------------------------------------------------- */
 NVFP4_API nvfp4_status_t moe_grouped_gemm_l2_scatter(const uint8_t* h, const uint8_t* sfh, const float* gs_h,
                                            const uint8_t* w2, const uint8_t* sfw2,

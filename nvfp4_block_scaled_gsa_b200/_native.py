@@ -32,8 +32,8 @@ SIGNATURES = {
     "nvfp4_grouped_gemm": (c_int, [c_void, c_void, c_void, c_void, c_void, c_void, c_void, c_int,
                                    c_int, c_int, c_i64, c_void, c_int, c_void, c_void]),
     "moe_grouped_gemm_l1_swiglu_q": (c_int, [c_void, c_void, c_void, c_void, c_void, c_void,
-                                             c_void, c_void, c_int, c_int, c_int, c_int, c_i64,
-                                             c_void, c_void, c_void, c_void, c_void]),
+                                             c_void, c_void, c_int, c_int, c_int, c_i64, c_void,
+                                             c_void, c_void, c_void, c_void]),
     "moe_grouped_gemm_l2_scatter": (c_int, [c_void, c_void, c_void, c_void, c_void, c_void, c_void,
                                             c_void, c_void, c_int, c_int, c_int, c_int, c_i64,
                                             c_void, c_void, c_void, c_void]),

@@ -127,17 +127,15 @@ def grouped_gemm(a_codes, a_sf, gs_a, w: NVFP4Weights, offs, out_dtype=F32, stat
     return out
 
 
-def l1_swiglu_q(a_codes, a_sf, gs_a, w1: NVFP4Weights, offs, gs_h, row_token=None, T=0,
-                status=None):
+def l1_swiglu_q(a_codes, a_sf, gs_a, w1: NVFP4Weights, offs, gs_h, row_token=None, status=None):
     """L1 GEMM + SwiGLU + NVFP4 re-quantization -> (h codes (R, I/2), h tiled scales).
-    With row_token, all-padding groups of 32 rows are skipped (left unwritten); with row_token
-    and 0 < T <= 32 the small-batch kernel runs."""
+    With row_token, all-padding groups of 32 rows are skipped (left unwritten)."""
     R = a_codes.shape[0]
     I = w1.N // 2
     h = torch.empty(R, I // 2, dtype=U8, device=a_codes.device)
     sfh = torch.empty(sf_bytes(R, I), dtype=U8, device=a_codes.device)
     call("moe_grouped_gemm_l1_swiglu_q", _p(a_codes), _p(a_sf), _p(gs_a), _p(w1.codes),
-         _p(w1.sf), _p(w1.gs), _p(offs), _p(row_token), T, w1.E, w1.K, I, R, _p(gs_h), _p(h),
+         _p(w1.sf), _p(w1.gs), _p(offs), _p(row_token), w1.E, w1.K, I, R, _p(gs_h), _p(h),
          _p(sfh), _p(status), _stream())
     return h, sfh
 

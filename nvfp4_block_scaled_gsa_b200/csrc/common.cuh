@@ -139,12 +139,6 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint
   d |= static_cast<uint64_t>(layout & 7u) << 61;
   return d;
 }
-// Copy a 32-row x 16-byte block of scale factors from shared memory into tensor memory,
-// replicated into all four 32-lane sub-partitions.
-__device__ __forceinline__ void tc_cp_sf(uint32_t taddr, uint64_t sdesc) {
-  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
-               : "memory");
-}
 // D(tmem) (+)= A(smem) * B(smem)^T with E2M1 operands and UE4M3 scales per 16 elements (K = 64).
 __device__ __forceinline__ void tc_mma_nvf4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
                                             uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,

@@ -35,7 +35,7 @@ nvfp4_status_t permute_launch(const float* logits, int T, int E, int k, int reno
                               int32_t* dev_status, cudaStream_t s);
 nvfp4_status_t gemm_l1(const uint8_t* a, const uint8_t* sfa, const float* gs_a, const uint8_t* w1,
                        const uint8_t* sfw1, const float* gs_w1, const int32_t* offs,
-                       const int32_t* row_token, int T, int E, int H, int I, int64_t R_max,
+                       const int32_t* row_token, int E, int H, int I, int64_t R_max,
                        const float* gs_h, uint8_t* h, uint8_t* sfh, int32_t* status,
                        cudaStream_t s);
 nvfp4_status_t gemm_l2(const uint8_t* h, const uint8_t* sfh, const float* gs_h, const uint8_t* w2,
@@ -95,7 +95,7 @@ extern "C" nvfp4_status_t moe_ffn_forward(const void* x_bf16, const float* logit
                                           nvfp4_stream_t stream) {
   if (T < 0 || E < 1 || E > 256 || k < 1 || k > 32 || k > E || H <= 0 || I <= 0)
     return NVFP4_ERR_UNSUPPORTED_SHAPE;
-  if (H % 256 || I % 128) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (H % 128 || I % 128) return NVFP4_ERR_UNSUPPORTED_SHAPE;
   if ((int64_t)T * k > (int64_t)1 << 30) return NVFP4_ERR_UNSUPPORTED_SHAPE;
   if (T == 0) return NVFP4_OK;
   if (!x_bf16 || !logits || !w1 || !sfw1 || !gs_w1 || !w2 || !sfw2 || !gs_w2 || !gs_h ||
@@ -121,8 +121,7 @@ extern "C" nvfp4_status_t moe_ffn_forward(const void* x_bf16, const float* logit
                        f32(L.gs_x), 1, base + L.amax, dev_status, s);
   if (st != NVFP4_OK) return st;
   st = gemm_l1(base + L.xq, base + L.xsf, f32(L.gs_x), w1, sfw1, gs_w1, i32(L.offs),
-               i32(L.row_token), T, E, H, I, L.R_max, gs_h, base + L.hq, base + L.hsf, dev_status,
-               s);
+               i32(L.row_token), E, H, I, L.R_max, gs_h, base + L.hq, base + L.hsf, dev_status, s);
   if (st != NVFP4_OK) return st;
   return gemm_l2(base + L.hq, base + L.hsf, gs_h, w2, sfw2, gs_w2, i32(L.offs), i32(L.row_token),
                  f32(L.row_w), E, H, I, T, L.R_max, f32(L.acc), out_bf16, dev_status, s);

@@ -45,24 +45,10 @@ namespace nvfp4 {
 namespace {
 
 constexpr int BM = 128;
-constexpr int BN = 256;
 constexpr int BK_BYTES = 128;  // 256 FP4 elements per stage along K
-constexpr int STAGES = 4;
 constexpr int A_BYTES = BM * BK_BYTES;                // 16 KB
-constexpr int B_BYTES = BN * BK_BYTES;                // 32 KB
 constexpr int SFA_BYTES = 4 * 512;                    // 128 rows x 16 scales
-constexpr int SFB_BYTES = 2 * 4 * 512;                // 256 rows x 16 scales
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024;
-static_assert(STAGE_BYTES % 1024 == 0, "stages must keep 1024-byte alignment (128B swizzle)");
-
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t TM_ACC = 0;                       // 256 FP32 columns
-constexpr uint32_t TM_SFA = 256;                     // 16 columns per stage
-constexpr uint32_t TM_SFB = TM_SFA + STAGES * 16;    // 32 columns per stage
-static_assert(TM_SFB + STAGES * 32 <= TMEM_COLS, "tensor memory budget");
-
-constexpr uint32_t IDESC = idesc_nvf4(BN);
 constexpr int NUM_THREADS = 512;  // 4 role warps + 8 epilogue warps + 4 scale-factor warps
 constexpr int EPI_WARP0 = 4;
 constexpr int EPI_WARPS = 8;
@@ -70,6 +56,27 @@ constexpr int SF_WARP0 = EPI_WARP0 + EPI_WARPS;
 constexpr int MAX_E = 256;
 
 enum Mode { PLAIN_F32 = 0, PLAIN_BF16 = 1, L1_SWIGLU = 2, L2_SCATTER = 3 };
+
+// Tile width N per epilogue.  The L2 scatter uses 128-column tiles: then two accumulators fit in
+// tensor memory next to the per-stage scale factors, so its long scatter epilogue overlaps the
+// next tile's main loop.  The other epilogues use 256 columns (half the MMA instructions per
+// output; one accumulator).  Shared memory holds as many stages as fit in 216 KB.
+template <int MODE>
+struct TileCfg {
+  static constexpr int BN = MODE == L2_SCATTER ? 128 : 256;
+  static constexpr int B_BYTES = BN * BK_BYTES;
+  static constexpr int SFB_BYTES = (BN / 128) * 4 * 512;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+  static constexpr int STAGES = (216 * 1024) / STAGE_BYTES;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024;
+  static constexpr uint32_t SFB_COLS = (BN / 128) * 16;  // scale columns of B per stage
+  static constexpr int ACC_BUFS = 2 * BN + STAGES * (16 + SFB_COLS) <= TMEM_COLS ? 2 : 1;
+  static constexpr uint32_t TM_SFA = ACC_BUFS * BN;        // 16 columns per stage
+  static constexpr uint32_t TM_SFB = TM_SFA + STAGES * 16;
+  static constexpr uint32_t IDESC = idesc_nvf4(BN);
+  static_assert(STAGE_BYTES % 1024 == 0, "stages must keep 1024-byte alignment (128B swizzle)");
+  static_assert(TM_SFB + STAGES * SFB_COLS <= TMEM_COLS, "tensor memory budget");
+};
 
 struct GemmArgs {
   const uint8_t* sfa;
@@ -125,12 +132,16 @@ template <int MODE>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_a,
                         const __grid_constant__ CUtensorMap tm_b, const GemmArgs args) {
+  using C = TileCfg<MODE>;
+  constexpr int STAGES = C::STAGES;
+  constexpr int BN = C::BN;
+  constexpr int ACC_BUFS = C::ACC_BUFS;
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t bar_full[STAGES];
   __shared__ __align__(8) uint64_t bar_empty[STAGES];
   __shared__ __align__(8) uint64_t bar_sf[STAGES];
-  __shared__ __align__(8) uint64_t bar_acc_full;
-  __shared__ __align__(8) uint64_t bar_acc_empty;
+  __shared__ __align__(8) uint64_t bar_acc_full[ACC_BUFS];
+  __shared__ __align__(8) uint64_t bar_acc_empty[ACC_BUFS];
   __shared__ __align__(8) uint64_t bar_drain;
   __shared__ uint32_t tmem_slot;
   __shared__ int seg[MAX_E + 1];
@@ -185,8 +196,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(smem_u32(&bar_empty[s]), 1);
       mbar_init(smem_u32(&bar_sf[s]), 4);
     }
-    mbar_init(smem_u32(&bar_acc_full), 1);
-    mbar_init(smem_u32(&bar_acc_empty), EPI_WARPS);
+    for (int b = 0; b < ACC_BUFS; ++b) {
+      mbar_init(smem_u32(&bar_acc_full[b]), 1);
+      mbar_init(smem_u32(&bar_acc_empty[b]), EPI_WARPS);
+    }
     mbar_init(smem_u32(&bar_drain), 1);
     fence_mbar_init();
   }
@@ -214,10 +227,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       bool ok = true;
       for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
         const Tile tl = decode_tile(t, tile_start, seg, E, args.n_tiles);
-        // B rows of this N-tile: 256 consecutive rows (for L1: 8 blocks of 16 gate rows followed
-        // by the 16 matching up rows)
+        // B rows of this N-tile: BN consecutive rows (for L1: 16-row gate blocks each followed by
+        // the 16 matching up rows)
         const int b_row0 = tl.e * args.N + tl.nt * BN;
-        const int b_row1 = b_row0 + 128;
         for (int kb = 0; kb < nk; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1u;
@@ -227,19 +239,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
           const int natoms = min(4, atoms_k - kb * 4);
           const uint32_t full = smem_u32(&bar_full[s]);
-          uint8_t* st = smem + s * STAGE_BYTES;
-          const uint32_t sA = smem_u32(st), sB = sA + A_BYTES, sSFA = sB + B_BYTES,
+          uint8_t* st = smem + s * C::STAGE_BYTES;
+          const uint32_t sA = smem_u32(st), sB = sA + A_BYTES, sSFA = sB + C::B_BYTES,
                          sSFB = sSFA + SFA_BYTES;
-          mbar_arrive_expect_tx(full, A_BYTES + B_BYTES + natoms * 512 * 3);
+          mbar_arrive_expect_tx(full, A_BYTES + C::B_BYTES + natoms * 512 * (1 + BN / 128));
           tma_load_2d(sA, &tm_a, full, kb * BK_BYTES, tl.m0);
-          tma_load_2d(sB, &tm_b, full, kb * BK_BYTES, b_row0);
-          tma_load_2d(sB + B_BYTES / 2, &tm_b, full, kb * BK_BYTES, b_row1);
           const int64_t a_atom = (int64_t)(tl.m0 >> 7) * atoms_k + kb * 4;
-          const int64_t b_atom0 = (int64_t)(b_row0 >> 7) * atoms_k + kb * 4;
-          const int64_t b_atom1 = (int64_t)(b_row1 >> 7) * atoms_k + kb * 4;
           bulk_load(sSFA, args.sfa + a_atom * 512, natoms * 512, full);
-          bulk_load(sSFB, args.sfb + b_atom0 * 512, natoms * 512, full);
-          bulk_load(sSFB + SFB_BYTES / 2, args.sfb + b_atom1 * 512, natoms * 512, full);
+#pragma unroll
+          for (int j = 0; j < BN / 128; ++j) {
+            tma_load_2d(sB + j * 128 * BK_BYTES, &tm_b, full, kb * BK_BYTES, b_row0 + 128 * j);
+            const int64_t b_atom = (int64_t)((b_row0 >> 7) + j) * atoms_k + kb * 4;
+            bulk_load(sSFB + j * 4 * 512, args.sfb + b_atom * 512, natoms * 512, full);
+          }
         }
       }
       if (!ok) {
@@ -263,11 +275,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t it = 0, tile_it = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++tile_it) {
-        if (!mbar_wait_bounded(smem_u32(&bar_acc_empty), (tile_it & 1u) ^ 1u, &abort_flag)) {
+        const int b = tile_it % ACC_BUFS;
+        if (!mbar_wait_bounded(smem_u32(&bar_acc_empty[b]), ((tile_it / ACC_BUFS) & 1u) ^ 1u,
+                               &abort_flag)) {
           ok = false;
           break;
         }
         tc_fence_after();
+        const uint32_t d_tmem = tmem + b * BN;
         for (int kb = 0; kb < nk; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1u;
@@ -277,26 +292,26 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             break;
           }
           tc_fence_after();
-          const uint64_t so = static_cast<uint64_t>(s) * (STAGE_BYTES >> 4);
-          const uint32_t t_sfa = tmem + TM_SFA + s * 16;
-          const uint32_t t_sfb = tmem + TM_SFB + s * 32;
+          const uint64_t so = static_cast<uint64_t>(s) * (C::STAGE_BYTES >> 4);
+          const uint32_t t_sfa = tmem + C::TM_SFA + s * 16;
+          const uint32_t t_sfb = tmem + C::TM_SFB + s * C::SFB_COLS;
           const uint32_t first = kb == 0 ? 0u : 1u;
           // scales of this stage are already in tensor memory (scale-factor warps)
           const int natoms = min(4, atoms_k - kb * 4);
           if (natoms == 4) {
 #pragma unroll
             for (int a = 0; a < 4; ++a)
-              tc_mma_nvf4(tmem + TM_ACC, a_desc0 + so + 2 * a, b_desc0 + so + 2 * a, IDESC,
-                          t_sfa + a * 4, t_sfb + a * 8, a == 0 ? first : 1u);
+              tc_mma_nvf4(d_tmem, a_desc0 + so + 2 * a, b_desc0 + so + 2 * a, C::IDESC,
+                          t_sfa + a * 4, t_sfb + a * (BN / 32), a == 0 ? first : 1u);
           } else {
             for (int a = 0; a < natoms; ++a)
-              tc_mma_nvf4(tmem + TM_ACC, a_desc0 + so + 2 * a, b_desc0 + so + 2 * a, IDESC,
-                          t_sfa + a * 4, t_sfb + a * 8, a == 0 ? first : 1u);
+              tc_mma_nvf4(d_tmem, a_desc0 + so + 2 * a, b_desc0 + so + 2 * a, C::IDESC,
+                          t_sfa + a * 4, t_sfb + a * (BN / 32), a == 0 ? first : 1u);
           }
           tc_commit(smem_u32(&bar_empty[s]));
         }
         if (!ok) break;
-        tc_commit(smem_u32(&bar_acc_full));
+        tc_commit(smem_u32(&bar_acc_full[b]));
       }
       // all MMAs issued by this thread complete before the CTA frees tensor memory
       tc_commit(smem_u32(&bar_drain));
@@ -318,10 +333,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           ok = false;
           break;
         }
-        const uint8_t* st = smem + s * STAGE_BYTES;
-        sf_rows128_to_tmem(tmem + lane_base + TM_SFA + s * 16, st + A_BYTES + B_BYTES, lane);
-        sf_rows256_to_tmem(tmem + lane_base + TM_SFB + s * 32, st + A_BYTES + B_BYTES + SFA_BYTES,
-                           lane);
+        const uint8_t* st = smem + s * C::STAGE_BYTES + A_BYTES + C::B_BYTES;
+        sf_rows128_to_tmem(tmem + lane_base + C::TM_SFA + s * 16, st, lane);
+        if (BN == 256)
+          sf_rows256_to_tmem(tmem + lane_base + C::TM_SFB + s * C::SFB_COLS, st + SFA_BYTES, lane);
+        else
+          sf_rows128_to_tmem(tmem + lane_base + C::TM_SFB + s * C::SFB_COLS, st + SFA_BYTES, lane);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
@@ -334,12 +351,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // `half` splits the tile's columns between them.
     const int q = warp & 3;
     const int half = (warp - EPI_WARP0) >> 2;
-    const uint32_t t_row = tmem + TM_ACC + (static_cast<uint32_t>(q * 32) << 16);
     uint32_t tile_it = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x, ++tile_it) {
       const Tile tl = decode_tile(t, tile_start, seg, E, args.n_tiles);
-      if (!mbar_wait_bounded(smem_u32(&bar_acc_full), tile_it & 1u, &abort_flag)) break;
+      const int b = tile_it % ACC_BUFS;
+      if (!mbar_wait_bounded(smem_u32(&bar_acc_full[b]), (tile_it / ACC_BUFS) & 1u, &abort_flag))
+        break;
       tc_fence_after();
+      const uint32_t t_row = tmem + b * BN + (static_cast<uint32_t>(q * 32) << 16);
       const float alpha = 1.0f / (__ldg(args.gs_a) * __ldg(args.gs_b + tl.e));
       const int64_t row = tl.m0 + q * 32 + lane;
       // rows of the row map that are padding produce nothing; skip groups of 32 of them
@@ -402,7 +421,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const int H = args.N;
           float* dst = args.acc + (int64_t)(tok >= 0 ? tok : 0) * H + tl.nt * BN;
 #pragma unroll 1
-          for (int c = 4 * half; c < 4 * half + 4; ++c) {
+          for (int c = (BN / 64) * half; c < (BN / 64) * (half + 1); ++c) {
             uint32_t v[32];
             tmem_ld32(t_row + 32 * c, v);
             tmem_wait_ld();
@@ -419,7 +438,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       } else {
         const int N = args.N;
 #pragma unroll 1
-        for (int c = 4 * half; c < 4 * half + 4; ++c) {
+        for (int c = (BN / 64) * half; c < (BN / 64) * (half + 1); ++c) {
           uint32_t v[32];
           tmem_ld32(t_row + 32 * c, v);
           tmem_wait_ld();
@@ -451,303 +470,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&bar_acc_empty));
-    }
-  }
-
-  __syncwarp();
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  if (warp == 2) tmem_dealloc(tmem, TMEM_COLS);
-  if (tid == 0 && abort_flag) report(args.status, NVFP4_DEVERR_TIMEOUT);
-}
-
-// ------------------------------------------------------------------------------ small batch
-// Swap-AB variant for batches of at most 32 tokens (so every expert has at most 32 rows): the
-// weights are the 128-row M operand and the expert's (at most 32) token rows the N operand, so no
-// tensor-core work and no shared memory goes to padding rows, and a 24 KB stage lets 9 stages
-// (144 KB of weights) stream per SM.  Accumulators are 32 TMEM columns, double buffered, so the
-// epilogue of one tile overlaps the main loop of the next.  A tile covers 128 weight rows of one
-// expert: 64 h features for L1 (16-row gate/up blocks: lane i and lane i+16 of a quadrant hold the
-// gate and up value of one feature), 128 output features for L2.
-constexpr int SB_N = 32;
-constexpr int SB_STAGES = 9;
-constexpr int SB_W_BYTES = 128 * BK_BYTES;
-constexpr int SB_X_BYTES = SB_N * BK_BYTES;
-constexpr int SB_SF_BYTES = 4 * 512;
-constexpr int SB_STAGE_BYTES = SB_W_BYTES + SB_X_BYTES + 2 * SB_SF_BYTES;
-constexpr int SB_SMEM_BYTES = SB_STAGES * SB_STAGE_BYTES + 1024;
-static_assert(SB_STAGE_BYTES % 1024 == 0, "stages must keep 1024-byte alignment (128B swizzle)");
-constexpr uint32_t SB_TM_ACC = 0;                           // 2 x 32 FP32 columns
-constexpr uint32_t SB_TM_SFW = 64;                          // 16 columns per stage
-constexpr uint32_t SB_TM_SFX = SB_TM_SFW + SB_STAGES * 16;  // 16 columns per stage
-static_assert(SB_TM_SFX + SB_STAGES * 16 <= TMEM_COLS, "tensor memory budget");
-constexpr uint32_t SB_IDESC = idesc_nvf4(SB_N);
-constexpr int SB_THREADS = 384;  // 4 role warps + 4 epilogue warps + 4 scale-factor warps
-constexpr int SB_SF_WARP0 = 8;
-
-template <int MODE>
-__global__ void __launch_bounds__(SB_THREADS, 1)
-    grouped_gemm_small_kernel(const __grid_constant__ CUtensorMap tm_x,
-                              const __grid_constant__ CUtensorMap tm_w, const GemmArgs args) {
-  extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t bar_full[SB_STAGES];
-  __shared__ __align__(8) uint64_t bar_empty[SB_STAGES];
-  __shared__ __align__(8) uint64_t bar_sf[SB_STAGES];
-  __shared__ __align__(8) uint64_t bar_acc_full[2];
-  __shared__ __align__(8) uint64_t bar_acc_empty[2];
-  __shared__ __align__(8) uint64_t bar_drain;
-  __shared__ uint32_t tmem_slot;
-  __shared__ int seg[MAX_E + 1];
-  __shared__ int tile_start[MAX_E + 1];
-  __shared__ int warp_sums[SB_THREADS / 32];
-  __shared__ int bad_offsets;
-  __shared__ volatile int abort_flag;
-
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~static_cast<uintptr_t>(1023));
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int E = args.E;
-
-  // ---- scheduler table: every non-empty expert segment is one 128-row block holding at most
-  // 32 tokens; it owns n_tiles weight tiles
-  if (tid == 0) {
-    bad_offsets = 0;
-    abort_flag = 0;
-  }
-  for (int i = tid; i <= E; i += SB_THREADS) seg[i] = __ldg(args.offs + i);
-  __syncthreads();
-  int my_tiles = 0;
-  if (tid < E) {
-    const int lo = seg[tid], hi = seg[tid + 1];
-    if (lo < 0 || hi < lo || (lo & 127) || hi > args.R_max || hi - lo > 128 ||
-        (hi > lo && __ldg(args.row_token + lo + SB_N) >= 0))
-      bad_offsets = 1;
-    else
-      my_tiles = ((hi - lo) >> 7) * args.n_tiles;
-  }
-  int incl = my_tiles;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int v = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += v;
-  }
-  if (lane == 31) warp_sums[warp] = incl;
-  __syncthreads();
-  if (tid == 0) {
-    int run = 0;
-    for (int w = 0; w < SB_THREADS / 32; ++w) {
-      const int c = warp_sums[w];
-      warp_sums[w] = run;
-      run += c;
-    }
-  }
-  __syncthreads();
-  const int excl = warp_sums[warp] + incl - my_tiles;
-  if (tid < E) tile_start[tid] = excl;
-  if (tid == E - 1) tile_start[E] = excl + my_tiles;
-
-  if (tid == 0) {
-    for (int s = 0; s < SB_STAGES; ++s) {
-      mbar_init(smem_u32(&bar_full[s]), 1);
-      mbar_init(smem_u32(&bar_empty[s]), 1);
-      mbar_init(smem_u32(&bar_sf[s]), 4);
-    }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(smem_u32(&bar_acc_full[b]), 1);
-      mbar_init(smem_u32(&bar_acc_empty[b]), 4);
-    }
-    mbar_init(smem_u32(&bar_drain), 1);
-    fence_mbar_init();
-  }
-  if (warp == 2) {
-    tmem_alloc(smem_u32(&tmem_slot), TMEM_COLS);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = tmem_slot;
-  const int total = bad_offsets ? 0 : tile_start[E];
-  if (tid == 0 && bad_offsets && blockIdx.x == 0) report(args.status, NVFP4_DEVERR_BAD_OFFSETS);
-
-  const int K = args.K;
-  const int nk = (K + 255) / 256;
-  const int atoms_k = K / 64;
-
-  if (warp == 0) {
-    // =========================== TMA producer ===========================
-    if (lane == 0) {
-      prefetch_tmap(&tm_x);
-      prefetch_tmap(&tm_w);
-      uint32_t it = 0;
-      bool ok = true;
-      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-        const Tile tl = decode_tile(t, tile_start, seg, E, args.n_tiles);
-        const int w_row = tl.e * args.N + tl.nt * 128;
-        for (int kb = 0; kb < nk; ++kb, ++it) {
-          const int s = it % SB_STAGES;
-          const uint32_t ph = (it / SB_STAGES) & 1u;
-          if (!mbar_wait_bounded(smem_u32(&bar_empty[s]), ph ^ 1u, &abort_flag)) {
-            ok = false;
-            break;
-          }
-          const int natoms = min(4, atoms_k - kb * 4);
-          const uint32_t full = smem_u32(&bar_full[s]);
-          const uint32_t sW = smem_u32(smem + s * SB_STAGE_BYTES), sX = sW + SB_W_BYTES,
-                         sSFW = sX + SB_X_BYTES, sSFX = sSFW + SB_SF_BYTES;
-          mbar_arrive_expect_tx(full, SB_W_BYTES + SB_X_BYTES + natoms * 512 * 2);
-          tma_load_2d(sW, &tm_w, full, kb * BK_BYTES, w_row);
-          tma_load_2d(sX, &tm_x, full, kb * BK_BYTES, tl.m0);
-          const int64_t w_atom = (int64_t)(w_row >> 7) * atoms_k + kb * 4;
-          const int64_t x_atom = (int64_t)(tl.m0 >> 7) * atoms_k + kb * 4;
-          bulk_load(sSFW, args.sfb + w_atom * 512, natoms * 512, full);
-          bulk_load(sSFX, args.sfa + x_atom * 512, natoms * 512, full);
-        }
-      }
-      if (!ok) {
-        volatile int never = 0;
-        const uint32_t first = it > (uint32_t)SB_STAGES ? it - SB_STAGES : 0u;
-        for (uint32_t j = first; j < it; ++j)
-          mbar_wait_bounded(smem_u32(&bar_full[j % SB_STAGES]), (j / SB_STAGES) & 1u, &never,
-                            NVFP4_WAIT_TIMEOUT_NS / 4);
-      }
-    }
-    __syncwarp();
-  } else if (warp == 1) {
-    // =========================== MMA issuer ===========================
-    if (lane == 0) {
-      const uint32_t s0 = smem_u32(smem);
-      const uint64_t w_desc0 = smem_desc(s0, 16, 1024, 2);
-      const uint64_t x_desc0 = smem_desc(s0 + SB_W_BYTES, 16, 1024, 2);
-      uint32_t it = 0, tile_it = 0;
-      bool ok = true;
-      for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++tile_it) {
-        const int b = tile_it & 1;
-        if (!mbar_wait_bounded(smem_u32(&bar_acc_empty[b]), ((tile_it >> 1) & 1u) ^ 1u,
-                               &abort_flag)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t d_tmem = tmem + SB_TM_ACC + b * SB_N;
-        for (int kb = 0; kb < nk; ++kb, ++it) {
-          const int s = it % SB_STAGES;
-          const uint32_t ph = (it / SB_STAGES) & 1u;
-          if (!mbar_wait_bounded(smem_u32(&bar_full[s]), ph, &abort_flag) ||
-              !mbar_wait_bounded(smem_u32(&bar_sf[s]), ph, &abort_flag)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint64_t so = static_cast<uint64_t>(s) * (SB_STAGE_BYTES >> 4);
-          const uint32_t t_sfw = tmem + SB_TM_SFW + s * 16;
-          const uint32_t t_sfx = tmem + SB_TM_SFX + s * 16;
-          const uint32_t first = kb == 0 ? 0u : 1u;
-          const int natoms = min(4, atoms_k - kb * 4);
-          for (int a = 0; a < natoms; ++a)
-            tc_mma_nvf4(d_tmem, w_desc0 + so + 2 * a, x_desc0 + so + 2 * a, SB_IDESC,
-                        t_sfw + a * 4, t_sfx + a * 4, a == 0 ? first : 1u);
-          tc_commit(smem_u32(&bar_empty[s]));
-        }
-        if (!ok) break;
-        tc_commit(smem_u32(&bar_acc_full[b]));
-      }
-      tc_commit(smem_u32(&bar_drain));
-      volatile int never = 0;
-      mbar_wait_bounded(smem_u32(&bar_drain), 0, &never);
-    }
-    __syncwarp();
-  } else if (warp >= SB_SF_WARP0) {
-    // =========================== scale-factor warps ===========================
-    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    uint32_t it = 0;
-    bool ok = true;
-    for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-      for (int kb = 0; kb < nk; ++kb, ++it) {
-        const int s = it % SB_STAGES;
-        const uint32_t ph = (it / SB_STAGES) & 1u;
-        if (!mbar_wait_bounded(smem_u32(&bar_full[s]), ph, &abort_flag)) {
-          ok = false;
-          break;
-        }
-        const uint8_t* st = smem + s * SB_STAGE_BYTES + SB_W_BYTES + SB_X_BYTES;
-        sf_rows128_to_tmem(tmem + lane_base + SB_TM_SFW + s * 16, st, lane);
-        sf_rows128_to_tmem(tmem + lane_base + SB_TM_SFX + s * 16, st + SB_SF_BYTES, lane);
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&bar_sf[s]));
-      }
-    }
-  } else if (warp >= EPI_WARP0) {
-    // =========================== epilogue ===========================
-    // warp q reads weight rows 32q..32q+31 of the tile (its TMEM lane quadrant) for the 32 token
-    // columns; column j is token row m0 + j, and the real rows of a segment come first
-    const int q = warp & 3;
-    uint32_t tile_it = 0;
-    for (int t = blockIdx.x; t < total; t += gridDim.x, ++tile_it) {
-      const int b = tile_it & 1;
-      const Tile tl = decode_tile(t, tile_start, seg, E, args.n_tiles);
-      if (!mbar_wait_bounded(smem_u32(&bar_acc_full[b]), (tile_it >> 1) & 1u, &abort_flag)) break;
-      tc_fence_after();
-      uint32_t v[32];
-      tmem_ld32(tmem + SB_TM_ACC + b * SB_N + (static_cast<uint32_t>(q * 32) << 16), v);
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&bar_acc_empty[b]));
-
-      const float alpha = 1.0f / (__ldg(args.gs_a) * __ldg(args.gs_b + tl.e));
-      const int my_tok = __ldg(args.row_token + tl.m0 + lane);
-      const int count = __popc(__ballot_sync(0xffffffffu, my_tok >= 0));
-      if (MODE == L2_SCATTER) {
-        const float my_w = __ldg(args.row_w + tl.m0 + lane);
-        const int H = args.N;
-        const int n = tl.nt * 128 + q * 32 + lane;  // output feature of this thread
-#pragma unroll
-        for (int j = 0; j < SB_N; ++j) {  // unrolled so v[j] stays in registers
-          if (j < count) {
-            const int tok = __shfl_sync(0xffffffffu, my_tok, j);
-            const float w = __shfl_sync(0xffffffffu, my_w, j);
-            if (tok < args.T) {
-              atomicAdd(args.acc + (int64_t)tok * H + n, __uint_as_float(v[j]) * (alpha * w));
-            } else if (lane == 0) {
-              report(args.status, NVFP4_DEVERR_BAD_INDEX);
-            }
-          }
-        }
-      } else {
-        // lanes 0..15: gate rows of h features f0..f0+15, lanes 16..31: the matching up rows
-        const float gs_h = __ldg(args.gs_h);
-        const int I = args.I;
-        const int f0 = tl.nt * 64 + q * 16;
-#pragma unroll
-        for (int j = 0; j < SB_N; ++j) {  // unrolled so v[j] stays in registers
-          if (j >= count) break;
-          const float x = __uint_as_float(v[j]) * alpha;
-          const float other = __shfl_xor_sync(0xffffffffu, x, 16);
-          const float h = lane < 16 ? __fdividef(x * other, 1.0f + __expf(-x)) : 0.0f;
-          float amax = fabsf(h);
-#pragma unroll
-          for (int o = 8; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-          float rcp;
-          const uint32_t sb = nvfp4_block_scale(amax, gs_h, rcp);
-          const uint32_t code = rcp == 0.0f ? 0u : (cvt_e2m1x2(scaled(h, rcp), 0.0f) & 0xFu);
-          // pack: byte of features (2i, 2i+1) in lane 2i, then bytes 0..7 into lanes 0 and 4
-          const uint32_t byte = code | (__shfl_down_sync(0xffffffffu, code, 1) << 4);
-          const uint32_t bb = __shfl_sync(0xffffffffu, byte, (2 * lane) & 31);
-          const uint32_t w2 = bb | (__shfl_down_sync(0xffffffffu, bb, 1) << 8);
-          const uint32_t w4 = w2 | (__shfl_down_sync(0xffffffffu, w2, 2) << 16);
-          const uint32_t hi = __shfl_sync(0xffffffffu, w4, 4);
-          if (lane == 0) {
-            const int64_t row = tl.m0 + j;
-            *reinterpret_cast<uint2*>(args.h + row * (I / 2) + f0 / 2) = make_uint2(w4, hi);
-            args.sfh[sf_offset(row, f0 / 16, I / 16)] = static_cast<uint8_t>(sb);
-          }
-        }
-      }
     }
   }
 
@@ -805,32 +528,12 @@ nvfp4_status_t launch(const uint8_t* a, const uint8_t* b, int64_t b_rows, GemmAr
     set_last_error("cuTensorMapEncodeTiled failed");
     return NVFP4_ERR_CUDA;
   }
-  static bool attr_set = false;  // per instantiation; idempotent, so a race is harmless
-  if (!attr_set) {
-    if (cudaFuncSetAttribute(grouped_gemm_kernel<MODE>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             SMEM_BYTES) != cudaSuccess)
-      return check_launch("cudaFuncSetAttribute");
-    attr_set = true;
-  }
-  grouped_gemm_kernel<MODE><<<num_sms(), NUM_THREADS, SMEM_BYTES, s>>>(ma, mb, args);
-  return check_launch("grouped_gemm_kernel");
-}
-
-template <int MODE>
-nvfp4_status_t launch_small(const uint8_t* x, const uint8_t* w, int64_t w_rows, GemmArgs args,
-                            cudaStream_t s) {
-  CUtensorMap mx, mw;
-  if (!make_map(&mx, x, args.K / 2, args.R_max, SB_N) || !make_map(&mw, w, args.K / 2, w_rows)) {
-    set_last_error("cuTensorMapEncodeTiled failed");
-    return NVFP4_ERR_CUDA;
-  }
-  if (cudaFuncSetAttribute(grouped_gemm_small_kernel<MODE>,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize, SB_SMEM_BYTES) !=
-      cudaSuccess)
+  constexpr int smem = TileCfg<MODE>::SMEM_BYTES;
+  if (cudaFuncSetAttribute(grouped_gemm_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           smem) != cudaSuccess)
     return check_launch("cudaFuncSetAttribute");
-  grouped_gemm_small_kernel<MODE><<<num_sms(), SB_THREADS, SB_SMEM_BYTES, s>>>(mx, mw, args);
-  return check_launch("grouped_gemm_small_kernel");
+  grouped_gemm_kernel<MODE><<<num_sms(), NUM_THREADS, smem, s>>>(ma, mb, args);
+  return check_launch("grouped_gemm_kernel");
 }
 
 __global__ void cast_bf16_kernel(const float* __restrict__ acc, __nv_bfloat16* __restrict__ out,
@@ -860,25 +563,21 @@ nvfp4_status_t gemm_plain(const uint8_t* a, const uint8_t* sfa, const float* gs_
                           cudaStream_t s) {
   GemmArgs g{};
   g.sfa = sfa; g.sfb = sfb; g.gs_a = gs_a; g.gs_b = gs_b; g.offs = offs;
-  g.E = E; g.N = N; g.K = K; g.n_tiles = N / BN; g.R_max = R_max; g.out = out; g.status = status;
+  g.E = E; g.N = N; g.K = K; g.n_tiles = N / TileCfg<PLAIN_F32>::BN; g.R_max = R_max; g.out = out;
+  g.status = status;
   const int64_t b_rows = (int64_t)E * N;
   return out_dtype == 0 ? launch<PLAIN_F32>(a, b, b_rows, g, s) : launch<PLAIN_BF16>(a, b, b_rows, g, s);
 }
 
 nvfp4_status_t gemm_l1(const uint8_t* a, const uint8_t* sfa, const float* gs_a, const uint8_t* w1,
                        const uint8_t* sfw1, const float* gs_w1, const int32_t* offs,
-                       const int32_t* row_token, int T, int E, int H, int I, int64_t R_max,
+                       const int32_t* row_token, int E, int H, int I, int64_t R_max,
                        const float* gs_h, uint8_t* h, uint8_t* sfh, int32_t* status,
                        cudaStream_t s) {
   GemmArgs g{};
   g.sfa = sfa; g.sfb = sfw1; g.gs_a = gs_a; g.gs_b = gs_w1; g.offs = offs;
-  g.E = E; g.N = 2 * I; g.K = H; g.R_max = R_max;
+  g.E = E; g.N = 2 * I; g.K = H; g.n_tiles = I / 128; g.R_max = R_max;
   g.gs_h = gs_h; g.h = h; g.sfh = sfh; g.I = I; g.row_token = row_token; g.status = status;
-  if (row_token != nullptr && T > 0 && T <= SB_N) {
-    g.n_tiles = 2 * I / 128;  // 128 weight rows (64 h features) per tile
-    return launch_small<L1_SWIGLU>(a, w1, (int64_t)E * 2 * I, g, s);
-  }
-  g.n_tiles = I / 128;
   return launch<L1_SWIGLU>(a, w1, (int64_t)E * 2 * I, g, s);
 }
 
@@ -894,14 +593,8 @@ nvfp4_status_t gemm_l2(const uint8_t* h, const uint8_t* sfh, const float* gs_h, 
   g.sfa = sfh; g.sfb = sfw2; g.gs_a = gs_h; g.gs_b = gs_w2; g.offs = offs;
   g.E = E; g.N = H; g.K = I; g.R_max = R_max;
   g.row_token = row_token; g.row_w = row_w; g.acc = acc; g.T = T; g.status = status;
-  nvfp4_status_t st;
-  if (T <= SB_N) {
-    g.n_tiles = H / 128;  // 128 output features per tile
-    st = launch_small<L2_SCATTER>(h, w2, (int64_t)E * H, g, s);
-  } else {
-    g.n_tiles = H / BN;
-    st = launch<L2_SCATTER>(h, w2, (int64_t)E * H, g, s);
-  }
+  g.n_tiles = H / TileCfg<L2_SCATTER>::BN;
+  nvfp4_status_t st = launch<L2_SCATTER>(h, w2, (int64_t)E * H, g, s);
   if (st != NVFP4_OK || out_bf16 == nullptr) return st;
   const int64_t n8 = (int64_t)T * H / 8;
   const int64_t want = (n8 + 255) / 256;
@@ -921,7 +614,7 @@ extern "C" nvfp4_status_t nvfp4_grouped_gemm(const uint8_t* a, const uint8_t* sf
                                              int64_t R_max, void* out, int out_dtype,
                                              int32_t* dev_status, nvfp4_stream_t stream) {
   if (E < 1 || E > MAX_E || N <= 0 || K <= 0 || R_max < 0) return NVFP4_ERR_INVALID_ARG;
-  if (K % 64 || N % BN || R_max % 128) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (K % 64 || N % TileCfg<PLAIN_F32>::BN || R_max % 128) return NVFP4_ERR_UNSUPPORTED_SHAPE;
   if (out_dtype != 0 && out_dtype != 1) return NVFP4_ERR_INVALID_ARG;
   if (!gs_a || !gs_b || !offs) return NVFP4_ERR_INVALID_ARG;
   if (R_max == 0) return NVFP4_OK;
@@ -933,17 +626,17 @@ extern "C" nvfp4_status_t nvfp4_grouped_gemm(const uint8_t* a, const uint8_t* sf
 
 extern "C" nvfp4_status_t moe_grouped_gemm_l1_swiglu_q(
     const uint8_t* a, const uint8_t* sfa, const float* gs_a, const uint8_t* w1,
-    const uint8_t* sfw1, const float* gs_w1, const int32_t* offs, const int32_t* row_token, int T,
-    int E, int H, int I, int64_t R_max, const float* gs_h, uint8_t* h, uint8_t* sfh,
-    int32_t* dev_status, nvfp4_stream_t stream) {
-  if (E < 1 || E > MAX_E || H <= 0 || I <= 0 || R_max < 0 || T < 0) return NVFP4_ERR_INVALID_ARG;
+    const uint8_t* sfw1, const float* gs_w1, const int32_t* offs, const int32_t* row_token, int E,
+    int H, int I, int64_t R_max, const float* gs_h, uint8_t* h, uint8_t* sfh, int32_t* dev_status,
+    nvfp4_stream_t stream) {
+  if (E < 1 || E > MAX_E || H <= 0 || I <= 0 || R_max < 0) return NVFP4_ERR_INVALID_ARG;
   if (H % 64 || I % 128 || R_max % 128) return NVFP4_ERR_UNSUPPORTED_SHAPE;
   if (!gs_a || !gs_w1 || !offs || !gs_h) return NVFP4_ERR_INVALID_ARG;
   if (R_max == 0) return NVFP4_OK;
   if (!ok_ptr(a) || !ok_ptr(sfa) || !ok_ptr(w1) || !ok_ptr(sfw1) || !ok_ptr(h) || !ok_ptr(sfh))
     return (a && sfa && w1 && sfw1 && h && sfh) ? NVFP4_ERR_MISALIGNED : NVFP4_ERR_INVALID_ARG;
   if (reinterpret_cast<uintptr_t>(row_token) & 3u) return NVFP4_ERR_MISALIGNED;
-  return gemm_l1(a, sfa, gs_a, w1, sfw1, gs_w1, offs, row_token, T, E, H, I, R_max, gs_h, h, sfh,
+  return gemm_l1(a, sfa, gs_a, w1, sfw1, gs_w1, offs, row_token, E, H, I, R_max, gs_h, h, sfh,
                  dev_status, reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -953,7 +646,7 @@ extern "C" nvfp4_status_t moe_grouped_gemm_l2_scatter(
     const float* row_w, int E, int H, int I, int T, int64_t R_max, float* acc_ws, void* out_bf16,
     int32_t* dev_status, nvfp4_stream_t stream) {
   if (E < 1 || E > MAX_E || H <= 0 || I <= 0 || T < 0 || R_max < 0) return NVFP4_ERR_INVALID_ARG;
-  if (H % BN || I % 64 || R_max % 128) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (H % TileCfg<L2_SCATTER>::BN || I % 64 || R_max % 128) return NVFP4_ERR_UNSUPPORTED_SHAPE;
   if (!gs_h || !gs_w2 || !offs || !row_token || !row_w) return NVFP4_ERR_INVALID_ARG;
   if (T == 0 || R_max == 0) return NVFP4_OK;
   if (!ok_ptr(h) || !ok_ptr(sfh) || !ok_ptr(w2) || !ok_ptr(sfw2) || !ok_ptr(acc_ws) ||
@@ -1000,7 +693,7 @@ extern "C" nvfp4_status_t moe_grouped_gemm_l2_scatter_noalloc(
     const float* row_w, int E, int H, int I, int T, int64_t R_max, void* out_bf16,
     int32_t* dev_status, nvfp4_stream_t stream) {
   if (E < 1 || E > MAX_E || H <= 0 || I <= 0 || T < 0 || R_max < 0) return NVFP4_ERR_INVALID_ARG;
-  if (H % BN || I % 64 || R_max % 128) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (H % TileCfg<L2_SCATTER>::BN || I % 64 || R_max % 128) return NVFP4_ERR_UNSUPPORTED_SHAPE;
   if (!gs_h || !gs_w2 || !offs || !row_token || !row_w || !out_bf16) return NVFP4_ERR_INVALID_ARG;
   if ((int64_t)T * H > NVFP4_L2_NOALLOC_MAX_ELEMS) {
     set_last_error("moe_grouped_gemm_l2_scatter_noalloc: T*H exceeds the static FP32 scratch "

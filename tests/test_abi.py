@@ -96,7 +96,7 @@ def test_gemms_reject_bad_shapes(L):
     assert L.nvfp4_grouped_gemm(f, f, f, f, f, f, f, 2, 256, 96, 128, f, 0, None, None) == 2
     assert L.nvfp4_grouped_gemm(f, f, f, f, f, f, f, 2, 256, 64, 100, f, 0, None, None) == 2
     assert L.nvfp4_grouped_gemm(f, f, f, f, f, f, f, 2, 256, 64, 128, f, 7, None, None) == 1
-    assert L.moe_grouped_gemm_l1_swiglu_q(f, f, f, f, f, f, f, None, 0, 8, 256, 96, 128, f, f, f,
+    assert L.moe_grouped_gemm_l1_swiglu_q(f, f, f, f, f, f, f, None, 8, 256, 96, 128, f, f, f,
                                           None, None) == 2  # I % 128
     assert L.moe_grouped_gemm_l2_scatter(f, f, f, f, f, f, f, f, f, 8, 200, 128, 4, 128, f, f,
                                          None, None) == 2  # H % 256

@@ -102,7 +102,7 @@ def test_ffn_rejects_small_workspace():
 
 @pytest.mark.parametrize("T", [16, 32, 3])
 def test_ffn_small_batch_end_to_end(T):
-    """T <= 32 runs the small-batch GEMM kernels inside moe_ffn_forward."""
+    """Decode-sized batches: a few tokens per expert, most rows of every M-tile padding."""
     from dataclasses import replace
     cfg = replace(CONFIGS["tiny"], T=T)
     got, ref = _ffn_check(cfg, gen_x(cfg), gen_logits(cfg))
