@@ -166,11 +166,11 @@ class Plan:
         e = lambda n, t: torch.empty(max(int(n), 1), dtype=t, device=dev)  # noqa: E731
         self.ids, self.w = e(T * k, i32), e(T * k, f32)
         self.offs, self.dst = e(E + 1, i32), e(T * k, i32)
-        self.row_token, self.row_w = e(self.R, i32), e(self.R, f32)
+        self.row_slot, self.row_w = e(self.R, i32), e(self.R, f32)
         self.xq, self.xsf = e(self.R * H // 2, u8), e(self.R * H // 16, u8)
         self.gs_x, self.qws = e(1, f32), e(256, u8)
         self.hq, self.hsf = e(self.R * I // 2, u8), e(self.R * I // 16, u8)
-        self.acc = e(T * H, f32)
+        self.ys = e(T * k * H, f32)
         self.out = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
         self.status = torch.zeros(1, dtype=i32, device=dev)
 
@@ -184,7 +184,7 @@ class Plan:
         if ev:
             ev[0].record()
         call("moe_permute", p(self.logits), T, E, k, 1, p(self.ids), p(self.w), p(self.offs),
-             p(self.dst), p(self.row_token), p(self.row_w), None, 0, p(self.status), s)
+             p(self.dst), p(self.row_slot), p(self.row_w), None, 0, p(self.status), s)
         if ev:
             ev[1].record()
         call("nvfp4_quantize", p(self.x), T, H, H, p(self.dst), k, self.R, p(self.xq), p(self.xsf),
@@ -192,19 +192,20 @@ class Plan:
         if ev:
             ev[2].record()
         call("moe_grouped_gemm_l1_swiglu_q", p(self.xq), p(self.xsf), p(self.gs_x),
-             p(self.w1.codes), p(self.w1.sf), p(self.w1.gs), p(self.offs), p(self.row_token),
+             p(self.w1.codes), p(self.w1.sf), p(self.w1.gs), p(self.offs), p(self.row_slot),
              E, H, I, self.R,
              p(self.gs_h), p(self.hq), p(self.hsf), p(self.status), s)
         if ev:
             ev[3].record()
         call("moe_grouped_gemm_l2_scatter", p(self.hq), p(self.hsf), p(self.gs_h),
-             p(self.w2.codes), p(self.w2.sf), p(self.w2.gs), p(self.offs), p(self.row_token),
-             p(self.row_w), E, H, I, T, self.R, p(self.acc), p(self.out), p(self.status), s)
+             p(self.w2.codes), p(self.w2.sf), p(self.w2.gs), p(self.offs), p(self.row_slot),
+             p(self.row_w), p(self.dst), E, H, I, T, k, self.R, p(self.ys), None, p(self.out),
+             p(self.status), s)
         if ev:
             ev[4].record()
 
 
-KERNELS_PER_STEP = 7  # topk, permute, amax, quantize, L1 GEMM, L2 GEMM, bf16 cast
+KERNELS_PER_STEP = 7  # topk, permute, amax, quantize, L1 GEMM, L2 GEMM, combine
 
 
 def make_config(args):

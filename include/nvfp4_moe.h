@@ -111,7 +111,8 @@ NVFP4_API nvfp4_status_t nvfp4_quantize(const void* x, int64_t rows, int64_t col
  *   topk_ids  int32 [T][k] (output when logits != NULL); topk_w float [T][k] likewise
  *   offs      int32 [E+1]: start row of each expert's segment, offs[E] = rows used
  *   dst_row   int32 [T*k]: row of slot (t, j), -1 when dropped
- *   row_token int32 [R_max]: token of each row, -1 for padding and unused rows
+ *   row_slot  int32 [R_max]: slot t*k + j of each row (its token is row_slot / k), -1 for padding
+ *             and unused rows
  *   row_w     float [R_max]: routing weight of each row, 0 for padding and unused rows
  *   R_max     = moe_rows_max(T, E, k)
  *   Constraints: 1 <= k <= E <= 256, k <= 32, T >= 0.
@@ -120,7 +121,7 @@ NVFP4_API int64_t moe_rows_max(int T, int E, int k);
 NVFP4_API size_t moe_permute_workspace_size(int T, int E, int k);
 NVFP4_API nvfp4_status_t moe_permute(const float* logits, int T, int E, int k, int renormalize,
                            int32_t* topk_ids, float* topk_w, int32_t* offs, int32_t* dst_row,
-                           int32_t* row_token, float* row_w, void* ws, size_t ws_bytes,
+                           int32_t* row_slot, float* row_w, void* ws, size_t ws_bytes,
                            int32_t* dev_status, nvfp4_stream_t stream);
 
 /* ---------------------------------------------------------------------------------------------
@@ -158,8 +159,8 @@ NVFP4_API nvfp4_status_t nvfp4_grouped_gemm(const uint8_t* a, const uint8_t* sfa
  *   a, sfa, gs_a    activations NVFP4 [R_max][H]
  *   w1, sfw1, gs_w1 NVFP4 [E*2I][H], gs_w1 float[E]
  *   offs            int32 [E+1] (from moe_permute)
- *   row_token       optional int32 [R_max] (from moe_permute).  NULL: every row of every segment
- *                   is written.  Given: groups of 32 rows that are all padding (row_token < 0)
+ *   row_slot        optional int32 [R_max] (from moe_permute).  NULL: every row of every segment
+ *                   is written.  Given: groups of 32 rows that are all padding (row_slot < 0)
  *                   are skipped and their h rows left unwritten.
  *   gs_h            device float[1]
  *   h, sfh          output NVFP4 [R_max][I] (tiled scales)
@@ -168,7 +169,7 @@ NVFP4_API nvfp4_status_t nvfp4_grouped_gemm(const uint8_t* a, const uint8_t* sfa
 NVFP4_API nvfp4_status_t moe_grouped_gemm_l1_swiglu_q(const uint8_t* a, const uint8_t* sfa, const float* gs_a,
                                             const uint8_t* w1, const uint8_t* sfw1,
                                             const float* gs_w1, const int32_t* offs,
-                                            const int32_t* row_token, int E, int H, int I,
+                                            const int32_t* row_slot, int E, int H, int I,
                                             int64_t R_max, const float* gs_h, uint8_t* h,
                                             uint8_t* sfh, int32_t* dev_status,
                                             nvfp4_stream_t stream);
@@ -182,25 +183,28 @@ NVFP4_API nvfp4_status_t moe_grouped_gemm_l1_swiglu_q(const uint8_t* a, const ui
 NVFP4_API nvfp4_status_t moe_w1_row_map(int I, int32_t* map);
 
 /* ---------------------------------------------------------------------------------------------
- * moe_grouped_gemm_l2_scatter — L2 grouped GEMM with the routing weight and the scatter-add in
- * its epilogue ("NVFP4 MegaMoE Kernel Rewrite — CuTeDSL", section "Our Adaptation": "Scatter
- * with routing weights"; section "Phase 3").
+ * moe_grouped_gemm_l2_scatter — L2 grouped GEMM with the routing weight and the scatter to token
+ * order in its epilogue ("NVFP4 MegaMoE Kernel Rewrite — CuTeDSL", section "Our Adaptation":
+ * "Scatter with routing weights"; section "Phase 3").
  *
- *   acc_ws[t][n] = sum over rows r of token t of  row_w[r] * (h_r . W2_e[n]) / (gs_h*gs_w2[e]),
- *   computed with FP32 reductions into acc_ws (zeroed by this call), then out = bf16_rn(acc_ws)
- *   when out_bf16 != NULL.  Padding rows (row_token < 0) contribute nothing.
+ *   ys[s] = row_w[r] * (h_r . W2_e^T) / (gs_h*gs_w2[e]) for the row r of slot s (FP32), then
+ *   out[t] = sum over j < k of ys[t*k + j], skipping dropped slots (dst_row < 0), added in j order
+ *   in FP32 (bitwise reproducible); written as FP32 (out_f32) and/or bf16 (out_bf16, RN).
+ *   Tokens whose slots are all dropped get exact zeros.
  *
  *   h, sfh, gs_h     NVFP4 [R_max][I]
  *   w2, sfw2, gs_w2  NVFP4 [E*H][I], gs_w2 float[E]
- *   offs, row_token, row_w  from moe_permute
- *   acc_ws           float [T][H] scratch/output;  out_bf16  bf16 [T][H] or NULL
- *   Constraints: H % 128 == 0, I % 64 == 0, R_max % 128 == 0, 1 <= E <= 256, T >= 0.
+ *   offs, row_slot, row_w, dst_row  from moe_permute
+ *   ys_ws            float [T*k][H] scratch (the weighted expert output of every slot)
+ *   out_f32          float [T][H] or NULL;  out_bf16  bf16 [T][H] or NULL (not both NULL)
+ *   Constraints: H % 256 == 0, I % 64 == 0, R_max % 128 == 0, 1 <= E <= 256, T >= 0, k >= 1.
  * ------------------------------------------------------------------------------------------- */
 NVFP4_API nvfp4_status_t moe_grouped_gemm_l2_scatter(const uint8_t* h, const uint8_t* sfh, const float* gs_h,
                                            const uint8_t* w2, const uint8_t* sfw2,
                                            const float* gs_w2, const int32_t* offs,
-                                           const int32_t* row_token, const float* row_w, int E,
-                                           int H, int I, int T, int64_t R_max, float* acc_ws,
+                                           const int32_t* row_slot, const float* row_w,
+                                           const int32_t* dst_row, int E, int H, int I, int T,
+                                           int k, int64_t R_max, float* ys_ws, float* out_f32,
                                            void* out_bf16, int32_t* dev_status,
                                            nvfp4_stream_t stream);
 
@@ -211,28 +215,29 @@ NVFP4_API nvfp4_status_t moe_grouped_gemm_l2_scatter(const uint8_t* h, const uin
  * (weights, KV cache, a fixed activation pool) and forbid later cudaMalloc, or foreign-language
  * callers that are handed input and output buffers but have no device allocator of their own.
  *
- *   Same arguments and result as moe_grouped_gemm_l2_scatter, minus acc_ws; out_bf16 is required.
- *   The FP32 accumulator lives in a static device array inside this library of
+ *   Same arguments and result as moe_grouped_gemm_l2_scatter, minus ys_ws and out_f32; out_bf16
+ *   is required.  The FP32 per-slot buffer lives in a static device array inside this library of
  *   NVFP4_L2_NOALLOC_MAX_ELEMS floats (4 MiB), which every GPU that loads the library holds until
- *   the process exits.  T*H beyond that returns NVFP4_ERR_WORKSPACE_TOO_SMALL (nothing launched;
+ *   the process exits.  T*k*H beyond that returns NVFP4_ERR_WORKSPACE_TOO_SMALL (nothing launched;
  *   nvfp4_last_error() says why).
  *   The array's device address is looked up once per device (cudaGetSymbolAddress) by the first
  *   call made with that device current; make that first call before any stream capture.
  *   No cudaMalloc / cudaFree or allocating library routine is called.  All calls share the one
- *   array: each call zeroes it on its stream before use, and calls that overlap on the GPU (other
+ *   array and every call rewrites the rows it reads back; calls that overlap on the GPU (other
  *   streams, other threads) race on it.
  * ------------------------------------------------------------------------------------------- */
 #define NVFP4_L2_NOALLOC_MAX_ELEMS (1 << 20)
 NVFP4_API nvfp4_status_t moe_grouped_gemm_l2_scatter_noalloc(
     const uint8_t* h, const uint8_t* sfh, const float* gs_h, const uint8_t* w2,
-    const uint8_t* sfw2, const float* gs_w2, const int32_t* offs, const int32_t* row_token,
-    const float* row_w, int E, int H, int I, int T, int64_t R_max, void* out_bf16,
-    int32_t* dev_status, nvfp4_stream_t stream);
+    const uint8_t* sfw2, const float* gs_w2, const int32_t* offs, const int32_t* row_slot,
+    const float* row_w, const int32_t* dst_row, int E, int H, int I, int T, int k, int64_t R_max,
+    void* out_bf16, int32_t* dev_status, nvfp4_stream_t stream);
 
 /* ---------------------------------------------------------------------------------------------
  * moe_ffn_forward — the whole expert FFN in one stream-ordered call:
  *   moe_permute -> nvfp4_quantize (amax -> gs on the GPU, permuted write) ->
- *   moe_grouped_gemm_l1_swiglu_q -> moe_grouped_gemm_l2_scatter -> bf16 out.
+ *   moe_grouped_gemm_l1_swiglu_q -> moe_grouped_gemm_l2_scatter (per-slot rows + combine) ->
+ *   bf16 out.
  *
  *   x_bf16   bf16 [T][H];  logits float [T][E] (softmax top-k routing, renormalized)
  *   w1.. / w2..  expert weights as above; gs_h device float[1] (static intermediate scale)

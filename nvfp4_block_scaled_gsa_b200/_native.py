@@ -35,11 +35,12 @@ SIGNATURES = {
                                              c_void, c_void, c_int, c_int, c_int, c_i64, c_void,
                                              c_void, c_void, c_void, c_void]),
     "moe_grouped_gemm_l2_scatter": (c_int, [c_void, c_void, c_void, c_void, c_void, c_void, c_void,
-                                            c_void, c_void, c_int, c_int, c_int, c_int, c_i64,
-                                            c_void, c_void, c_void, c_void]),
+                                            c_void, c_void, c_void, c_int, c_int, c_int, c_int,
+                                            c_int, c_i64, c_void, c_void, c_void, c_void, c_void]),
     "moe_grouped_gemm_l2_scatter_noalloc": (c_int, [c_void, c_void, c_void, c_void, c_void,
-                                                    c_void, c_void, c_void, c_void, c_int, c_int,
-                                                    c_int, c_int, c_i64, c_void, c_void, c_void]),
+                                                    c_void, c_void, c_void, c_void, c_void, c_int,
+                                                    c_int, c_int, c_int, c_int, c_i64, c_void,
+                                                    c_void, c_void]),
     "moe_w1_row_map": (c_int, [c_int, c_void]),
     "moe_ffn_workspace_size": (c_size, [c_int, c_int, c_int, c_int, c_int]),
     "moe_ffn_forward": (c_int, [c_void, c_void, c_int, c_int, c_int, c_int, c_int, c_void, c_void,

@@ -110,11 +110,11 @@ def permute(logits, k, renormalize=True, ids=None, weights=None, E=None, status=
     R = rows_max(T, E, k)
     offs = torch.empty(E + 1, dtype=I32, device=dev)
     dst_row = torch.empty(T * k, dtype=I32, device=dev)
-    row_token = torch.empty(max(R, 1), dtype=I32, device=dev)
+    row_slot = torch.empty(max(R, 1), dtype=I32, device=dev)
     row_w = torch.empty(max(R, 1), dtype=F32, device=dev)
     call("moe_permute", _p(logits), T, E, k, int(renormalize), _p(ids), _p(weights), _p(offs),
-         _p(dst_row), _p(row_token), _p(row_w), None, 0, _p(status), _stream())
-    return dict(ids=ids, weights=weights, offs=offs, dst_row=dst_row, row_token=row_token,
+         _p(dst_row), _p(row_slot), _p(row_w), None, 0, _p(status), _stream())
+    return dict(ids=ids, weights=weights, offs=offs, dst_row=dst_row, row_slot=row_slot,
                 row_w=row_w, R_max=R, E=E, T=T, k=k)
 
 
@@ -127,31 +127,31 @@ def grouped_gemm(a_codes, a_sf, gs_a, w: NVFP4Weights, offs, out_dtype=F32, stat
     return out
 
 
-def l1_swiglu_q(a_codes, a_sf, gs_a, w1: NVFP4Weights, offs, gs_h, row_token=None, status=None):
+def l1_swiglu_q(a_codes, a_sf, gs_a, w1: NVFP4Weights, offs, gs_h, row_slot=None, status=None):
     """L1 GEMM + SwiGLU + NVFP4 re-quantization -> (h codes (R, I/2), h tiled scales).
-    With row_token, all-padding groups of 32 rows are skipped (left unwritten)."""
+    With row_slot, all-padding groups of 32 rows are skipped (left unwritten)."""
     R = a_codes.shape[0]
     I = w1.N // 2
     h = torch.empty(R, I // 2, dtype=U8, device=a_codes.device)
     sfh = torch.empty(sf_bytes(R, I), dtype=U8, device=a_codes.device)
     call("moe_grouped_gemm_l1_swiglu_q", _p(a_codes), _p(a_sf), _p(gs_a), _p(w1.codes),
-         _p(w1.sf), _p(w1.gs), _p(offs), _p(row_token), w1.E, w1.K, I, R, _p(gs_h), _p(h),
+         _p(w1.sf), _p(w1.gs), _p(offs), _p(row_slot), w1.E, w1.K, I, R, _p(gs_h), _p(h),
          _p(sfh), _p(status), _stream())
     return h, sfh
 
 
-def l2_scatter(h, sfh, gs_h, w2: NVFP4Weights, offs, row_token, row_w, T, out_bf16=True,
-               status=None):
-    """L2 GEMM + routing weight + scatter-add -> (acc fp32 (T, H), out bf16 (T, H) or None)."""
+def l2_scatter(h, sfh, gs_h, w2: NVFP4Weights, offs, row_slot, row_w, dst_row, T, k, status=None):
+    """L2 GEMM + routing weight + scatter to token order -> (out fp32 (T, H), out bf16 (T, H))."""
     R = h.shape[0]
     H = w2.N
     I = w2.K
-    acc = torch.empty(T, H, dtype=F32, device=h.device)
-    out = torch.empty(T, H, dtype=BF16, device=h.device) if out_bf16 else None
+    ys = torch.empty(max(T * k, 1), H, dtype=F32, device=h.device)
+    out32 = torch.empty(T, H, dtype=F32, device=h.device)
+    out16 = torch.empty(T, H, dtype=BF16, device=h.device)
     call("moe_grouped_gemm_l2_scatter", _p(h), _p(sfh), _p(gs_h), _p(w2.codes), _p(w2.sf),
-         _p(w2.gs), _p(offs), _p(row_token), _p(row_w), w2.E, H, I, T, R, _p(acc), _p(out),
-         _p(status), _stream())
-    return acc, out
+         _p(w2.gs), _p(offs), _p(row_slot), _p(row_w), _p(dst_row), w2.E, H, I, T, k, R, _p(ys),
+         _p(out32), _p(out16), _p(status), _stream())
+    return out32, out16
 
 
 def ffn_workspace_bytes(T, H, I, E, k):

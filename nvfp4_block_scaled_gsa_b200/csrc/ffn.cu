@@ -4,7 +4,7 @@
 // Pipeline ("NVFP4 MegaMoE Kernel Rewrite — CuTeDSL", section "Phase 3: Full MoE pipeline";
 // "May 24, 2026 — Session Start Plan", section 5 "NVFP4-1.1"):
 //   topk + permute  ->  amax -> quantize (permuted write)  ->  L1 GEMM + SwiGLU + FP4 pack
-//   ->  L2 GEMM + routing weight + scatter-add  ->  bf16 cast
+//   ->  L2 GEMM + routing weight, per-slot rows  ->  combine (k-sum per token) + bf16
 // No host synchronization anywhere; every intermediate lives in the caller's workspace.
 #include <cstdio>
 
@@ -31,22 +31,22 @@ nvfp4_status_t quantize_launch(const void* x, int64_t rows, int64_t cols, int64_
                                int32_t* dev_status, cudaStream_t s);
 nvfp4_status_t permute_launch(const float* logits, int T, int E, int k, int renorm,
                               int32_t* topk_ids, float* topk_w, int32_t* offs, int32_t* dst_row,
-                              int32_t* row_token, float* row_w, int64_t R_max,
+                              int32_t* row_slot, float* row_w, int64_t R_max,
                               int32_t* dev_status, cudaStream_t s);
 nvfp4_status_t gemm_l1(const uint8_t* a, const uint8_t* sfa, const float* gs_a, const uint8_t* w1,
                        const uint8_t* sfw1, const float* gs_w1, const int32_t* offs,
-                       const int32_t* row_token, int E, int H, int I, int64_t R_max,
+                       const int32_t* row_slot, int E, int H, int I, int64_t R_max,
                        const float* gs_h, uint8_t* h, uint8_t* sfh, int32_t* status,
                        cudaStream_t s);
 nvfp4_status_t gemm_l2(const uint8_t* h, const uint8_t* sfh, const float* gs_h, const uint8_t* w2,
                        const uint8_t* sfw2, const float* gs_w2, const int32_t* offs,
-                       const int32_t* row_token, const float* row_w, int E, int H, int I, int T,
-                       int64_t R_max, float* acc, void* out_bf16, int32_t* status,
-                       cudaStream_t s);
+                       const int32_t* row_slot, const float* row_w, const int32_t* dst_row, int E,
+                       int H, int I, int T, int k, int64_t R_max, float* ys, float* out_f32,
+                       void* out_bf16, int32_t* status, cudaStream_t s);
 
 // Byte offsets of the moe_ffn_forward workspace regions (each 256-byte aligned).
 struct FfnLayout {
-  int64_t amax, gs_x, ids, w, offs, dst_row, row_token, row_w, xq, xsf, hq, hsf, acc, total;
+  int64_t amax, gs_x, ids, w, offs, dst_row, row_slot, row_w, xq, xsf, hq, hsf, ys, total;
   int64_t R_max;
 };
 
@@ -66,13 +66,13 @@ FfnLayout ffn_layout(int T, int H, int I, int E, int k) {
   L.w = take(S * 4);
   L.offs = take((int64_t)(E + 1) * 4);
   L.dst_row = take(S * 4);
-  L.row_token = take(L.R_max * 4);
+  L.row_slot = take(L.R_max * 4);
   L.row_w = take(L.R_max * 4);
   L.xq = take(L.R_max * H / 2);
   L.xsf = take(L.R_max * H / 16);
   L.hq = take(L.R_max * I / 2);
   L.hsf = take(L.R_max * I / 16);
-  L.acc = take((int64_t)T * H * 4);
+  L.ys = take(S * H * 4);
   L.total = o;
   return L;
 }
@@ -95,7 +95,7 @@ extern "C" nvfp4_status_t moe_ffn_forward(const void* x_bf16, const float* logit
                                           nvfp4_stream_t stream) {
   if (T < 0 || E < 1 || E > 256 || k < 1 || k > 32 || k > E || H <= 0 || I <= 0)
     return NVFP4_ERR_UNSUPPORTED_SHAPE;
-  if (H % 128 || I % 128) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (H % 256 || I % 128) return NVFP4_ERR_UNSUPPORTED_SHAPE;
   if ((int64_t)T * k > (int64_t)1 << 30) return NVFP4_ERR_UNSUPPORTED_SHAPE;
   if (T == 0) return NVFP4_OK;
   if (!x_bf16 || !logits || !w1 || !sfw1 || !gs_w1 || !w2 || !sfw2 || !gs_w2 || !gs_h ||
@@ -114,17 +114,18 @@ extern "C" nvfp4_status_t moe_ffn_forward(const void* x_bf16, const float* logit
   auto f32 = [&](int64_t off) { return reinterpret_cast<float*>(base + off); };
 
   nvfp4_status_t st = permute_launch(logits, T, E, k, 1, i32(L.ids), f32(L.w), i32(L.offs),
-                                     i32(L.dst_row), i32(L.row_token), f32(L.row_w), L.R_max,
+                                     i32(L.dst_row), i32(L.row_slot), f32(L.row_w), L.R_max,
                                      dev_status, s);
   if (st != NVFP4_OK) return st;
   st = quantize_launch(x_bf16, T, H, H, i32(L.dst_row), k, L.R_max, base + L.xq, base + L.xsf,
                        f32(L.gs_x), 1, base + L.amax, dev_status, s);
   if (st != NVFP4_OK) return st;
   st = gemm_l1(base + L.xq, base + L.xsf, f32(L.gs_x), w1, sfw1, gs_w1, i32(L.offs),
-               i32(L.row_token), E, H, I, L.R_max, gs_h, base + L.hq, base + L.hsf, dev_status, s);
+               i32(L.row_slot), E, H, I, L.R_max, gs_h, base + L.hq, base + L.hsf, dev_status, s);
   if (st != NVFP4_OK) return st;
-  return gemm_l2(base + L.hq, base + L.hsf, gs_h, w2, sfw2, gs_w2, i32(L.offs), i32(L.row_token),
-                 f32(L.row_w), E, H, I, T, L.R_max, f32(L.acc), out_bf16, dev_status, s);
+  return gemm_l2(base + L.hq, base + L.hsf, gs_h, w2, sfw2, gs_w2, i32(L.offs), i32(L.row_slot),
+                 f32(L.row_w), i32(L.dst_row), E, H, I, T, k, L.R_max, f32(L.ys), nullptr,
+                 out_bf16, dev_status, s);
 }
 
 extern "C" nvfp4_status_t nvfp4_read_status(const int32_t* dev_status, int32_t* host_code,

@@ -25,7 +25,9 @@
 //       section 5 "NVFP4-1.1"): W1 is stored gate/up interleaved in 16-row blocks, so the
 //       256-row B tile holds gate and up rows of the same 128 h features and each epilogue
 //       thread finds matching gate and up values 16 accumulator columns apart.
-//   L2  routing weight + scatter-add: red.global.add.v4.f32 into an FP32 [T][H] buffer.
+//   L2  routing weight + scatter: each row's weighted output is stored to its slot's row of an
+//       FP32 [T*k][H] buffer; a combine kernel then sums each token's k rows in a fixed order
+//       (no atomics: FP32 reductions into a shared accumulator were the bottleneck).
 //
 // Tile scheduler: each expert's 128-padded row segment gives (rows/128) M-tiles; tiles are
 // numbered expert by expert with the N-tile outer and the M-tile inner, so CTAs running at the
@@ -57,18 +59,20 @@ constexpr int MAX_E = 256;
 
 enum Mode { PLAIN_F32 = 0, PLAIN_BF16 = 1, L1_SWIGLU = 2, L2_SCATTER = 3 };
 
-// Tile width N per epilogue.  The L2 scatter uses 128-column tiles: then two accumulators fit in
-// tensor memory next to the per-stage scale factors, so its long scatter epilogue overlaps the
-// next tile's main loop.  The other epilogues use 256 columns (half the MMA instructions per
-// output; one accumulator).  Shared memory holds as many stages as fit in 216 KB.
+// Tile shape: M = 128 rows, N = 256 columns, K = 256 per stage.  One MMA instruction has a fixed
+// cost, so the widest N moves the most weight bytes per instruction; one 256-column accumulator
+// and 4 stages of per-stage scale columns fill tensor memory (448 of 512 columns).  The L2 mode
+// keeps 3 stages and gives the fourth stage's shared memory to its epilogue's staging blocks.
 template <int MODE>
 struct TileCfg {
-  static constexpr int BN = MODE == L2_SCATTER ? 128 : 256;
+  static constexpr int BN = 256;
   static constexpr int B_BYTES = BN * BK_BYTES;
   static constexpr int SFB_BYTES = (BN / 128) * 4 * 512;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
-  static constexpr int STAGES = (216 * 1024) / STAGE_BYTES;
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024;
+  // L2: each epilogue warp stages a 32 x 32 FP32 block in shared memory to write whole lines
+  static constexpr int EPI_STAGE_BYTES = MODE == L2_SCATTER ? EPI_WARPS * 4096 : 0;
+  static constexpr int STAGES = (216 * 1024 - EPI_STAGE_BYTES) / STAGE_BYTES;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_STAGE_BYTES + 1024;
   static constexpr uint32_t SFB_COLS = (BN / 128) * 16;  // scale columns of B per stage
   static constexpr int ACC_BUFS = 2 * BN + STAGES * (16 + SFB_COLS) <= TMEM_COLS ? 2 : 1;
   static constexpr uint32_t TM_SFA = ACC_BUFS * BN;        // 16 columns per stage
@@ -94,18 +98,12 @@ struct GemmArgs {
   uint8_t* h;         // L1: [R_max][I/2]
   uint8_t* sfh;       // L1
   int I;              // L1
-  const int32_t* row_token;  // L2 (required), L1 (optional: skip padding rows)
+  const int32_t* row_slot;   // L2 (required), L1 (optional: skip padding rows)
   const float* row_w;        // L2
-  float* acc;                // L2: [T][H]
-  int T;                     // L2
+  float* ys;                 // L2: weighted expert outputs per slot [S][H]
+  int S;                     // L2: slots (T*k)
   int32_t* status;
 };
-
-__device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c),
-               "f"(d)
-               : "memory");
-}
 
 struct Tile {
   int e, m0, nt;
@@ -362,11 +360,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const float alpha = 1.0f / (__ldg(args.gs_a) * __ldg(args.gs_b + tl.e));
       const int64_t row = tl.m0 + q * 32 + lane;
       // rows of the row map that are padding produce nothing; skip groups of 32 of them
-      int tok = 0;
+      int slot = 0;
       if (MODE == L1_SWIGLU || MODE == L2_SCATTER) {
-        if (args.row_token != nullptr) tok = __ldg(args.row_token + row);
+        if (args.row_slot != nullptr) slot = __ldg(args.row_slot + row);
       }
-      const bool live = __any_sync(0xffffffffu, tok >= 0);
+      const bool live = __any_sync(0xffffffffu, slot >= 0);
+      bool released = false;  // accumulator buffer b handed back to the MMA warp
 
       if (MODE == L1_SWIGLU) {
         if (live) {
@@ -412,27 +411,49 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               sfw;
         }
       } else if (MODE == L2_SCATTER) {
+        // this row's weighted expert output goes to its slot's row of ys; the combine kernel sums
+        // a token's k slot rows.  Each 32-column chunk passes through shared memory (16-byte
+        // units XOR-swizzled by row) so that 8 lanes write one row's 128 contiguous bytes.
         if (live) {
-          if (tok >= args.T) {
+          if (slot >= args.S) {
             report(args.status, NVFP4_DEVERR_BAD_INDEX);
-            tok = -1;
+            slot = -1;
           }
-          const float scale = alpha * (tok >= 0 ? __ldg(args.row_w + row) : 0.0f);
+          const float scale = alpha * (slot >= 0 ? __ldg(args.row_w + row) : 0.0f);
           const int H = args.N;
-          float* dst = args.acc + (int64_t)(tok >= 0 ? tok : 0) * H + tl.nt * BN;
+          float4* stg = reinterpret_cast<float4*>(smem + STAGES * C::STAGE_BYTES +
+                                                  (warp - EPI_WARP0) * 4096);
+          const int sub = lane >> 3, c4 = lane & 7;
+          int sl[8];  // slot of row 4i + sub of this warp's 32 rows
+#pragma unroll
+          for (int i = 0; i < 8; ++i) sl[i] = __shfl_sync(0xffffffffu, slot, 4 * i + sub);
+          const int c_lo = (BN / 64) * half, c_hi = c_lo + BN / 64;
 #pragma unroll 1
-          for (int c = (BN / 64) * half; c < (BN / 64) * (half + 1); ++c) {
+          for (int c = c_lo; c < c_hi; ++c) {
             uint32_t v[32];
             tmem_ld32(t_row + 32 * c, v);
             tmem_wait_ld();
-            if (tok >= 0) {
-#pragma unroll
-              for (int i = 0; i < 8; ++i)
-                red_add_v4(dst + 32 * c + 4 * i, __uint_as_float(v[4 * i]) * scale,
-                           __uint_as_float(v[4 * i + 1]) * scale,
-                           __uint_as_float(v[4 * i + 2]) * scale,
-                           __uint_as_float(v[4 * i + 3]) * scale);
+            if (c == c_hi - 1) {  // last read of this tile's accumulator: hand it back now
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(smem_u32(&bar_acc_empty[b]));
+              released = true;
             }
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              stg[lane * 8 + (j ^ (lane & 7))] =
+                  make_float4(__uint_as_float(v[4 * j]) * scale, __uint_as_float(v[4 * j + 1]) * scale,
+                              __uint_as_float(v[4 * j + 2]) * scale,
+                              __uint_as_float(v[4 * j + 3]) * scale);
+            __syncwarp();
+            const int64_t col = (int64_t)tl.nt * BN + 32 * c + 4 * c4;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const int r = 4 * i + sub;
+              const float4 val = stg[r * 8 + (c4 ^ (r & 7))];
+              if (sl[i] >= 0) *reinterpret_cast<float4*>(args.ys + (int64_t)sl[i] * H + col) = val;
+            }
+            __syncwarp();
           }
         }
       } else {
@@ -468,9 +489,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&bar_acc_empty[b]));
+      if (!released) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&bar_acc_empty[b]));
+      }
     }
   }
 
@@ -536,20 +559,40 @@ nvfp4_status_t launch(const uint8_t* a, const uint8_t* b, int64_t b_rows, GemmAr
   return check_launch("grouped_gemm_kernel");
 }
 
-__global__ void cast_bf16_kernel(const float* __restrict__ acc, __nv_bfloat16* __restrict__ out,
-                                 int64_t n8) {
-  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n8;
+// out[t] = sum over the token's slots j (in order, skipping dropped ones) of ys[t*k + j]; FP32
+// adds in a fixed order, so the output is bitwise reproducible.  8 columns per thread.
+__global__ void combine_kernel(const float* __restrict__ ys, const int32_t* __restrict__ dst_row,
+                               int T, int k, int H, float* __restrict__ out_f32,
+                               __nv_bfloat16* __restrict__ out_bf16) {
+  const int n8 = H / 8;
+  const int64_t total = (int64_t)T * n8;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
        i += (int64_t)gridDim.x * blockDim.x) {
-    const float4 a = reinterpret_cast<const float4*>(acc)[2 * i];
-    const float4 b = reinterpret_cast<const float4*>(acc)[2 * i + 1];
-    const __nv_bfloat162 p0 = __floats2bfloat162_rn(a.x, a.y), p1 = __floats2bfloat162_rn(a.z, a.w),
-                         p2 = __floats2bfloat162_rn(b.x, b.y), p3 = __floats2bfloat162_rn(b.z, b.w);
-    uint4 o;
-    o.x = *reinterpret_cast<const uint32_t*>(&p0);
-    o.y = *reinterpret_cast<const uint32_t*>(&p1);
-    o.z = *reinterpret_cast<const uint32_t*>(&p2);
-    o.w = *reinterpret_cast<const uint32_t*>(&p3);
-    reinterpret_cast<uint4*>(out)[i] = o;
+    const int64_t t = i / n8;
+    const int c = static_cast<int>(i - t * n8) * 8;
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
+    for (int j = 0; j < k; ++j) {
+      if (__ldg(dst_row + t * k + j) < 0) continue;
+      const float4* p = reinterpret_cast<const float4*>(ys + (t * k + j) * H + c);
+      const float4 p0 = __ldg(p), p1 = __ldg(p + 1);
+      a.x += p0.x; a.y += p0.y; a.z += p0.z; a.w += p0.w;
+      b.x += p1.x; b.y += p1.y; b.z += p1.z; b.w += p1.w;
+    }
+    if (out_f32 != nullptr) {
+      float4* o = reinterpret_cast<float4*>(out_f32 + t * H + c);
+      o[0] = a;
+      o[1] = b;
+    }
+    if (out_bf16 != nullptr) {
+      const __nv_bfloat162 q0 = __floats2bfloat162_rn(a.x, a.y), q1 = __floats2bfloat162_rn(a.z, a.w),
+                           q2 = __floats2bfloat162_rn(b.x, b.y), q3 = __floats2bfloat162_rn(b.z, b.w);
+      uint4 o;
+      o.x = *reinterpret_cast<const uint32_t*>(&q0);
+      o.y = *reinterpret_cast<const uint32_t*>(&q1);
+      o.z = *reinterpret_cast<const uint32_t*>(&q2);
+      o.w = *reinterpret_cast<const uint32_t*>(&q3);
+      *reinterpret_cast<uint4*>(out_bf16 + t * H + c) = o;
+    }
   }
 }
 
@@ -571,36 +614,33 @@ nvfp4_status_t gemm_plain(const uint8_t* a, const uint8_t* sfa, const float* gs_
 
 nvfp4_status_t gemm_l1(const uint8_t* a, const uint8_t* sfa, const float* gs_a, const uint8_t* w1,
                        const uint8_t* sfw1, const float* gs_w1, const int32_t* offs,
-                       const int32_t* row_token, int E, int H, int I, int64_t R_max,
+                       const int32_t* row_slot, int E, int H, int I, int64_t R_max,
                        const float* gs_h, uint8_t* h, uint8_t* sfh, int32_t* status,
                        cudaStream_t s) {
   GemmArgs g{};
   g.sfa = sfa; g.sfb = sfw1; g.gs_a = gs_a; g.gs_b = gs_w1; g.offs = offs;
   g.E = E; g.N = 2 * I; g.K = H; g.n_tiles = I / 128; g.R_max = R_max;
-  g.gs_h = gs_h; g.h = h; g.sfh = sfh; g.I = I; g.row_token = row_token; g.status = status;
+  g.gs_h = gs_h; g.h = h; g.sfh = sfh; g.I = I; g.row_slot = row_slot; g.status = status;
   return launch<L1_SWIGLU>(a, w1, (int64_t)E * 2 * I, g, s);
 }
 
 nvfp4_status_t gemm_l2(const uint8_t* h, const uint8_t* sfh, const float* gs_h, const uint8_t* w2,
                        const uint8_t* sfw2, const float* gs_w2, const int32_t* offs,
-                       const int32_t* row_token, const float* row_w, int E, int H, int I, int T,
-                       int64_t R_max, float* acc, void* out_bf16, int32_t* status,
-                       cudaStream_t s) {
+                       const int32_t* row_slot, const float* row_w, const int32_t* dst_row, int E,
+                       int H, int I, int T, int k, int64_t R_max, float* ys, float* out_f32,
+                       void* out_bf16, int32_t* status, cudaStream_t s) {
   if (T == 0) return NVFP4_OK;
-  if (cudaMemsetAsync(acc, 0, (size_t)T * H * sizeof(float), s) != cudaSuccess)
-    return check_launch("memset acc");
   GemmArgs g{};
   g.sfa = sfh; g.sfb = sfw2; g.gs_a = gs_h; g.gs_b = gs_w2; g.offs = offs;
-  g.E = E; g.N = H; g.K = I; g.R_max = R_max;
-  g.row_token = row_token; g.row_w = row_w; g.acc = acc; g.T = T; g.status = status;
-  g.n_tiles = H / TileCfg<L2_SCATTER>::BN;
+  g.E = E; g.N = H; g.K = I; g.R_max = R_max; g.n_tiles = H / TileCfg<L2_SCATTER>::BN;
+  g.row_slot = row_slot; g.row_w = row_w; g.ys = ys; g.S = T * k; g.status = status;
   nvfp4_status_t st = launch<L2_SCATTER>(h, w2, (int64_t)E * H, g, s);
-  if (st != NVFP4_OK || out_bf16 == nullptr) return st;
-  const int64_t n8 = (int64_t)T * H / 8;
-  const int64_t want = (n8 + 255) / 256;
-  cast_bf16_kernel<<<(unsigned)(want < 148 * 16 ? want : 148 * 16), 256, 0, s>>>(
-      acc, static_cast<__nv_bfloat16*>(out_bf16), n8);
-  return check_launch("cast_bf16_kernel");
+  if (st != NVFP4_OK) return st;
+  const int64_t n = (int64_t)T * H / 8;
+  const int64_t want = (n + 255) / 256;
+  combine_kernel<<<(unsigned)(want < 148 * 16 ? want : 148 * 16), 256, 0, s>>>(
+      ys, dst_row, T, k, H, out_f32, static_cast<__nv_bfloat16*>(out_bf16));
+  return check_launch("combine_kernel");
 }
 
 }  // namespace nvfp4
@@ -626,7 +666,7 @@ extern "C" nvfp4_status_t nvfp4_grouped_gemm(const uint8_t* a, const uint8_t* sf
 
 extern "C" nvfp4_status_t moe_grouped_gemm_l1_swiglu_q(
     const uint8_t* a, const uint8_t* sfa, const float* gs_a, const uint8_t* w1,
-    const uint8_t* sfw1, const float* gs_w1, const int32_t* offs, const int32_t* row_token, int E,
+    const uint8_t* sfw1, const float* gs_w1, const int32_t* offs, const int32_t* row_slot, int E,
     int H, int I, int64_t R_max, const float* gs_h, uint8_t* h, uint8_t* sfh, int32_t* dev_status,
     nvfp4_stream_t stream) {
   if (E < 1 || E > MAX_E || H <= 0 || I <= 0 || R_max < 0) return NVFP4_ERR_INVALID_ARG;
@@ -635,30 +675,32 @@ extern "C" nvfp4_status_t moe_grouped_gemm_l1_swiglu_q(
   if (R_max == 0) return NVFP4_OK;
   if (!ok_ptr(a) || !ok_ptr(sfa) || !ok_ptr(w1) || !ok_ptr(sfw1) || !ok_ptr(h) || !ok_ptr(sfh))
     return (a && sfa && w1 && sfw1 && h && sfh) ? NVFP4_ERR_MISALIGNED : NVFP4_ERR_INVALID_ARG;
-  if (reinterpret_cast<uintptr_t>(row_token) & 3u) return NVFP4_ERR_MISALIGNED;
-  return gemm_l1(a, sfa, gs_a, w1, sfw1, gs_w1, offs, row_token, E, H, I, R_max, gs_h, h, sfh,
+  if (reinterpret_cast<uintptr_t>(row_slot) & 3u) return NVFP4_ERR_MISALIGNED;
+  return gemm_l1(a, sfa, gs_a, w1, sfw1, gs_w1, offs, row_slot, E, H, I, R_max, gs_h, h, sfh,
                  dev_status, reinterpret_cast<cudaStream_t>(stream));
 }
 
 extern "C" nvfp4_status_t moe_grouped_gemm_l2_scatter(
     const uint8_t* h, const uint8_t* sfh, const float* gs_h, const uint8_t* w2,
-    const uint8_t* sfw2, const float* gs_w2, const int32_t* offs, const int32_t* row_token,
-    const float* row_w, int E, int H, int I, int T, int64_t R_max, float* acc_ws, void* out_bf16,
-    int32_t* dev_status, nvfp4_stream_t stream) {
-  if (E < 1 || E > MAX_E || H <= 0 || I <= 0 || T < 0 || R_max < 0) return NVFP4_ERR_INVALID_ARG;
+    const uint8_t* sfw2, const float* gs_w2, const int32_t* offs, const int32_t* row_slot,
+    const float* row_w, const int32_t* dst_row, int E, int H, int I, int T, int k, int64_t R_max,
+    float* ys_ws, float* out_f32, void* out_bf16, int32_t* dev_status, nvfp4_stream_t stream) {
+  if (E < 1 || E > MAX_E || H <= 0 || I <= 0 || T < 0 || k < 1 || R_max < 0)
+    return NVFP4_ERR_INVALID_ARG;
   if (H % TileCfg<L2_SCATTER>::BN || I % 64 || R_max % 128) return NVFP4_ERR_UNSUPPORTED_SHAPE;
-  if (!gs_h || !gs_w2 || !offs || !row_token || !row_w) return NVFP4_ERR_INVALID_ARG;
+  if (!gs_h || !gs_w2 || !offs || !row_slot || !row_w || !dst_row || (!out_f32 && !out_bf16))
+    return NVFP4_ERR_INVALID_ARG;
   if (T == 0 || R_max == 0) return NVFP4_OK;
-  if (!ok_ptr(h) || !ok_ptr(sfh) || !ok_ptr(w2) || !ok_ptr(sfw2) || !ok_ptr(acc_ws) ||
-      (out_bf16 && !aligned16(out_bf16)))
-    return (h && sfh && w2 && sfw2 && acc_ws) ? NVFP4_ERR_MISALIGNED : NVFP4_ERR_INVALID_ARG;
-  return gemm_l2(h, sfh, gs_h, w2, sfw2, gs_w2, offs, row_token, row_w, E, H, I, T, R_max, acc_ws,
-                 out_bf16, dev_status, reinterpret_cast<cudaStream_t>(stream));
+  if (!ok_ptr(h) || !ok_ptr(sfh) || !ok_ptr(w2) || !ok_ptr(sfw2) || !ok_ptr(ys_ws) ||
+      (out_f32 && !aligned16(out_f32)) || (out_bf16 && !aligned16(out_bf16)))
+    return (h && sfh && w2 && sfw2 && ys_ws) ? NVFP4_ERR_MISALIGNED : NVFP4_ERR_INVALID_ARG;
+  return gemm_l2(h, sfh, gs_h, w2, sfw2, gs_w2, offs, row_slot, row_w, dst_row, E, H, I, T, k,
+                 R_max, ys_ws, out_f32, out_bf16, dev_status, reinterpret_cast<cudaStream_t>(stream));
 }
 
 // ------------------------------------------------------------------------------ no-alloc variant
-// The FP32 accumulator of moe_grouped_gemm_l2_scatter_noalloc: one static array per device that
-// loads the library.  Host code must not pass its name to a kernel (on the host it is only a
+// The FP32 per-slot buffer of moe_grouped_gemm_l2_scatter_noalloc: one static array per device
+// that loads the library.  Host code must not pass its name to a kernel (on the host it is only a
 // stand-in symbol); its device address comes from cudaGetSymbolAddress, looked up once per device.
 static __device__ __align__(256) float g_l2_noalloc_acc[NVFP4_L2_NOALLOC_MAX_ELEMS];
 
@@ -689,22 +731,24 @@ float* l2_noalloc_scratch() {
 
 extern "C" nvfp4_status_t moe_grouped_gemm_l2_scatter_noalloc(
     const uint8_t* h, const uint8_t* sfh, const float* gs_h, const uint8_t* w2,
-    const uint8_t* sfw2, const float* gs_w2, const int32_t* offs, const int32_t* row_token,
-    const float* row_w, int E, int H, int I, int T, int64_t R_max, void* out_bf16,
-    int32_t* dev_status, nvfp4_stream_t stream) {
-  if (E < 1 || E > MAX_E || H <= 0 || I <= 0 || T < 0 || R_max < 0) return NVFP4_ERR_INVALID_ARG;
+    const uint8_t* sfw2, const float* gs_w2, const int32_t* offs, const int32_t* row_slot,
+    const float* row_w, const int32_t* dst_row, int E, int H, int I, int T, int k, int64_t R_max,
+    void* out_bf16, int32_t* dev_status, nvfp4_stream_t stream) {
+  if (E < 1 || E > MAX_E || H <= 0 || I <= 0 || T < 0 || k < 1 || R_max < 0)
+    return NVFP4_ERR_INVALID_ARG;
   if (H % TileCfg<L2_SCATTER>::BN || I % 64 || R_max % 128) return NVFP4_ERR_UNSUPPORTED_SHAPE;
-  if (!gs_h || !gs_w2 || !offs || !row_token || !row_w || !out_bf16) return NVFP4_ERR_INVALID_ARG;
-  if ((int64_t)T * H > NVFP4_L2_NOALLOC_MAX_ELEMS) {
-    set_last_error("moe_grouped_gemm_l2_scatter_noalloc: T*H exceeds the static FP32 scratch "
+  if (!gs_h || !gs_w2 || !offs || !row_slot || !row_w || !dst_row || !out_bf16)
+    return NVFP4_ERR_INVALID_ARG;
+  if ((int64_t)T * k * H > NVFP4_L2_NOALLOC_MAX_ELEMS) {
+    set_last_error("moe_grouped_gemm_l2_scatter_noalloc: T*k*H exceeds the static FP32 scratch "
                    "(NVFP4_L2_NOALLOC_MAX_ELEMS floats)");
     return NVFP4_ERR_WORKSPACE_TOO_SMALL;
   }
   if (T == 0 || R_max == 0) return NVFP4_OK;
   if (!ok_ptr(h) || !ok_ptr(sfh) || !ok_ptr(w2) || !ok_ptr(sfw2) || !aligned16(out_bf16))
     return (h && sfh && w2 && sfw2) ? NVFP4_ERR_MISALIGNED : NVFP4_ERR_INVALID_ARG;
-  float* acc = l2_noalloc_scratch();
-  if (acc == nullptr) return NVFP4_ERR_CUDA;
-  return gemm_l2(h, sfh, gs_h, w2, sfw2, gs_w2, offs, row_token, row_w, E, H, I, T, R_max, acc,
-                 out_bf16, dev_status, reinterpret_cast<cudaStream_t>(stream));
+  float* ys = l2_noalloc_scratch();
+  if (ys == nullptr) return NVFP4_ERR_CUDA;
+  return gemm_l2(h, sfh, gs_h, w2, sfw2, gs_w2, offs, row_slot, row_w, dst_row, E, H, I, T, k,
+                 R_max, ys, nullptr, out_bf16, dev_status, reinterpret_cast<cudaStream_t>(stream));
 }

@@ -5,8 +5,8 @@
 // used here: top-k of the logits (ties to the lower id; -inf = dropped slot), weights
 // softmax(logits)[e] renormalized over the k; rows bucketed by expert in ascending id, every
 // segment padded to a multiple of 128 rows (the GEMM's M tile), slots inside a segment in
-// ascending (token, j).  Everything stays on the device: no host sync between routing and the
-// GEMMs (the commit log's zero-.item() rule).
+// ascending (token, j); each row records its slot t*k + j.  Everything stays on the device: no
+// host sync between routing and the GEMMs (the commit log's zero-.item() rule).
 #include <float.h>
 
 #include "common.cuh"
@@ -90,7 +90,7 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
 __global__ void __launch_bounds__(1024) permute_kernel(
     const int32_t* __restrict__ ids, const float* __restrict__ w, int S, int k, int E,
     int64_t R_max, int32_t* __restrict__ offs_out, int32_t* __restrict__ dst_row,
-    int32_t* __restrict__ row_token, float* __restrict__ row_w, int32_t* __restrict__ dev_status) {
+    int32_t* __restrict__ row_slot, float* __restrict__ row_w, int32_t* __restrict__ dev_status) {
   __shared__ int hist[32][kMaxE];
   __shared__ int cnt[kMaxE];
   __shared__ int offs[kMaxE + 1];
@@ -139,7 +139,7 @@ __global__ void __launch_bounds__(1024) permute_kernel(
       if (e >= 0) {
         const int row = offs[e] + hist[warp][e] + rank;
         dst_row[s] = row;
-        row_token[row] = s / k;
+        row_slot[row] = s;
         row_w[row] = __ldg(w + s);
       } else {
         dst_row[s] = -1;
@@ -152,12 +152,12 @@ __global__ void __launch_bounds__(1024) permute_kernel(
   // padding rows of every segment, then the unused tail up to R_max
   for (int e = warp; e < E; e += 32) {
     for (int r = offs[e] + cnt[e] + lane; r < offs[e + 1]; r += 32) {
-      row_token[r] = -1;
+      row_slot[r] = -1;
       row_w[r] = 0.0f;
     }
   }
   for (int64_t r = offs[E] + tid; r < R_max; r += blockDim.x) {
-    row_token[r] = -1;
+    row_slot[r] = -1;
     row_w[r] = 0.0f;
   }
 }
@@ -166,7 +166,7 @@ __global__ void __launch_bounds__(1024) permute_kernel(
 
 nvfp4_status_t permute_launch(const float* logits, int T, int E, int k, int renorm,
                               int32_t* topk_ids, float* topk_w, int32_t* offs, int32_t* dst_row,
-                              int32_t* row_token, float* row_w, int64_t R_max,
+                              int32_t* row_slot, float* row_w, int64_t R_max,
                               int32_t* dev_status, cudaStream_t s) {
   if (logits != nullptr && T > 0) {
     topk_kernel<<<(T + 7) / 8, 256, 0, s>>>(logits, T, E, k, renorm, topk_ids, topk_w);
@@ -174,7 +174,7 @@ nvfp4_status_t permute_launch(const float* logits, int T, int E, int k, int reno
     if (st != NVFP4_OK) return st;
   }
   permute_kernel<<<1, 1024, 0, s>>>(topk_ids, topk_w, T * k, k, E, R_max, offs, dst_row,
-                                    row_token, row_w, dev_status);
+                                    row_slot, row_w, dev_status);
   return check_launch("permute_kernel");
 }
 
@@ -191,19 +191,19 @@ extern "C" size_t moe_permute_workspace_size(int, int, int) { return 0; }
 
 extern "C" nvfp4_status_t moe_permute(const float* logits, int T, int E, int k, int renormalize,
                                       int32_t* topk_ids, float* topk_w, int32_t* offs,
-                                      int32_t* dst_row, int32_t* row_token, float* row_w, void*,
+                                      int32_t* dst_row, int32_t* row_slot, float* row_w, void*,
                                       size_t, int32_t* dev_status, nvfp4_stream_t stream) {
   using namespace nvfp4;
   if (T < 0 || E < 1 || E > kMaxE || k < 1 || k > kMaxK || k > E) return NVFP4_ERR_UNSUPPORTED_SHAPE;
   if ((int64_t)T * k > (int64_t)1 << 30) return NVFP4_ERR_UNSUPPORTED_SHAPE;
   if (offs == nullptr) return NVFP4_ERR_INVALID_ARG;
   if (T > 0 && (topk_ids == nullptr || topk_w == nullptr || dst_row == nullptr ||
-                row_token == nullptr || row_w == nullptr))
+                row_slot == nullptr || row_w == nullptr))
     return NVFP4_ERR_INVALID_ARG;
-  const void* ptrs[] = {logits, topk_ids, topk_w, offs, dst_row, row_token, row_w};
+  const void* ptrs[] = {logits, topk_ids, topk_w, offs, dst_row, row_slot, row_w};
   for (const void* p : ptrs)
     if (reinterpret_cast<uintptr_t>(p) & 3u) return NVFP4_ERR_MISALIGNED;
-  return permute_launch(logits, T, E, k, renormalize, topk_ids, topk_w, offs, dst_row, row_token,
+  return permute_launch(logits, T, E, k, renormalize, topk_ids, topk_w, offs, dst_row, row_slot,
                         row_w, moe_rows_max(T, E, k), dev_status,
                         reinterpret_cast<cudaStream_t>(stream));
 }

@@ -59,6 +59,7 @@ def permute(ids, w, E):
       offs    int64 (E+1,)   start row of each expert's 128-padded segment; offs[E] = R
       dst_row int64 (T, k)   permuted row of slot (t, j), -1 for a dropped slot
       row_token int64 (R,)   token of each row, -1 for padding rows
+      row_slot  int64 (R,)   slot t*k + j of each row, -1 for padding rows
       row_w   float64 (R,)   routing weight of each row, 0 for padding rows
     """
     ids = np.asarray(ids)
@@ -74,6 +75,7 @@ def permute(ids, w, E):
     R = int(offs[E])
     dst_row = np.full((T, k), -1, dtype=np.int64)
     row_token = np.full(R, -1, dtype=np.int64)
+    row_slot = np.full(R, -1, dtype=np.int64)
     row_w = np.zeros(R, dtype=np.float64)
     fill = offs[:E].copy()
     for t in range(T):  # ascending token, then ascending slot j
@@ -85,5 +87,7 @@ def permute(ids, w, E):
             fill[e] += 1
             dst_row[t, j] = r
             row_token[r] = t
+            row_slot[r] = t * k + j
             row_w[r] = w[t, j]
-    return dict(counts=counts, offs=offs, dst_row=dst_row, row_token=row_token, row_w=row_w, R=R)
+    return dict(counts=counts, offs=offs, dst_row=dst_row, row_token=row_token, row_slot=row_slot,
+                row_w=row_w, R=R)

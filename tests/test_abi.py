@@ -98,8 +98,12 @@ def test_gemms_reject_bad_shapes(L):
     assert L.nvfp4_grouped_gemm(f, f, f, f, f, f, f, 2, 256, 64, 128, f, 7, None, None) == 1
     assert L.moe_grouped_gemm_l1_swiglu_q(f, f, f, f, f, f, f, None, 8, 256, 96, 128, f, f, f,
                                           None, None) == 2  # I % 128
-    assert L.moe_grouped_gemm_l2_scatter(f, f, f, f, f, f, f, f, f, 8, 200, 128, 4, 128, f, f,
-                                         None, None) == 2  # H % 256
+    assert L.moe_grouped_gemm_l2_scatter(f, f, f, f, f, f, f, f, f, f, 8, 200, 128, 4, 2, 128, f,
+                                         f, None, None, None) == 2  # H % 128
+    assert L.moe_grouped_gemm_l2_scatter(f, f, f, f, f, f, f, f, f, f, 8, 256, 128, 4, 2, 128, f,
+                                         None, None, None, None) == 1  # no output
+    assert L.moe_grouped_gemm_l2_scatter_noalloc(f, f, f, f, f, f, f, f, f, f, 8, 256, 128, 4096,
+                                                 2, 128, f, None, None) == 4  # T*k*H > 1<<20
     assert L.moe_ffn_forward(f, f, 4, 256, 128, 8, 2, f, f, f, f, f, f, f, f, f, 10, None,
                              None) == 4  # workspace too small
     assert L.moe_ffn_forward(f, f, 4, 256, 128, 8, 2, f, f, f, f, f, f, f, f, None, 1 << 30, None,

@@ -2,7 +2,8 @@
 
 * L1 + SwiGLU + NVFP4 re-quantization: h codes may differ by one E2M1 step on at most 0.1% of
   the elements (a block whose scale byte differs counts whole);
-* L2 + routing weight + scatter-add: FP32 result within relative Frobenius 1e-5 of the oracle.
+* L2 + routing weight + scatter to token order: FP32 result within relative Frobenius 1e-5 of
+  the oracle.
 """
 
 import numpy as np
@@ -67,10 +68,9 @@ def test_l1_and_l2_match_oracle(T, H, I, E, k):
     # ---- L1 fused SwiGLU + re-quantization (every row; and with the row map, which skips
     # all-padding row groups but must give the same bytes on real rows)
     h, sfh = nv.l1_swiglu_q(a, asf, gs_x, w1d, offs, gs_h_d)
-    row_token_d = to_dev(perm["row_token"].astype(np.int32))
+    row_slot = to_dev(perm["row_slot"].astype(np.int32))
     status = torch.zeros(1, dtype=torch.int32, device=DEV)
-    h2, sfh2 = nv.l1_swiglu_q(a, asf, gs_x, w1d, offs, gs_h_d, row_token=row_token_d,
-                              status=status)
+    h2, sfh2 = nv.l1_swiglu_q(a, asf, gs_x, w1d, offs, gs_h_d, row_slot=row_slot, status=status)
     torch.cuda.synchronize()
     hc2, hs2 = download_nvfp4(h2, sfh2, Rr, I)
     c1_logical = c1.cpu().numpy()[:, nv.w1_row_map(I).numpy()]  # stored -> logical columns
@@ -88,9 +88,10 @@ def test_l1_and_l2_match_oracle(T, H, I, E, k):
 
     # ---- L2 + scatter on the oracle's h codes (identical operands)
     h_o, sfh_o = upload_nvfp4(ref["h_codes"], ref["h_sf"])
-    row_token = to_dev(perm["row_token"].astype(np.int32))
     row_w = to_dev(perm["row_w"].astype(np.float32))
-    acc, out = nv.l2_scatter(h_o, sfh_o, gs_h_d, w2d, offs, row_token, row_w, T, status=status)
+    dst_row = to_dev(perm["dst_row"].reshape(-1).astype(np.int32))
+    acc, out = nv.l2_scatter(h_o, sfh_o, gs_h_d, w2d, offs, row_slot, row_w, dst_row, T, k,
+                             status=status)
     torch.cuda.synchronize()
     code, rc = nv.read_status(status)
     assert code == 0 and rc == 0
@@ -100,16 +101,17 @@ def test_l1_and_l2_match_oracle(T, H, I, E, k):
     assert np.all(acc.cpu().numpy()[dropped] == 0)
 
 
-def test_l2_bad_row_token_is_flagged():
+def test_l2_bad_row_slot_is_flagged():
     x, ids, w32, w1, w1d, w2, w2d = _setup(16, 256, 128, 2, 1)
     perm = R.permute(ids, w32, 2)
     Rr = perm["R"]
     h = torch.zeros(Rr, 64, dtype=torch.uint8, device=DEV)
     sfh = torch.zeros(nv.sf_bytes(Rr, 128), dtype=torch.uint8, device=DEV)
-    rt = perm["row_token"].astype(np.int32).copy()
-    rt[0] = 999  # out of range token
+    rs = perm["row_slot"].astype(np.int32).copy()
+    rs[0] = 999  # out of range slot (T*k = 16)
     status = torch.zeros(1, dtype=torch.int32, device=DEV)
     nv.l2_scatter(h, sfh, torch.ones(1, device=DEV), w2d, to_dev(perm["offs"].astype(np.int32)),
-                  to_dev(rt), to_dev(perm["row_w"].astype(np.float32)), 16, status=status)
+                  to_dev(rs), to_dev(perm["row_w"].astype(np.float32)),
+                  to_dev(perm["dst_row"].reshape(-1).astype(np.int32)), 16, 1, status=status)
     code, rc = nv.read_status(status)
     assert code & 2 and rc == 7

@@ -22,11 +22,11 @@ def _compare(p, ids_ref, w_ref, E, k):
     assert np.array_equal(p["offs"].cpu().numpy(), pr["offs"])
     assert np.array_equal(p["dst_row"].cpu().numpy().reshape(T, k), pr["dst_row"])
     Rm = p["R_max"]
-    rt = p["row_token"].cpu().numpy()[:Rm]
+    rs = p["row_slot"].cpu().numpy()[:Rm]
     rw = p["row_w"].cpu().numpy()[:Rm]
     n = pr["R"]
-    assert np.array_equal(rt[:n], pr["row_token"])
-    assert np.all(rt[n:] == -1) and np.all(rw[n:] == 0)
+    assert np.array_equal(rs[:n], pr["row_slot"])
+    assert np.all(rs[n:] == -1) and np.all(rw[n:] == 0)
     assert np.allclose(rw[:n], pr["row_w"], rtol=2e-6, atol=1e-7)
 
 

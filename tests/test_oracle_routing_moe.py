@@ -58,6 +58,8 @@ def test_permute_offsets_order_and_padding():
     # expert 2 rows: (t0,j0), (t1,j1), (t2,j0), (t3,j1) in that order
     assert p["dst_row"].tolist() == [[256, 0], [1, 257], [258, -1], [128, 259]]
     assert p["row_token"][256:260].tolist() == [0, 1, 2, 3]
+    assert p["row_slot"][256:260].tolist() == [0, 3, 4, 7]
+    assert p["row_slot"][128] == 6 and np.all(p["row_slot"][2:128] == -1)
     assert np.allclose(p["row_w"][256:260], [0.0, 0.3, 0.4, 0.7])
     assert np.all(p["row_token"][2:128] == -1) and np.all(p["row_w"][2:128] == 0)
     assert p["R"] == 384
