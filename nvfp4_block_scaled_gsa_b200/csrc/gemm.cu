@@ -57,11 +57,16 @@ constexpr int EPI_WARPS = 8;
 constexpr int SF_WARP0 = EPI_WARP0 + EPI_WARPS;
 constexpr int MAX_E = 256;
 
-enum Mode { PLAIN_F32 = 0, PLAIN_BF16 = 1, L1_SWIGLU = 2, L2_SCATTER = 3 };
+// L2_DIRECT: each epilogue lane stores its own row (4 stages; suits a few rows per expert).
+// L2_STAGED: rows pass through shared memory so a warp writes whole lines (3 stages).
+enum Mode { PLAIN_F32 = 0, PLAIN_BF16 = 1, L1_SWIGLU = 2, L2_DIRECT = 3, L2_STAGED = 4 };
+
+// Average routed rows per expert from which the L2 epilogue stages its output
+constexpr int kL2StagedMinRowsPerExpert = 32;
 
 // Tile shape: M = 128 rows, N = 256 columns, K = 256 per stage.  One MMA instruction has a fixed
 // cost, so the widest N moves the most weight bytes per instruction; one 256-column accumulator
-// and 4 stages of per-stage scale columns fill tensor memory (448 of 512 columns).  The L2 mode
+// and 4 stages of per-stage scale columns fill tensor memory (448 of 512 columns).  L2_STAGED
 // keeps 3 stages and gives the fourth stage's shared memory to its epilogue's staging blocks.
 template <int MODE>
 struct TileCfg {
@@ -70,7 +75,7 @@ struct TileCfg {
   static constexpr int SFB_BYTES = (BN / 128) * 4 * 512;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
   // L2: each epilogue warp stages a 32 x 32 FP32 block in shared memory to write whole lines
-  static constexpr int EPI_STAGE_BYTES = MODE == L2_SCATTER ? EPI_WARPS * 4096 : 0;
+  static constexpr int EPI_STAGE_BYTES = MODE == L2_STAGED ? EPI_WARPS * 4096 : 0;
   static constexpr int STAGES = (216 * 1024 - EPI_STAGE_BYTES) / STAGE_BYTES;
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_STAGE_BYTES + 1024;
   static constexpr uint32_t SFB_COLS = (BN / 128) * 16;  // scale columns of B per stage
@@ -361,7 +366,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int64_t row = tl.m0 + q * 32 + lane;
       // rows of the row map that are padding produce nothing; skip groups of 32 of them
       int slot = 0;
-      if (MODE == L1_SWIGLU || MODE == L2_SCATTER) {
+      if (MODE == L1_SWIGLU || MODE == L2_DIRECT || MODE == L2_STAGED) {
         if (args.row_slot != nullptr) slot = __ldg(args.row_slot + row);
       }
       const bool live = __any_sync(0xffffffffu, slot >= 0);
@@ -410,10 +415,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           *reinterpret_cast<uint32_t*>(args.sfh + sf_offset(row, tl.nt * 8 + 4 * half, I / 16)) =
               sfw;
         }
-      } else if (MODE == L2_SCATTER) {
+      } else if (MODE == L2_DIRECT || MODE == L2_STAGED) {
         // this row's weighted expert output goes to its slot's row of ys; the combine kernel sums
-        // a token's k slot rows.  Each 32-column chunk passes through shared memory (16-byte
-        // units XOR-swizzled by row) so that 8 lanes write one row's 128 contiguous bytes.
+        // a token's k slot rows
         if (live) {
           if (slot >= args.S) {
             report(args.status, NVFP4_DEVERR_BAD_INDEX);
@@ -421,39 +425,59 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
           const float scale = alpha * (slot >= 0 ? __ldg(args.row_w + row) : 0.0f);
           const int H = args.N;
-          float4* stg = reinterpret_cast<float4*>(smem + STAGES * C::STAGE_BYTES +
-                                                  (warp - EPI_WARP0) * 4096);
-          const int sub = lane >> 3, c4 = lane & 7;
-          int sl[8];  // slot of row 4i + sub of this warp's 32 rows
-#pragma unroll
-          for (int i = 0; i < 8; ++i) sl[i] = __shfl_sync(0xffffffffu, slot, 4 * i + sub);
           const int c_lo = (BN / 64) * half, c_hi = c_lo + BN / 64;
+          if constexpr (MODE == L2_STAGED) {
+            // each 32-column chunk passes through shared memory (16-byte units XOR-swizzled by
+            // row) so that 8 lanes write one row's 128 contiguous bytes
+            float4* stg = reinterpret_cast<float4*>(smem + STAGES * C::STAGE_BYTES +
+                                                    (warp - EPI_WARP0) * 4096);
+            const int sub = lane >> 3, c4 = lane & 7;
+            int sl[8];  // slot of row 4i + sub of this warp's 32 rows
+#pragma unroll
+            for (int i = 0; i < 8; ++i) sl[i] = __shfl_sync(0xffffffffu, slot, 4 * i + sub);
 #pragma unroll 1
-          for (int c = c_lo; c < c_hi; ++c) {
-            uint32_t v[32];
-            tmem_ld32(t_row + 32 * c, v);
-            tmem_wait_ld();
-            if (c == c_hi - 1) {  // last read of this tile's accumulator: hand it back now
-              tc_fence_before();
+            for (int c = c_lo; c < c_hi; ++c) {
+              uint32_t v[32];
+              tmem_ld32(t_row + 32 * c, v);
+              tmem_wait_ld();
+              if (c == c_hi - 1) {  // last read of this tile's accumulator: hand it back now
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&bar_acc_empty[b]));
+                released = true;
+              }
+#pragma unroll
+              for (int j = 0; j < 8; ++j)
+                stg[lane * 8 + (j ^ (lane & 7))] = make_float4(
+                    __uint_as_float(v[4 * j]) * scale, __uint_as_float(v[4 * j + 1]) * scale,
+                    __uint_as_float(v[4 * j + 2]) * scale, __uint_as_float(v[4 * j + 3]) * scale);
               __syncwarp();
-              if (lane == 0) mbar_arrive(smem_u32(&bar_acc_empty[b]));
-              released = true;
-            }
+              const int64_t col = (int64_t)tl.nt * BN + 32 * c + 4 * c4;
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
-              stg[lane * 8 + (j ^ (lane & 7))] =
-                  make_float4(__uint_as_float(v[4 * j]) * scale, __uint_as_float(v[4 * j + 1]) * scale,
-                              __uint_as_float(v[4 * j + 2]) * scale,
-                              __uint_as_float(v[4 * j + 3]) * scale);
-            __syncwarp();
-            const int64_t col = (int64_t)tl.nt * BN + 32 * c + 4 * c4;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              const int r = 4 * i + sub;
-              const float4 val = stg[r * 8 + (c4 ^ (r & 7))];
-              if (sl[i] >= 0) *reinterpret_cast<float4*>(args.ys + (int64_t)sl[i] * H + col) = val;
+              for (int i = 0; i < 8; ++i) {
+                const int r = 4 * i + sub;
+                const float4 val = stg[r * 8 + (c4 ^ (r & 7))];
+                if (sl[i] >= 0) *reinterpret_cast<float4*>(args.ys + (int64_t)sl[i] * H + col) = val;
+              }
+              __syncwarp();
             }
-            __syncwarp();
+          } else {
+            float* dst = args.ys + (int64_t)(slot >= 0 ? slot : 0) * H + tl.nt * BN;
+#pragma unroll 1
+            for (int c = c_lo; c < c_hi; ++c) {
+              uint32_t v[32];
+              tmem_ld32(t_row + 32 * c, v);
+              tmem_wait_ld();
+              if (slot >= 0) {
+                float4* o = reinterpret_cast<float4*>(dst + 32 * c);
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                  o[i] = make_float4(__uint_as_float(v[4 * i]) * scale,
+                                     __uint_as_float(v[4 * i + 1]) * scale,
+                                     __uint_as_float(v[4 * i + 2]) * scale,
+                                     __uint_as_float(v[4 * i + 3]) * scale);
+              }
+            }
           }
         }
       } else {
@@ -632,9 +656,11 @@ nvfp4_status_t gemm_l2(const uint8_t* h, const uint8_t* sfh, const float* gs_h, 
   if (T == 0) return NVFP4_OK;
   GemmArgs g{};
   g.sfa = sfh; g.sfb = sfw2; g.gs_a = gs_h; g.gs_b = gs_w2; g.offs = offs;
-  g.E = E; g.N = H; g.K = I; g.R_max = R_max; g.n_tiles = H / TileCfg<L2_SCATTER>::BN;
+  g.E = E; g.N = H; g.K = I; g.R_max = R_max; g.n_tiles = H / TileCfg<L2_DIRECT>::BN;
   g.row_slot = row_slot; g.row_w = row_w; g.ys = ys; g.S = T * k; g.status = status;
-  nvfp4_status_t st = launch<L2_SCATTER>(h, w2, (int64_t)E * H, g, s);
+  const bool staged = (int64_t)T * k >= (int64_t)kL2StagedMinRowsPerExpert * E;
+  nvfp4_status_t st = staged ? launch<L2_STAGED>(h, w2, (int64_t)E * H, g, s)
+                             : launch<L2_DIRECT>(h, w2, (int64_t)E * H, g, s);
   if (st != NVFP4_OK) return st;
   const int64_t n = (int64_t)T * H / 8;
   const int64_t want = (n + 255) / 256;
@@ -687,7 +713,7 @@ extern "C" nvfp4_status_t moe_grouped_gemm_l2_scatter(
     float* ys_ws, float* out_f32, void* out_bf16, int32_t* dev_status, nvfp4_stream_t stream) {
   if (E < 1 || E > MAX_E || H <= 0 || I <= 0 || T < 0 || k < 1 || R_max < 0)
     return NVFP4_ERR_INVALID_ARG;
-  if (H % TileCfg<L2_SCATTER>::BN || I % 64 || R_max % 128) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (H % TileCfg<L2_DIRECT>::BN || I % 64 || R_max % 128) return NVFP4_ERR_UNSUPPORTED_SHAPE;
   if (!gs_h || !gs_w2 || !offs || !row_slot || !row_w || !dst_row || (!out_f32 && !out_bf16))
     return NVFP4_ERR_INVALID_ARG;
   if (T == 0 || R_max == 0) return NVFP4_OK;
@@ -736,7 +762,7 @@ extern "C" nvfp4_status_t moe_grouped_gemm_l2_scatter_noalloc(
     void* out_bf16, int32_t* dev_status, nvfp4_stream_t stream) {
   if (E < 1 || E > MAX_E || H <= 0 || I <= 0 || T < 0 || k < 1 || R_max < 0)
     return NVFP4_ERR_INVALID_ARG;
-  if (H % TileCfg<L2_SCATTER>::BN || I % 64 || R_max % 128) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (H % TileCfg<L2_DIRECT>::BN || I % 64 || R_max % 128) return NVFP4_ERR_UNSUPPORTED_SHAPE;
   if (!gs_h || !gs_w2 || !offs || !row_slot || !row_w || !dst_row || !out_bf16)
     return NVFP4_ERR_INVALID_ARG;
   if ((int64_t)T * k * H > NVFP4_L2_NOALLOC_MAX_ELEMS) {
