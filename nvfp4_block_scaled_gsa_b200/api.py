@@ -118,10 +118,14 @@ def permute(logits, k, renormalize=True, ids=None, weights=None, E=None, status=
                 row_w=row_w, R_max=R, E=E, T=T, k=k)
 
 
-def grouped_gemm(a_codes, a_sf, gs_a, w: NVFP4Weights, offs, out_dtype=F32, status=None):
-    """Plain 2D x 3D grouped GEMM: out[r] = A[r] . W_e^T / (gs_a * gs_w[e])."""
+def grouped_gemm(a_codes, a_sf, gs_a, w: NVFP4Weights, offs, out_dtype=F32, status=None,
+                 out=None):
+    """Plain 2D x 3D grouped GEMM: out[r] = A[r] . W_e^T / (gs_a * gs_w[e]).  Rows past
+    offs[E] are left as they are (``out`` may be given, (R, N) of ``out_dtype``)."""
     R = a_codes.shape[0]
-    out = torch.empty(R, w.N, dtype=out_dtype, device=a_codes.device)
+    if out is None:
+        out = torch.empty(R, w.N, dtype=out_dtype, device=a_codes.device)
+    assert out.shape == (R, w.N) and out.dtype == out_dtype and out.is_contiguous()
     call("nvfp4_grouped_gemm", _p(a_codes), _p(a_sf), _p(gs_a), _p(w.codes), _p(w.sf), _p(w.gs),
          _p(offs), w.E, w.N, w.K, R, _p(out), 0 if out_dtype == F32 else 1, _p(status), _stream())
     return out

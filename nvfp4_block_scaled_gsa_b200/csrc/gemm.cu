@@ -64,17 +64,22 @@ enum Mode { PLAIN_F32 = 0, PLAIN_BF16 = 1, L1_SWIGLU = 2, L2_DIRECT = 3, L2_STAG
 // Average routed rows per expert from which the L2 epilogue stages its output
 constexpr int kL2StagedMinRowsPerExpert = 32;
 
-// Tile shape: M = 128 rows, N = 256 columns, K = 256 per stage.  One MMA instruction has a fixed
-// cost, so the widest N moves the most weight bytes per instruction; one 256-column accumulator
-// and 4 stages of per-stage scale columns fill tensor memory (448 of 512 columns).  L2_STAGED
-// keeps 3 stages and gives the fourth stage's shared memory to its epilogue's staging blocks.
-template <int MODE>
+// Tile shape: M = 128 rows per CTA, N = 256 columns, K = 256 per stage.  One MMA instruction
+// has a fixed cost, so the widest N moves the most weight bytes per instruction; one 256-column
+// accumulator and the per-stage scale columns fill tensor memory.
+//
+// CTAS = 2 runs the pair form (cta_group::2) on a cluster of 2 CTAs: a 256 x 256 tile, each CTA
+// holding 128 rows of A and 128 rows (N) of B per stage, so each SM moves 2/3 of the operand
+// bytes of a 128 x 256 tile for the same MMA work.  The even CTA (the leader) issues the MMAs;
+// both CTAs run producer, scale-factor and epilogue warps.
+template <int MODE, int CTAS>
 struct TileCfg {
   static constexpr int BN = 256;
-  static constexpr int B_BYTES = BN * BK_BYTES;
-  static constexpr int SFB_BYTES = (BN / 128) * 4 * 512;
+  static constexpr int B_ROWS = BN / CTAS;                 // B rows (N) per CTA per stage
+  static constexpr int B_BYTES = B_ROWS * BK_BYTES;
+  static constexpr int SFB_BYTES = (BN / 128) * 4 * 512;   // scales of all BN rows of B
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
-  // L2: each epilogue warp stages a 32 x 32 FP32 block in shared memory to write whole lines
+  // L2_STAGED: each epilogue warp stages a 32 x 32 FP32 block in shared memory
   static constexpr int EPI_STAGE_BYTES = MODE == L2_STAGED ? EPI_WARPS * 4096 : 0;
   static constexpr int STAGES = (216 * 1024 - EPI_STAGE_BYTES) / STAGE_BYTES;
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_STAGE_BYTES + 1024;
@@ -82,7 +87,7 @@ struct TileCfg {
   static constexpr int ACC_BUFS = 2 * BN + STAGES * (16 + SFB_COLS) <= TMEM_COLS ? 2 : 1;
   static constexpr uint32_t TM_SFA = ACC_BUFS * BN;        // 16 columns per stage
   static constexpr uint32_t TM_SFB = TM_SFA + STAGES * 16;
-  static constexpr uint32_t IDESC = idesc_nvf4(BN);
+  static constexpr uint32_t IDESC = idesc_nvf4(BN, 128 * CTAS);
   static_assert(STAGE_BYTES % 1024 == 0, "stages must keep 1024-byte alignment (128B swizzle)");
   static_assert(TM_SFB + STAGES * SFB_COLS <= TMEM_COLS, "tensor memory budget");
 };
@@ -114,6 +119,9 @@ struct Tile {
   int e, m0, nt;
 };
 
+// Tile t -> (expert, first row, N-tile).  Each expert's segment gives ceil(rows / (128*CTAS))
+// M-tiles of 128*CTAS rows.
+template <int CTAS>
 __device__ __forceinline__ Tile decode_tile(int t, const int* tile_start, const int* seg, int E,
                                             int n_tiles) {
   int lo = 0, hi = E;  // tile_start[lo] <= t < tile_start[hi]
@@ -123,26 +131,28 @@ __device__ __forceinline__ Tile decode_tile(int t, const int* tile_start, const 
     else hi = mid;
   }
   const int local = t - tile_start[lo];
-  const int mt_cnt = (seg[lo + 1] - seg[lo]) >> 7;
+  const int mt_cnt = (((seg[lo + 1] - seg[lo]) >> 7) + CTAS - 1) / CTAS;
   Tile r;
   r.e = lo;
   r.nt = local / mt_cnt;
-  r.m0 = seg[lo] + (local - r.nt * mt_cnt) * BM;
+  r.m0 = seg[lo] + (local - r.nt * mt_cnt) * (BM * CTAS);
   return r;
 }
 
-template <int MODE>
+template <int MODE, int CTAS>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_a,
                         const __grid_constant__ CUtensorMap tm_b, const GemmArgs args) {
-  using C = TileCfg<MODE>;
+  using C = TileCfg<MODE, CTAS>;
   constexpr int STAGES = C::STAGES;
   constexpr int BN = C::BN;
   constexpr int ACC_BUFS = C::ACC_BUFS;
+  constexpr bool PAIR = CTAS == 2;
   extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t bar_full[STAGES];
-  __shared__ __align__(8) uint64_t bar_empty[STAGES];
-  __shared__ __align__(8) uint64_t bar_sf[STAGES];
+  __shared__ __align__(8) uint64_t bar_full[STAGES];   // A/B landed (a pair: both CTAs')
+  __shared__ __align__(8) uint64_t bar_empty[STAGES];  // MMAs done with the stage
+  __shared__ __align__(8) uint64_t bar_sf[STAGES];     // scales in tensor memory (all CTAs)
+  __shared__ __align__(8) uint64_t bar_sfin[STAGES];   // this CTA's scale atoms landed
   __shared__ __align__(8) uint64_t bar_acc_full[ACC_BUFS];
   __shared__ __align__(8) uint64_t bar_acc_empty[ACC_BUFS];
   __shared__ __align__(8) uint64_t bar_drain;
@@ -157,6 +167,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                                              ~static_cast<uintptr_t>(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int E = args.E;
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;  // 0 = leader
+  const int cluster_id = blockIdx.x / CTAS, num_clusters = gridDim.x / CTAS;
+  // shared::cluster address of this CTA's barrier `bar` in the leader / in the other CTA
+  auto at_leader = [&](const uint64_t* bar) {
+    return PAIR ? mapa_shared(smem_u32(bar), 0u) : smem_u32(bar);
+  };
+  auto at_peer = [&](const uint64_t* bar) { return mapa_shared(smem_u32(bar), rank ^ 1u); };
 
   // ---- scheduler table: tiles per expert, exclusive scan over experts
   if (tid == 0) {
@@ -169,7 +186,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (tid < E) {
     const int lo = seg[tid], hi = seg[tid + 1];
     if (lo < 0 || hi < lo || (lo & 127) || (hi & 127) || hi > args.R_max) bad_offsets = 1;
-    else my_tiles = ((hi - lo) >> 7) * args.n_tiles;
+    else my_tiles = ((((hi - lo) >> 7) + CTAS - 1) / CTAS) * args.n_tiles;
   }
   int incl = my_tiles;
 #pragma unroll
@@ -197,21 +214,28 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(smem_u32(&bar_full[s]), 1);
       mbar_init(smem_u32(&bar_empty[s]), 1);
-      mbar_init(smem_u32(&bar_sf[s]), 4);
+      mbar_init(smem_u32(&bar_sf[s]), 4 * CTAS);
+      mbar_init(smem_u32(&bar_sfin[s]), 1);
     }
     for (int b = 0; b < ACC_BUFS; ++b) {
       mbar_init(smem_u32(&bar_acc_full[b]), 1);
-      mbar_init(smem_u32(&bar_acc_empty[b]), EPI_WARPS);
+      mbar_init(smem_u32(&bar_acc_empty[b]), EPI_WARPS * CTAS);
     }
     mbar_init(smem_u32(&bar_drain), 1);
     fence_mbar_init();
   }
   if (warp == 2) {
-    tmem_alloc(smem_u32(&tmem_slot), TMEM_COLS);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc_pair(smem_u32(&tmem_slot), TMEM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(smem_u32(&tmem_slot), TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
   __syncthreads();
+  if constexpr (PAIR) cluster_sync();  // the peer's barriers are initialised before any remote use
   tc_fence_after();
   const uint32_t tmem = tmem_slot;
   const int total = bad_offsets ? 0 : tile_start[E];
@@ -228,10 +252,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       prefetch_tmap(&tm_b);
       uint32_t it = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-        const Tile tl = decode_tile(t, tile_start, seg, E, args.n_tiles);
+      for (int t = cluster_id; t < total && ok; t += num_clusters) {
+        const Tile tl = decode_tile<CTAS>(t, tile_start, seg, E, args.n_tiles);
+        const int m_cta = tl.m0 + BM * rank;  // this CTA's rows
+        // a pair's second half past the expert's segment computes rows it never writes; its
+        // scale atoms are taken from the first half so that every read stays inside the tensor
+        const int a_blk = (m_cta < seg[tl.e + 1] ? m_cta : tl.m0) >> 7;
         // B rows of this N-tile: BN consecutive rows (for L1: 16-row gate blocks each followed by
-        // the 16 matching up rows)
+        // the 16 matching up rows); a pair's CTA r loads rows B_ROWS*r .. B_ROWS*r + B_ROWS-1
         const int b_row0 = tl.e * args.N + tl.nt * BN;
         for (int kb = 0; kb < nk; ++kb, ++it) {
           const int s = it % STAGES;
@@ -241,19 +269,32 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             break;
           }
           const int natoms = min(4, atoms_k - kb * 4);
-          const uint32_t full = smem_u32(&bar_full[s]);
           uint8_t* st = smem + s * C::STAGE_BYTES;
           const uint32_t sA = smem_u32(st), sB = sA + A_BYTES, sSFA = sB + C::B_BYTES,
                          sSFB = sSFA + SFA_BYTES;
-          mbar_arrive_expect_tx(full, A_BYTES + C::B_BYTES + natoms * 512 * (1 + BN / 128));
-          tma_load_2d(sA, &tm_a, full, kb * BK_BYTES, tl.m0);
-          const int64_t a_atom = (int64_t)(tl.m0 >> 7) * atoms_k + kb * 4;
-          bulk_load(sSFA, args.sfa + a_atom * 512, natoms * 512, full);
+          // the scales first, on their own barrier: the scale-factor warps move them to tensor
+          // memory while the A/B boxes are still in flight
+          const uint32_t sf_bar = smem_u32(&bar_sfin[s]);
+          mbar_arrive_expect_tx(sf_bar, natoms * 512 * (1 + BN / 128));
+          bulk_load(sSFA, args.sfa + ((int64_t)a_blk * atoms_k + kb * 4) * 512, natoms * 512,
+                    sf_bar);
 #pragma unroll
           for (int j = 0; j < BN / 128; ++j) {
-            tma_load_2d(sB + j * 128 * BK_BYTES, &tm_b, full, kb * BK_BYTES, b_row0 + 128 * j);
             const int64_t b_atom = (int64_t)((b_row0 >> 7) + j) * atoms_k + kb * 4;
-            bulk_load(sSFB + j * 4 * 512, args.sfb + b_atom * 512, natoms * 512, full);
+            bulk_load(sSFB + j * 4 * 512, args.sfb + b_atom * 512, natoms * 512, sf_bar);
+          }
+          if constexpr (PAIR) {
+            const uint32_t full = at_leader(&bar_full[s]);
+            if (rank == 0) mbar_arrive_expect_tx(smem_u32(&bar_full[s]), 2 * (A_BYTES + C::B_BYTES));
+            tma_load_2d_pair(sA, &tm_a, full, kb * BK_BYTES, m_cta);
+            tma_load_2d_pair(sB, &tm_b, full, kb * BK_BYTES, b_row0 + C::B_ROWS * (int)rank);
+          } else {
+            const uint32_t full = smem_u32(&bar_full[s]);
+            mbar_arrive_expect_tx(full, A_BYTES + C::B_BYTES);
+            tma_load_2d(sA, &tm_a, full, kb * BK_BYTES, m_cta);
+#pragma unroll
+            for (int j = 0; j < BN / 128; ++j)
+              tma_load_2d(sB + j * 128 * BK_BYTES, &tm_b, full, kb * BK_BYTES, b_row0 + 128 * j);
           }
         }
       }
@@ -261,15 +302,26 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // let the copies already issued land before the CTA can exit
         volatile int never = 0;
         const uint32_t first = it > (uint32_t)STAGES ? it - STAGES : 0u;
-        for (uint32_t j = first; j < it; ++j)
-          mbar_wait_bounded(smem_u32(&bar_full[j % STAGES]), (j / STAGES) & 1u, &never,
+        for (uint32_t j = first; j < it; ++j) {
+          mbar_wait_bounded(smem_u32(&bar_sfin[j % STAGES]), (j / STAGES) & 1u, &never,
                             NVFP4_WAIT_TIMEOUT_NS / 4);
+          if (!PAIR)
+            mbar_wait_bounded(smem_u32(&bar_full[j % STAGES]), (j / STAGES) & 1u, &never,
+                              NVFP4_WAIT_TIMEOUT_NS / 4);
+        }
+        if (PAIR) {  // this CTA's A/B boxes complete on the leader's barrier: give them time
+          const uint64_t t0 = global_timer_ns();
+          while (global_timer_ns() - t0 < 2000000ull) {
+          }
+        }
       }
     }
     __syncwarp();
   } else if (warp == 1) {
-    // =========================== MMA issuer ===========================
-    if (lane == 0) {
+    // =========================== MMA issuer (the leader's, for a pair) ===========================
+    // The whole warp runs the loop; elect.sync picks the issuing lane.  Waits are agreed across
+    // the warp so that every lane leaves the loop together.
+    if (rank == 0) {
       // Descriptors of stage 0; stage s adds s * STAGE_BYTES / 16 to the start-address field
       // (bits [0,14) hold address >> 4, and every stage address fits, so the add never carries).
       const uint32_t s0 = smem_u32(smem);
@@ -277,10 +329,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const uint64_t b_desc0 = smem_desc(s0 + A_BYTES, 16, 1024, 2);
       uint32_t it = 0, tile_it = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++tile_it) {
+      auto mma = [&](uint32_t d, uint64_t ad, uint64_t bd, uint32_t sfa, uint32_t sfb,
+                     uint32_t acc) {
+        if constexpr (PAIR) tc_mma_nvf4_pair_warp(d, ad, bd, C::IDESC, sfa, sfb, acc);
+        else tc_mma_nvf4_warp(d, ad, bd, C::IDESC, sfa, sfb, acc);
+      };
+      auto commit_all = [&](const uint64_t* bar) {  // arrive on `bar` of every CTA
+        if constexpr (PAIR) {
+          tc_commit_pair_warp(smem_u32(bar));
+          tc_commit_pair_warp(at_peer(bar));
+        } else {
+          tc_commit_warp(smem_u32(bar));
+        }
+      };
+      auto wait_all = [&](const uint64_t* bar, uint32_t parity) {
+        return __all_sync(0xffffffffu, mbar_wait_bounded(smem_u32(bar), parity, &abort_flag));
+      };
+      for (int t = cluster_id; t < total && ok; t += num_clusters, ++tile_it) {
         const int b = tile_it % ACC_BUFS;
-        if (!mbar_wait_bounded(smem_u32(&bar_acc_empty[b]), ((tile_it / ACC_BUFS) & 1u) ^ 1u,
-                               &abort_flag)) {
+        if (!wait_all(&bar_acc_empty[b], ((tile_it / ACC_BUFS) & 1u) ^ 1u)) {
           ok = false;
           break;
         }
@@ -289,8 +356,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int kb = 0; kb < nk; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1u;
-          if (!mbar_wait_bounded(smem_u32(&bar_full[s]), ph, &abort_flag) ||
-              !mbar_wait_bounded(smem_u32(&bar_sf[s]), ph, &abort_flag)) {
+          if (!wait_all(&bar_full[s], ph) || !wait_all(&bar_sf[s], ph)) {
             ok = false;
             break;
           }
@@ -304,20 +370,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if (natoms == 4) {
 #pragma unroll
             for (int a = 0; a < 4; ++a)
-              tc_mma_nvf4(d_tmem, a_desc0 + so + 2 * a, b_desc0 + so + 2 * a, C::IDESC,
-                          t_sfa + a * 4, t_sfb + a * (BN / 32), a == 0 ? first : 1u);
+              mma(d_tmem, a_desc0 + so + 2 * a, b_desc0 + so + 2 * a, t_sfa + a * 4,
+                  t_sfb + a * (BN / 32), a == 0 ? first : 1u);
           } else {
             for (int a = 0; a < natoms; ++a)
-              tc_mma_nvf4(d_tmem, a_desc0 + so + 2 * a, b_desc0 + so + 2 * a, C::IDESC,
-                          t_sfa + a * 4, t_sfb + a * (BN / 32), a == 0 ? first : 1u);
+              mma(d_tmem, a_desc0 + so + 2 * a, b_desc0 + so + 2 * a, t_sfa + a * 4,
+                  t_sfb + a * (BN / 32), a == 0 ? first : 1u);
           }
-          tc_commit(smem_u32(&bar_empty[s]));
+          commit_all(&bar_empty[s]);
         }
         if (!ok) break;
-        tc_commit(smem_u32(&bar_acc_full[b]));
+        commit_all(&bar_acc_full[b]);
       }
-      // all MMAs issued by this thread complete before the CTA frees tensor memory
-      tc_commit(smem_u32(&bar_drain));
+      // all MMAs issued by this warp complete before tensor memory is freed
+      if constexpr (PAIR) tc_commit_pair_warp(smem_u32(&bar_drain));
+      else tc_commit_warp(smem_u32(&bar_drain));
       volatile int never = 0;
       mbar_wait_bounded(smem_u32(&bar_drain), 0, &never);
     }
@@ -328,24 +395,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     uint32_t it = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+    for (int t = cluster_id; t < total && ok; t += num_clusters) {
       for (int kb = 0; kb < nk; ++kb, ++it) {
         const int s = it % STAGES;
         const uint32_t ph = (it / STAGES) & 1u;
-        if (!mbar_wait_bounded(smem_u32(&bar_full[s]), ph, &abort_flag)) {
+        if (!mbar_wait_bounded(smem_u32(&bar_sfin[s]), ph, &abort_flag)) {
           ok = false;
           break;
         }
         const uint8_t* st = smem + s * C::STAGE_BYTES + A_BYTES + C::B_BYTES;
         sf_rows128_to_tmem(tmem + lane_base + C::TM_SFA + s * 16, st, lane);
-        if (BN == 256)
-          sf_rows256_to_tmem(tmem + lane_base + C::TM_SFB + s * C::SFB_COLS, st + SFA_BYTES, lane);
-        else
-          sf_rows128_to_tmem(tmem + lane_base + C::TM_SFB + s * C::SFB_COLS, st + SFA_BYTES, lane);
+        sf_rows256_to_tmem(tmem + lane_base + C::TM_SFB + s * C::SFB_COLS, st + SFA_BYTES, lane);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&bar_sf[s]));
+        if (lane == 0) {
+          if constexpr (PAIR) mbar_arrive_cluster(at_leader(&bar_sf[s]));
+          else mbar_arrive(smem_u32(&bar_sf[s]));
+        }
       }
     }
   } else if (warp >= EPI_WARP0) {
@@ -355,22 +422,33 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int q = warp & 3;
     const int half = (warp - EPI_WARP0) >> 2;
     uint32_t tile_it = 0;
-    for (int t = blockIdx.x; t < total; t += gridDim.x, ++tile_it) {
-      const Tile tl = decode_tile(t, tile_start, seg, E, args.n_tiles);
+    for (int t = cluster_id; t < total; t += num_clusters, ++tile_it) {
+      const Tile tl = decode_tile<CTAS>(t, tile_start, seg, E, args.n_tiles);
       const int b = tile_it % ACC_BUFS;
       if (!mbar_wait_bounded(smem_u32(&bar_acc_full[b]), (tile_it / ACC_BUFS) & 1u, &abort_flag))
         break;
       tc_fence_after();
+      const int m_cta = tl.m0 + BM * rank;
+      const bool rows_valid = m_cta < seg[tl.e + 1];  // false: a pair's half past the segment
       const uint32_t t_row = tmem + b * BN + (static_cast<uint32_t>(q * 32) << 16);
       const float alpha = 1.0f / (__ldg(args.gs_a) * __ldg(args.gs_b + tl.e));
-      const int64_t row = tl.m0 + q * 32 + lane;
+      const int64_t row = m_cta + q * 32 + lane;
       // rows of the row map that are padding produce nothing; skip groups of 32 of them
-      int slot = 0;
+      int slot = rows_valid ? 0 : -1;
       if (MODE == L1_SWIGLU || MODE == L2_DIRECT || MODE == L2_STAGED) {
-        if (args.row_slot != nullptr) slot = __ldg(args.row_slot + row);
+        if (rows_valid && args.row_slot != nullptr) slot = __ldg(args.row_slot + row);
       }
       const bool live = __any_sync(0xffffffffu, slot >= 0);
       bool released = false;  // accumulator buffer b handed back to the MMA warp
+      auto release = [&] {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          if constexpr (PAIR) mbar_arrive_cluster(at_leader(&bar_acc_empty[b]));
+          else mbar_arrive(smem_u32(&bar_acc_empty[b]));
+        }
+        released = true;
+      };
 
       if (MODE == L1_SWIGLU) {
         if (live) {
@@ -397,15 +475,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             }
             uint32_t packed[4];
 #pragma unroll
-            for (int b = 0; b < 2; ++b) {
+            for (int bb = 0; bb < 2; ++bb) {
               float amax = 0.0f;
 #pragma unroll
-              for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(hv[16 * b + i]));
+              for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(hv[16 * bb + i]));
               float rcp;
               const uint32_t sb = nvfp4_block_scale(amax, gs_h, rcp);
-              packed[2 * b] = nvfp4_pack8(hv + 16 * b, rcp);
-              packed[2 * b + 1] = nvfp4_pack8(hv + 16 * b + 8, rcp);
-              const int sc = 2 * c + b;  // scale column inside the tile (0..7)
+              packed[2 * bb] = nvfp4_pack8(hv + 16 * bb, rcp);
+              packed[2 * bb + 1] = nvfp4_pack8(hv + 16 * bb + 8, rcp);
+              const int sc = 2 * c + bb;  // scale column inside the tile (0..7)
               sfw |= sb << (8 * (sc & 3));
             }
             *reinterpret_cast<uint4*>(hrow + 16 * c) =
@@ -440,12 +518,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               uint32_t v[32];
               tmem_ld32(t_row + 32 * c, v);
               tmem_wait_ld();
-              if (c == c_hi - 1) {  // last read of this tile's accumulator: hand it back now
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(smem_u32(&bar_acc_empty[b]));
-                released = true;
-              }
+              if (c == c_hi - 1) release();  // last read of the accumulator: hand it back now
 #pragma unroll
               for (int j = 0; j < 8; ++j)
                 stg[lane * 8 + (j ^ (lane & 7))] = make_float4(
@@ -480,7 +553,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             }
           }
         }
-      } else {
+      } else if (rows_valid) {
         const int N = args.N;
 #pragma unroll 1
         for (int c = (BN / 64) * half; c < (BN / 64) * (half + 1); ++c) {
@@ -513,19 +586,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
         }
       }
-      if (!released) {
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&bar_acc_empty[b]));
-      }
+      if (!released) release();
     }
   }
 
   __syncwarp();
   tc_fence_before();
   __syncthreads();
+  // a pair: the leader's MMAs (which write both CTAs' tensor memory) are drained and no remote
+  // arrival or copy is still headed for the other CTA before either frees or exits
+  if constexpr (PAIR) cluster_sync();
   tc_fence_after();
-  if (warp == 2) tmem_dealloc(tmem, TMEM_COLS);
+  if (warp == 2) {
+    if constexpr (PAIR) tmem_dealloc_pair(tmem, TMEM_COLS);
+    else tmem_dealloc(tmem, TMEM_COLS);
+  }
   if (tid == 0 && abort_flag) report(args.status, NVFP4_DEVERR_TIMEOUT);
 }
 
@@ -567,6 +642,47 @@ int num_sms() {
   return n > 0 ? n : 148;
 }
 
+// Pair tiles (CTAS = 2) from this many 128-row blocks of capacity per expert on average.  A pair
+// tile covers 256 rows, so an expert with an odd number of blocks computes a half tile that
+// nobody writes; with ~2.5 blocks per expert that waste (about 20%) outweighs the pair's smaller
+// operand traffic, with 16 blocks per expert the pair is ahead.
+constexpr int kPairMinBlocksPerExpert = 8;
+
+template <int MODE, int CTAS>
+nvfp4_status_t launch_cfg(const CUtensorMap& ma, const CUtensorMap& mb, const GemmArgs& args,
+                          cudaStream_t s) {
+  constexpr int smem = TileCfg<MODE, CTAS>::SMEM_BYTES;
+  auto kernel = grouped_gemm_kernel<MODE, CTAS>;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+      cudaSuccess)
+    return check_launch("cudaFuncSetAttribute");
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  cfg.blockDim = dim3(NUM_THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  if (CTAS == 1) {
+    cfg.gridDim = dim3(num_sms());
+  } else {
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = CTAS;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cfg.gridDim = dim3(num_sms());
+    int clusters = 0;  // persistent: as many pairs as can be resident at once
+    if (cudaOccupancyMaxActiveClusters(&clusters, kernel, &cfg) != cudaSuccess || clusters <= 0) {
+      (void)cudaGetLastError();
+      clusters = num_sms() / CTAS;
+    }
+    cfg.gridDim = dim3(clusters * CTAS);
+  }
+  if (cudaLaunchKernelEx(&cfg, kernel, ma, mb, args) != cudaSuccess)
+    return check_launch("grouped_gemm_kernel");
+  return check_launch("grouped_gemm_kernel");
+}
+
 template <int MODE>
 nvfp4_status_t launch(const uint8_t* a, const uint8_t* b, int64_t b_rows, GemmArgs args,
                       cudaStream_t s) {
@@ -575,12 +691,8 @@ nvfp4_status_t launch(const uint8_t* a, const uint8_t* b, int64_t b_rows, GemmAr
     set_last_error("cuTensorMapEncodeTiled failed");
     return NVFP4_ERR_CUDA;
   }
-  constexpr int smem = TileCfg<MODE>::SMEM_BYTES;
-  if (cudaFuncSetAttribute(grouped_gemm_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           smem) != cudaSuccess)
-    return check_launch("cudaFuncSetAttribute");
-  grouped_gemm_kernel<MODE><<<num_sms(), NUM_THREADS, smem, s>>>(ma, mb, args);
-  return check_launch("grouped_gemm_kernel");
+  const bool pair = args.R_max >= (int64_t)kPairMinBlocksPerExpert * BM * args.E;
+  return pair ? launch_cfg<MODE, 2>(ma, mb, args, s) : launch_cfg<MODE, 1>(ma, mb, args, s);
 }
 
 // out[t] = sum over the token's slots j (in order, skipping dropped ones) of ys[t*k + j]; FP32
@@ -630,7 +742,7 @@ nvfp4_status_t gemm_plain(const uint8_t* a, const uint8_t* sfa, const float* gs_
                           cudaStream_t s) {
   GemmArgs g{};
   g.sfa = sfa; g.sfb = sfb; g.gs_a = gs_a; g.gs_b = gs_b; g.offs = offs;
-  g.E = E; g.N = N; g.K = K; g.n_tiles = N / TileCfg<PLAIN_F32>::BN; g.R_max = R_max; g.out = out;
+  g.E = E; g.N = N; g.K = K; g.n_tiles = N / TileCfg<PLAIN_F32, 1>::BN; g.R_max = R_max; g.out = out;
   g.status = status;
   const int64_t b_rows = (int64_t)E * N;
   return out_dtype == 0 ? launch<PLAIN_F32>(a, b, b_rows, g, s) : launch<PLAIN_BF16>(a, b, b_rows, g, s);
@@ -656,7 +768,7 @@ nvfp4_status_t gemm_l2(const uint8_t* h, const uint8_t* sfh, const float* gs_h, 
   if (T == 0) return NVFP4_OK;
   GemmArgs g{};
   g.sfa = sfh; g.sfb = sfw2; g.gs_a = gs_h; g.gs_b = gs_w2; g.offs = offs;
-  g.E = E; g.N = H; g.K = I; g.R_max = R_max; g.n_tiles = H / TileCfg<L2_DIRECT>::BN;
+  g.E = E; g.N = H; g.K = I; g.R_max = R_max; g.n_tiles = H / TileCfg<L2_DIRECT, 1>::BN;
   g.row_slot = row_slot; g.row_w = row_w; g.ys = ys; g.S = T * k; g.status = status;
   const bool staged = (int64_t)T * k >= (int64_t)kL2StagedMinRowsPerExpert * E;
   nvfp4_status_t st = staged ? launch<L2_STAGED>(h, w2, (int64_t)E * H, g, s)
@@ -680,7 +792,7 @@ extern "C" nvfp4_status_t nvfp4_grouped_gemm(const uint8_t* a, const uint8_t* sf
                                              int64_t R_max, void* out, int out_dtype,
                                              int32_t* dev_status, nvfp4_stream_t stream) {
   if (E < 1 || E > MAX_E || N <= 0 || K <= 0 || R_max < 0) return NVFP4_ERR_INVALID_ARG;
-  if (K % 64 || N % TileCfg<PLAIN_F32>::BN || R_max % 128) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (K % 64 || N % TileCfg<PLAIN_F32, 1>::BN || R_max % 128) return NVFP4_ERR_UNSUPPORTED_SHAPE;
   if (out_dtype != 0 && out_dtype != 1) return NVFP4_ERR_INVALID_ARG;
   if (!gs_a || !gs_b || !offs) return NVFP4_ERR_INVALID_ARG;
   if (R_max == 0) return NVFP4_OK;
@@ -713,7 +825,7 @@ extern "C" nvfp4_status_t moe_grouped_gemm_l2_scatter(
     float* ys_ws, float* out_f32, void* out_bf16, int32_t* dev_status, nvfp4_stream_t stream) {
   if (E < 1 || E > MAX_E || H <= 0 || I <= 0 || T < 0 || k < 1 || R_max < 0)
     return NVFP4_ERR_INVALID_ARG;
-  if (H % TileCfg<L2_DIRECT>::BN || I % 64 || R_max % 128) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (H % TileCfg<L2_DIRECT, 1>::BN || I % 64 || R_max % 128) return NVFP4_ERR_UNSUPPORTED_SHAPE;
   if (!gs_h || !gs_w2 || !offs || !row_slot || !row_w || !dst_row || (!out_f32 && !out_bf16))
     return NVFP4_ERR_INVALID_ARG;
   if (T == 0 || R_max == 0) return NVFP4_OK;
@@ -762,7 +874,7 @@ extern "C" nvfp4_status_t moe_grouped_gemm_l2_scatter_noalloc(
     void* out_bf16, int32_t* dev_status, nvfp4_stream_t stream) {
   if (E < 1 || E > MAX_E || H <= 0 || I <= 0 || T < 0 || k < 1 || R_max < 0)
     return NVFP4_ERR_INVALID_ARG;
-  if (H % TileCfg<L2_DIRECT>::BN || I % 64 || R_max % 128) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (H % TileCfg<L2_DIRECT, 1>::BN || I % 64 || R_max % 128) return NVFP4_ERR_UNSUPPORTED_SHAPE;
   if (!gs_h || !gs_w2 || !offs || !row_slot || !row_w || !dst_row || !out_bf16)
     return NVFP4_ERR_INVALID_ARG;
   if ((int64_t)T * k * H > NVFP4_L2_NOALLOC_MAX_ELEMS) {

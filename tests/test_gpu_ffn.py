@@ -109,3 +109,16 @@ def test_ffn_small_batch_end_to_end(T):
     want = M.bf16_round(ref["out"])
     assert rel_fro(got, want) <= 1e-3
     assert cosine(got, want) >= 0.9999
+
+
+@pytest.mark.parametrize("T", [640, 4096])
+def test_ffn_prefill_sized_batch_end_to_end(T):
+    """160 / 1024 rows per expert on average: the L2 epilogue stages its rows through shared
+    memory; at 1024 both GEMMs also take 256-row tiles on CTA pairs."""
+    from dataclasses import replace
+    cfg = replace(CONFIGS["tiny"], T=T)
+    assert nv.rows_max(cfg.T, cfg.E, cfg.k) >= (1024 if T == 4096 else 256) * cfg.E
+    got, ref = _ffn_check(cfg, gen_x(cfg), gen_logits(cfg))
+    want = M.bf16_round(ref["out"])
+    assert rel_fro(got, want) <= 1e-3
+    assert cosine(got, want) >= 0.9999

@@ -78,6 +78,25 @@ def test_grouped_gemm_full_k_and_n():
     assert rel_fro(out.cpu().numpy()[rows], ref[rows]) <= 1e-5
 
 
+@pytest.mark.parametrize("m_sizes,K", [([1100, 0, 2200], 320), ([1153, 900], 1024)])
+def test_grouped_gemm_pair_tiles(m_sizes, K):
+    """Enough rows per group for 256-row tiles on CTA pairs: groups with an odd number of
+    128-row blocks (the pair's second half past the group, for the last group past the end of A),
+    an empty group, a partial last K stage, two N-tiles."""
+    E = len(m_sizes)
+    a, asf, gs_a, w, offs_d, ref, offs = _problem(11 + K, E, 512, K, m_sizes)
+    assert offs[-1] >= 1024 * E  # the library's pair-tile rule
+    out = torch.full((int(offs[-1]), 512), 7.0, dtype=torch.float32, device=DEV)
+    nv.grouped_gemm(a, asf, gs_a, w, offs_d, out_dtype=torch.float32, out=out)
+    torch.cuda.synchronize()
+    rows = _valid_rows(offs, m_sizes)
+    got = out.cpu().numpy()
+    assert rel_fro(got[rows], ref[rows]) <= 1e-5
+    # every row of every segment is written (padding rows of A are zero -> zero output)
+    pad = np.setdiff1d(np.arange(offs[-1]), rows)
+    assert np.all(got[pad] == 0)
+
+
 def test_grouped_gemm_rejects_bad_shapes():
     z = torch.zeros(256, dtype=torch.uint8, device=DEV)
     f = torch.ones(4, dtype=torch.float32, device=DEV)

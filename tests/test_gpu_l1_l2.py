@@ -45,7 +45,11 @@ def _setup(T, H, I, E, k, seed=0, drop=0.0):
     (64, 256, 128, 8, 2), (200, 512, 256, 6, 3), (33, 7168, 2048, 2, 2), (96, 256, 128, 256, 8),
     # decode-like batches (few tokens per expert)
     (16, 256, 128, 8, 2), (32, 512, 256, 6, 3), (20, 7168, 2048, 3, 2), (16, 256, 128, 256, 8),
-    (1, 256, 128, 4, 1)])
+    (1, 256, 128, 4, 1),
+    # 128+ rows per expert (the L2 epilogue staged through shared memory)
+    (640, 256, 128, 4, 2), (640, 1024, 512, 2, 1),
+    # 1024+ rows per expert: 256-row tiles on CTA pairs (odd block counts: half-empty pair tiles)
+    (2304, 256, 128, 2, 1)])
 def test_l1_and_l2_match_oracle(T, H, I, E, k):
     x, ids, w32, w1, w1d, w2, w2d = _setup(T, H, I, E, k, drop=0.1)
     gs_h = np.float32(64.0 if H <= 512 else 1.0)
