@@ -64,6 +64,15 @@ enum Mode { PLAIN_F32 = 0, PLAIN_BF16 = 1, L1_SWIGLU = 2, L2_DIRECT = 3, L2_STAG
 // Average routed rows per expert from which the L2 epilogue stages its output
 constexpr int kL2StagedMinRowsPerExpert = 32;
 
+// Tile width (N) per epilogue.  256 columns fill tensor memory with one accumulator; 128 leave
+// room for two, so the epilogue of one tile overlaps the MMAs of the next.
+constexpr int kL1TileN = 256;
+constexpr int kL2TileN = 256;
+template <int MODE>
+constexpr int tile_n() {
+  return MODE == L1_SWIGLU ? kL1TileN : (MODE == L2_DIRECT || MODE == L2_STAGED) ? kL2TileN : 256;
+}
+
 // Tile shape: M = 128 rows per CTA, N = 256 columns, K = 256 per stage.  One MMA instruction
 // has a fixed cost, so the widest N moves the most weight bytes per instruction; one 256-column
 // accumulator and the per-stage scale columns fill tensor memory.
@@ -74,7 +83,9 @@ constexpr int kL2StagedMinRowsPerExpert = 32;
 // both CTAs run producer, scale-factor and epilogue warps.
 template <int MODE, int CTAS>
 struct TileCfg {
-  static constexpr int BN = 256;
+  static constexpr int BN = tile_n<MODE>();
+  static_assert(BN == 128 || BN == 256, "tile width");
+  static_assert(CTAS == 1 || BN == 256, "pair tiles are 256 columns wide");
   static constexpr int B_ROWS = BN / CTAS;                 // B rows (N) per CTA per stage
   static constexpr int B_BYTES = B_ROWS * BK_BYTES;
   static constexpr int SFB_BYTES = (BN / 128) * 4 * 512;   // scales of all BN rows of B
@@ -405,7 +416,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         const uint8_t* st = smem + s * C::STAGE_BYTES + A_BYTES + C::B_BYTES;
         sf_rows128_to_tmem(tmem + lane_base + C::TM_SFA + s * 16, st, lane);
-        sf_rows256_to_tmem(tmem + lane_base + C::TM_SFB + s * C::SFB_COLS, st + SFA_BYTES, lane);
+        if constexpr (BN == 256)
+          sf_rows256_to_tmem(tmem + lane_base + C::TM_SFB + s * C::SFB_COLS, st + SFA_BYTES, lane);
+        else
+          sf_rows128_to_tmem(tmem + lane_base + C::TM_SFB + s * C::SFB_COLS, st + SFA_BYTES, lane);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
@@ -454,16 +468,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (live) {
           const float gs_h = __ldg(args.gs_h);
           const int I = args.I;
-          uint8_t* hrow = args.h + row * (I / 2) + tl.nt * 64;
+          constexpr int n_chunks = BN / 128;  // 64-column chunks per warp
+          uint8_t* hrow = args.h + row * (I / 2) + tl.nt * (BN / 4);
           uint32_t sfw = 0u;
 #pragma unroll 1
-          for (int c = 2 * half; c < 2 * half + 2; ++c) {
+          for (int cc = 0; cc < n_chunks; ++cc) {
             // h features 32c..32c+31 of the tile live in accumulator columns 64c..64c+63 as two
             // 32-column blocks, each 16 gate columns followed by the 16 matching up columns
+            const int c = half * n_chunks + cc;
             uint32_t v0[32], v1[32];
             tmem_ld32(t_row + 64 * c, v0);
             tmem_ld32(t_row + 64 * c + 32, v1);
             tmem_wait_ld();
+            // the accumulator's last columns of this warp are in registers: hand it back, so the
+            // next tile's MMAs overlap the rest of this epilogue
+            if (cc == n_chunks - 1) release();
             float hv[32];
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
@@ -483,15 +502,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               const uint32_t sb = nvfp4_block_scale(amax, gs_h, rcp);
               packed[2 * bb] = nvfp4_pack8(hv + 16 * bb, rcp);
               packed[2 * bb + 1] = nvfp4_pack8(hv + 16 * bb + 8, rcp);
-              const int sc = 2 * c + bb;  // scale column inside the tile (0..7)
-              sfw |= sb << (8 * (sc & 3));
+              sfw |= sb << (8 * (2 * cc + bb));  // this warp's scale columns, in order
             }
             *reinterpret_cast<uint4*>(hrow + 16 * c) =
                 make_uint4(packed[0], packed[1], packed[2], packed[3]);
           }
-          // this half's 4 scale columns are one 4-byte group of the tiled layout
-          *reinterpret_cast<uint32_t*>(args.sfh + sf_offset(row, tl.nt * 8 + 4 * half, I / 16)) =
-              sfw;
+          // this warp's 2 * n_chunks scale columns are consecutive bytes of one 4-byte group of
+          // the tiled layout
+          const int sc0 = tl.nt * (BN / 32) + half * (BN / 64);
+          uint8_t* sfp = args.sfh + sf_offset(row, sc0, I / 16);
+          if constexpr (n_chunks == 2) *reinterpret_cast<uint32_t*>(sfp) = sfw;
+          else *reinterpret_cast<uint16_t*>(sfp) = static_cast<uint16_t>(sfw);
         }
       } else if (MODE == L2_DIRECT || MODE == L2_STAGED) {
         // this row's weighted expert output goes to its slot's row of ys; the combine kernel sums
@@ -504,6 +525,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const float scale = alpha * (slot >= 0 ? __ldg(args.row_w + row) : 0.0f);
           const int H = args.N;
           const int c_lo = (BN / 64) * half, c_hi = c_lo + BN / 64;
+          // 32-column chunks are read from tensor memory two at a time; once the last two are in
+          // registers the accumulator goes back to the MMA warp
           if constexpr (MODE == L2_STAGED) {
             // each 32-column chunk passes through shared memory (16-byte units XOR-swizzled by
             // row) so that 8 lanes write one row's 128 contiguous bytes
@@ -513,12 +536,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             int sl[8];  // slot of row 4i + sub of this warp's 32 rows
 #pragma unroll
             for (int i = 0; i < 8; ++i) sl[i] = __shfl_sync(0xffffffffu, slot, 4 * i + sub);
-#pragma unroll 1
-            for (int c = c_lo; c < c_hi; ++c) {
-              uint32_t v[32];
-              tmem_ld32(t_row + 32 * c, v);
-              tmem_wait_ld();
-              if (c == c_hi - 1) release();  // last read of the accumulator: hand it back now
+            auto emit = [&](int c, const uint32_t (&v)[32]) {
 #pragma unroll
               for (int j = 0; j < 8; ++j)
                 stg[lane * 8 + (j ^ (lane & 7))] = make_float4(
@@ -533,33 +551,44 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 if (sl[i] >= 0) *reinterpret_cast<float4*>(args.ys + (int64_t)sl[i] * H + col) = val;
               }
               __syncwarp();
+            };
+#pragma unroll 1
+            for (int c = c_lo; c < c_hi; c += 2) {
+              uint32_t v0[32], v1[32];
+              tmem_ld32(t_row + 32 * c, v0);
+              tmem_ld32(t_row + 32 * (c + 1), v1);
+              tmem_wait_ld();
+              if (c + 2 >= c_hi) release();
+              emit(c, v0);
+              emit(c + 1, v1);
             }
           } else {
             float* dst = args.ys + (int64_t)(slot >= 0 ? slot : 0) * H + tl.nt * BN;
-#pragma unroll 1
-            for (int c = c_lo; c < c_hi; ++c) {
-              uint32_t v[32];
-              tmem_ld32(t_row + 32 * c, v);
-              tmem_wait_ld();
-              if (slot >= 0) {
-                float4* o = reinterpret_cast<float4*>(dst + 32 * c);
+            auto emit = [&](int c, const uint32_t (&v)[32]) {
+              if (slot < 0) return;
+              float4* o = reinterpret_cast<float4*>(dst + 32 * c);
 #pragma unroll
-                for (int i = 0; i < 8; ++i)
-                  o[i] = make_float4(__uint_as_float(v[4 * i]) * scale,
-                                     __uint_as_float(v[4 * i + 1]) * scale,
-                                     __uint_as_float(v[4 * i + 2]) * scale,
-                                     __uint_as_float(v[4 * i + 3]) * scale);
-              }
+              for (int i = 0; i < 8; ++i)
+                o[i] = make_float4(__uint_as_float(v[4 * i]) * scale,
+                                   __uint_as_float(v[4 * i + 1]) * scale,
+                                   __uint_as_float(v[4 * i + 2]) * scale,
+                                   __uint_as_float(v[4 * i + 3]) * scale);
+            };
+#pragma unroll 1
+            for (int c = c_lo; c < c_hi; c += 2) {
+              uint32_t v0[32], v1[32];
+              tmem_ld32(t_row + 32 * c, v0);
+              tmem_ld32(t_row + 32 * (c + 1), v1);
+              tmem_wait_ld();
+              if (c + 2 >= c_hi) release();
+              emit(c, v0);
+              emit(c + 1, v1);
             }
           }
         }
       } else if (rows_valid) {
         const int N = args.N;
-#pragma unroll 1
-        for (int c = (BN / 64) * half; c < (BN / 64) * (half + 1); ++c) {
-          uint32_t v[32];
-          tmem_ld32(t_row + 32 * c, v);
-          tmem_wait_ld();
+        auto emit = [&](int c, const uint32_t (&v)[32]) {
           const int64_t col = (int64_t)tl.nt * BN + 32 * c;
           if (MODE == PLAIN_F32) {
             float4* o = reinterpret_cast<float4*>(static_cast<float*>(args.out) + row * N + col);
@@ -584,6 +613,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               o[i] = make_uint4(wds[0], wds[1], wds[2], wds[3]);
             }
           }
+        };
+        const int c_lo = (BN / 64) * half, c_hi = c_lo + BN / 64;
+#pragma unroll 1
+        for (int c = c_lo; c < c_hi; c += 2) {
+          uint32_t v0[32], v1[32];
+          tmem_ld32(t_row + 32 * c, v0);
+          tmem_ld32(t_row + 32 * (c + 1), v1);
+          tmem_wait_ld();
+          if (c + 2 >= c_hi) release();
+          emit(c, v0);
+          emit(c + 1, v1);
         }
       }
       if (!released) release();
@@ -691,8 +731,11 @@ nvfp4_status_t launch(const uint8_t* a, const uint8_t* b, int64_t b_rows, GemmAr
     set_last_error("cuTensorMapEncodeTiled failed");
     return NVFP4_ERR_CUDA;
   }
-  const bool pair = args.R_max >= (int64_t)kPairMinBlocksPerExpert * BM * args.E;
-  return pair ? launch_cfg<MODE, 2>(ma, mb, args, s) : launch_cfg<MODE, 1>(ma, mb, args, s);
+  if constexpr (TileCfg<MODE, 1>::BN == 256) {
+    if (args.R_max >= (int64_t)kPairMinBlocksPerExpert * BM * args.E)
+      return launch_cfg<MODE, 2>(ma, mb, args, s);
+  }
+  return launch_cfg<MODE, 1>(ma, mb, args, s);
 }
 
 // out[t] = sum over the token's slots j (in order, skipping dropped ones) of ys[t*k + j]; FP32
@@ -755,7 +798,7 @@ nvfp4_status_t gemm_l1(const uint8_t* a, const uint8_t* sfa, const float* gs_a, 
                        cudaStream_t s) {
   GemmArgs g{};
   g.sfa = sfa; g.sfb = sfw1; g.gs_a = gs_a; g.gs_b = gs_w1; g.offs = offs;
-  g.E = E; g.N = 2 * I; g.K = H; g.n_tiles = I / 128; g.R_max = R_max;
+  g.E = E; g.N = 2 * I; g.K = H; g.n_tiles = 2 * I / TileCfg<L1_SWIGLU, 1>::BN; g.R_max = R_max;
   g.gs_h = gs_h; g.h = h; g.sfh = sfh; g.I = I; g.row_slot = row_slot; g.status = status;
   return launch<L1_SWIGLU>(a, w1, (int64_t)E * 2 * I, g, s);
 }
@@ -808,7 +851,8 @@ extern "C" nvfp4_status_t moe_grouped_gemm_l1_swiglu_q(
     int H, int I, int64_t R_max, const float* gs_h, uint8_t* h, uint8_t* sfh, int32_t* dev_status,
     nvfp4_stream_t stream) {
   if (E < 1 || E > MAX_E || H <= 0 || I <= 0 || R_max < 0) return NVFP4_ERR_INVALID_ARG;
-  if (H % 64 || I % 128 || R_max % 128) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (H % 64 || I % 64 || (2 * I) % TileCfg<L1_SWIGLU, 1>::BN || R_max % 128)
+    return NVFP4_ERR_UNSUPPORTED_SHAPE;
   if (!gs_a || !gs_w1 || !offs || !gs_h) return NVFP4_ERR_INVALID_ARG;
   if (R_max == 0) return NVFP4_OK;
   if (!ok_ptr(a) || !ok_ptr(sfa) || !ok_ptr(w1) || !ok_ptr(sfw1) || !ok_ptr(h) || !ok_ptr(sfh))
