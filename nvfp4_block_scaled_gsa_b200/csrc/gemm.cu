@@ -55,6 +55,11 @@ constexpr int NUM_THREADS = 512;  // 4 role warps + 8 epilogue warps + 4 scale-f
 constexpr int EPI_WARP0 = 4;
 constexpr int EPI_WARPS = 8;
 constexpr int SF_WARP0 = EPI_WARP0 + EPI_WARPS;
+// Register budgets per warpgroup (the block is launched with 128 per thread): the two epilogue
+// warpgroups hold a whole 128-column accumulator slice in registers; the producer / MMA group
+// and the scale-factor group need few.
+constexpr uint32_t REGS_EPI = 176, REGS_OTHER = 80;
+static_assert(2 * REGS_EPI + 2 * REGS_OTHER == 4 * 128, "register budgets exceed the launch's");
 constexpr int MAX_E = 256;
 
 // L2_DIRECT: each epilogue lane stores its own row (4 stages; suits a few rows per expert).
@@ -256,151 +261,158 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int nk = (K + 255) / 256;  // stages along K
   const int atoms_k = K / 64;      // 64-element scale atoms along K
 
-  if (warp == 0) {
-    // =========================== TMA producer ===========================
-    if (lane == 0) {
-      prefetch_tmap(&tm_a);
-      prefetch_tmap(&tm_b);
-      uint32_t it = 0;
-      bool ok = true;
-      for (int t = cluster_id; t < total && ok; t += num_clusters) {
-        const Tile tl = decode_tile<CTAS>(t, tile_start, seg, E, args.n_tiles);
-        const int m_cta = tl.m0 + BM * rank;  // this CTA's rows
-        // a pair's second half past the expert's segment computes rows it never writes; its
-        // scale atoms are taken from the first half so that every read stays inside the tensor
-        const int a_blk = (m_cta < seg[tl.e + 1] ? m_cta : tl.m0) >> 7;
-        // B rows of this N-tile: BN consecutive rows (for L1: 16-row gate blocks each followed by
-        // the 16 matching up rows); a pair's CTA r loads rows B_ROWS*r .. B_ROWS*r + B_ROWS-1
-        const int b_row0 = tl.e * args.N + tl.nt * BN;
-        for (int kb = 0; kb < nk; ++kb, ++it) {
-          const int s = it % STAGES;
-          const uint32_t ph = (it / STAGES) & 1u;
-          if (!mbar_wait_bounded(smem_u32(&bar_empty[s]), ph ^ 1u, &abort_flag)) {
-            ok = false;
-            break;
-          }
-          const int natoms = min(4, atoms_k - kb * 4);
-          uint8_t* st = smem + s * C::STAGE_BYTES;
-          const uint32_t sA = smem_u32(st), sB = sA + A_BYTES, sSFA = sB + C::B_BYTES,
-                         sSFB = sSFA + SFA_BYTES;
-          // the scales first, on their own barrier: the scale-factor warps move them to tensor
-          // memory while the A/B boxes are still in flight
-          const uint32_t sf_bar = smem_u32(&bar_sfin[s]);
-          mbar_arrive_expect_tx(sf_bar, natoms * 512 * (1 + BN / 128));
-          bulk_load(sSFA, args.sfa + ((int64_t)a_blk * atoms_k + kb * 4) * 512, natoms * 512,
-                    sf_bar);
-#pragma unroll
-          for (int j = 0; j < BN / 128; ++j) {
-            const int64_t b_atom = (int64_t)((b_row0 >> 7) + j) * atoms_k + kb * 4;
-            bulk_load(sSFB + j * 4 * 512, args.sfb + b_atom * 512, natoms * 512, sf_bar);
-          }
-          if constexpr (PAIR) {
-            const uint32_t full = at_leader(&bar_full[s]);
-            if (rank == 0) mbar_arrive_expect_tx(smem_u32(&bar_full[s]), 2 * (A_BYTES + C::B_BYTES));
-            tma_load_2d_pair(sA, &tm_a, full, kb * BK_BYTES, m_cta);
-            tma_load_2d_pair(sB, &tm_b, full, kb * BK_BYTES, b_row0 + C::B_ROWS * (int)rank);
-          } else {
-            const uint32_t full = smem_u32(&bar_full[s]);
-            mbar_arrive_expect_tx(full, A_BYTES + C::B_BYTES);
-            tma_load_2d(sA, &tm_a, full, kb * BK_BYTES, m_cta);
-#pragma unroll
-            for (int j = 0; j < BN / 128; ++j)
-              tma_load_2d(sB + j * 128 * BK_BYTES, &tm_b, full, kb * BK_BYTES, b_row0 + 128 * j);
+  // Roles by warpgroup (4 warps each).  setmaxnreg is executed by a whole warpgroup at the top
+  // of its own branch: warpgroups 0 (producer, MMA) and 3 (scale factors) give registers to
+  // warpgroups 1 and 2 (epilogue).
+  if (warp < EPI_WARP0) {
+    regs_release_to<REGS_OTHER>();
+    if (warp == 0) {
+      // =========================== TMA producer ===========================
+      if (lane == 0) {
+        prefetch_tmap(&tm_a);
+        prefetch_tmap(&tm_b);
+        uint32_t it = 0;
+        bool ok = true;
+        for (int t = cluster_id; t < total && ok; t += num_clusters) {
+          const Tile tl = decode_tile<CTAS>(t, tile_start, seg, E, args.n_tiles);
+          const int m_cta = tl.m0 + BM * rank;  // this CTA's rows
+          // a pair's second half past the expert's segment computes rows it never writes; its
+          // scale atoms are taken from the first half so that every read stays inside the tensor
+          const int a_blk = (m_cta < seg[tl.e + 1] ? m_cta : tl.m0) >> 7;
+          // B rows of this N-tile: BN consecutive rows (for L1: 16-row gate blocks each followed by
+          // the 16 matching up rows); a pair's CTA r loads rows B_ROWS*r .. B_ROWS*r + B_ROWS-1
+          const int b_row0 = tl.e * args.N + tl.nt * BN;
+          for (int kb = 0; kb < nk; ++kb, ++it) {
+            const int s = it % STAGES;
+            const uint32_t ph = (it / STAGES) & 1u;
+            if (!mbar_wait_bounded(smem_u32(&bar_empty[s]), ph ^ 1u, &abort_flag)) {
+              ok = false;
+              break;
+            }
+            const int natoms = min(4, atoms_k - kb * 4);
+            uint8_t* st = smem + s * C::STAGE_BYTES;
+            const uint32_t sA = smem_u32(st), sB = sA + A_BYTES, sSFA = sB + C::B_BYTES,
+                           sSFB = sSFA + SFA_BYTES;
+            // the scales first, on their own barrier: the scale-factor warps move them to tensor
+            // memory while the A/B boxes are still in flight
+            const uint32_t sf_bar = smem_u32(&bar_sfin[s]);
+            mbar_arrive_expect_tx(sf_bar, natoms * 512 * (1 + BN / 128));
+            bulk_load(sSFA, args.sfa + ((int64_t)a_blk * atoms_k + kb * 4) * 512, natoms * 512,
+                      sf_bar);
+  #pragma unroll
+            for (int j = 0; j < BN / 128; ++j) {
+              const int64_t b_atom = (int64_t)((b_row0 >> 7) + j) * atoms_k + kb * 4;
+              bulk_load(sSFB + j * 4 * 512, args.sfb + b_atom * 512, natoms * 512, sf_bar);
+            }
+            if constexpr (PAIR) {
+              const uint32_t full = at_leader(&bar_full[s]);
+              if (rank == 0) mbar_arrive_expect_tx(smem_u32(&bar_full[s]), 2 * (A_BYTES + C::B_BYTES));
+              tma_load_2d_pair(sA, &tm_a, full, kb * BK_BYTES, m_cta);
+              tma_load_2d_pair(sB, &tm_b, full, kb * BK_BYTES, b_row0 + C::B_ROWS * (int)rank);
+            } else {
+              const uint32_t full = smem_u32(&bar_full[s]);
+              mbar_arrive_expect_tx(full, A_BYTES + C::B_BYTES);
+              tma_load_2d(sA, &tm_a, full, kb * BK_BYTES, m_cta);
+  #pragma unroll
+              for (int j = 0; j < BN / 128; ++j)
+                tma_load_2d(sB + j * 128 * BK_BYTES, &tm_b, full, kb * BK_BYTES, b_row0 + 128 * j);
+            }
           }
         }
-      }
-      if (!ok) {
-        // let the copies already issued land before the CTA can exit
-        volatile int never = 0;
-        const uint32_t first = it > (uint32_t)STAGES ? it - STAGES : 0u;
-        for (uint32_t j = first; j < it; ++j) {
-          mbar_wait_bounded(smem_u32(&bar_sfin[j % STAGES]), (j / STAGES) & 1u, &never,
-                            NVFP4_WAIT_TIMEOUT_NS / 4);
-          if (!PAIR)
-            mbar_wait_bounded(smem_u32(&bar_full[j % STAGES]), (j / STAGES) & 1u, &never,
+        if (!ok) {
+          // let the copies already issued land before the CTA can exit
+          volatile int never = 0;
+          const uint32_t first = it > (uint32_t)STAGES ? it - STAGES : 0u;
+          for (uint32_t j = first; j < it; ++j) {
+            mbar_wait_bounded(smem_u32(&bar_sfin[j % STAGES]), (j / STAGES) & 1u, &never,
                               NVFP4_WAIT_TIMEOUT_NS / 4);
-        }
-        if (PAIR) {  // this CTA's A/B boxes complete on the leader's barrier: give them time
-          const uint64_t t0 = global_timer_ns();
-          while (global_timer_ns() - t0 < 2000000ull) {
+            if (!PAIR)
+              mbar_wait_bounded(smem_u32(&bar_full[j % STAGES]), (j / STAGES) & 1u, &never,
+                                NVFP4_WAIT_TIMEOUT_NS / 4);
+          }
+          if (PAIR) {  // this CTA's A/B boxes complete on the leader's barrier: give them time
+            const uint64_t t0 = global_timer_ns();
+            while (global_timer_ns() - t0 < 2000000ull) {
+            }
           }
         }
       }
-    }
-    __syncwarp();
-  } else if (warp == 1) {
-    // =========================== MMA issuer (the leader's, for a pair) ===========================
-    // The whole warp runs the loop; elect.sync picks the issuing lane.  Waits are agreed across
-    // the warp so that every lane leaves the loop together.
-    if (rank == 0) {
-      // Descriptors of stage 0; stage s adds s * STAGE_BYTES / 16 to the start-address field
-      // (bits [0,14) hold address >> 4, and every stage address fits, so the add never carries).
-      const uint32_t s0 = smem_u32(smem);
-      const uint64_t a_desc0 = smem_desc(s0, 16, 1024, 2);
-      const uint64_t b_desc0 = smem_desc(s0 + A_BYTES, 16, 1024, 2);
-      uint32_t it = 0, tile_it = 0;
-      bool ok = true;
-      auto mma = [&](uint32_t d, uint64_t ad, uint64_t bd, uint32_t sfa, uint32_t sfb,
-                     uint32_t acc) {
-        if constexpr (PAIR) tc_mma_nvf4_pair_warp(d, ad, bd, C::IDESC, sfa, sfb, acc);
-        else tc_mma_nvf4_warp(d, ad, bd, C::IDESC, sfa, sfb, acc);
-      };
-      auto commit_all = [&](const uint64_t* bar) {  // arrive on `bar` of every CTA
-        if constexpr (PAIR) {
-          tc_commit_pair_warp(smem_u32(bar));
-          tc_commit_pair_warp(at_peer(bar));
-        } else {
-          tc_commit_warp(smem_u32(bar));
-        }
-      };
-      auto wait_all = [&](const uint64_t* bar, uint32_t parity) {
-        return __all_sync(0xffffffffu, mbar_wait_bounded(smem_u32(bar), parity, &abort_flag));
-      };
-      for (int t = cluster_id; t < total && ok; t += num_clusters, ++tile_it) {
-        const int b = tile_it % ACC_BUFS;
-        if (!wait_all(&bar_acc_empty[b], ((tile_it / ACC_BUFS) & 1u) ^ 1u)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t d_tmem = tmem + b * BN;
-        for (int kb = 0; kb < nk; ++kb, ++it) {
-          const int s = it % STAGES;
-          const uint32_t ph = (it / STAGES) & 1u;
-          if (!wait_all(&bar_full[s], ph) || !wait_all(&bar_sf[s], ph)) {
+      __syncwarp();
+    } else if (warp == 1) {
+      // =========================== MMA issuer (the leader's, for a pair) ===========================
+      // The whole warp runs the loop; elect.sync picks the issuing lane.  Waits are agreed across
+      // the warp so that every lane leaves the loop together.
+      if (rank == 0) {
+        // Descriptors of stage 0; stage s adds s * STAGE_BYTES / 16 to the start-address field
+        // (bits [0,14) hold address >> 4, and every stage address fits, so the add never carries).
+        const uint32_t s0 = smem_u32(smem);
+        const uint64_t a_desc0 = smem_desc(s0, 16, 1024, 2);
+        const uint64_t b_desc0 = smem_desc(s0 + A_BYTES, 16, 1024, 2);
+        uint32_t it = 0, tile_it = 0;
+        bool ok = true;
+        auto mma = [&](uint32_t d, uint64_t ad, uint64_t bd, uint32_t sfa, uint32_t sfb,
+                       uint32_t acc) {
+          if constexpr (PAIR) tc_mma_nvf4_pair_warp(d, ad, bd, C::IDESC, sfa, sfb, acc);
+          else tc_mma_nvf4_warp(d, ad, bd, C::IDESC, sfa, sfb, acc);
+        };
+        auto commit_all = [&](const uint64_t* bar) {  // arrive on `bar` of every CTA
+          if constexpr (PAIR) {
+            tc_commit_pair_warp(smem_u32(bar));
+            tc_commit_pair_warp(at_peer(bar));
+          } else {
+            tc_commit_warp(smem_u32(bar));
+          }
+        };
+        auto wait_all = [&](const uint64_t* bar, uint32_t parity) {
+          return __all_sync(0xffffffffu, mbar_wait_bounded(smem_u32(bar), parity, &abort_flag));
+        };
+        for (int t = cluster_id; t < total && ok; t += num_clusters, ++tile_it) {
+          const int b = tile_it % ACC_BUFS;
+          if (!wait_all(&bar_acc_empty[b], ((tile_it / ACC_BUFS) & 1u) ^ 1u)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint64_t so = static_cast<uint64_t>(s) * (C::STAGE_BYTES >> 4);
-          const uint32_t t_sfa = tmem + C::TM_SFA + s * 16;
-          const uint32_t t_sfb = tmem + C::TM_SFB + s * C::SFB_COLS;
-          const uint32_t first = kb == 0 ? 0u : 1u;
-          // scales of this stage are already in tensor memory (scale-factor warps)
-          const int natoms = min(4, atoms_k - kb * 4);
-          if (natoms == 4) {
-#pragma unroll
-            for (int a = 0; a < 4; ++a)
-              mma(d_tmem, a_desc0 + so + 2 * a, b_desc0 + so + 2 * a, t_sfa + a * 4,
-                  t_sfb + a * (BN / 32), a == 0 ? first : 1u);
-          } else {
-            for (int a = 0; a < natoms; ++a)
-              mma(d_tmem, a_desc0 + so + 2 * a, b_desc0 + so + 2 * a, t_sfa + a * 4,
-                  t_sfb + a * (BN / 32), a == 0 ? first : 1u);
+          const uint32_t d_tmem = tmem + b * BN;
+          for (int kb = 0; kb < nk; ++kb, ++it) {
+            const int s = it % STAGES;
+            const uint32_t ph = (it / STAGES) & 1u;
+            if (!wait_all(&bar_full[s], ph) || !wait_all(&bar_sf[s], ph)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint64_t so = static_cast<uint64_t>(s) * (C::STAGE_BYTES >> 4);
+            const uint32_t t_sfa = tmem + C::TM_SFA + s * 16;
+            const uint32_t t_sfb = tmem + C::TM_SFB + s * C::SFB_COLS;
+            const uint32_t first = kb == 0 ? 0u : 1u;
+            // scales of this stage are already in tensor memory (scale-factor warps)
+            const int natoms = min(4, atoms_k - kb * 4);
+            if (natoms == 4) {
+  #pragma unroll
+              for (int a = 0; a < 4; ++a)
+                mma(d_tmem, a_desc0 + so + 2 * a, b_desc0 + so + 2 * a, t_sfa + a * 4,
+                    t_sfb + a * (BN / 32), a == 0 ? first : 1u);
+            } else {
+              for (int a = 0; a < natoms; ++a)
+                mma(d_tmem, a_desc0 + so + 2 * a, b_desc0 + so + 2 * a, t_sfa + a * 4,
+                    t_sfb + a * (BN / 32), a == 0 ? first : 1u);
+            }
+            commit_all(&bar_empty[s]);
           }
-          commit_all(&bar_empty[s]);
+          if (!ok) break;
+          commit_all(&bar_acc_full[b]);
         }
-        if (!ok) break;
-        commit_all(&bar_acc_full[b]);
+        // all MMAs issued by this warp complete before tensor memory is freed
+        if constexpr (PAIR) tc_commit_pair_warp(smem_u32(&bar_drain));
+        else tc_commit_warp(smem_u32(&bar_drain));
+        volatile int never = 0;
+        mbar_wait_bounded(smem_u32(&bar_drain), 0, &never);
       }
-      // all MMAs issued by this warp complete before tensor memory is freed
-      if constexpr (PAIR) tc_commit_pair_warp(smem_u32(&bar_drain));
-      else tc_commit_warp(smem_u32(&bar_drain));
-      volatile int never = 0;
-      mbar_wait_bounded(smem_u32(&bar_drain), 0, &never);
-    }
-    __syncwarp();
+      __syncwarp();
+  }
   } else if (warp >= SF_WARP0) {
+    regs_release_to<REGS_OTHER>();
     // =========================== scale-factor warps ===========================
     // warp (SF_WARP0 + q) writes lane quadrant q of each stage's scale-factor columns
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
@@ -429,7 +441,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
       }
     }
-  } else if (warp >= EPI_WARP0) {
+  } else {
+    regs_raise_to<REGS_EPI>();
     // =========================== epilogue ===========================
     // Two warps per tensor-memory lane quadrant (a warp may only read lanes 32*(warp%4)..+31);
     // `half` splits the tile's columns between them.
@@ -470,25 +483,30 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const int I = args.I;
           constexpr int n_chunks = BN / 128;  // 64-column chunks per warp
           uint8_t* hrow = args.h + row * (I / 2) + tl.nt * (BN / 4);
+          // the warp's whole accumulator slice into registers, then tensor memory goes back to
+          // the MMA warp and the next tile's MMAs overlap this epilogue
+          uint32_t v[n_chunks][2][32];
+#pragma unroll
+          for (int cc = 0; cc < n_chunks; ++cc) {
+            tmem_ld32(t_row + 64 * (half * n_chunks + cc), v[cc][0]);
+            tmem_ld32(t_row + 64 * (half * n_chunks + cc) + 32, v[cc][1]);
+          }
+          tmem_wait_ld();
+          release();
           uint32_t sfw = 0u;
-#pragma unroll 1
+#pragma unroll
           for (int cc = 0; cc < n_chunks; ++cc) {
             // h features 32c..32c+31 of the tile live in accumulator columns 64c..64c+63 as two
             // 32-column blocks, each 16 gate columns followed by the 16 matching up columns
             const int c = half * n_chunks + cc;
-            uint32_t v0[32], v1[32];
-            tmem_ld32(t_row + 64 * c, v0);
-            tmem_ld32(t_row + 64 * c + 32, v1);
-            tmem_wait_ld();
-            // the accumulator's last columns of this warp are in registers: hand it back, so the
-            // next tile's MMAs overlap the rest of this epilogue
-            if (cc == n_chunks - 1) release();
             float hv[32];
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
               // h = silu(g) * u = g * u / (1 + e^-g), g and u de-scaled by alpha
-              const float g0 = __uint_as_float(v0[i]) * alpha, u0 = __uint_as_float(v0[16 + i]) * alpha;
-              const float g1 = __uint_as_float(v1[i]) * alpha, u1 = __uint_as_float(v1[16 + i]) * alpha;
+              const float g0 = __uint_as_float(v[cc][0][i]) * alpha;
+              const float u0 = __uint_as_float(v[cc][0][16 + i]) * alpha;
+              const float g1 = __uint_as_float(v[cc][1][i]) * alpha;
+              const float u1 = __uint_as_float(v[cc][1][16 + i]) * alpha;
               hv[i] = __fdividef(g0 * u0, 1.0f + __expf(-g0));
               hv[16 + i] = __fdividef(g1 * u1, 1.0f + __expf(-g1));
             }
@@ -524,9 +542,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
           const float scale = alpha * (slot >= 0 ? __ldg(args.row_w + row) : 0.0f);
           const int H = args.N;
-          const int c_lo = (BN / 64) * half, c_hi = c_lo + BN / 64;
-          // 32-column chunks are read from tensor memory two at a time; once the last two are in
-          // registers the accumulator goes back to the MMA warp
+          const int c_lo = (BN / 64) * half;
+          // the warp's whole slice (BN/2 columns) is read from tensor memory first; then the
+          // accumulator goes back to the MMA warp and the stores overlap the next tile's MMAs
           if constexpr (MODE == L2_STAGED) {
             // each 32-column chunk passes through shared memory (16-byte units XOR-swizzled by
             // row) so that 8 lanes write one row's 128 contiguous bytes
@@ -552,16 +570,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               }
               __syncwarp();
             };
-#pragma unroll 1
-            for (int c = c_lo; c < c_hi; c += 2) {
-              uint32_t v0[32], v1[32];
-              tmem_ld32(t_row + 32 * c, v0);
-              tmem_ld32(t_row + 32 * (c + 1), v1);
-              tmem_wait_ld();
-              if (c + 2 >= c_hi) release();
-              emit(c, v0);
-              emit(c + 1, v1);
-            }
+            uint32_t v[BN / 64][32];
+#pragma unroll
+            for (int j = 0; j < BN / 64; ++j) tmem_ld32(t_row + 32 * (c_lo + j), v[j]);
+            tmem_wait_ld();
+            release();
+#pragma unroll
+            for (int j = 0; j < BN / 64; ++j) emit(c_lo + j, v[j]);
           } else {
             float* dst = args.ys + (int64_t)(slot >= 0 ? slot : 0) * H + tl.nt * BN;
             auto emit = [&](int c, const uint32_t (&v)[32]) {
@@ -574,16 +589,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                                    __uint_as_float(v[4 * i + 2]) * scale,
                                    __uint_as_float(v[4 * i + 3]) * scale);
             };
-#pragma unroll 1
-            for (int c = c_lo; c < c_hi; c += 2) {
-              uint32_t v0[32], v1[32];
-              tmem_ld32(t_row + 32 * c, v0);
-              tmem_ld32(t_row + 32 * (c + 1), v1);
-              tmem_wait_ld();
-              if (c + 2 >= c_hi) release();
-              emit(c, v0);
-              emit(c + 1, v1);
-            }
+            uint32_t v[BN / 64][32];
+#pragma unroll
+            for (int j = 0; j < BN / 64; ++j) tmem_ld32(t_row + 32 * (c_lo + j), v[j]);
+            tmem_wait_ld();
+            release();
+#pragma unroll
+            for (int j = 0; j < BN / 64; ++j) emit(c_lo + j, v[j]);
           }
         }
       } else if (rows_valid) {
@@ -614,17 +626,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             }
           }
         };
-        const int c_lo = (BN / 64) * half, c_hi = c_lo + BN / 64;
-#pragma unroll 1
-        for (int c = c_lo; c < c_hi; c += 2) {
-          uint32_t v0[32], v1[32];
-          tmem_ld32(t_row + 32 * c, v0);
-          tmem_ld32(t_row + 32 * (c + 1), v1);
-          tmem_wait_ld();
-          if (c + 2 >= c_hi) release();
-          emit(c, v0);
-          emit(c + 1, v1);
-        }
+        const int c_lo = (BN / 64) * half;
+        uint32_t v[BN / 64][32];
+#pragma unroll
+        for (int j = 0; j < BN / 64; ++j) tmem_ld32(t_row + 32 * (c_lo + j), v[j]);
+        tmem_wait_ld();
+        release();
+#pragma unroll
+        for (int j = 0; j < BN / 64; ++j) emit(c_lo + j, v[j]);
       }
       if (!released) release();
     }
