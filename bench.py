@@ -1,7 +1,7 @@
 """Throughput of the NVFP4 MoE expert-FFN hot path on B200 (one JSON line on rank 0).
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--config decode|mid|prefill|tiny]
-                    [--impl ours|reference] [--no-cpu-baseline] [--experts E]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config decode|mid|prefill|tiny|sweep]
+                    [--impl ours|reference] [--no-cpu-baseline] [--experts E] [--tokens T]
 
 A step is one pass of the whole path over one batch: routing (top-k + expert buckets), amax ->
 global scale -> NVFP4 quantization of the activations, L1 grouped GEMM with SwiGLU + FP4
@@ -14,6 +14,9 @@ The default workload is the decode configuration (T=16 tokens, hidden 7168, inte
 algorithmic HBM traffic per second (GB/s) and `tflops` rides along.  Multi-GPU runs are
 independent replicas (the path has no exchange step on one node's data-parallel batch), so the
 scaling is weak and `value` sums the ranks' bytes over the slowest rank's time.
+
+--config sweep times the standalone 2D x 3D grouped GEMM instead (E=32 groups, M_g ~ U{0..4096},
+K=7168, N=4096, bf16 output): a step is one grouped-GEMM launch over NVFP4 operands already in HBM.
 
 --impl reference times the CPU oracle (numpy, float64) on a bounded sample of the same workload.
 """
@@ -31,6 +34,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "MoE FFN TFLOPS & HBM GB/s on 1 B200, % of NVFP4 tensor/HBM roofline"
 FP4_ELEM_BYTES = 0.5 + 1.0 / 16.0  # E2M1 code + one E4M3 scale per 16 elements
+FP4_PER_BF16 = 4.0  # nominal dense tensor throughput ratio FP4 : BF16 on B200 (9 : 2.25 PFLOP/s)
 
 
 def parse():
@@ -82,11 +86,10 @@ def kernel_sources_sha16():
 
 
 def captured_traffic(cfg):
-    """DRAM bytes per L1 launch from the committed ncu summary, or None when the kernel sources
-    changed since that capture (or the workload is not the one it covers)."""
-    if cfg.name != "decode":
-        return None
-    path = os.path.join(ROOT, "profiles", "grouped_gemm_l1_decode.md")
+    """DRAM bytes per L1 launch from the committed ncu summary of this workload
+    (profiles/grouped_gemm_l1_<workload>.md), or None when there is none or the kernel sources
+    changed since that capture."""
+    path = os.path.join(ROOT, "profiles", f"grouped_gemm_l1_{cfg.name}.md")
     if not os.path.exists(path):
         return None
     fields = {}
@@ -96,7 +99,7 @@ def captured_traffic(cfg):
             fields[k.strip()] = v.strip()
     if fields.get("kernel_sources_sha256_16") != kernel_sources_sha16():
         return None
-    v = fields.get("decode_l1_traffic_bytes_per_launch")
+    v = fields.get("l1_traffic_bytes_per_launch")
     return int(v) if v else None
 
 
@@ -274,10 +277,12 @@ def run_ours(args):
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
+    torch.cuda.nvtx.range_push("timed")
     start.record()
     for i in range(K):
         plan.step(evs[i])
     stop.record()
+    torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -343,6 +348,24 @@ def run_ours(args):
         return
     peaks = load_peaks()
     l1_gbs = acc["l1_bytes"] / (l1_ms * 1e-3) / 1e9
+    l1_tflops = acc["l1_flops"] / (l1_ms * 1e-3) / 1e12
+    fp4_peak = peaks["bf16"] * FP4_PER_BF16
+    tensor_bound = acc["l1_flops"] / acc["l1_bytes"] > fp4_peak * 1e12 / (peaks["hbm"] * 1e9)
+    if tensor_bound:
+        roof = {"bound": "tensor", "kernel": "grouped_gemm_kernel<L1_SWIGLU>",
+                "achieved": round(l1_tflops, 1), "peak": round(fp4_peak, 1), "unit": "TFLOP/s",
+                "frac": round(l1_tflops / fp4_peak, 4), "traffic": captured_traffic(cfg),
+                "algorithmic_flops_per_launch": int(acc["l1_flops"]),
+                "peak_source": f"{peaks['src']} bf16 burst x {FP4_PER_BF16} (nominal FP4/BF16 "
+                               "dense ratio)",
+                "step_frac": round(tflops / world / fp4_peak, 4)}
+    else:
+        roof = {"bound": "hbm", "kernel": "grouped_gemm_kernel<L1_SWIGLU>",
+                "achieved": round(l1_gbs, 1), "peak": peaks["hbm"], "unit": "GB/s",
+                "frac": round(l1_gbs / peaks["hbm"], 4), "traffic": captured_traffic(cfg),
+                "algorithmic_bytes_per_launch": int(acc["l1_bytes"]),
+                "peak_source": peaks["src"],
+                "step_frac": round(value / world / peaks["hbm"], 4)}
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True,
@@ -358,12 +381,7 @@ def run_ours(args):
         "tflops": round(tflops, 3),
         "algorithmic": {"bytes_per_step": int(acc["bytes"]), "flops_per_step": int(acc["flops"]),
                         "active_experts": acc["active"], "slots": acc["slots"]},
-        "roofline": {"bound": "hbm", "kernel": "grouped_gemm_kernel<L1_SWIGLU>",
-                     "achieved": round(l1_gbs, 1), "peak": peaks["hbm"], "unit": "GB/s",
-                     "frac": round(l1_gbs / peaks["hbm"], 4), "traffic": captured_traffic(cfg),
-                     "algorithmic_bytes_per_launch": int(acc["l1_bytes"]),
-                     "peak_source": peaks["src"],
-                     "step_frac": round(value / world / peaks["hbm"], 4)},
+        "roofline": roof,
         "stages_ms": {"route": round(statistics.mean(stage[0]), 4),
                       "quantize": round(statistics.mean(stage[1]), 4),
                       "l1_gemm_swiglu_q": round(l1_ms, 4), "l2_gemm_scatter": round(l2_ms, 4)},
@@ -388,8 +406,9 @@ class _SparseWeights:
         return self.parts[e].dequant(0)
 
 
-def _oracle_sample(cfg, logits_cpu, x_cpu, dev, n_tokens=1):
-    """Bounded oracle sample: the first n_tokens tokens and the experts they route to.  Weight
+def _oracle_sample(cfg, logits_cpu, x_cpu, dev, n_tokens=1, n_experts=1):
+    """Bounded oracle sample: the first n_tokens tokens of the workload, evaluated through the
+    first n_experts of the experts they route to (the oracle's `experts` restriction).  Weight
     pre-packing (quantizing the float weights with the oracle) is done here, untimed."""
     import numpy as np
 
@@ -399,7 +418,11 @@ def _oracle_sample(cfg, logits_cpu, x_cpu, dev, n_tokens=1):
     lg = logits_cpu[:n_tokens].numpy()
     x = x_cpu[:n_tokens].float().numpy()
     ids, _ = R.route_topk(lg, cfg.k)
-    experts = sorted(set(int(e) for e in ids.ravel() if e >= 0))
+    routed = []
+    for e in ids.ravel():
+        if e >= 0 and int(e) not in routed:
+            routed.append(int(e))
+    experts = sorted(routed[:n_experts])
     p1, p2 = {}, {}
     for e in experts:
         w1 = gen_weight_expert(cfg.seed, 1, e, 2 * cfg.I, cfg.H, device=dev).float().cpu().numpy()
@@ -410,11 +433,11 @@ def _oracle_sample(cfg, logits_cpu, x_cpu, dev, n_tokens=1):
     W2 = _SparseWeights(cfg.E, cfg.H, p2)
 
     def run():
-        return M.moe_ffn(x, lg, cfg.k, W1, W2, np.float32(cfg.gs_h))
+        return M.moe_ffn(x, lg, cfg.k, W1, W2, np.float32(cfg.gs_h), experts=experts)
 
     counts = [0] * cfg.E
     for e in ids.ravel():
-        if e >= 0:
+        if int(e) in experts:
             counts[int(e)] += 1
     from dataclasses import replace
     return run, algorithmic(replace(cfg, T=n_tokens), counts), experts
@@ -430,20 +453,71 @@ def _threads():
 
 
 def cpu_baseline(cfg, logits_cpu, x_cpu, dev):
+    """The oracle on a bounded sample (about 10-30 s of CPU work): the first tokens of the
+    workload through their first routed expert each, repeated until 10 s have passed."""
     run, acc, experts = _oracle_sample(cfg, logits_cpu, x_cpu, dev)
-    t0 = time.perf_counter()
-    run()
-    dt = time.perf_counter() - t0
-    return {"value": round(acc["bytes"] / dt / 1e9, 4), "unit": "GB/s", "cores": _threads(),
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        run()
+        reps += 1
+        dt = time.perf_counter() - t0
+        if dt >= 10.0:
+            break
+    return {"value": round(acc["bytes"] * reps / dt / 1e9, 4), "unit": "GB/s", "cores": _threads(),
             "kind": "oracle",
-            "sample": f"1 of {cfg.T} tokens of the {cfg.name} workload ({len(experts)} experts, "
-                      f"{acc['bytes'] / 1e6:.0f} MB algorithmic) in {dt:.1f} s; numpy float64, "
-                      "BLAS threads for the matmuls, elementwise work single-threaded"}
+            "sample": f"token 0 of the {cfg.name} workload through expert {experts[0]} "
+                      f"({acc['bytes'] / 1e6:.0f} MB algorithmic), {reps} repetitions in "
+                      f"{dt:.1f} s; numpy float64, BLAS threads for the matmuls, elementwise "
+                      "work single-threaded"}
+
+
+def run_reference_sweep(args):
+    """The oracle's grouped GEMM on a bounded sample of the sweep: 256 rows of the largest group
+    against that group's weights, both quantized by the oracle (untimed), float64 matmul per step."""
+    import numpy as np
+
+    from oracle import moe as M
+    from oracle import quant as Q
+    from synth import CONFIGS, gen_weight_expert
+    from synth.inputs import gen_sweep, gen_sweep_a
+    cfg = CONFIGS["sweep"]
+    m = gen_sweep(cfg)
+    g = int(np.argmax(m))
+    n = min(256, m[g])
+    r0 = sum(m[:g])
+    a = gen_sweep_a(cfg, r0 + n)[r0:].to(__import__("torch").bfloat16).float().numpy()
+    gs_a = Q.global_scale(a)
+    a_deq = Q.dequantize(*Q.quantize(a, gs_a), gs_a)
+    wq = M.QuantWeights.from_float(gen_weight_expert(cfg.seed, 1, g, cfg.N, cfg.K).float().numpy()[None])
+    b = wq.dequant(0)
+    flops = 2 * n * cfg.N * cfg.K
+    for _ in range(args.warmup):
+        a_deq @ b.T
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        a_deq @ b.T
+    dt = time.perf_counter() - t0
+    value = flops * args.steps / dt / 1e12
+    sample = f"each step: {n} rows of group {g} x {cfg.N} x {cfg.K}, float64 matmul of the decoded operands"
+    print(json.dumps({
+        "impl": "reference", "metric": SWEEP_METRIC, "value": round(value, 6), "unit": "TFLOP/s",
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"grouped GEMM sweep: E={cfg.E} groups, M_g ~ U{{0..{cfg.m_max}}}, "
+                               f"K={cfg.K}, N={cfg.N}, bf16 out"},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": _threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0}}), flush=True)
 
 
 def run_reference(args):
     rank = int(os.environ.get("RANK", 0))
     if rank != 0:
+        return
+    if args.config == "sweep":
+        run_reference_sweep(args)
         return
     import torch
     cfg = make_config(args)
@@ -458,8 +532,8 @@ def run_reference(args):
         run()
     dt = time.perf_counter() - t0
     value = acc["bytes"] * args.steps / dt / 1e9
-    sample = (f"each step: 1 of {cfg.T} tokens of the {cfg.name} workload ({len(experts)} experts, "
-              f"{acc['bytes'] / 1e6:.0f} MB algorithmic)")
+    sample = (f"each step: token 0 of {cfg.T} of the {cfg.name} workload through {len(experts)} "
+              f"of its experts ({acc['bytes'] / 1e6:.0f} MB algorithmic)")
     line = {
         "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
         "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
@@ -475,9 +549,190 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+# ----------------------------------------------------------------------------- sweep
+
+SWEEP_METRIC = "grouped GEMM TFLOP/s on 1 B200 (NVFP4 2D x 3D, bf16 out), % of NVFP4 tensor peak"
+
+
+def sweep_operands(cfg, dev):
+    """Group sizes, 128-padded offsets and NVFP4 operands of the grouped-GEMM sweep: A rows
+    N(0,1) (zero padding rows), B = per-group weights N(0,0.02), both quantized on the GPU."""
+    import torch
+
+    import nvfp4_block_scaled_gsa_b200 as nv
+    from synth import gen_weight_expert
+    from synth.inputs import gen_sweep, gen_sweep_a
+    m = gen_sweep(cfg)
+    pad = [(x + 127) // 128 * 128 for x in m]
+    offs_l = [0]
+    for p_ in pad:
+        offs_l.append(offs_l[-1] + p_)
+    R = offs_l[-1]
+    a_rows = gen_sweep_a(cfg, sum(m), device=dev).to(torch.bfloat16)
+    a = torch.zeros(R, cfg.K, dtype=torch.bfloat16, device=dev)
+    r0 = 0
+    for g, mg in enumerate(m):
+        a[offs_l[g]:offs_l[g] + mg] = a_rows[r0:r0 + mg]
+        r0 += mg
+    w = nv.quantize_weights(lambda e: gen_weight_expert(cfg.seed, 1, e, cfg.N, cfg.K, device=dev),
+                            cfg.E, cfg.N, cfg.K, device=dev)
+    offs = torch.tensor(offs_l, dtype=torch.int32, device=dev)
+    return m, offs, a, w
+
+
+def run_sweep(args):
+    import torch
+    import torch.distributed as dist
+
+    import nvfp4_block_scaled_gsa_b200 as nv
+    from synth import CONFIGS
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local = int(os.environ.get("LOCAL_RANK", 0))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    cfg = CONFIGS["sweep"]
+    m, offs, a_bf16, w = sweep_operands(cfg, dev)
+    R = a_bf16.shape[0]
+    codes, sf, gs = nv.quantize(a_bf16)
+    out = torch.empty(R, cfg.N, dtype=torch.bfloat16, device=dev)
+    flops = 2 * sum(m) * cfg.N * cfg.K
+
+    def step():
+        nv.grouped_gemm(codes, sf, gs, w, offs, out_dtype=torch.bfloat16, out=out)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local) if rank == 0 else None
+    t_end = time.time() + args.soak
+    while time.time() < t_end:
+        for _ in range(8):
+            step()
+        torch.cuda.synchronize()
+    K = args.steps
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    torch.cuda.nvtx.range_push("timed")
+    start.record()
+    for _ in range(K):
+        step()
+    stop.record()
+    torch.cuda.nvtx.range_pop()
+    torch.cuda.synchronize()
+    clocks = sampler.stop() if sampler else None
+    t = torch.tensor([start.elapsed_time(stop)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.barrier()
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms = float(t.item()) / K
+    value = world * flops / (ms * 1e-3) / 1e12
+
+    # end to end: bf16 A from pinned host memory, quantize, GEMM, bf16 result back to the host
+    a_h = a_bf16.cpu().pin_memory()
+    out_h = torch.empty(R, cfg.N, dtype=torch.bfloat16).pin_memory()
+    a_d = torch.empty_like(a_bf16)
+
+    def e2e_step():
+        a_d.copy_(a_h, non_blocking=True)
+        c2, s2_, g2 = nv.quantize(a_d)
+        nv.grouped_gemm(c2, s2_, g2, w, offs, out_dtype=torch.bfloat16, out=out)
+        out_h.copy_(out, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ke = max(1, min(K, 5))
+    e0.record()
+    for _ in range(ke):
+        e2e_step()
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / ke
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = sweep_cpu_baseline(cfg, m, offs, codes, sf, gs, w)
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    peaks = load_peaks()
+    fp4_peak = peaks["bf16"] * FP4_PER_BF16
+    line = {
+        "metric": SWEEP_METRIC, "value": round(value, 1), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4 (e2m1 + e4m3/16), fp32 accumulate",
+        "data": "synthetic (seeded N(0,1) A rows, N(0,0.02) weights, quantized on the GPU)",
+        "config": {"workload": f"grouped GEMM sweep: E={cfg.E} groups, M_g ~ U{{0..{cfg.m_max}}} "
+                               f"(sum {sum(m)}), K={cfg.K}, N={cfg.N}, bf16 out",
+                   "parallelism": f"replicas x{world}",
+                   "l2": "no flush: A (NVFP4, %.0f MB) + B (%.0f MB) > 126 MB L2" % (
+                       R * cfg.K * FP4_ELEM_BYTES / 1e6, cfg.E * cfg.N * cfg.K * FP4_ELEM_BYTES / 1e6)},
+        "roofline": {"bound": "tensor", "kernel": "grouped_gemm_kernel<PLAIN_BF16>",
+                     "achieved": round(value / world, 1), "peak": round(fp4_peak, 1),
+                     "unit": "TFLOP/s", "frac": round(value / world / fp4_peak, 4), "traffic": None,
+                     "algorithmic_flops_per_launch": int(flops),
+                     "peak_source": f"{peaks['src']} bf16 burst x {FP4_PER_BF16} (nominal FP4/BF16 "
+                                    "dense ratio)"},
+        "e2e": {"value": round(world * flops / (e2e_ms * 1e-3) / 1e12, 1), "unit": "TFLOP/s",
+                "h2d_bytes_per_step": a_h.numel() * 2, "d2h_bytes_per_step": out_h.numel() * 2,
+                "ms_per_step": round(e2e_ms, 4)},
+        "gpu_launches": K,
+        "clocks": clocks,
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def _sweep_oracle_sample(cfg, m, offs, codes, sf, gs, w, rows=4096):
+    """The oracle's grouped GEMM on (up to `rows` rows of) the largest group, decoded from the
+    same NVFP4 operands the GPU used."""
+    import numpy as np
+
+    from oracle import quant as Q
+    g = int(np.argmax(m))
+    o = int(offs[g])
+    n = min(rows, m[g])
+    K, N = cfg.K, cfg.N
+    cols = np.arange(K // 16)
+
+    def scales(flat, r0, nrows):
+        rr, cc = np.meshgrid(np.arange(r0, r0 + nrows), cols, indexing="ij")
+        return flat[Q.sf_tile_offset(rr, cc, K // 16)]
+
+    a = Q.dequantize_packed(codes[o:o + n].cpu().numpy(), scales(sf.cpu().numpy(), o, n),
+                           float(gs.item()))
+    b = Q.dequantize_packed(w.codes[g * N:(g + 1) * N].cpu().numpy(),
+                            scales(w.sf.cpu().numpy(), g * N, N), float(w.gs[g].item()))
+
+    def run():
+        return a @ b.T
+
+    return run, 2 * n * N * K, n, g
+
+
+def sweep_cpu_baseline(cfg, m, offs, codes, sf, gs, w):
+    run, flops, n, g = _sweep_oracle_sample(cfg, m, offs, codes, sf, gs, w)
+    t0 = time.perf_counter()
+    run()
+    dt = time.perf_counter() - t0
+    return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": _threads(),
+            "kind": "oracle",
+            "sample": f"{n} rows of group {g} x {cfg.N} x {cfg.K} (float64 matmul of the decoded "
+                      f"NVFP4 operands) in {dt:.2f} s"}
+
+
 def main():
     args = parse()
-    if args.impl == "reference":
+    if args.config == "sweep" and args.impl == "ours":
+        run_sweep(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)
