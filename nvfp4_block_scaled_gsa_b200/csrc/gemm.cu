@@ -6,18 +6,20 @@
 // accumulation.  The pages' kernel is a 7-warp CuTeDSL design; this one is written directly in
 // PTX for sm_100a:
 //
-//   warp 0      TMA producer: A and B tiles (cp.async.bulk.tensor, 128-byte swizzle) and the
-//               pre-tiled scale atoms (cp.async.bulk) into a 4-stage shared-memory ring
-//   warp 1      MMA issuer: tcgen05.mma.kind::mxf4nvf4.block_scale (M=128, N=256, K=64) into a
-//               TMEM accumulator; it issues nothing else, because the tensor pipe runs its
-//               instructions one after another and scale copies in that stream cost as much as
-//               the MMAs themselves
+//   warp 0      TMA producer: A and B tiles (cp.async.bulk.tensor, 128-byte swizzle) into a
+//               4-stage shared-memory ring
+//   warp 3      scale producer: the pre-tiled scale atoms (cp.async.bulk) into a ring of their
+//               own, ahead of the A/B ring
+//   warp 1      MMA issuer (whole warp, elect.sync): tcgen05.mma.kind::mxf4nvf4.block_scale
+//               (M=128, N=256, K=64) into a TMEM accumulator; it issues nothing else, because
+//               the tensor pipe runs its instructions one after another and scale copies in that
+//               stream cost as much as the MMAs themselves
 //   warp 2      owns the tensor-memory allocation (512 columns)
-//   warps 4..11 epilogue: tcgen05.ld of the accumulator (warp w reads lanes 32*(w%4)..+31),
-//               then one of the fused epilogues below
-//   warps 12..15 scale-factor warps: each stage's scale atoms go from shared memory to the
+//   warps 4..11 epilogue (176 registers each, setmaxnreg): tcgen05.ld of the accumulator (warp w
+//               reads lanes 32*(w%4)..+31), then one of the fused epilogues below
+//   warps 12..15 scale-factor warps: each stage's scale atoms go from the scale ring to the
 //               tensor-memory layout the MMA reads, by ld.shared + tcgen05.st, one warp per
-//               lane quadrant
+//               lane quadrant, as soon as the stage's tensor-memory columns are free
 //
 // Epilogues (the MODE template parameter):
 //   PLAIN_F32 / PLAIN_BF16  C = acc / (gs_a * gs_b[e])
@@ -94,17 +96,28 @@ struct TileCfg {
   static constexpr int B_ROWS = BN / CTAS;                 // B rows (N) per CTA per stage
   static constexpr int B_BYTES = B_ROWS * BK_BYTES;
   static constexpr int SFB_BYTES = (BN / 128) * 4 * 512;   // scales of all BN rows of B
-  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+  // A/B ring: STAGES slots of AB_BYTES.  Scale atoms have a ring of their own (SF_STAGES slots of
+  // SF_BYTES), filled ahead of the A/B ring by a separate producer warp, so a stage's scales are
+  // already in shared memory when its tensor-memory columns become free.
+  static constexpr int AB_BYTES = A_BYTES + B_BYTES;
+  static constexpr int SF_BYTES = SFA_BYTES + SFB_BYTES;
+  static constexpr int SF_STAGES = 4;
   // L2_STAGED: each epilogue warp stages a 32 x 32 FP32 block in shared memory
   static constexpr int EPI_STAGE_BYTES = MODE == L2_STAGED ? EPI_WARPS * 4096 : 0;
-  static constexpr int STAGES = (216 * 1024 - EPI_STAGE_BYTES) / STAGE_BYTES;
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_STAGE_BYTES + 1024;
   static constexpr uint32_t SFB_COLS = (BN / 128) * 16;  // scale columns of B per stage
+  static constexpr int STAGES_SMEM =
+      (216 * 1024 - EPI_STAGE_BYTES - SF_STAGES * SF_BYTES) / AB_BYTES;
+  static constexpr int STAGES_TMEM = (TMEM_COLS - BN) / (16 + SFB_COLS);
+  static constexpr int STAGES = STAGES_SMEM < STAGES_TMEM ? STAGES_SMEM : STAGES_TMEM;
+  static constexpr int SF_OFFSET = STAGES * AB_BYTES;
+  static constexpr int EPI_OFFSET = SF_OFFSET + SF_STAGES * SF_BYTES;
+  static constexpr int SMEM_BYTES = EPI_OFFSET + EPI_STAGE_BYTES + 1024;
   static constexpr int ACC_BUFS = 2 * BN + STAGES * (16 + SFB_COLS) <= TMEM_COLS ? 2 : 1;
   static constexpr uint32_t TM_SFA = ACC_BUFS * BN;        // 16 columns per stage
   static constexpr uint32_t TM_SFB = TM_SFA + STAGES * 16;
   static constexpr uint32_t IDESC = idesc_nvf4(BN, 128 * CTAS);
-  static_assert(STAGE_BYTES % 1024 == 0, "stages must keep 1024-byte alignment (128B swizzle)");
+  static_assert(AB_BYTES % 1024 == 0, "stages must keep 1024-byte alignment (128B swizzle)");
+  static_assert(SF_BYTES % 16 == 0, "bulk copies need 16-byte alignment");
   static_assert(TM_SFB + STAGES * SFB_COLS <= TMEM_COLS, "tensor memory budget");
 };
 
@@ -168,7 +181,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   __shared__ __align__(8) uint64_t bar_full[STAGES];   // A/B landed (a pair: both CTAs')
   __shared__ __align__(8) uint64_t bar_empty[STAGES];  // MMAs done with the stage
   __shared__ __align__(8) uint64_t bar_sf[STAGES];     // scales in tensor memory (all CTAs)
-  __shared__ __align__(8) uint64_t bar_sfin[STAGES];   // this CTA's scale atoms landed
+  __shared__ __align__(8) uint64_t bar_sfin[C::SF_STAGES];     // scale atoms landed in a slot
+  __shared__ __align__(8) uint64_t bar_sfempty[C::SF_STAGES];  // scale slot copied out
   __shared__ __align__(8) uint64_t bar_acc_full[ACC_BUFS];
   __shared__ __align__(8) uint64_t bar_acc_empty[ACC_BUFS];
   __shared__ __align__(8) uint64_t bar_drain;
@@ -231,7 +245,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(smem_u32(&bar_full[s]), 1);
       mbar_init(smem_u32(&bar_empty[s]), 1);
       mbar_init(smem_u32(&bar_sf[s]), 4 * CTAS);
-      mbar_init(smem_u32(&bar_sfin[s]), 1);
+    }
+    for (int j = 0; j < C::SF_STAGES; ++j) {
+      mbar_init(smem_u32(&bar_sfin[j]), 1);
+      mbar_init(smem_u32(&bar_sfempty[j]), 4);
     }
     for (int b = 0; b < ACC_BUFS; ++b) {
       mbar_init(smem_u32(&bar_acc_full[b]), 1);
@@ -276,9 +293,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int t = cluster_id; t < total && ok; t += num_clusters) {
           const Tile tl = decode_tile<CTAS>(t, tile_start, seg, E, args.n_tiles);
           const int m_cta = tl.m0 + BM * rank;  // this CTA's rows
-          // a pair's second half past the expert's segment computes rows it never writes; its
-          // scale atoms are taken from the first half so that every read stays inside the tensor
-          const int a_blk = (m_cta < seg[tl.e + 1] ? m_cta : tl.m0) >> 7;
           // B rows of this N-tile: BN consecutive rows (for L1: 16-row gate blocks each followed by
           // the 16 matching up rows); a pair's CTA r loads rows B_ROWS*r .. B_ROWS*r + B_ROWS-1
           const int b_row0 = tl.e * args.N + tl.nt * BN;
@@ -289,21 +303,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               ok = false;
               break;
             }
-            const int natoms = min(4, atoms_k - kb * 4);
-            uint8_t* st = smem + s * C::STAGE_BYTES;
-            const uint32_t sA = smem_u32(st), sB = sA + A_BYTES, sSFA = sB + C::B_BYTES,
-                           sSFB = sSFA + SFA_BYTES;
-            // the scales first, on their own barrier: the scale-factor warps move them to tensor
-            // memory while the A/B boxes are still in flight
-            const uint32_t sf_bar = smem_u32(&bar_sfin[s]);
-            mbar_arrive_expect_tx(sf_bar, natoms * 512 * (1 + BN / 128));
-            bulk_load(sSFA, args.sfa + ((int64_t)a_blk * atoms_k + kb * 4) * 512, natoms * 512,
-                      sf_bar);
-  #pragma unroll
-            for (int j = 0; j < BN / 128; ++j) {
-              const int64_t b_atom = (int64_t)((b_row0 >> 7) + j) * atoms_k + kb * 4;
-              bulk_load(sSFB + j * 4 * 512, args.sfb + b_atom * 512, natoms * 512, sf_bar);
-            }
+            uint8_t* st = smem + s * C::AB_BYTES;
+            const uint32_t sA = smem_u32(st), sB = sA + A_BYTES;
             if constexpr (PAIR) {
               const uint32_t full = at_leader(&bar_full[s]);
               if (rank == 0) mbar_arrive_expect_tx(smem_u32(&bar_full[s]), 2 * (A_BYTES + C::B_BYTES));
@@ -323,13 +324,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           // let the copies already issued land before the CTA can exit
           volatile int never = 0;
           const uint32_t first = it > (uint32_t)STAGES ? it - STAGES : 0u;
-          for (uint32_t j = first; j < it; ++j) {
-            mbar_wait_bounded(smem_u32(&bar_sfin[j % STAGES]), (j / STAGES) & 1u, &never,
+          for (uint32_t j = first; j < it && !PAIR; ++j)
+            mbar_wait_bounded(smem_u32(&bar_full[j % STAGES]), (j / STAGES) & 1u, &never,
                               NVFP4_WAIT_TIMEOUT_NS / 4);
-            if (!PAIR)
-              mbar_wait_bounded(smem_u32(&bar_full[j % STAGES]), (j / STAGES) & 1u, &never,
-                                NVFP4_WAIT_TIMEOUT_NS / 4);
-          }
           if (PAIR) {  // this CTA's A/B boxes complete on the leader's barrier: give them time
             const uint64_t t0 = global_timer_ns();
             while (global_timer_ns() - t0 < 2000000ull) {
@@ -338,12 +335,56 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
       }
       __syncwarp();
+    } else if (warp == 3) {
+      // =========================== scale producer ===========================
+      // Scale atoms of every stage (this CTA's 128 A rows, all BN rows of B) into the scale ring;
+      // it runs ahead of the A/B producer by up to SF_STAGES stages.
+      if (lane == 0) {
+        uint32_t it = 0;
+        bool ok = true;
+        for (int t = cluster_id; t < total && ok; t += num_clusters) {
+          const Tile tl = decode_tile<CTAS>(t, tile_start, seg, E, args.n_tiles);
+          const int m_cta = tl.m0 + BM * rank;
+          // a pair's second half past the expert's segment computes rows it never writes; its
+          // scale atoms are taken from the first half so that every read stays inside the tensor
+          const int a_blk = (m_cta < seg[tl.e + 1] ? m_cta : tl.m0) >> 7;
+          const int b_blk = (tl.e * args.N + tl.nt * BN) >> 7;
+          for (int kb = 0; kb < nk; ++kb, ++it) {
+            const int j = it % C::SF_STAGES;
+            const uint32_t ph = (it / C::SF_STAGES) & 1u;
+            if (!mbar_wait_bounded(smem_u32(&bar_sfempty[j]), ph ^ 1u, &abort_flag)) {
+              ok = false;
+              break;
+            }
+            const int natoms = min(4, atoms_k - kb * 4);
+            const uint32_t sSFA = smem_u32(smem + C::SF_OFFSET + j * C::SF_BYTES);
+            const uint32_t sf_bar = smem_u32(&bar_sfin[j]);
+            mbar_arrive_expect_tx(sf_bar, natoms * 512 * (1 + BN / 128));
+            bulk_load(sSFA, args.sfa + ((int64_t)a_blk * atoms_k + kb * 4) * 512, natoms * 512,
+                      sf_bar);
+#pragma unroll
+            for (int jj = 0; jj < BN / 128; ++jj) {
+              const int64_t b_atom = (int64_t)(b_blk + jj) * atoms_k + kb * 4;
+              bulk_load(sSFA + SFA_BYTES + jj * 4 * 512, args.sfb + b_atom * 512, natoms * 512,
+                        sf_bar);
+            }
+          }
+        }
+        if (!ok) {  // let the copies already issued land before the CTA can exit
+          volatile int never = 0;
+          const uint32_t first = it > (uint32_t)C::SF_STAGES ? it - C::SF_STAGES : 0u;
+          for (uint32_t j = first; j < it; ++j)
+            mbar_wait_bounded(smem_u32(&bar_sfin[j % C::SF_STAGES]), (j / C::SF_STAGES) & 1u,
+                              &never, NVFP4_WAIT_TIMEOUT_NS / 4);
+        }
+      }
+      __syncwarp();
     } else if (warp == 1) {
       // =========================== MMA issuer (the leader's, for a pair) ===========================
       // The whole warp runs the loop; elect.sync picks the issuing lane.  Waits are agreed across
       // the warp so that every lane leaves the loop together.
       if (rank == 0) {
-        // Descriptors of stage 0; stage s adds s * STAGE_BYTES / 16 to the start-address field
+        // Descriptors of stage 0; stage s adds s * AB_BYTES / 16 to the start-address field
         // (bits [0,14) hold address >> 4, and every stage address fits, so the add never carries).
         const uint32_t s0 = smem_u32(smem);
         const uint64_t a_desc0 = smem_desc(s0, 16, 1024, 2);
@@ -382,7 +423,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               break;
             }
             tc_fence_after();
-            const uint64_t so = static_cast<uint64_t>(s) * (C::STAGE_BYTES >> 4);
+            const uint64_t so = static_cast<uint64_t>(s) * (C::AB_BYTES >> 4);
             const uint32_t t_sfa = tmem + C::TM_SFA + s * 16;
             const uint32_t t_sfb = tmem + C::TM_SFB + s * C::SFB_COLS;
             const uint32_t first = kb == 0 ? 0u : 1u;
@@ -422,11 +463,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       for (int kb = 0; kb < nk; ++kb, ++it) {
         const int s = it % STAGES;
         const uint32_t ph = (it / STAGES) & 1u;
-        if (!mbar_wait_bounded(smem_u32(&bar_sfin[s]), ph, &abort_flag)) {
+        const int j = it % C::SF_STAGES;
+        // the stage's scales are in the scale ring, and its tensor-memory columns are free once
+        // the MMAs of the stage's previous use have completed (the A/B producer waits the same)
+        if (!mbar_wait_bounded(smem_u32(&bar_sfin[j]), (it / C::SF_STAGES) & 1u, &abort_flag) ||
+            !mbar_wait_bounded(smem_u32(&bar_empty[s]), ph ^ 1u, &abort_flag)) {
           ok = false;
           break;
         }
-        const uint8_t* st = smem + s * C::STAGE_BYTES + A_BYTES + C::B_BYTES;
+        tc_fence_after();
+        const uint8_t* st = smem + C::SF_OFFSET + j * C::SF_BYTES;
         sf_rows128_to_tmem(tmem + lane_base + C::TM_SFA + s * 16, st, lane);
         if constexpr (BN == 256)
           sf_rows256_to_tmem(tmem + lane_base + C::TM_SFB + s * C::SFB_COLS, st + SFA_BYTES, lane);
@@ -436,6 +482,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) {
+          mbar_arrive(smem_u32(&bar_sfempty[j]));
           if constexpr (PAIR) mbar_arrive_cluster(at_leader(&bar_sf[s]));
           else mbar_arrive(smem_u32(&bar_sf[s]));
         }
@@ -548,7 +595,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if constexpr (MODE == L2_STAGED) {
             // each 32-column chunk passes through shared memory (16-byte units XOR-swizzled by
             // row) so that 8 lanes write one row's 128 contiguous bytes
-            float4* stg = reinterpret_cast<float4*>(smem + STAGES * C::STAGE_BYTES +
+            float4* stg = reinterpret_cast<float4*>(smem + C::EPI_OFFSET +
                                                     (warp - EPI_WARP0) * 4096);
             const int sub = lane >> 3, c4 = lane & 7;
             int sl[8];  // slot of row 4i + sub of this warp's 32 rows
