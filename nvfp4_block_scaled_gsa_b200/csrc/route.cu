@@ -86,7 +86,11 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
 
 // Single CTA of 32 warps.  Warp w owns the contiguous slot range [w*chunk, (w+1)*chunk), so a
 // per-warp histogram plus an exclusive scan over warps gives every slot a stable rank inside
-// its expert; __match_any_sync ranks the slots of one 32-slot step that share an expert.
+// its expert; __match_any_sync ranks the slots of one 32-slot step that share an expert.  Both
+// passes over the slots load kUnroll steps ahead (independent loads in flight), and one warp
+// scans the expert counts.
+constexpr int kUnroll = 8;
+
 __global__ void __launch_bounds__(1024) permute_kernel(
     const int32_t* __restrict__ ids, const float* __restrict__ w, int S, int k, int E,
     int64_t R_max, int32_t* __restrict__ offs_out, int32_t* __restrict__ dst_row,
@@ -100,10 +104,18 @@ __global__ void __launch_bounds__(1024) permute_kernel(
   const int chunk = (S + 31) / 32;
   const int lo = min(S, warp * chunk), hi = min(S, lo + chunk);
   bool bad = false;
-  for (int s = lo + lane; s < hi; s += 32) {
-    const int e = __ldg(ids + s);
-    if (e >= E) bad = true;
-    else if (e >= 0) atomicAdd(&hist[warp][e], 1);
+  for (int base = lo; base < hi; base += 32 * kUnroll) {
+    int e[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int s = base + 32 * u + lane;
+      e[u] = s < hi ? __ldg(ids + s) : -1;
+    }
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      if (e[u] >= E) bad = true;
+      else if (e[u] >= 0) atomicAdd(&hist[warp][e[u]], 1);
+    }
   }
   if (bad) report(dev_status, NVFP4_DEVERR_BAD_INDEX);
   __syncthreads();
@@ -117,37 +129,63 @@ __global__ void __launch_bounds__(1024) permute_kernel(
     cnt[tid] = run;
   }
   __syncthreads();
-  if (tid == 0) {
-    int o = 0;
-    for (int e = 0; e < E; ++e) {
-      offs[e] = o;
-      o += (cnt[e] + 127) & ~127;
+  if (warp == 0) {  // offs = exclusive scan of the 128-padded counts (lane l: experts 8l..8l+7)
+    int p[kMaxE / 32];
+    int sum = 0;
+#pragma unroll
+    for (int i = 0; i < kMaxE / 32; ++i) {
+      const int e = lane * (kMaxE / 32) + i;
+      p[i] = e < E ? (cnt[e] + 127) & ~127 : 0;
+      sum += p[i];
     }
-    offs[E] = o;
+    int incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    int run = incl - sum;
+#pragma unroll
+    for (int i = 0; i < kMaxE / 32; ++i) {
+      const int e = lane * (kMaxE / 32) + i;
+      if (e <= E) offs[e] = run;
+      run += p[i];
+    }
+    if (lane == 31 && E == kMaxE) offs[E] = run;
   }
   __syncthreads();
   if (tid <= E) offs_out[tid] = offs[tid];
   const unsigned lt_mask = (1u << lane) - 1u;
-  for (int base = lo; base < hi; base += 32) {
-    const int s = base + lane;
-    const bool valid = s < hi;
-    int e = valid ? __ldg(ids + s) : -1;
-    if (e >= E) e = -1;
-    const unsigned peers = __match_any_sync(0xffffffffu, e);
-    const int rank = __popc(peers & lt_mask);
-    if (valid) {
-      if (e >= 0) {
-        const int row = offs[e] + hist[warp][e] + rank;
-        dst_row[s] = row;
-        row_slot[row] = s;
-        row_w[row] = __ldg(w + s);
-      } else {
-        dst_row[s] = -1;
-      }
+  for (int base = lo; base < hi; base += 32 * kUnroll) {
+    int e[kUnroll];
+    float wv[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int s = base + 32 * u + lane;
+      e[u] = s < hi ? __ldg(ids + s) : -1;
+      wv[u] = s < hi ? __ldg(w + s) : 0.0f;
     }
-    __syncwarp();
-    if (e >= 0 && rank == 0) hist[warp][e] += __popc(peers);
-    __syncwarp();
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int s = base + 32 * u + lane;
+      const bool valid = s < hi;
+      const int eu = (e[u] >= E) ? -1 : e[u];
+      const unsigned peers = __match_any_sync(0xffffffffu, eu);
+      const int rank = __popc(peers & lt_mask);
+      if (valid) {
+        if (eu >= 0) {
+          const int row = offs[eu] + hist[warp][eu] + rank;
+          dst_row[s] = row;
+          row_slot[row] = s;
+          row_w[row] = wv[u];
+        } else {
+          dst_row[s] = -1;
+        }
+      }
+      __syncwarp();
+      if (eu >= 0 && rank == 0) hist[warp][eu] += __popc(peers);
+      __syncwarp();
+    }
   }
   // padding rows of every segment, then the unused tail up to R_max
   for (int e = warp; e < E; e += 32) {
