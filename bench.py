@@ -170,6 +170,7 @@ class Plan:
         self.ids, self.w = e(T * k, i32), e(T * k, f32)
         self.offs, self.dst = e(E + 1, i32), e(T * k, i32)
         self.row_slot, self.row_w = e(self.R, i32), e(self.R, f32)
+        self.pws = e(max(nv.lib().moe_permute_workspace_size(T, E, k), 1), torch.uint8)
         self.xq, self.xsf = e(self.R * H // 2, u8), e(self.R * H // 16, u8)
         self.gs_x, self.qws = e(1, f32), e(256, u8)
         self.hq, self.hsf = e(self.R * I // 2, u8), e(self.R * I // 16, u8)
@@ -187,7 +188,8 @@ class Plan:
         if ev:
             ev[0].record()
         call("moe_permute", p(self.logits), T, E, k, 1, p(self.ids), p(self.w), p(self.offs),
-             p(self.dst), p(self.row_slot), p(self.row_w), None, 0, p(self.status), s)
+             p(self.dst), p(self.row_slot), p(self.row_w), p(self.pws), self.pws.numel(),
+             p(self.status), s)
         if ev:
             ev[1].record()
         call("nvfp4_quantize", p(self.x), T, H, H, p(self.dst), k, self.R, p(self.xq), p(self.xsf),
@@ -208,7 +210,8 @@ class Plan:
             ev[4].record()
 
 
-KERNELS_PER_STEP = 7  # topk, permute, amax, quantize, L1 GEMM, L2 GEMM, combine
+KERNELS_PER_STEP = 7  # topk, permute, amax, quantize, L1 GEMM, L2 GEMM, combine (+ a count
+#                       kernel before permute from 4096 slots)
 
 
 def make_config(args):
@@ -387,7 +390,8 @@ def run_ours(args):
                       "l1_gemm_swiglu_q": round(l1_ms, 4), "l2_gemm_scatter": round(l2_ms, 4)},
         "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms / K, 4)},
-        "gpu_launches": KERNELS_PER_STEP * K,
+        "gpu_launches": (KERNELS_PER_STEP + (1 if nv.lib().moe_permute_workspace_size(
+            cfg.T, cfg.E, cfg.k) else 0)) * K,
         "clocks": clocks,
         "cpu_baseline": cpu,
     }

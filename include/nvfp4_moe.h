@@ -115,6 +115,9 @@ NVFP4_API nvfp4_status_t nvfp4_quantize(const void* x, int64_t rows, int64_t col
  *             and unused rows
  *   row_w     float [R_max]: routing weight of each row, 0 for padding and unused rows
  *   R_max     = moe_rows_max(T, E, k)
+ *   ws        device scratch of moe_permute_workspace_size(T, E, k) bytes (4-byte aligned): from
+ *             4096 slots the map is built by many CTAs, which exchange per-chunk expert counts
+ *             there.  NULL or smaller: one CTA builds the same map (slower for large T*k).
  *   Constraints: 1 <= k <= E <= 256, k <= 32, T >= 0.
  * ------------------------------------------------------------------------------------------- */
 NVFP4_API int64_t moe_rows_max(int T, int E, int k);

@@ -112,8 +112,10 @@ def permute(logits, k, renormalize=True, ids=None, weights=None, E=None, status=
     dst_row = torch.empty(T * k, dtype=I32, device=dev)
     row_slot = torch.empty(max(R, 1), dtype=I32, device=dev)
     row_w = torch.empty(max(R, 1), dtype=F32, device=dev)
+    ws_bytes = lib().moe_permute_workspace_size(T, E, k)
+    ws = torch.empty(max(ws_bytes, 1), dtype=U8, device=dev)
     call("moe_permute", _p(logits), T, E, k, int(renormalize), _p(ids), _p(weights), _p(offs),
-         _p(dst_row), _p(row_slot), _p(row_w), None, 0, _p(status), _stream())
+         _p(dst_row), _p(row_slot), _p(row_w), _p(ws), ws_bytes, _p(status), _stream())
     return dict(ids=ids, weights=weights, offs=offs, dst_row=dst_row, row_slot=row_slot,
                 row_w=row_w, R_max=R, E=E, T=T, k=k)
 

@@ -31,8 +31,9 @@ nvfp4_status_t quantize_launch(const void* x, int64_t rows, int64_t cols, int64_
                                int32_t* dev_status, cudaStream_t s);
 nvfp4_status_t permute_launch(const float* logits, int T, int E, int k, int renorm,
                               int32_t* topk_ids, float* topk_w, int32_t* offs, int32_t* dst_row,
-                              int32_t* row_slot, float* row_w, int64_t R_max,
+                              int32_t* row_slot, float* row_w, int64_t R_max, int32_t* hist_ws,
                               int32_t* dev_status, cudaStream_t s);
+size_t permute_workspace_bytes(int T, int E, int k);
 nvfp4_status_t gemm_l1(const uint8_t* a, const uint8_t* sfa, const float* gs_a, const uint8_t* w1,
                        const uint8_t* sfw1, const float* gs_w1, const int32_t* offs,
                        const int32_t* row_slot, int E, int H, int I, int64_t R_max,
@@ -46,7 +47,7 @@ nvfp4_status_t gemm_l2(const uint8_t* h, const uint8_t* sfh, const float* gs_h, 
 
 // Byte offsets of the moe_ffn_forward workspace regions (each 256-byte aligned).
 struct FfnLayout {
-  int64_t amax, gs_x, ids, w, offs, dst_row, row_slot, row_w, xq, xsf, hq, hsf, ys, total;
+  int64_t amax, gs_x, ids, w, offs, dst_row, row_slot, row_w, hist, xq, xsf, hq, hsf, ys, total;
   int64_t R_max;
 };
 
@@ -68,6 +69,7 @@ FfnLayout ffn_layout(int T, int H, int I, int E, int k) {
   L.dst_row = take(S * 4);
   L.row_slot = take(L.R_max * 4);
   L.row_w = take(L.R_max * 4);
+  L.hist = take((int64_t)permute_workspace_bytes(T, E, k));
   L.xq = take(L.R_max * H / 2);
   L.xsf = take(L.R_max * H / 16);
   L.hq = take(L.R_max * I / 2);
@@ -115,6 +117,7 @@ extern "C" nvfp4_status_t moe_ffn_forward(const void* x_bf16, const float* logit
 
   nvfp4_status_t st = permute_launch(logits, T, E, k, 1, i32(L.ids), f32(L.w), i32(L.offs),
                                      i32(L.dst_row), i32(L.row_slot), f32(L.row_w), L.R_max,
+                                     permute_workspace_bytes(T, E, k) ? i32(L.hist) : nullptr,
                                      dev_status, s);
   if (st != NVFP4_OK) return st;
   st = quantize_launch(x_bf16, T, H, H, i32(L.dst_row), k, L.R_max, base + L.xq, base + L.xsf,

@@ -84,26 +84,19 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
   }
 }
 
-// Single CTA of 32 warps.  Warp w owns the contiguous slot range [w*chunk, (w+1)*chunk), so a
-// per-warp histogram plus an exclusive scan over warps gives every slot a stable rank inside
-// its expert; __match_any_sync ranks the slots of one 32-slot step that share an expert.  Both
-// passes over the slots load kUnroll steps ahead (independent loads in flight), and one warp
-// scans the expert counts.
+// Slots [lo, hi) of one CTA of 32 warps.  Warp w owns a contiguous part of the range, so a
+// per-warp histogram plus an exclusive scan over warps gives every slot a stable rank inside its
+// expert; __match_any_sync ranks the slots of one 32-slot step that share an expert.  Both passes
+// over the slots load kUnroll steps ahead (independent loads in flight).
 constexpr int kUnroll = 8;
+// From this many slots the row map is built by many CTAs (two launches: per-chunk expert
+// histograms, then ranks and writes): one SM issuing every scattered row store was the limit.
+constexpr int kMultiMinSlots = 4096;
+constexpr int kChunkSlots = 2048;  // slots per CTA in the multi-CTA form
 
-__global__ void __launch_bounds__(1024) permute_kernel(
-    const int32_t* __restrict__ ids, const float* __restrict__ w, int S, int k, int E,
-    int64_t R_max, int32_t* __restrict__ offs_out, int32_t* __restrict__ dst_row,
-    int32_t* __restrict__ row_slot, float* __restrict__ row_w, int32_t* __restrict__ dev_status) {
-  __shared__ int hist[32][kMaxE];
-  __shared__ int cnt[kMaxE];
-  __shared__ int offs[kMaxE + 1];
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  for (int i = tid; i < 32 * kMaxE; i += blockDim.x) (&hist[0][0])[i] = 0;
-  __syncthreads();
-  const int chunk = (S + 31) / 32;
-  const int lo = min(S, warp * chunk), hi = min(S, lo + chunk);
-  bool bad = false;
+__device__ __forceinline__ void warp_histogram(const int32_t* __restrict__ ids, int lo, int hi,
+                                               int E, int lane, int* __restrict__ hist_w,
+                                               bool& bad) {
   for (int base = lo; base < hi; base += 32 * kUnroll) {
     int e[kUnroll];
 #pragma unroll
@@ -114,19 +107,69 @@ __global__ void __launch_bounds__(1024) permute_kernel(
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
       if (e[u] >= E) bad = true;
-      else if (e[u] >= 0) atomicAdd(&hist[warp][e[u]], 1);
+      else if (e[u] >= 0) atomicAdd(&hist_w[e[u]], 1);
     }
   }
+}
+
+// Per-chunk expert histograms of the multi-CTA form: hist_g[c][e] = slots of chunk c routed to e.
+__global__ void __launch_bounds__(1024) permute_count_kernel(const int32_t* __restrict__ ids, int S,
+                                                              int E, int32_t* __restrict__ hist_g,
+                                                              int32_t* __restrict__ dev_status) {
+  __shared__ int hist[kMaxE];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  for (int i = tid; i < kMaxE; i += blockDim.x) hist[i] = 0;
+  __syncthreads();
+  const int c0 = blockIdx.x * kChunkSlots, c1 = min(S, c0 + kChunkSlots);
+  const int per = (c1 - c0 + 31) / 32;
+  const int lo = min(c1, c0 + warp * per), hi = min(c1, lo + per);
+  bool bad = false;
+  warp_histogram(ids, lo, hi, E, lane, hist, bad);
   if (bad) report(dev_status, NVFP4_DEVERR_BAD_INDEX);
+  __syncthreads();
+  for (int e = tid; e < E; e += blockDim.x) hist_g[(int64_t)blockIdx.x * E + e] = hist[e];
+}
+
+// kMulti = false: one CTA over all S slots.  kMulti = true: CTA c over chunk c, with the expert
+// totals and the chunk's base per expert taken from hist_g (nch chunks).
+template <bool kMulti>
+__global__ void __launch_bounds__(1024) permute_kernel(
+    const int32_t* __restrict__ ids, const float* __restrict__ w, int S, int E, int64_t R_max,
+    const int32_t* __restrict__ hist_g, int nch, int32_t* __restrict__ offs_out,
+    int32_t* __restrict__ dst_row, int32_t* __restrict__ row_slot, float* __restrict__ row_w,
+    int32_t* __restrict__ dev_status) {
+  __shared__ int hist[32][kMaxE];
+  __shared__ int cnt[kMaxE];
+  __shared__ int offs[kMaxE + 1];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  for (int i = tid; i < 32 * kMaxE; i += blockDim.x) (&hist[0][0])[i] = 0;
+  __syncthreads();
+  const int c0 = kMulti ? blockIdx.x * kChunkSlots : 0;
+  const int c1 = kMulti ? min(S, c0 + kChunkSlots) : S;
+  const int per = (c1 - c0 + 31) / 32;
+  const int lo = min(c1, c0 + warp * per), hi = min(c1, lo + per);
+  bool bad = false;
+  warp_histogram(ids, lo, hi, E, lane, hist[warp], bad);
+  if (bad && !kMulti) report(dev_status, NVFP4_DEVERR_BAD_INDEX);  // multi: the count kernel
   __syncthreads();
   if (tid < E) {
     int run = 0;
+    if (kMulti) {  // this chunk's base and the expert's total over all chunks
+      int before = 0, total = 0;
+      for (int c = 0; c < nch; ++c) {
+        const int v = __ldg(hist_g + (int64_t)c * E + tid);
+        if (c < (int)blockIdx.x) before += v;
+        total += v;
+      }
+      run = before;
+      cnt[tid] = total;
+    }
     for (int ww = 0; ww < 32; ++ww) {
       const int c = hist[ww][tid];
       hist[ww][tid] = run;
       run += c;
     }
-    cnt[tid] = run;
+    if (!kMulti) cnt[tid] = run;
   }
   __syncthreads();
   if (warp == 0) {  // offs = exclusive scan of the 128-padded counts (lane l: experts 8l..8l+7)
@@ -154,7 +197,7 @@ __global__ void __launch_bounds__(1024) permute_kernel(
     if (lane == 31 && E == kMaxE) offs[E] = run;
   }
   __syncthreads();
-  if (tid <= E) offs_out[tid] = offs[tid];
+  if (blockIdx.x == 0 && tid <= E) offs_out[tid] = offs[tid];
   const unsigned lt_mask = (1u << lane) - 1u;
   for (int base = lo; base < hi; base += 32 * kUnroll) {
     int e[kUnroll];
@@ -187,14 +230,17 @@ __global__ void __launch_bounds__(1024) permute_kernel(
       __syncwarp();
     }
   }
-  // padding rows of every segment, then the unused tail up to R_max
-  for (int e = warp; e < E; e += 32) {
+  // padding rows of every segment, then the unused tail up to R_max (spread over the CTAs)
+  const int nwarps = 32 * gridDim.x;
+  const int gwarp = blockIdx.x * 32 + warp;
+  for (int e = gwarp; e < E; e += nwarps) {
     for (int r = offs[e] + cnt[e] + lane; r < offs[e + 1]; r += 32) {
       row_slot[r] = -1;
       row_w[r] = 0.0f;
     }
   }
-  for (int64_t r = offs[E] + tid; r < R_max; r += blockDim.x) {
+  for (int64_t r = offs[E] + blockIdx.x * (int64_t)blockDim.x + tid; r < R_max;
+       r += (int64_t)gridDim.x * blockDim.x) {
     row_slot[r] = -1;
     row_w[r] = 0.0f;
   }
@@ -202,17 +248,36 @@ __global__ void __launch_bounds__(1024) permute_kernel(
 
 }  // namespace
 
+int permute_chunks(int T, int k) {
+  const int64_t S = (int64_t)T * k;
+  return S >= kMultiMinSlots ? static_cast<int>((S + kChunkSlots - 1) / kChunkSlots) : 0;
+}
+
+size_t permute_workspace_bytes(int T, int E, int k) {
+  return (size_t)permute_chunks(T, k) * (size_t)E * sizeof(int32_t);
+}
+
 nvfp4_status_t permute_launch(const float* logits, int T, int E, int k, int renorm,
                               int32_t* topk_ids, float* topk_w, int32_t* offs, int32_t* dst_row,
-                              int32_t* row_slot, float* row_w, int64_t R_max,
+                              int32_t* row_slot, float* row_w, int64_t R_max, int32_t* hist_ws,
                               int32_t* dev_status, cudaStream_t s) {
   if (logits != nullptr && T > 0) {
     topk_kernel<<<(T + 7) / 8, 256, 0, s>>>(logits, T, E, k, renorm, topk_ids, topk_w);
     nvfp4_status_t st = check_launch("topk_kernel");
     if (st != NVFP4_OK) return st;
   }
-  permute_kernel<<<1, 1024, 0, s>>>(topk_ids, topk_w, T * k, k, E, R_max, offs, dst_row,
-                                    row_slot, row_w, dev_status);
+  const int S = T * k;
+  const int nch = permute_chunks(T, k);
+  if (nch > 0 && hist_ws != nullptr) {
+    permute_count_kernel<<<nch, 1024, 0, s>>>(topk_ids, S, E, hist_ws, dev_status);
+    nvfp4_status_t st = check_launch("permute_count_kernel");
+    if (st != NVFP4_OK) return st;
+    permute_kernel<true><<<nch, 1024, 0, s>>>(topk_ids, topk_w, S, E, R_max, hist_ws, nch, offs,
+                                              dst_row, row_slot, row_w, dev_status);
+    return check_launch("permute_kernel");
+  }
+  permute_kernel<false><<<1, 1024, 0, s>>>(topk_ids, topk_w, S, E, R_max, nullptr, 0, offs,
+                                           dst_row, row_slot, row_w, dev_status);
   return check_launch("permute_kernel");
 }
 
@@ -225,12 +290,16 @@ extern "C" int64_t moe_rows_max(int T, int E, int k) {
   return nvfp4::round_up(S + 127 * busy, 128);
 }
 
-extern "C" size_t moe_permute_workspace_size(int, int, int) { return 0; }
+extern "C" size_t moe_permute_workspace_size(int T, int E, int k) {
+  if (T <= 0 || E <= 0 || k <= 0) return 0;
+  return nvfp4::permute_workspace_bytes(T, E, k);
+}
 
 extern "C" nvfp4_status_t moe_permute(const float* logits, int T, int E, int k, int renormalize,
                                       int32_t* topk_ids, float* topk_w, int32_t* offs,
-                                      int32_t* dst_row, int32_t* row_slot, float* row_w, void*,
-                                      size_t, int32_t* dev_status, nvfp4_stream_t stream) {
+                                      int32_t* dst_row, int32_t* row_slot, float* row_w, void* ws,
+                                      size_t ws_bytes, int32_t* dev_status,
+                                      nvfp4_stream_t stream) {
   using namespace nvfp4;
   if (T < 0 || E < 1 || E > kMaxE || k < 1 || k > kMaxK || k > E) return NVFP4_ERR_UNSUPPORTED_SHAPE;
   if ((int64_t)T * k > (int64_t)1 << 30) return NVFP4_ERR_UNSUPPORTED_SHAPE;
@@ -238,10 +307,14 @@ extern "C" nvfp4_status_t moe_permute(const float* logits, int T, int E, int k, 
   if (T > 0 && (topk_ids == nullptr || topk_w == nullptr || dst_row == nullptr ||
                 row_slot == nullptr || row_w == nullptr))
     return NVFP4_ERR_INVALID_ARG;
-  const void* ptrs[] = {logits, topk_ids, topk_w, offs, dst_row, row_slot, row_w};
+  const void* ptrs[] = {logits, topk_ids, topk_w, offs, dst_row, row_slot, row_w, ws};
   for (const void* p : ptrs)
     if (reinterpret_cast<uintptr_t>(p) & 3u) return NVFP4_ERR_MISALIGNED;
+  // the multi-CTA form needs the workspace; without it one CTA builds the map (same result)
+  int32_t* hist_ws = ws != nullptr && ws_bytes >= permute_workspace_bytes(T, E, k)
+                         ? static_cast<int32_t*>(ws)
+                         : nullptr;
   return permute_launch(logits, T, E, k, renormalize, topk_ids, topk_w, offs, dst_row, row_slot,
-                        row_w, moe_rows_max(T, E, k), dev_status,
+                        row_w, moe_rows_max(T, E, k), hist_ws, dev_status,
                         reinterpret_cast<cudaStream_t>(stream));
 }

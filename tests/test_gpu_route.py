@@ -64,3 +64,27 @@ def test_route_empty_batch():
     p = nv.permute(lg, 2)
     torch.cuda.synchronize()
     assert p["offs"].cpu().tolist() == [0] * 9 and p["R_max"] == 0
+
+
+def test_permute_without_workspace_matches_multi_cta():
+    """From 4096 slots the row map is built by many CTAs through the workspace; without one, a
+    single CTA builds it.  Both must give the same map."""
+    from nvfp4_block_scaled_gsa_b200._native import call, lib
+    cfg = CONFIGS["mid"]
+    lg = gen_logits(cfg).to(DEV)
+    a = nv.permute(lg, cfg.k)
+    assert lib().moe_permute_workspace_size(cfg.T, cfg.E, cfg.k) > 0
+    T, E, k = cfg.T, cfg.E, cfg.k
+    R = a["R_max"]
+    ids = torch.empty(T, k, dtype=torch.int32, device=DEV)
+    w = torch.empty(T, k, dtype=torch.float32, device=DEV)
+    offs = torch.empty(E + 1, dtype=torch.int32, device=DEV)
+    dst = torch.empty(T * k, dtype=torch.int32, device=DEV)
+    rs = torch.empty(R, dtype=torch.int32, device=DEV)
+    rw = torch.empty(R, dtype=torch.float32, device=DEV)
+    call("moe_permute", lg.data_ptr(), T, E, k, 1, ids.data_ptr(), w.data_ptr(), offs.data_ptr(),
+         dst.data_ptr(), rs.data_ptr(), rw.data_ptr(), None, 0, None,
+         torch.cuda.current_stream().cuda_stream)
+    torch.cuda.synchronize()
+    assert torch.equal(offs, a["offs"]) and torch.equal(dst, a["dst_row"])
+    assert torch.equal(rs, a["row_slot"]) and torch.equal(rw, a["row_w"])
