@@ -261,6 +261,19 @@ NVFP4_API nvfp4_status_t moe_ffn_forward(const void* x_bf16, const float* logits
  *   the stream; returns NVFP4_ERR_TIMEOUT / NVFP4_ERR_BAD_INDEX when the matching bit is set.
  *   nvfp4_last_error: the last CUDA error string seen by this library on this thread.
  * ------------------------------------------------------------------------------------------- */
+/* ---------------------------------------------------------------------------------------------
+ * nvfp4_wait_selftest — diagnostic (no counterpart in the pages): runs one CTA whose first warp
+ * waits, with the library's bounded wait and a limit of limit_ns, on an mbarrier that nothing
+ * arrives on.  When the wait runs out it raises the CTA's abort flag; a second warp waiting on
+ * another such barrier (default 2 s limit) must then give up early, as the grouped GEMM's roles
+ * do; NVFP4_DEVERR_TIMEOUT is ORed into *dev_status.  No fault, no trap, no unbounded wait: it
+ * checks the timeout path on a GPU and leaves the context usable.
+ *   limit_ns    1 .. 2e9
+ *   elapsed_ns  optional device uint64: time from the start of the waits to the report
+ * ------------------------------------------------------------------------------------------- */
+NVFP4_API nvfp4_status_t nvfp4_wait_selftest(int64_t limit_ns, int32_t* dev_status,
+                                             uint64_t* elapsed_ns, nvfp4_stream_t stream);
+
 NVFP4_API nvfp4_status_t nvfp4_read_status(const int32_t* dev_status, int32_t* host_code,
                                  nvfp4_stream_t stream);
 NVFP4_API const char* nvfp4_last_error(void);

@@ -47,6 +47,7 @@ SIGNATURES = {
                                 c_void, c_void, c_void, c_void, c_void, c_void, c_void, c_size,
                                 c_void, c_void]),
     "nvfp4_read_status": (c_int, [c_void, c_void, c_void]),
+    "nvfp4_wait_selftest": (c_int, [c_i64, c_void, c_void, c_void]),
     "nvfp4_last_error": (c_char_p, []),
     "nvfp4_abi_version": (c_int, []),
 }

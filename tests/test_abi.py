@@ -110,6 +110,13 @@ def test_gemms_reject_bad_shapes(L):
                              None) == 1
 
 
+def test_wait_selftest_rejects_bad_arguments(L):
+    f = FAKE
+    assert L.nvfp4_wait_selftest(0, f, None, None) == 1
+    assert L.nvfp4_wait_selftest(3_000_000_000, f, None, None) == 1  # above the 2 s wait limit
+    assert L.nvfp4_wait_selftest(10_000_000, None, None, None) == 1
+
+
 def test_w1_row_map_is_the_documented_interleave(L):
     I = 192
     buf = (ctypes.c_int32 * (2 * I))()
