@@ -112,6 +112,24 @@ def load_peaks():
     return dict(hbm=6650.0, bf16=1590.0, bf16_sust=1400.0, src="fallback")
 
 
+# ----------------------------------------------------------------------------- ranks
+
+def slowest_rank_ms(ms, world, device="cpu"):
+    """The timed region's length on the slowest rank: every rank passes its own CUDA-event time
+    and gets the maximum over ranks (a no-op for one process)."""
+    import torch
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_step_per_rank, steps, world, total_ms):
+    """Units per second of the whole job: every rank's units over the slowest rank's time."""
+    return world * units_per_step_per_rank * steps / (total_ms * 1e-3)
+
+
 # ----------------------------------------------------------------------------- clocks
 
 class ClockSampler:
@@ -304,13 +322,10 @@ def run_ours(args):
     if code != 0:
         raise RuntimeError(f"device status {code} after the timed region")
 
-    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms = float(t.item())
+    total_ms = slowest_rank_ms(total_ms, world, dev)
     ms_step = total_ms / K
-    value = world * acc["bytes"] * K / (total_ms * 1e-3) / 1e9
-    tflops = world * acc["flops"] * K / (total_ms * 1e-3) / 1e12
+    value = whole_job_rate(acc["bytes"], K, world, total_ms) / 1e9
+    tflops = whole_job_rate(acc["flops"], K, world, total_ms) / 1e12
 
     # ---- end to end through moe_ffn_forward with host buffers (pinned), copies timed
     x_h = x_cpu.pin_memory()
@@ -338,12 +353,10 @@ def run_ours(args):
         e2e_step()
     e2.record()
     torch.cuda.synchronize()
-    t2 = torch.tensor([s2.elapsed_time(e2)], dtype=torch.float64, device=dev)
     if world > 1:
         dist.barrier()
-        dist.all_reduce(t2, op=dist.ReduceOp.MAX)
-    e2e_ms = float(t2.item())
-    e2e_value = world * acc["bytes"] * K / (e2e_ms * 1e-3) / 1e9
+    e2e_ms = slowest_rank_ms(s2.elapsed_time(e2), world, dev)
+    e2e_value = whole_job_rate(acc["bytes"], K, world, e2e_ms) / 1e9
     h2d = x_h.numel() * x_h.element_size() + lg_h.numel() * lg_h.element_size()
     d2h = out_h.numel() * out_h.element_size()
 
@@ -636,12 +649,11 @@ def run_sweep(args):
     torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize()
     clocks = sampler.stop() if sampler else None
-    t = torch.tensor([start.elapsed_time(stop)], dtype=torch.float64, device=dev)
     if world > 1:
         dist.barrier()
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms = float(t.item()) / K
-    value = world * flops / (ms * 1e-3) / 1e12
+    total_ms = slowest_rank_ms(start.elapsed_time(stop), world, dev)
+    ms = total_ms / K
+    value = whole_job_rate(flops, K, world, total_ms) / 1e12
 
     # end to end: bf16 A from pinned host memory, quantize, GEMM, bf16 result back to the host
     a_h = a_bf16.cpu().pin_memory()
