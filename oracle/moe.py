@@ -103,7 +103,7 @@ def grouped_gemm(a, b_dequant, offs, rows_valid=None):
 
 
 def moe_ffn(x, logits, k, w1, w2, gs_h, renormalize=True, ids=None, weights=None,
-            keep=False, experts=None):
+            keep=False, experts=None, gs_x=None):
     """The whole expert FFN, step by step.
 
     x        (T, H) float (the bf16 activations, as float32)
@@ -112,6 +112,9 @@ def moe_ffn(x, logits, k, w1, w2, gs_h, renormalize=True, ids=None, weights=None
              then up rows) and N = H
     gs_h     float32 static global scale of the intermediate
     experts  optional iterable restricting which experts are evaluated (for sampled checks)
+    gs_x     optional global scale of x; by default computed from x.  A sampled check passes the
+             scale of the whole batch when x holds only some of its rows (a token's output
+             depends on the batch only through this scale)
 
     Returns dict: out float64 (T, H), routing, permutation, gs_x, and (keep=True) per-row
     intermediates c1 (R, 2I), h32 (R, I), h_codes (R, I), h_sf (R, I/16), y (R, H).
@@ -123,7 +126,9 @@ def moe_ffn(x, logits, k, w1, w2, gs_h, renormalize=True, ids=None, weights=None
     if ids is None:
         ids, weights = route_topk(logits, k, renormalize)
     perm = permute(ids, weights, E)
-    gs_x = global_scale(x)
+    if gs_x is None:
+        gs_x = global_scale(x)
+    gs_x = np.float32(gs_x)
     xc, xsf = quantize(x, gs_x)
     out = np.zeros((T, H), dtype=np.float64)
     R = perm["R"]
