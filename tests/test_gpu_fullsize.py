@@ -68,3 +68,34 @@ def test_ffn_full_size_sampled_token(name, tok, pool):
     want = M.bf16_round(ref)
     assert rel_fro(got, want) <= 1e-3
     assert cosine(got, want) >= 0.9999
+
+
+def test_grouped_gemm_sweep_full_size_sampled_rows(pool):
+    """The standalone grouped GEMM at the sweep shape (E=32, M_g ~ U{0..4096}, K=7168, N=4096,
+    bf16 out, pair tiles): rows sampled from two groups against the oracle, which quantizes those
+    rows itself with the global scale of the whole A (from its amax, taken on the host)."""
+    import sys
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    import bench
+    cfg = CONFIGS["sweep"]
+    m, offs, a, w = bench.sweep_operands(cfg, DEV)
+    codes, sf, gs = nv.quantize(a)
+    out = nv.grouped_gemm(codes, sf, gs, w, offs, out_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    a_cpu = a.cpu()
+    gs_ref = Q.global_scale(np.array([[float(a_cpu.abs().max())]], np.float32))
+    order = np.argsort(m)
+    groups = [int(order[-1]), int(order[len(order) // 2])]  # the largest and a middle-sized one
+    wf = [gen_weight_expert(cfg.seed, 1, g, cfg.N, cfg.K, device=DEV).float().cpu().numpy()
+          for g in groups]
+    qw = pool.map(M.QuantWeights.from_float, [x[None] for x in wf])
+    offs_h = offs.cpu().numpy()
+    for g, q in zip(groups, qw):
+        rows = offs_h[g] + np.array([0, m[g] // 2, m[g] - 1])
+        xr = a_cpu[rows].float().numpy()
+        c, s = Q.quantize(xr, gs_ref)
+        ref = Q.dequantize(c, s, gs_ref) @ q.dequant(0).T
+        got = out[torch.as_tensor(rows, device=DEV)].float().cpu().numpy().astype(np.float64)
+        want = M.bf16_round(ref)
+        assert rel_fro(got, want) <= 1e-3
+        assert cosine(got, want) >= 0.9999
