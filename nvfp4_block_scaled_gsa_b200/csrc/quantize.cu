@@ -19,18 +19,30 @@ __global__ void __launch_bounds__(kThreads) amax_kernel(const __nv_bfloat16* __r
                                                         uint32_t* __restrict__ amax_bits) {
   const int64_t vec_per_row = cols / 8;
   const int64_t nvec = rows * vec_per_row;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   uint32_t m = 0;  // max of |bf16| bit patterns (sign cleared)
-  for (int64_t v = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; v < nvec;
-       v += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t r = v / vec_per_row, c = (v - r * vec_per_row) * 8;
-    const uint4 q = __ldg(reinterpret_cast<const uint4*>(x + r * ld + c));
+  auto fold = [&](const uint4& q) {
     const uint32_t w[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       m = max(m, w[i] & 0x7FFFu);
       m = max(m, (w[i] >> 16) & 0x7FFFu);
     }
+  };
+  auto load = [&](int64_t v) {
+    const int64_t r = v / vec_per_row, c = (v - r * vec_per_row) * 8;
+    return __ldg(reinterpret_cast<const uint4*>(x + r * ld + c));
+  };
+  int64_t v = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  for (; v + 3 * stride < nvec; v += 4 * stride) {  // four independent loads in flight
+    const uint4 q0 = load(v), q1 = load(v + stride), q2 = load(v + 2 * stride),
+                q3 = load(v + 3 * stride);
+    fold(q0);
+    fold(q1);
+    fold(q2);
+    fold(q3);
   }
+  for (; v < nvec; v += stride) fold(load(v));
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
   __shared__ uint32_t red[kThreads / 32];
@@ -61,28 +73,44 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(
   } else {
     gs = __ldg(gs_io);
   }
-  if (gid >= nblk) return;
-  const int64_t r = gid / nblk_row, c = gid - r * nblk_row;
-  const uint4* src = reinterpret_cast<const uint4*>(x + r * ld + c * 16);
-  const uint4 q0 = __ldg(src), q1 = __ldg(src + 1);
-  const uint32_t w[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
-  float v[16];
-  float amax = 0.0f;
+  // no early return: the 4 lanes of a 4-block group exchange their scale bytes with shuffles
+  // (blocks 4g..4g+3 of a row are 4 consecutive lanes, since cols % 64 == 0)
+  const bool valid = gid < nblk;
+  const int64_t r = valid ? gid / nblk_row : 0, c = valid ? gid - r * nblk_row : 0;
+  uint32_t sbyte = 0;
+  uint2 packed = make_uint2(0u, 0u);
+  if (valid) {
+    const uint4* src = reinterpret_cast<const uint4*>(x + r * ld + c * 16);
+    const uint4 q0 = __ldg(src), q1 = __ldg(src + 1);
+    const uint32_t w[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+    float v[16];
+    float amax = 0.0f;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    v[2 * i] = __uint_as_float(w[i] << 16);
-    v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-    amax = fmaxf(amax, fmaxf(fabsf(v[2 * i]), fabsf(v[2 * i + 1])));
+    for (int i = 0; i < 8; ++i) {
+      v[2 * i] = __uint_as_float(w[i] << 16);
+      v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+      amax = fmaxf(amax, fmaxf(fabsf(v[2 * i]), fabsf(v[2 * i + 1])));
+    }
+    float rcp;
+    sbyte = nvfp4_block_scale(amax, gs, rcp);
+    packed.x = nvfp4_pack8(v, rcp);
+    packed.y = nvfp4_pack8(v + 8, rcp);
   }
-  float rcp;
-  const uint32_t sbyte = nvfp4_block_scale(amax, gs, rcp);
-  uint2 packed;
-  packed.x = nvfp4_pack8(v, rcp);
-  packed.y = nvfp4_pack8(v + 8, rcp);
+  // the group's 4 scale bytes, assembled in its first lane (scale columns 4g..4g+3 are one
+  // aligned 4-byte group of the tiled layout)
+  uint32_t sword = sbyte;
+  sword |= __shfl_down_sync(0xffffffffu, sbyte, 1) << 8;
+  sword |= __shfl_down_sync(0xffffffffu, sbyte, 2) << 16;
+  sword |= __shfl_down_sync(0xffffffffu, sbyte, 3) << 24;
+  if (!valid) return;
+  const bool leader = (c & 3) == 0;
   const int64_t row_bytes = cols / 2;
+  auto put = [&](int64_t d) {
+    *reinterpret_cast<uint2*>(codes + d * row_bytes + c * 8) = packed;
+    if (leader) *reinterpret_cast<uint32_t*>(sf + sf_offset(d, c, nblk_row)) = sword;
+  };
   if (dst_row == nullptr) {
-    *reinterpret_cast<uint2*>(codes + r * row_bytes + c * 8) = packed;
-    sf[sf_offset(r, c, nblk_row)] = static_cast<uint8_t>(sbyte);
+    put(r);
     return;
   }
   for (int j = 0; j < k; ++j) {
@@ -92,8 +120,7 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(
       report(dev_status, NVFP4_DEVERR_BAD_INDEX);
       continue;
     }
-    *reinterpret_cast<uint2*>(codes + d * row_bytes + c * 8) = packed;
-    sf[sf_offset(d, c, nblk_row)] = static_cast<uint8_t>(sbyte);
+    put(d);
   }
 }
 
