@@ -182,17 +182,6 @@ __device__ __forceinline__ void tc_fence_before() {
 __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
-__device__ __forceinline__ void tc_commit(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                   bar)
-               : "memory");
-}
-// Arrive on `cluster_bar` (this CTA's or the peer's) once the pair MMAs issued so far complete.
-__device__ __forceinline__ void tc_commit_pair(uint32_t cluster_bar) {
-  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                   cluster_bar)
-               : "memory");
-}
 // Shared-memory matrix descriptor (sm_100 format): start>>4 in [0,14), LBO>>4 in [16,30),
 // SBO>>4 in [32,46), version 1 in [46,48), layout type in [61,64) (0 none, 2 = 128-byte swizzle).
 __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo,
@@ -205,32 +194,11 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint
   d |= static_cast<uint64_t>(layout & 7u) << 61;
   return d;
 }
-// D(tmem) (+)= A(smem) * B(smem)^T with E2M1 operands and UE4M3 scales per 16 elements (K = 64).
-__device__ __forceinline__ void tc_mma_nvf4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
-                                            uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
-                                            uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X"
-      " [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
-      : "memory");
-}
+// D(tmem) (+)= A(smem) * B(smem)^T with E2M1 operands and UE4M3 scales per 16 elements (K = 64),
+// from tensor memory addresses of the scales.
 // Pair form: M = 256 rows, 128 from each CTA's shared memory; B's N columns split in halves,
 // the first from the leader's shared memory; every CTA keeps its 128 rows x N accumulator and
 // reads its own scale factors (its A rows, all N of B) from its own tensor memory.
-__device__ __forceinline__ void tc_mma_nvf4_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
-                                                 uint32_t idesc, uint32_t sfa_tmem,
-                                                 uint32_t sfb_tmem, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.scale_vec::4X"
-      " [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
-      : "memory");
-}
 // Whole-warp forms: every lane of the warp executes them and elect.sync picks the one lane that
 // issues (the lowest active lane, so MMAs and their commits come from the same thread).  A loop
 // that issues MMAs from a single divergent lane costs about twice as many cycles per MMA.
