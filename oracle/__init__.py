@@ -12,9 +12,10 @@ quant     NVFP4 quantizer (global scale from amax, FP8-round-tripped block scale
           dequantizer, and the 128x4 scale-factor tile index map
 routing   softmax top-k routing and the expert-bucketed row permutation
 moe       grouped GEMM, SwiGLU, re-quantization, weighted scatter, whole FFN
+dense     dense NVFP4 linear, and the RMSNorm fused in front of the quantizer
 
 Every function says which page passage it follows.  Functions with no independent pin say
 "parity unpinned" in their docstring.
 """
 
-from . import formats, quant, routing, moe  # noqa: F401
+from . import formats, quant, routing, moe, dense  # noqa: F401
