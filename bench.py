@@ -1,6 +1,7 @@
 """Throughput of the NVFP4 MoE expert-FFN hot path on B200 (one JSON line on rank 0).
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--config decode|mid|prefill|tiny|sweep]
+    python bench.py [--gpus N] [--steps K] [--warmup W]
+                    [--config decode|mid|prefill|tiny|sweep|dense_decode|dense_prefill]
                     [--impl ours|reference] [--no-cpu-baseline] [--experts E] [--tokens T]
 
 A step is one pass of the whole path over one batch: routing (top-k + expert buckets), amax ->
@@ -17,6 +18,11 @@ scaling is weak and `value` sums the ranks' bytes over the slowest rank's time.
 
 --config sweep times the standalone 2D x 3D grouped GEMM instead (E=32 groups, M_g ~ U{0..4096},
 K=7168, N=4096, bf16 output): a step is one grouped-GEMM launch over NVFP4 operands already in HBM.
+
+--config dense_decode | dense_prefill times the dense NVFP4 linear with the RMSNorm fused into its
+activation quantizer (the MoE shared expert's gate/up projection: M = 16 or 8192 rows, K = 7168,
+N = 4096): a step is RMSNorm + amax -> quantize -> dense GEMM, bf16 out, with L2 flushed before
+every step (the 16.5 MB weight would otherwise stay in the 126 MB L2).
 
 --impl reference times the CPU oracle (numpy, float64) on a bounded sample of the same workload.
 """
@@ -750,12 +756,270 @@ def sweep_cpu_baseline(cfg, m, offs, codes, sf, gs, w):
                       f"NVFP4 operands) in {dt:.2f} s"}
 
 
+# ----------------------------------------------------------------------------- dense linear
+
+DENSE_METRIC = ("dense NVFP4 linear (RMSNorm fused) on 1 B200, % of NVFP4 tensor/HBM roofline")
+L2_FLUSH_BYTES = 256 << 20  # written between steps: larger than the 126 MB L2
+
+
+def dense_algorithmic(cfg):
+    """Bytes and FLOPs of one dense step and of its GEMM launch: x read as bf16 (and gamma),
+    activation codes written and read once, weight codes + scales read once, bf16 out written."""
+    a_q = cfg.M * cfg.K * FP4_ELEM_BYTES
+    w_q = cfg.N * cfg.K * FP4_ELEM_BYTES
+    out = cfg.M * cfg.N * 2
+    return dict(flops=cfg.flops(), bytes=cfg.M * cfg.K * 2 + cfg.K * 2 + 2 * a_q + w_q + out,
+                gemm_bytes=a_q + w_q + out)
+
+
+def dense_operands(cfg, dev):
+    import torch
+
+    import nvfp4_block_scaled_gsa_b200 as nv
+    from synth import gen_dense
+    x, gamma, w = gen_dense(cfg, device=dev)
+    wd = nv.quantize_weights(lambda e: w, 1, cfg.N, cfg.K, device=dev)
+    return x, gamma.to(dev), wd, torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+
+def _timed_steps(step, flush, K):
+    """Device time of K steps, each timed by its own pair of events after an L2 flush."""
+    import torch
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(K)]
+    for a, b in evs:
+        flush.zero_()
+        a.record()
+        step()
+        b.record()
+    torch.cuda.synchronize()
+    return sum(a.elapsed_time(b) for a, b in evs)
+
+
+def run_dense(args):
+    import torch
+    import torch.distributed as dist
+
+    import nvfp4_block_scaled_gsa_b200 as nv
+    from synth import CONFIGS
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local = int(os.environ.get("LOCAL_RANK", 0))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    cfg = CONFIGS[args.config]
+    x_cpu, gamma, wd, flush = dense_operands(cfg, dev)
+    x = x_cpu.to(dev)
+    out = torch.empty(cfg.M, cfg.N, dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(nv.linear_workspace_bytes(cfg.M, cfg.N, cfg.K), dtype=torch.uint8, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    acc = dense_algorithmic(cfg)
+
+    def step():
+        nv.linear(x, wd, gamma=gamma, eps=cfg.eps, out=out, ws=ws, status=status)
+
+    # the step as a CUDA graph (one launch of its 3-4 kernels: no host gaps at decode sizes)
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, capture_error_mode="thread_local"):
+        step()
+    torch.cuda.synchronize()
+
+    sampler = ClockSampler(local) if rank == 0 else None
+    t_end = time.time() + args.soak
+    while time.time() < t_end:
+        for _ in range(8):
+            graph.replay()
+        torch.cuda.synchronize()
+    K = args.steps
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    torch.cuda.nvtx.range_push("timed")
+    total_ms = _timed_steps(graph.replay, flush, K)
+    torch.cuda.nvtx.range_pop()
+    clocks = sampler.stop() if sampler else None
+    if world > 1:
+        dist.barrier()
+    eager_ms = _timed_steps(step, flush, max(1, min(K, 50)))
+    eager_ms /= max(1, min(K, 50))
+
+    # the GEMM stage alone (the dominant kernel, plus its split-K reduction), on the codes the
+    # fused quantizer wrote
+    Mp = (cfg.M + 127) // 128 * 128
+    codes, sf, gs = nv.rmsnorm_quantize(x, gamma, cfg.eps, out_rows=Mp)
+    gws_n = int(nv.lib().nvfp4_gemm_dense_workspace_size(cfg.M, cfg.N, cfg.K))
+    gws = torch.empty(max(gws_n, 256), dtype=torch.uint8, device=dev)
+    kg = max(1, min(K, 50))
+    gemm_ms = _timed_steps(lambda: nv.gemm_dense(codes, sf, gs, cfg.M, wd, out=out, ws=gws), flush,
+                           kg) / kg
+    split = nv.lib().nvfp4_gemm_dense_workspace_size(cfg.M, cfg.N, cfg.K) > 0
+    code, rc = nv.read_status(status)
+    if code != 0:
+        raise RuntimeError(f"device status {code} after the timed region")
+
+    total_ms = slowest_rank_ms(total_ms, world, dev)
+    ms_step = total_ms / K
+    gbs = whole_job_rate(acc["bytes"], K, world, total_ms) / 1e9
+    tflops = whole_job_rate(acc["flops"], K, world, total_ms) / 1e12
+
+    # end to end through nvfp4_linear: x from pinned host memory, bf16 result back to the host
+    x_h = x_cpu.pin_memory()
+    out_h = torch.empty(cfg.M, cfg.N, dtype=torch.bfloat16).pin_memory()
+    x_d = torch.empty_like(x)
+
+    def e2e_step():
+        x_d.copy_(x_h, non_blocking=True)
+        nv.linear(x_d, wd, gamma=gamma, eps=cfg.eps, out=out, ws=ws, status=status)
+        out_h.copy_(out, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    ke = max(1, min(K, 50))
+    e2e_ms = slowest_rank_ms(_timed_steps(e2e_step, flush, ke), world, dev) / ke
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = dense_cpu_baseline(cfg)
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    peaks = load_peaks()
+    fp4_peak = peaks["bf16"] * FP4_PER_BF16
+    tensor_bound = acc["flops"] / acc["gemm_bytes"] > fp4_peak * 1e12 / (peaks["hbm"] * 1e9)
+    kname = "grouped_gemm_kernel<PLAIN_F32> + splitk_reduce_kernel" if split else \
+        "grouped_gemm_kernel<PLAIN_BF16>"
+    g_tflops = acc["flops"] / (gemm_ms * 1e-3) / 1e12
+    g_gbs = acc["gemm_bytes"] / (gemm_ms * 1e-3) / 1e9
+    if tensor_bound:
+        value, unit = tflops, "TFLOP/s"
+        roof = {"bound": "tensor", "kernel": kname, "achieved": round(g_tflops, 1),
+                "peak": round(fp4_peak, 1), "unit": "TFLOP/s", "frac": round(g_tflops / fp4_peak, 4),
+                "traffic": None, "algorithmic_flops_per_launch": int(acc["flops"]),
+                "peak_source": f"{peaks['src']} bf16 burst x {FP4_PER_BF16} (nominal FP4/BF16 "
+                               "dense ratio)",
+                "step_frac": round(tflops / world / fp4_peak, 4)}
+    else:
+        value, unit = gbs, "GB/s"
+        roof = {"bound": "hbm", "kernel": kname, "achieved": round(g_gbs, 1),
+                "peak": peaks["hbm"], "unit": "GB/s", "frac": round(g_gbs / peaks["hbm"], 4),
+                "traffic": None, "algorithmic_bytes_per_launch": int(acc["gemm_bytes"]),
+                "peak_source": peaks["src"], "step_frac": round(gbs / world / peaks["hbm"], 4)}
+    e2e_rate = (world * acc["flops"] / (e2e_ms * 1e-3) / 1e12 if tensor_bound
+                else world * acc["bytes"] / (e2e_ms * 1e-3) / 1e9)
+    line = {
+        "metric": DENSE_METRIC, "value": round(value, 2), "unit": unit, "n_gpus": world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "nvfp4 (e2m1 + e4m3/16), fp32 accumulate",
+        "data": "synthetic (seeded N(0,1) bf16 activations, gamma 1 + 0.1 N(0,1), N(0,0.02) "
+                "weight quantized to NVFP4 on the GPU)",
+        "config": {"workload": f"{cfg.name}: RMSNorm + dense NVFP4 linear, M={cfg.M}, "
+                               f"K={cfg.K}, N={cfg.N}, bf16 out",
+                   "parallelism": f"replicas x{world}",
+                   "l2": "flushed before every step (256 MB write, outside the timed events)",
+                   "cuda_graph": True, "k_splits": bool(split)},
+        "tflops": round(tflops, 3), "gbs": round(gbs, 2),
+        "algorithmic": {"bytes_per_step": int(acc["bytes"]), "flops_per_step": int(acc["flops"]),
+                        "gemm_bytes_per_launch": int(acc["gemm_bytes"])},
+        "roofline": roof,
+        "stages_ms": {"gemm": round(gemm_ms, 5), "eager_step": round(eager_ms, 5)},
+        "e2e": {"value": round(e2e_rate, 2), "unit": unit,
+                "h2d_bytes_per_step": x_h.numel() * 2, "d2h_bytes_per_step": out_h.numel() * 2,
+                "ms_per_step": round(e2e_ms, 5)},
+        "gpu_launches": (4 if split else 3) * K,
+        "clocks": clocks,
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def _dense_oracle_sample(cfg, rows=16):
+    """The oracle's RMSNorm + linear on the first `rows` rows of the workload (the global scale
+    then comes from those rows' amax); weight pre-packing by the oracle, untimed."""
+    from oracle import dense as D
+    from oracle import formats as F
+    from oracle import moe as M
+    from synth import gen_dense
+    x, gamma, w = gen_dense(cfg)
+    x = x[:rows].float().numpy()
+    g = gamma.float().numpy()
+    qw = M.QuantWeights.from_float(w.float().numpy()[None])
+    wc = F.unpack_nibbles(qw.codes[0])
+
+    def run():
+        y, _ = D.rmsnorm(x, g, cfg.eps)
+        return D.linear(y, wc, qw.sf[0], qw.gs[0])
+
+    n = x.shape[0]
+    flops = 2 * n * cfg.N * cfg.K
+    nbytes = n * cfg.K * 2 + cfg.K * 2 + 2 * n * cfg.K * FP4_ELEM_BYTES + \
+        cfg.N * cfg.K * FP4_ELEM_BYTES + n * cfg.N * 2
+    return run, flops, nbytes, n
+
+
+def dense_cpu_baseline(cfg):
+    run, flops, nbytes, n = _dense_oracle_sample(cfg)
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        run()
+        reps += 1
+        dt = time.perf_counter() - t0
+        if dt >= 10.0:
+            break
+    unit = "GB/s" if cfg.M <= 128 else "TFLOP/s"
+    val = nbytes * reps / dt / 1e9 if unit == "GB/s" else flops * reps / dt / 1e12
+    return {"value": round(val, 6), "unit": unit, "cores": _threads(), "kind": "oracle",
+            "sample": f"first {n} rows of {cfg.name}: RMSNorm, quantize, decode and float64 matmul "
+                      f"against the {cfg.N} x {cfg.K} weight, {reps} repetitions in {dt:.1f} s"}
+
+
+def run_reference_dense(args):
+    from synth import CONFIGS
+    cfg = CONFIGS[args.config]
+    run, flops, nbytes, n = _dense_oracle_sample(cfg)
+    for _ in range(args.warmup):
+        run()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        run()
+    dt = time.perf_counter() - t0
+    unit = "GB/s" if cfg.M <= 128 else "TFLOP/s"
+    value = nbytes * args.steps / dt / 1e9 if unit == "GB/s" else flops * args.steps / dt / 1e12
+    sample = f"each step: the first {n} rows of {cfg.name} through the oracle's RMSNorm + linear"
+    print(json.dumps({
+        "impl": "reference", "metric": DENSE_METRIC, "value": round(value, 6), "unit": unit,
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{cfg.name}: RMSNorm + dense NVFP4 linear, M={cfg.M}, "
+                               f"K={cfg.K}, N={cfg.N}, bf16 out"},
+        "cpu_baseline": {"value": round(value, 6), "unit": unit, "cores": _threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 6), "unit": unit, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0}}), flush=True)
+
+
 def main():
     args = parse()
-    if args.config == "sweep" and args.impl == "ours":
+    dense = args.config.startswith("dense_")
+    if args.impl == "reference":
+        if dense:
+            if int(os.environ.get("RANK", 0)) == 0:
+                run_reference_dense(args)
+        else:
+            run_reference(args)
+    elif args.config == "sweep":
         run_sweep(args)
-    elif args.impl == "reference":
-        run_reference(args)
+    elif dense:
+        run_dense(args)
     else:
         run_ours(args)
 

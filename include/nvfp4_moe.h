@@ -98,6 +98,32 @@ NVFP4_API nvfp4_status_t nvfp4_quantize(const void* x, int64_t rows, int64_t col
                               nvfp4_stream_t stream);
 
 /* ---------------------------------------------------------------------------------------------
+ * nvfp4_rmsnorm_quantize — RMSNorm fused in front of the BF16 -> NVFP4 quantizer.
+ *
+ * The commit log of dsv4/kernels/cuda (nvfp4-megamoe-kernel) fuses the RMSNorm with the amax and
+ * the quantize (its kernel keeps the row's inverse RMS, s_inv_rms, beside the amax).  Reading:
+ *
+ *   ss = sum of x_i^2 over the row in float64;  ms = fl32(ss / cols);  rstd = 1 / sqrt_rn(ms + eps)
+ *   y_i = fl32(fl32(x_i * rstd) * gamma_i)      (float32, one rounding per operation)
+ *
+ * then y is quantized exactly as nvfp4_quantize quantizes x (gs = 2688 / max|y| when
+ * compute_gs = 1).  Two kernels: per-row rstd + the amax of y, then the quantize, which
+ * normalizes each block as it loads it; the normalized tensor is never written.
+ *
+ *   gamma    bf16 [cols] (16-byte aligned);  eps >= 0
+ *   ws       device scratch of nvfp4_rmsnorm_quantize_workspace_size(rows) bytes (the amax word
+ *            and one float per row)
+ *   everything else as nvfp4_quantize.
+ * ------------------------------------------------------------------------------------------- */
+NVFP4_API size_t nvfp4_rmsnorm_quantize_workspace_size(int64_t rows);
+NVFP4_API nvfp4_status_t nvfp4_rmsnorm_quantize(const void* x, int64_t rows, int64_t cols,
+                              int64_t ld, const void* gamma, float eps,
+                              const int32_t* dst_row, int k, int64_t out_rows,
+                              uint8_t* codes, uint8_t* sf, float* gs, int compute_gs,
+                              void* ws, size_t ws_bytes, int32_t* dev_status,
+                              nvfp4_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------------
  * moe_permute — top-k softmax routing and the expert-bucketed row map.
  *
  * The pages list "the MoE routing logic (top-k selection, slot mapping)" as work outside the
@@ -146,6 +172,58 @@ NVFP4_API nvfp4_status_t nvfp4_grouped_gemm(const uint8_t* a, const uint8_t* sfa
                                   const int32_t* offs, int E, int N, int K, int64_t R_max,
                                   void* out, int out_dtype, int32_t* dev_status,
                                   nvfp4_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------------
+ * nvfp4_gemm_dense — dense block-scaled GEMM on NVFP4 activations: out = A W^T, bf16 out.
+ *
+ * The GEMM of the pages' dense layer (Nvfp4Linear; the shared expert), commit log of
+ * dsv4/kernels/cuda (nvfp4-megamoe-kernel), on the grouped GEMM's core ("NVFP4 MegaMoE Kernel
+ * Rewrite — CuTeDSL", section "The Reference Kernel: ScaledGroupedGemmKernel") with one dense
+ * segment in place of expert offsets.
+ *
+ *   a, sfa    NVFP4 activations for round_up(M, 128) rows (codes [.][K/2], tiled scales);
+ *             rows at or past M are padding: read, never stored, their content is irrelevant
+ *   gs_a      device float[1]
+ *   w, sfw    NVFP4 [N][K], gs_w device float[1]
+ *   out       bf16 [M][N]:  out[m][n] = bf16( sum_k a[m][k] * w[n][k] / (gs_a * gs_w) )
+ *   ws        device scratch of nvfp4_gemm_dense_workspace_size(M, N, K) bytes (0 = none
+ *             needed): when M gives fewer output tiles than half the SMs, several CTAs share
+ *             an output tile, each over one range of K, and their FP32 partial products are
+ *             added afterwards in a fixed order (split-K; the result is reproducible)
+ *   Constraints: K % 64 == 0, N % 256 == 0, M >= 0.
+ * ------------------------------------------------------------------------------------------- */
+NVFP4_API size_t nvfp4_gemm_dense_workspace_size(int64_t M, int N, int K);
+NVFP4_API nvfp4_status_t nvfp4_gemm_dense(const uint8_t* a, const uint8_t* sfa,
+                                          const float* gs_a, int64_t M, const uint8_t* w,
+                                          const uint8_t* sfw, const float* gs_w, int N, int K,
+                                          void* out, void* ws, size_t ws_bytes,
+                                          int32_t* dev_status, nvfp4_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------------
+ * nvfp4_linear — dense NVFP4 linear: out = x W^T, bf16 in and out.
+ *
+ * The dense layer of the pages (Nvfp4Linear; the MoE shared expert's projections), commit log
+ * of dsv4/kernels/cuda (nvfp4-megamoe-kernel), "Updated layers" of the fused amax + quantize
+ * commit: the activation is quantized with a GPU-computed global scale (no host sync) and
+ * multiplied by pre-packed NVFP4 weights.
+ *
+ *   x         bf16 [M][ld] (ld >= K, ld % 8 == 0)
+ *   gamma     NULL, or bf16 [K]: x is first RMSNorm'd with gamma and eps (as in
+ *             nvfp4_rmsnorm_quantize), fused into the quantizer
+ *   w, sfw    NVFP4 [N][K] (codes [N][K/2], tiled scales), gs_w device float[1]
+ *   out       bf16 [M][N]:  out[m][n] = bf16( sum_k xq[m][k] * wq[n][k] / (gs_x * gs_w) )
+ *   ws        device scratch of nvfp4_linear_workspace_size(M, N, K) bytes: the quantized
+ *             activation (rows padded to 128), its global scale and nvfp4_gemm_dense's
+ *             partial products.  The steps are nvfp4_quantize (or nvfp4_rmsnorm_quantize) and
+ *             nvfp4_gemm_dense.
+ *   Constraints: K % 64 == 0, N % 256 == 0, M >= 0.
+ * ------------------------------------------------------------------------------------------- */
+NVFP4_API size_t nvfp4_linear_workspace_size(int64_t M, int N, int K);
+NVFP4_API nvfp4_status_t nvfp4_linear(const void* x, int64_t M, int K, int64_t ld,
+                                      const void* gamma, float eps, const uint8_t* w,
+                                      const uint8_t* sfw, const float* gs_w, int N, void* out,
+                                      void* ws, size_t ws_bytes, int32_t* dev_status,
+                                      nvfp4_stream_t stream);
 
 /* ---------------------------------------------------------------------------------------------
  * moe_grouped_gemm_l1_swiglu_q — L1 grouped GEMM with SwiGLU and NVFP4 re-quantization fused in

@@ -8,14 +8,18 @@ tensors and the current CUDA stream into its calls.
 from .api import (  # noqa: F401
     NVFP4Weights,
     ffn_workspace_bytes,
+    gemm_dense,
     grouped_gemm,
     l1_swiglu_q,
     l2_scatter,
+    linear,
+    linear_workspace_bytes,
     moe_ffn_forward,
     permute,
     quantize,
     quantize_w1,
     quantize_weights,
+    rmsnorm_quantize,
     w1_row_map,
     read_status,
     rows_max,

@@ -13,6 +13,7 @@ c_i64 = ctypes.c_int64
 c_size = ctypes.c_size_t
 c_void = ctypes.c_void_p
 c_char_p = ctypes.c_char_p
+c_float = ctypes.c_float
 
 STATUS = {
     0: "NVFP4_OK", 1: "NVFP4_ERR_INVALID_ARG", 2: "NVFP4_ERR_UNSUPPORTED_SHAPE",
@@ -25,12 +26,22 @@ SIGNATURES = {
     "nvfp4_quantize_workspace_size": (c_size, []),
     "nvfp4_quantize": (c_int, [c_void, c_i64, c_i64, c_i64, c_void, c_int, c_i64, c_void, c_void,
                                c_void, c_int, c_void, c_size, c_void, c_void]),
+    "nvfp4_rmsnorm_quantize_workspace_size": (c_size, [c_i64]),
+    "nvfp4_rmsnorm_quantize": (c_int, [c_void, c_i64, c_i64, c_i64, c_void, c_float, c_void, c_int,
+                                       c_i64, c_void, c_void, c_void, c_int, c_void, c_size, c_void,
+                                       c_void]),
     "moe_rows_max": (c_i64, [c_int, c_int, c_int]),
     "moe_permute_workspace_size": (c_size, [c_int, c_int, c_int]),
     "moe_permute": (c_int, [c_void, c_int, c_int, c_int, c_int, c_void, c_void, c_void, c_void,
                             c_void, c_void, c_void, c_size, c_void, c_void]),
     "nvfp4_grouped_gemm": (c_int, [c_void, c_void, c_void, c_void, c_void, c_void, c_void, c_int,
                                    c_int, c_int, c_i64, c_void, c_int, c_void, c_void]),
+    "nvfp4_gemm_dense_workspace_size": (c_size, [c_i64, c_int, c_int]),
+    "nvfp4_gemm_dense": (c_int, [c_void, c_void, c_void, c_i64, c_void, c_void, c_void, c_int, c_int,
+                                 c_void, c_void, c_size, c_void, c_void]),
+    "nvfp4_linear_workspace_size": (c_size, [c_i64, c_int, c_int]),
+    "nvfp4_linear": (c_int, [c_void, c_i64, c_int, c_i64, c_void, c_float, c_void, c_void, c_void,
+                             c_int, c_void, c_void, c_size, c_void, c_void]),
     "moe_grouped_gemm_l1_swiglu_q": (c_int, [c_void, c_void, c_void, c_void, c_void, c_void,
                                              c_void, c_void, c_int, c_int, c_int, c_i64, c_void,
                                              c_void, c_void, c_void, c_void]),

@@ -60,6 +60,60 @@ def quantize(x, gs=None, dst_row=None, k=1, out_rows=None, status=None):
     return codes, sf, gs
 
 
+def rmsnorm_quantize(x, gamma, eps, gs=None, dst_row=None, k=1, out_rows=None, status=None):
+    """RMSNorm of bf16 x (rows, cols) with bf16 gamma (cols,), fused into the NVFP4 quantizer.
+    Same outputs and options as quantize(); the normalized tensor itself is never written."""
+    assert x.dtype == BF16 and x.dim() == 2 and x.stride(1) == 1
+    assert gamma.dtype == BF16 and gamma.is_contiguous() and gamma.numel() == x.shape[1]
+    rows, cols = x.shape
+    if out_rows is None:
+        out_rows = rows
+    dev = x.device
+    codes = torch.empty(out_rows, cols // 2, dtype=U8, device=dev)
+    sf = torch.empty(sf_bytes(out_rows, cols), dtype=U8, device=dev)
+    compute = gs is None
+    if compute:
+        gs = torch.empty(1, dtype=F32, device=dev)
+    ws = torch.empty(int(lib().nvfp4_rmsnorm_quantize_workspace_size(rows)), dtype=U8, device=dev)
+    call("nvfp4_rmsnorm_quantize", _p(x), rows, cols, x.stride(0), _p(gamma), float(eps),
+         _p(dst_row), k, out_rows, _p(codes), _p(sf), _p(gs), int(compute), _p(ws), ws.numel(),
+         _p(status), _stream())
+    return codes, sf, gs
+
+
+def gemm_dense(a_codes, a_sf, gs_a, M, w: "NVFP4Weights", out=None, ws=None, status=None):
+    """Dense GEMM on NVFP4 activations (round_up(M, 128) rows of codes and tiled scales):
+    bf16 (M, N) = A W^T with W one NVFP4 matrix (w.E == 1)."""
+    assert w.E == 1
+    if out is None:
+        out = torch.empty(M, w.N, dtype=BF16, device=a_codes.device)
+    need = int(lib().nvfp4_gemm_dense_workspace_size(M, w.N, w.K))
+    if ws is None and need > 0:
+        ws = torch.empty(need, dtype=U8, device=a_codes.device)
+    call("nvfp4_gemm_dense", _p(a_codes), _p(a_sf), _p(gs_a), M, _p(w.codes), _p(w.sf), _p(w.gs),
+         w.N, w.K, _p(out), _p(ws), 0 if ws is None else ws.numel(), _p(status), _stream())
+    return out
+
+
+def linear_workspace_bytes(M, N, K):
+    return int(lib().nvfp4_linear_workspace_size(M, N, K))
+
+
+def linear(x, w: "NVFP4Weights", gamma=None, eps=1e-6, out=None, ws=None, status=None):
+    """Dense NVFP4 linear: bf16 x (M, K) -> bf16 (M, N) = x W^T, with W one NVFP4 matrix
+    (w.E == 1, shape N x K).  gamma (bf16 (K,)) fuses an RMSNorm into the activation quantizer."""
+    assert x.dtype == BF16 and x.dim() == 2 and x.stride(1) == 1 and w.E == 1
+    M, K = x.shape
+    assert K == w.K
+    if out is None:
+        out = torch.empty(M, w.N, dtype=BF16, device=x.device)
+    if ws is None:
+        ws = torch.empty(max(linear_workspace_bytes(M, w.N, K), 256), dtype=U8, device=x.device)
+    call("nvfp4_linear", _p(x), M, K, x.stride(0), _p(gamma), float(eps), _p(w.codes), _p(w.sf),
+         _p(w.gs), w.N, _p(out), _p(ws), ws.numel(), _p(status), _stream())
+    return out
+
+
 def quantize_weights(get_expert, E, N, K, device="cuda", row_map=None):
     """Pre-pack expert weights: get_expert(e) -> bf16 (N, K) on the device; each expert gets its
     own global scale from its amax.  row_map (device int32 [N]): stored row of each row."""

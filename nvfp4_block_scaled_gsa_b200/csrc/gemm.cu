@@ -142,6 +142,9 @@ struct GemmArgs {
   float* ys;                 // L2: weighted expert outputs per slot [S][H]
   int S;                     // L2: slots (T*k)
   int32_t* status;
+  int64_t out_rows;          // PLAIN: rows of `out`; rows at or past it are not stored
+  int k_splits;              // PLAIN_F32: each tile's K is cut into this many ranges
+  int64_t split_stride;      // PLAIN_F32, k_splits > 1: floats between two ranges' outputs
 };
 
 struct Tile {
@@ -210,7 +213,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     bad_offsets = 0;
     abort_flag = 0;
   }
-  for (int i = tid; i <= E; i += NUM_THREADS) seg[i] = __ldg(args.offs + i);  // E + 1 entries
+  // E + 1 segment starts; no offsets = one dense segment of R_max rows (E = 1)
+  for (int i = tid; i <= E; i += NUM_THREADS)
+    seg[i] = args.offs != nullptr ? __ldg(args.offs + i) : (i == 0 ? 0 : (int)args.R_max);
   __syncthreads();
   int my_tiles = 0;
   if (tid < E) {
@@ -271,12 +276,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if constexpr (PAIR) cluster_sync();  // the peer's barriers are initialised before any remote use
   tc_fence_after();
   const uint32_t tmem = tmem_slot;
-  const int total = bad_offsets ? 0 : tile_start[E];
+  // PLAIN_F32 may cut each tile's K into KS ranges (split-K, for a dense product with fewer
+  // tiles than SMs): work item t is K range t % KS of tile t / KS.  KS is 1 in every other mode.
+  const int KS = MODE == PLAIN_F32 ? args.k_splits : 1;
+  const int total = bad_offsets ? 0 : tile_start[E] * KS;
   if (tid == 0 && bad_offsets && blockIdx.x == 0) report(args.status, NVFP4_DEVERR_BAD_OFFSETS);
 
   const int K = args.K;
   const int nk = (K + 255) / 256;  // stages along K
   const int atoms_k = K / 64;      // 64-element scale atoms along K
+  // stages [lo, hi) of work item t (the host keeps KS <= nk, so no range is empty)
+  auto k_range = [&](int t, int& lo, int& hi) {
+    const int ks = t % KS;
+    lo = ks * nk / KS;
+    hi = (ks + 1) * nk / KS;
+  };
 
   // Roles by warpgroup (4 warps each).  setmaxnreg is executed by a whole warpgroup at the top
   // of its own branch: warpgroups 0 (producer, MMA) and 3 (scale factors) give registers to
@@ -291,12 +305,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         uint32_t it = 0;
         bool ok = true;
         for (int t = cluster_id; t < total && ok; t += num_clusters) {
-          const Tile tl = decode_tile<CTAS>(t, tile_start, seg, E, args.n_tiles);
+          const Tile tl = decode_tile<CTAS>(t / KS, tile_start, seg, E, args.n_tiles);
           const int m_cta = tl.m0 + BM * rank;  // this CTA's rows
           // B rows of this N-tile: BN consecutive rows (for L1: 16-row gate blocks each followed by
           // the 16 matching up rows); a pair's CTA r loads rows B_ROWS*r .. B_ROWS*r + B_ROWS-1
           const int b_row0 = tl.e * args.N + tl.nt * BN;
-          for (int kb = 0; kb < nk; ++kb, ++it) {
+          int kb_lo, kb_hi;
+          k_range(t, kb_lo, kb_hi);
+          for (int kb = kb_lo; kb < kb_hi; ++kb, ++it) {
             const int s = it % STAGES;
             const uint32_t ph = (it / STAGES) & 1u;
             if (!mbar_wait_bounded(smem_u32(&bar_empty[s]), ph ^ 1u, &abort_flag)) {
@@ -343,13 +359,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         uint32_t it = 0;
         bool ok = true;
         for (int t = cluster_id; t < total && ok; t += num_clusters) {
-          const Tile tl = decode_tile<CTAS>(t, tile_start, seg, E, args.n_tiles);
+          const Tile tl = decode_tile<CTAS>(t / KS, tile_start, seg, E, args.n_tiles);
           const int m_cta = tl.m0 + BM * rank;
           // a pair's second half past the expert's segment computes rows it never writes; its
           // scale atoms are taken from the first half so that every read stays inside the tensor
           const int a_blk = (m_cta < seg[tl.e + 1] ? m_cta : tl.m0) >> 7;
           const int b_blk = (tl.e * args.N + tl.nt * BN) >> 7;
-          for (int kb = 0; kb < nk; ++kb, ++it) {
+          int kb_lo, kb_hi;
+          k_range(t, kb_lo, kb_hi);
+          for (int kb = kb_lo; kb < kb_hi; ++kb, ++it) {
             const int j = it % C::SF_STAGES;
             const uint32_t ph = (it / C::SF_STAGES) & 1u;
             if (!mbar_wait_bounded(smem_u32(&bar_sfempty[j]), ph ^ 1u, &abort_flag)) {
@@ -415,7 +433,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
           tc_fence_after();
           const uint32_t d_tmem = tmem + b * BN;
-          for (int kb = 0; kb < nk; ++kb, ++it) {
+          int kb_lo, kb_hi;
+          k_range(t, kb_lo, kb_hi);
+          for (int kb = kb_lo; kb < kb_hi; ++kb, ++it) {
             const int s = it % STAGES;
             const uint32_t ph = (it / STAGES) & 1u;
             if (!wait_all(&bar_full[s], ph) || !wait_all(&bar_sf[s], ph)) {
@@ -426,7 +446,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const uint64_t so = static_cast<uint64_t>(s) * (C::AB_BYTES >> 4);
             const uint32_t t_sfa = tmem + C::TM_SFA + s * 16;
             const uint32_t t_sfb = tmem + C::TM_SFB + s * C::SFB_COLS;
-            const uint32_t first = kb == 0 ? 0u : 1u;
+            const uint32_t first = kb == kb_lo ? 0u : 1u;
             // scales of this stage are already in tensor memory (scale-factor warps)
             const int natoms = min(4, atoms_k - kb * 4);
             if (natoms == 4) {
@@ -460,7 +480,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint32_t it = 0;
     bool ok = true;
     for (int t = cluster_id; t < total && ok; t += num_clusters) {
-      for (int kb = 0; kb < nk; ++kb, ++it) {
+      int kb_lo, kb_hi;
+      k_range(t, kb_lo, kb_hi);
+      for (int kb = kb_lo; kb < kb_hi; ++kb, ++it) {
         const int s = it % STAGES;
         const uint32_t ph = (it / STAGES) & 1u;
         const int j = it % C::SF_STAGES;
@@ -497,7 +519,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int half = (warp - EPI_WARP0) >> 2;
     uint32_t tile_it = 0;
     for (int t = cluster_id; t < total; t += num_clusters, ++tile_it) {
-      const Tile tl = decode_tile<CTAS>(t, tile_start, seg, E, args.n_tiles);
+      const Tile tl = decode_tile<CTAS>(t / KS, tile_start, seg, E, args.n_tiles);
       const int b = tile_it % ACC_BUFS;
       if (!mbar_wait_bounded(smem_u32(&bar_acc_full[b]), (tile_it / ACC_BUFS) & 1u, &abort_flag))
         break;
@@ -648,9 +670,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       } else if (rows_valid) {
         const int N = args.N;
         auto emit = [&](int c, const uint32_t (&v)[32]) {
+          if (row >= args.out_rows) return;
           const int64_t col = (int64_t)tl.nt * BN + 32 * c;
           if (MODE == PLAIN_F32) {
-            float4* o = reinterpret_cast<float4*>(static_cast<float*>(args.out) + row * N + col);
+            float* base = static_cast<float*>(args.out) + (int64_t)(t % KS) * args.split_stride;
+            float4* o = reinterpret_cast<float4*>(base + row * N + col);
 #pragma unroll
             for (int i = 0; i < 8; ++i)
               o[i] = make_float4(__uint_as_float(v[4 * i]) * alpha,
@@ -743,6 +767,8 @@ int num_sms() {
 // nobody writes; with ~2.5 blocks per expert that waste (about 20%) outweighs the pair's smaller
 // operand traffic, with 16 blocks per expert the pair is ahead.
 constexpr int kPairMinBlocksPerExpert = 8;
+// At most this many K ranges per tile of a dense product.
+constexpr int kMaxKSplits = 16;
 
 template <int MODE, int CTAS>
 nvfp4_status_t launch_cfg(const CUtensorMap& ma, const CUtensorMap& mb, const GemmArgs& args,
@@ -831,9 +857,83 @@ __global__ void combine_kernel(const float* __restrict__ ys, const int32_t* __re
   }
 }
 
+// out[i] = bf16 of the sum over the K ranges r = 0 .. ks-1 of part[r * n + i], added in that
+// order (reproducible).  8 consecutive outputs per thread.
+__global__ void splitk_reduce_kernel(const float* __restrict__ part, int ks, int64_t n,
+                                     __nv_bfloat16* __restrict__ out) {
+  for (int64_t i = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) * 8; i < n;
+       i += (int64_t)gridDim.x * blockDim.x * 8) {
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
+    for (int r = 0; r < ks; ++r) {
+      const float4* p = reinterpret_cast<const float4*>(part + r * n + i);
+      const float4 p0 = __ldg(p), p1 = __ldg(p + 1);
+      a.x += p0.x; a.y += p0.y; a.z += p0.z; a.w += p0.w;
+      b.x += p1.x; b.y += p1.y; b.z += p1.z; b.w += p1.w;
+    }
+    const __nv_bfloat162 q0 = __floats2bfloat162_rn(a.x, a.y), q1 = __floats2bfloat162_rn(a.z, a.w),
+                         q2 = __floats2bfloat162_rn(b.x, b.y), q3 = __floats2bfloat162_rn(b.z, b.w);
+    uint4 o;
+    o.x = *reinterpret_cast<const uint32_t*>(&q0);
+    o.y = *reinterpret_cast<const uint32_t*>(&q1);
+    o.z = *reinterpret_cast<const uint32_t*>(&q2);
+    o.w = *reinterpret_cast<const uint32_t*>(&q3);
+    *reinterpret_cast<uint4*>(out + i) = o;
+  }
+}
+
 bool ok_ptr(const void* p) { return p != nullptr && aligned16(p); }
 
 }  // namespace
+
+// K ranges of a dense product: split while the tiles fill at most half of the SMs and the
+// caller's partial-sum buffer holds them; each range keeps at least one 256-element stage.
+int dense_k_splits(int64_t M, int N, int K, int sms, int64_t part_floats) {
+  const int64_t Mp = round_up(M, 128);
+  const int64_t tiles = (Mp / BM) * (N / TileCfg<PLAIN_F32, 1>::BN);
+  if (M <= 0 || tiles <= 0 || Mp >= (int64_t)kPairMinBlocksPerExpert * BM || tiles * 2 > sms)
+    return 1;
+  int64_t ks = sms / tiles;
+  ks = ks < kMaxKSplits ? ks : kMaxKSplits;
+  const int64_t nk = (K + 255) / 256;
+  ks = ks < nk ? ks : nk;
+  const int64_t fit = part_floats / (M * (int64_t)N);
+  ks = ks < fit ? ks : fit;
+  return ks >= 2 ? static_cast<int>(ks) : 1;
+}
+
+int device_sms() { return num_sms(); }
+
+// Dense C = A B^T for A NVFP4 [round_up(M, 128)][K] (rows past M are padding that is never
+// stored) and B NVFP4 [N][K]: one segment, no offsets.  With K splits the ranges' FP32 partial
+// products go to `part` and splitk_reduce_kernel adds them; otherwise the bf16 result is stored
+// straight from the epilogue.
+nvfp4_status_t gemm_dense(const uint8_t* a, const uint8_t* sfa, const float* gs_a,
+                          const uint8_t* b, const uint8_t* sfb, const float* gs_b, int64_t M, int N,
+                          int K, void* out_bf16, float* part, int64_t part_floats, int32_t* status,
+                          cudaStream_t s) {
+  if (M == 0) return NVFP4_OK;
+  const int64_t Mp = round_up(M, 128);
+  const int ks = dense_k_splits(M, N, K, num_sms(), part != nullptr ? part_floats : 0);
+  GemmArgs g{};
+  g.sfa = sfa; g.sfb = sfb; g.gs_a = gs_a; g.gs_b = gs_b; g.offs = nullptr;
+  g.E = 1; g.N = N; g.K = K; g.n_tiles = N / TileCfg<PLAIN_F32, 1>::BN; g.R_max = Mp;
+  g.out_rows = M; g.status = status;
+  if (ks == 1) {
+    g.out = out_bf16;
+    g.k_splits = 1;
+    return launch<PLAIN_BF16>(a, b, N, g, s);
+  }
+  g.out = part;
+  g.k_splits = ks;
+  g.split_stride = M * (int64_t)N;
+  nvfp4_status_t st = launch<PLAIN_F32>(a, b, N, g, s);
+  if (st != NVFP4_OK) return st;
+  const int64_t n = M * (int64_t)N;
+  const int64_t want = (n / 8 + 255) / 256;
+  splitk_reduce_kernel<<<(unsigned)(want < 148 * 8 ? want : 148 * 8), 256, 0, s>>>(
+      part, ks, n, static_cast<__nv_bfloat16*>(out_bf16));
+  return check_launch("splitk_reduce_kernel");
+}
 
 nvfp4_status_t gemm_plain(const uint8_t* a, const uint8_t* sfa, const float* gs_a, const uint8_t* b,
                           const uint8_t* sfb, const float* gs_b, const int32_t* offs, int E, int N,
@@ -842,7 +942,7 @@ nvfp4_status_t gemm_plain(const uint8_t* a, const uint8_t* sfa, const float* gs_
   GemmArgs g{};
   g.sfa = sfa; g.sfb = sfb; g.gs_a = gs_a; g.gs_b = gs_b; g.offs = offs;
   g.E = E; g.N = N; g.K = K; g.n_tiles = N / TileCfg<PLAIN_F32, 1>::BN; g.R_max = R_max; g.out = out;
-  g.status = status;
+  g.status = status; g.out_rows = R_max; g.k_splits = 1;
   const int64_t b_rows = (int64_t)E * N;
   return out_dtype == 0 ? launch<PLAIN_F32>(a, b, b_rows, g, s) : launch<PLAIN_BF16>(a, b, b_rows, g, s);
 }
@@ -856,6 +956,7 @@ nvfp4_status_t gemm_l1(const uint8_t* a, const uint8_t* sfa, const float* gs_a, 
   g.sfa = sfa; g.sfb = sfw1; g.gs_a = gs_a; g.gs_b = gs_w1; g.offs = offs;
   g.E = E; g.N = 2 * I; g.K = H; g.n_tiles = 2 * I / TileCfg<L1_SWIGLU, 1>::BN; g.R_max = R_max;
   g.gs_h = gs_h; g.h = h; g.sfh = sfh; g.I = I; g.row_slot = row_slot; g.status = status;
+  g.out_rows = R_max; g.k_splits = 1;
   return launch<L1_SWIGLU>(a, w1, (int64_t)E * 2 * I, g, s);
 }
 
@@ -869,6 +970,7 @@ nvfp4_status_t gemm_l2(const uint8_t* h, const uint8_t* sfh, const float* gs_h, 
   g.sfa = sfh; g.sfb = sfw2; g.gs_a = gs_h; g.gs_b = gs_w2; g.offs = offs;
   g.E = E; g.N = H; g.K = I; g.R_max = R_max; g.n_tiles = H / TileCfg<L2_DIRECT, 1>::BN;
   g.row_slot = row_slot; g.row_w = row_w; g.ys = ys; g.S = T * k; g.status = status;
+  g.out_rows = R_max; g.k_splits = 1;
   const bool staged = (int64_t)T * k >= (int64_t)kL2StagedMinRowsPerExpert * E;
   nvfp4_status_t st = staged ? launch<L2_STAGED>(h, w2, (int64_t)E * H, g, s)
                              : launch<L2_DIRECT>(h, w2, (int64_t)E * H, g, s);

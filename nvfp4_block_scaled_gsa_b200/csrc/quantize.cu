@@ -5,6 +5,11 @@
 // one device word, and the quantize kernel derives gs = 2688 / amax from that word itself (no
 // host sync, no .item()).  Codes are computed against the decoded FP8 block scale (the commit
 // log's "quantize must use the FP8-round-tripped block scale").
+//
+// The same pair of kernels with an RMSNorm in front (the fused RMSNorm + quantize of the same
+// commit log, whose kernel keeps the row's inverse RMS beside the amax): a row-statistics
+// kernel writes each row's 1/rms and reduces the amax of the normalized tensor, and the
+// quantize kernel normalizes each block as it loads it.
 #include "common.cuh"
 
 namespace nvfp4 {
@@ -55,13 +60,82 @@ __global__ void __launch_bounds__(kThreads) amax_kernel(const __nv_bfloat16* __r
   }
 }
 
+// RMSNorm of one element, FP32 with one rounding per step: y = (x * rstd) * gamma.
+__device__ __forceinline__ float rms_apply(float x, float rstd, float g) {
+  return __fmul_rn(__fmul_rn(x, rstd), g);
+}
+
+// One warp per row: rstd = 1 / sqrt(mean(x^2) + eps), then the amax of the normalized row.
+// The sum of squares is taken in float64 (each square of a bf16 value is exact), its mean is
+// rounded once to float32, and the rest is float32 with one rounding per operation:
+//   ms = fl32(ss / cols); v = ms + eps; s = sqrt_rn(v); rstd = 1 / s (rn); y = (x*rstd)*gamma.
+// The amax is an unsigned max over the float bits with the sign cleared, so a NaN wins (and
+// then gives gs = 1), as in the plain amax kernel.
+__global__ void __launch_bounds__(kThreads) rms_stats_kernel(
+    const __nv_bfloat16* __restrict__ x, int64_t rows, int64_t cols, int64_t ld,
+    const __nv_bfloat16* __restrict__ gamma, float eps, float* __restrict__ rstd_out,
+    uint32_t* __restrict__ amax_bits) {
+  const int lane = threadIdx.x & 31;
+  const int64_t row = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
+  uint32_t m = 0;
+  if (row < rows) {
+    const __nv_bfloat16* xr = x + row * ld;
+    double ss = 0.0;
+#pragma unroll 4
+    for (int64_t c = lane * 8; c < cols; c += 256) {
+      const uint4 q = __ldg(reinterpret_cast<const uint4*>(xr + c));
+      const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const double lo = __uint_as_float(w[i] << 16), hi = __uint_as_float(w[i] & 0xFFFF0000u);
+        ss += lo * lo;
+        ss += hi * hi;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    const float ms = __double2float_rn(ss / static_cast<double>(cols));
+    const float rstd = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, eps)));
+    if (lane == 0) rstd_out[row] = rstd;
+    if (amax_bits != nullptr) {
+      for (int64_t c = lane * 8; c < cols; c += 256) {
+        const uint4 q = __ldg(reinterpret_cast<const uint4*>(xr + c));
+        const uint4 g = __ldg(reinterpret_cast<const uint4*>(gamma + c));
+        const uint32_t w[4] = {q.x, q.y, q.z, q.w}, gw[4] = {g.x, g.y, g.z, g.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float y0 = rms_apply(__uint_as_float(w[i] << 16), rstd, __uint_as_float(gw[i] << 16));
+          const float y1 = rms_apply(__uint_as_float(w[i] & 0xFFFF0000u), rstd,
+                                     __uint_as_float(gw[i] & 0xFFFF0000u));
+          m = max(m, __float_as_uint(y0) & 0x7FFFFFFFu);
+          m = max(m, __float_as_uint(y1) & 0x7FFFFFFFu);
+        }
+      }
+    }
+  }
+  if (amax_bits == nullptr) return;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+  __shared__ uint32_t red[kThreads / 32];
+  if (lane == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    uint32_t b = 0;
+    for (int i = 0; i < kThreads / 32; ++i) b = max(b, red[i]);
+    atomicMax(amax_bits, b);
+  }
+}
+
 // One thread per 16-element block.  gs comes from the amax word (compute mode, and thread 0
 // publishes it to *gs) or is read from *gs.  Codes and the scale byte go to output row i
-// (dst_row == nullptr) or to the k rows dst_row[i*k + j].
+// (dst_row == nullptr) or to the k rows dst_row[i*k + j].  NORM: each element is first
+// normalized with its row's rstd and gamma (rms_apply), exactly as rms_stats_kernel did.
+template <bool NORM>
 __global__ void __launch_bounds__(kThreads) quantize_kernel(
     const __nv_bfloat16* __restrict__ x, int64_t rows, int64_t cols, int64_t ld,
     const int32_t* __restrict__ dst_row, int k, int64_t out_rows, uint8_t* __restrict__ codes,
     uint8_t* __restrict__ sf, float* __restrict__ gs_io, const uint32_t* __restrict__ amax_bits,
+    const float* __restrict__ rstd, const __nv_bfloat16* __restrict__ gamma,
     int32_t* __restrict__ dev_status) {
   const int64_t nblk_row = cols / 16;
   const int64_t nblk = rows * nblk_row;
@@ -89,8 +163,20 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(
     for (int i = 0; i < 8; ++i) {
       v[2 * i] = __uint_as_float(w[i] << 16);
       v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-      amax = fmaxf(amax, fmaxf(fabsf(v[2 * i]), fabsf(v[2 * i + 1])));
     }
+    if constexpr (NORM) {
+      const float rs = __ldg(rstd + r);
+      const uint4* gsrc = reinterpret_cast<const uint4*>(gamma + c * 16);
+      const uint4 g0 = __ldg(gsrc), g1 = __ldg(gsrc + 1);
+      const uint32_t gw[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        v[2 * i] = rms_apply(v[2 * i], rs, __uint_as_float(gw[i] << 16));
+        v[2 * i + 1] = rms_apply(v[2 * i + 1], rs, __uint_as_float(gw[i] & 0xFFFF0000u));
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
     float rcp;
     sbyte = nvfp4_block_scale(amax, gs, rcp);
     packed.x = nvfp4_pack8(v, rcp);
@@ -147,15 +233,48 @@ nvfp4_status_t quantize_launch(const void* x, int64_t rows, int64_t cols, int64_
   }
   const int64_t nblk = rows * (cols / 16);
   const int64_t grid = nblk > 0 ? (nblk + kThreads - 1) / kThreads : 1;
-  quantize_kernel<<<static_cast<unsigned>(grid), kThreads, 0, s>>>(
+  quantize_kernel<false><<<static_cast<unsigned>(grid), kThreads, 0, s>>>(
       static_cast<const __nv_bfloat16*>(x), rows, cols, ld, dst_row, k, out_rows, codes, sf, gs,
-      amax, dev_status);
+      amax, nullptr, nullptr, dev_status);
+  return check_launch("quantize_kernel");
+}
+
+// Workspace of the fused RMSNorm + quantize: the amax word, then rstd float[rows].
+constexpr int64_t kRmsRstdOffset = 256;
+
+nvfp4_status_t rmsnorm_quantize_launch(const void* x, int64_t rows, int64_t cols, int64_t ld,
+                                       const void* gamma, float eps, const int32_t* dst_row,
+                                       int k, int64_t out_rows, uint8_t* codes, uint8_t* sf,
+                                       float* gs, int compute_gs, void* ws, int32_t* dev_status,
+                                       cudaStream_t s) {
+  uint32_t* amax = compute_gs ? static_cast<uint32_t*>(ws) : nullptr;
+  float* rstd = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + kRmsRstdOffset);
+  const auto* xb = static_cast<const __nv_bfloat16*>(x);
+  const auto* gb = static_cast<const __nv_bfloat16*>(gamma);
+  if (amax != nullptr && cudaMemsetAsync(amax, 0, sizeof(uint32_t), s) != cudaSuccess)
+    return check_launch("memset amax");
+  if (rows > 0) {
+    const int64_t blocks = (rows * 32 + kThreads - 1) / kThreads;
+    rms_stats_kernel<<<static_cast<unsigned>(blocks), kThreads, 0, s>>>(xb, rows, cols, ld, gb,
+                                                                        eps, rstd, amax);
+    nvfp4_status_t st = check_launch("rms_stats_kernel");
+    if (st != NVFP4_OK) return st;
+  }
+  const int64_t nblk = rows * (cols / 16);
+  const int64_t grid = nblk > 0 ? (nblk + kThreads - 1) / kThreads : 1;
+  quantize_kernel<true><<<static_cast<unsigned>(grid), kThreads, 0, s>>>(
+      xb, rows, cols, ld, dst_row, k, out_rows, codes, sf, gs, amax, rstd, gb, dev_status);
   return check_launch("quantize_kernel");
 }
 
 }  // namespace nvfp4
 
 extern "C" size_t nvfp4_quantize_workspace_size(void) { return 256; }
+
+extern "C" size_t nvfp4_rmsnorm_quantize_workspace_size(int64_t rows) {
+  return static_cast<size_t>(nvfp4::kRmsRstdOffset +
+                             nvfp4::round_up((rows > 0 ? rows : 0) * 4, 256));
+}
 
 extern "C" nvfp4_status_t nvfp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t ld,
                                          const int32_t* dst_row, int k, int64_t out_rows,
@@ -181,4 +300,31 @@ extern "C" nvfp4_status_t nvfp4_quantize(const void* x, int64_t rows, int64_t co
     return NVFP4_ERR_MISALIGNED;
   return quantize_launch(x, rows, cols, ld, dst_row, k, out_rows, codes, sf, gs, compute_gs, ws,
                          dev_status, reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" nvfp4_status_t nvfp4_rmsnorm_quantize(const void* x, int64_t rows, int64_t cols,
+                                                 int64_t ld, const void* gamma, float eps,
+                                                 const int32_t* dst_row, int k, int64_t out_rows,
+                                                 uint8_t* codes, uint8_t* sf, float* gs,
+                                                 int compute_gs, void* ws, size_t ws_bytes,
+                                                 int32_t* dev_status, nvfp4_stream_t stream) {
+  using namespace nvfp4;
+  if (rows < 0 || out_rows < 0 || cols <= 0 || ld < cols) return NVFP4_ERR_INVALID_ARG;
+  if (cols % 64 != 0 || ld % 8 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (gs == nullptr || ws == nullptr || !(eps >= 0.0f)) return NVFP4_ERR_INVALID_ARG;
+  if (rows > 0 && (x == nullptr || gamma == nullptr || codes == nullptr || sf == nullptr))
+    return NVFP4_ERR_INVALID_ARG;
+  if (dst_row == nullptr) {
+    if (out_rows < rows) return NVFP4_ERR_INVALID_ARG;
+  } else if (k < 1 || k > 64) {
+    return NVFP4_ERR_INVALID_ARG;
+  }
+  if (ws_bytes < nvfp4_rmsnorm_quantize_workspace_size(rows)) return NVFP4_ERR_WORKSPACE_TOO_SMALL;
+  if (!aligned16(x) || !aligned16(gamma) || !aligned16(codes) || !aligned16(sf) ||
+      !aligned16(ws) || (reinterpret_cast<uintptr_t>(gs) & 3u) ||
+      (reinterpret_cast<uintptr_t>(dst_row) & 3u))
+    return NVFP4_ERR_MISALIGNED;
+  return rmsnorm_quantize_launch(x, rows, cols, ld, gamma, eps, dst_row, k, out_rows, codes, sf,
+                                 gs, compute_gs, ws, dev_status,
+                                 reinterpret_cast<cudaStream_t>(stream));
 }

@@ -50,12 +50,30 @@ class SweepConfig:
     seed: int = 0
 
 
+@dataclass(frozen=True)
+class DenseConfig:
+    """A dense NVFP4 linear out = RMSNorm(x) W^T (M x K activations, N x K weight): the MoE
+    shared expert's gate/up projection, hidden 7168 -> 2 * 2048."""
+    name: str
+    M: int
+    N: int
+    K: int
+    norm: bool = True
+    eps: float = 1e-6
+    seed: int = 0
+
+    def flops(self):
+        return 2 * self.M * self.N * self.K
+
+
 CONFIGS = {
     "tiny": MoEConfig("tiny", T=64, H=256, I=128, E=8, k=2, logits="normal", gs_h=64.0),
     "decode": MoEConfig("decode", T=16, H=7168, I=2048, E=256, k=8, logits="uniform"),
     "mid": MoEConfig("mid", T=512, H=7168, I=2048, E=256, k=8, logits="zipf_gumbel", x_outliers=True),
     "prefill": MoEConfig("prefill", T=8192, H=7168, I=2048, E=256, k=8, logits="uniform"),
     "sweep": SweepConfig("sweep", E=32, K=7168, N=4096, m_max=4096),
+    "dense_decode": DenseConfig("dense_decode", M=16, N=4096, K=7168),
+    "dense_prefill": DenseConfig("dense_prefill", M=8192, N=4096, K=7168),
 }
 
 
@@ -121,3 +139,15 @@ def gen_sweep(cfg, device="cpu"):
 def gen_sweep_a(cfg, rows, device="cpu"):
     g = torch.Generator(device=device).manual_seed(cfg.seed + 7)
     return torch.randn(rows, cfg.K, generator=g, dtype=torch.float32, device=device)
+
+
+def gen_dense(cfg, device="cpu"):
+    """Inputs of a dense workload: x bf16 (M, K) N(0, 1) (seed + 11), gamma bf16 (K,)
+    1 + 0.1 N(0, 1) (seed + 12), W bf16 (N, K) N(0, 0.02) (seed + 13, on `device`)."""
+    g = torch.Generator().manual_seed(cfg.seed + 11)
+    x = torch.randn(cfg.M, cfg.K, generator=g, dtype=torch.float32).to(torch.bfloat16)
+    g = torch.Generator().manual_seed(cfg.seed + 12)
+    gamma = (1.0 + 0.1 * torch.randn(cfg.K, generator=g, dtype=torch.float32)).to(torch.bfloat16)
+    g = torch.Generator(device=device).manual_seed(cfg.seed + 13)
+    w = (torch.randn(cfg.N, cfg.K, generator=g, dtype=torch.float32, device=device) * 0.02)
+    return x, gamma, w.to(torch.bfloat16)

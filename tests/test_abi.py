@@ -128,3 +128,44 @@ def test_w1_row_map_is_the_documented_interleave(L):
         assert m[I + r] == 32 * (r // 16) + 16 + r % 16   # up row r
     assert m[:3] == [0, 1, 2] and m[16] == 32 and m[I] == 16
     assert L.moe_w1_row_map(100, ctypes.cast(buf, ctypes.c_void_p)) == 1  # I % 16
+
+
+def test_dense_workspace_sizes(L):
+    # amax word + one float per row, in 256-byte units
+    assert L.nvfp4_rmsnorm_quantize_workspace_size(8192) == 256 + 8192 * 4
+    assert L.nvfp4_rmsnorm_quantize_workspace_size(1) == 512
+    assert L.nvfp4_rmsnorm_quantize_workspace_size(0) == 256
+    # M = 16, N = 4096, K = 7168: quantizer scratch, gs, 128 padded code rows and their scales,
+    # and 9 K ranges of FP32 partials (16 output tiles, 148 // 16 = 9 CTAs per tile)
+    want = 512 + 256 + 128 * 3584 + 128 * 448 + 9 * 16 * 4096 * 4
+    assert L.nvfp4_linear_workspace_size(16, 4096, 7168) == want
+    # 8192 rows give 512 tiles: no split, no partials
+    assert L.nvfp4_linear_workspace_size(8192, 4096, 7168) == (
+        256 + 8192 * 4 + 256 + 8192 * 3584 + 8192 * 448)
+    # K = 256 has one stage: no split either
+    assert L.nvfp4_linear_workspace_size(16, 4096, 256) == 512 + 256 + 128 * 128 + 128 * 16
+    assert L.nvfp4_linear_workspace_size(-1, 4096, 256) == 0
+
+
+def test_dense_entry_points_reject_bad_arguments(L):
+    f = FAKE
+    odd = ctypes.c_void_p((1 << 20) + 8)
+    big = 1 << 40
+    lin = L.nvfp4_linear
+    # x, M, K, ld, gamma, eps, w, sfw, gs_w, N, out, ws, ws_bytes, status, stream
+    assert lin(f, 16, 100, 128, None, 0.0, f, f, f, 256, f, f, big, None, None) == 2  # K % 64
+    assert lin(f, 16, 128, 128, None, 0.0, f, f, f, 200, f, f, big, None, None) == 2  # N % 256
+    assert lin(f, 16, 128, 64, None, 0.0, f, f, f, 256, f, f, big, None, None) == 1   # ld < K
+    assert lin(f, 16, 128, 128, None, -1.0, f, f, f, 256, f, f, big, None, None) == 1  # eps < 0
+    assert lin(f, 16, 128, 128, None, 0.0, f, f, f, 256, f, f, 64, None, None) == 4   # workspace
+    assert lin(odd, 16, 128, 128, None, 0.0, f, f, f, 256, f, f, big, None, None) == 3
+    assert lin(f, 16, 128, 128, odd, 0.0, f, f, f, 256, f, f, big, None, None) == 3  # gamma
+    assert lin(f, 16, 128, 128, None, 0.0, None, f, f, 256, f, f, big, None, None) == 1
+    assert lin(None, 0, 128, 128, None, 0.0, f, f, f, 256, None, f, big, None, None) == 0  # M = 0
+    rq = L.nvfp4_rmsnorm_quantize
+    # x, rows, cols, ld, gamma, eps, dst, k, out_rows, codes, sf, gs, compute, ws, ws_bytes, ...
+    assert rq(f, 4, 64, 64, f, float("nan"), None, 1, 4, f, f, f, 1, f, big, None, None) == 1
+    assert rq(f, 4, 64, 64, None, 0.0, None, 1, 4, f, f, f, 1, f, big, None, None) == 1  # gamma
+    assert rq(f, 4, 64, 64, f, 0.0, None, 1, 4, f, f, f, 1, f, 256, None, None) == 4   # ws
+    assert rq(f, 4, 96, 96, f, 0.0, None, 1, 4, f, f, f, 1, f, big, None, None) == 2   # cols % 64
+    assert rq(f, 4, 64, 64, odd, 0.0, None, 1, 4, f, f, f, 1, f, big, None, None) == 3
