@@ -858,26 +858,28 @@ __global__ void combine_kernel(const float* __restrict__ ys, const int32_t* __re
 }
 
 // out[i] = bf16 of the sum over the K ranges r = 0 .. ks-1 of part[r * n + i], added in that
-// order (reproducible).  8 consecutive outputs per thread.
-__global__ void splitk_reduce_kernel(const float* __restrict__ part, int ks, int64_t n,
-                                     __nv_bfloat16* __restrict__ out) {
-  for (int64_t i = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) * 8; i < n;
-       i += (int64_t)gridDim.x * blockDim.x * 8) {
-    float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
-    for (int r = 0; r < ks; ++r) {
-      const float4* p = reinterpret_cast<const float4*>(part + r * n + i);
-      const float4 p0 = __ldg(p), p1 = __ldg(p + 1);
-      a.x += p0.x; a.y += p0.y; a.z += p0.z; a.w += p0.w;
-      b.x += p1.x; b.y += p1.y; b.z += p1.z; b.w += p1.w;
+// order (reproducible).  4 consecutive outputs per thread, all ks loads in flight at once.
+__global__ void __launch_bounds__(256) splitk_reduce_kernel(const float* __restrict__ part, int ks,
+                                                            int64_t n,
+                                                            __nv_bfloat16* __restrict__ out) {
+  for (int64_t i = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) * 4; i < n;
+       i += (int64_t)gridDim.x * blockDim.x * 4) {
+    float4 p[kMaxKSplits];
+#pragma unroll
+    for (int r = 0; r < kMaxKSplits; ++r)
+      if (r < ks) p[r] = __ldg(reinterpret_cast<const float4*>(part + r * n + i));
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int r = 0; r < kMaxKSplits; ++r) {
+      if (r < ks) {
+        a.x += p[r].x; a.y += p[r].y; a.z += p[r].z; a.w += p[r].w;
+      }
     }
-    const __nv_bfloat162 q0 = __floats2bfloat162_rn(a.x, a.y), q1 = __floats2bfloat162_rn(a.z, a.w),
-                         q2 = __floats2bfloat162_rn(b.x, b.y), q3 = __floats2bfloat162_rn(b.z, b.w);
-    uint4 o;
+    const __nv_bfloat162 q0 = __floats2bfloat162_rn(a.x, a.y), q1 = __floats2bfloat162_rn(a.z, a.w);
+    uint2 o;
     o.x = *reinterpret_cast<const uint32_t*>(&q0);
     o.y = *reinterpret_cast<const uint32_t*>(&q1);
-    o.z = *reinterpret_cast<const uint32_t*>(&q2);
-    o.w = *reinterpret_cast<const uint32_t*>(&q3);
-    *reinterpret_cast<uint4*>(out + i) = o;
+    *reinterpret_cast<uint2*>(out + i) = o;
   }
 }
 
@@ -929,7 +931,7 @@ nvfp4_status_t gemm_dense(const uint8_t* a, const uint8_t* sfa, const float* gs_
   nvfp4_status_t st = launch<PLAIN_F32>(a, b, N, g, s);
   if (st != NVFP4_OK) return st;
   const int64_t n = M * (int64_t)N;
-  const int64_t want = (n / 8 + 255) / 256;
+  const int64_t want = (n / 4 + 255) / 256;
   splitk_reduce_kernel<<<(unsigned)(want < 148 * 8 ? want : 148 * 8), 256, 0, s>>>(
       part, ks, n, static_cast<__nv_bfloat16*>(out_bf16));
   return check_launch("splitk_reduce_kernel");

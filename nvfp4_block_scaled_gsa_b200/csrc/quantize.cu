@@ -65,61 +65,94 @@ __device__ __forceinline__ float rms_apply(float x, float rstd, float g) {
   return __fmul_rn(__fmul_rn(x, rstd), g);
 }
 
-// One warp per row: rstd = 1 / sqrt(mean(x^2) + eps), then the amax of the normalized row.
-// The sum of squares is taken in float64 (each square of a bf16 value is exact), its mean is
-// rounded once to float32, and the rest is float32 with one rounding per operation:
+// rstd = 1 / sqrt(mean(x^2) + eps) of each row, then the amax of the normalized rows.  One
+// 256-thread block per row (grid-stride over rows): the row's first 8192 columns are loaded
+// into registers at once (every load in flight), summed, and reused for the amax.  The sum of
+// squares is taken in float64 (each square of a bf16 value is exact) with the warps' partial
+// sums added in warp order; its mean is rounded once to float32, and the rest is float32 with
+// one rounding per operation:
 //   ms = fl32(ss / cols); v = ms + eps; s = sqrt_rn(v); rstd = 1 / s (rn); y = (x*rstd)*gamma.
 // The amax is an unsigned max over the float bits with the sign cleared, so a NaN wins (and
-// then gives gs = 1), as in the plain amax kernel.
+// then gives gs = 1), as in the plain amax kernel; one atomic per block.
+constexpr int kRmsChunks = 4;  // uint4 chunks (8 columns each) per thread held in registers
+
 __global__ void __launch_bounds__(kThreads) rms_stats_kernel(
     const __nv_bfloat16* __restrict__ x, int64_t rows, int64_t cols, int64_t ld,
     const __nv_bfloat16* __restrict__ gamma, float eps, float* __restrict__ rstd_out,
     uint32_t* __restrict__ amax_bits) {
-  const int lane = threadIdx.x & 31;
-  const int64_t row = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t n8 = cols / 8;
+  __shared__ double part[kThreads / 32];
+  __shared__ float s_rstd;
+  __shared__ uint32_t red[kThreads / 32];
   uint32_t m = 0;
-  if (row < rows) {
-    const __nv_bfloat16* xr = x + row * ld;
-    double ss = 0.0;
-#pragma unroll 4
-    for (int64_t c = lane * 8; c < cols; c += 256) {
-      const uint4 q = __ldg(reinterpret_cast<const uint4*>(xr + c));
-      const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+  auto sq = [](const uint4& q) {
+    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+    double t = 0.0;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const double lo = __uint_as_float(w[i] << 16), hi = __uint_as_float(w[i] & 0xFFFF0000u);
-        ss += lo * lo;
-        ss += hi * hi;
-      }
+    for (int i = 0; i < 4; ++i) {
+      const double lo = __uint_as_float(w[i] << 16), hi = __uint_as_float(w[i] & 0xFFFF0000u);
+      t += lo * lo;
+      t += hi * hi;
     }
+    return t;
+  };
+  auto fold_amax = [&](const uint4& q, const uint4& g, float rstd) {
+    const uint32_t w[4] = {q.x, q.y, q.z, q.w}, gw[4] = {g.x, g.y, g.z, g.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float y0 = rms_apply(__uint_as_float(w[i] << 16), rstd, __uint_as_float(gw[i] << 16));
+      const float y1 = rms_apply(__uint_as_float(w[i] & 0xFFFF0000u), rstd,
+                                 __uint_as_float(gw[i] & 0xFFFF0000u));
+      m = max(m, __float_as_uint(y0) & 0x7FFFFFFFu);
+      m = max(m, __float_as_uint(y1) & 0x7FFFFFFFu);
+    }
+  };
+  for (int64_t row = blockIdx.x; row < rows; row += gridDim.x) {
+    const uint4* xr = reinterpret_cast<const uint4*>(x + row * ld);
+    uint4 q[kRmsChunks];
+#pragma unroll
+    for (int j = 0; j < kRmsChunks; ++j) {
+      const int64_t c = tid + (int64_t)j * kThreads;
+      q[j] = c < n8 ? __ldg(xr + c) : make_uint4(0u, 0u, 0u, 0u);
+    }
+    double ss = 0.0;
+#pragma unroll
+    for (int j = 0; j < kRmsChunks; ++j) ss += sq(q[j]);
+    for (int64_t c = tid + (int64_t)kRmsChunks * kThreads; c < n8; c += kThreads)
+      ss += sq(__ldg(xr + c));
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    const float ms = __double2float_rn(ss / static_cast<double>(cols));
-    const float rstd = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, eps)));
-    if (lane == 0) rstd_out[row] = rstd;
-    if (amax_bits != nullptr) {
-      for (int64_t c = lane * 8; c < cols; c += 256) {
-        const uint4 q = __ldg(reinterpret_cast<const uint4*>(xr + c));
-        const uint4 g = __ldg(reinterpret_cast<const uint4*>(gamma + c));
-        const uint32_t w[4] = {q.x, q.y, q.z, q.w}, gw[4] = {g.x, g.y, g.z, g.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float y0 = rms_apply(__uint_as_float(w[i] << 16), rstd, __uint_as_float(gw[i] << 16));
-          const float y1 = rms_apply(__uint_as_float(w[i] & 0xFFFF0000u), rstd,
-                                     __uint_as_float(gw[i] & 0xFFFF0000u));
-          m = max(m, __float_as_uint(y0) & 0x7FFFFFFFu);
-          m = max(m, __float_as_uint(y1) & 0x7FFFFFFFu);
-        }
-      }
+    if (lane == 0) part[warp] = ss;
+    __syncthreads();
+    if (tid == 0) {
+      double t = 0.0;
+      for (int w = 0; w < kThreads / 32; ++w) t += part[w];
+      const float ms = __double2float_rn(t / static_cast<double>(cols));
+      const float rstd = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, eps)));
+      s_rstd = rstd;
+      rstd_out[row] = rstd;
     }
+    __syncthreads();
+    const float rstd = s_rstd;
+    if (amax_bits != nullptr) {
+      const uint4* gr = reinterpret_cast<const uint4*>(gamma);
+#pragma unroll
+      for (int j = 0; j < kRmsChunks; ++j) {
+        const int64_t c = tid + (int64_t)j * kThreads;
+        if (c < n8) fold_amax(q[j], __ldg(gr + c), rstd);
+      }
+      for (int64_t c = tid + (int64_t)kRmsChunks * kThreads; c < n8; c += kThreads)
+        fold_amax(__ldg(xr + c), __ldg(gr + c), rstd);
+    }
+    __syncthreads();  // part[] and s_rstd are rewritten for the next row
   }
   if (amax_bits == nullptr) return;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
-  __shared__ uint32_t red[kThreads / 32];
-  if (lane == 0) red[threadIdx.x >> 5] = m;
+  if (lane == 0) red[warp] = m;
   __syncthreads();
-  if (threadIdx.x == 0) {
+  if (tid == 0) {
     uint32_t b = 0;
     for (int i = 0; i < kThreads / 32; ++i) b = max(b, red[i]);
     atomicMax(amax_bits, b);
@@ -254,7 +287,7 @@ nvfp4_status_t rmsnorm_quantize_launch(const void* x, int64_t rows, int64_t cols
   if (amax != nullptr && cudaMemsetAsync(amax, 0, sizeof(uint32_t), s) != cudaSuccess)
     return check_launch("memset amax");
   if (rows > 0) {
-    const int64_t blocks = (rows * 32 + kThreads - 1) / kThreads;
+    const int64_t blocks = rows < 148 * 4 ? rows : 148 * 4;  // 4 resident blocks per SM (64 regs)
     rms_stats_kernel<<<static_cast<unsigned>(blocks), kThreads, 0, s>>>(xb, rows, cols, ld, gb,
                                                                         eps, rstd, amax);
     nvfp4_status_t st = check_launch("rms_stats_kernel");
