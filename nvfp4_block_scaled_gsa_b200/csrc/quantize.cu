@@ -67,7 +67,8 @@ __device__ __forceinline__ float rms_apply(float x, float rstd, float g) {
 
 // rstd = 1 / sqrt(mean(x^2) + eps) of each row, then the amax of the normalized rows.  One
 // 256-thread block per row (grid-stride over rows): the row's first 8192 columns are loaded
-// into registers at once (every load in flight), summed, and reused for the amax.  The sum of
+// into registers at once (every load in flight), summed, and reused for the amax; the block's
+// next row is loaded meanwhile.  The sum of
 // squares is taken in float64 (each square of a bf16 value is exact) with the warps' partial
 // sums added in warp order; its mean is rounded once to float32, and the rest is float32 with
 // one rounding per operation:
@@ -76,7 +77,7 @@ __device__ __forceinline__ float rms_apply(float x, float rstd, float g) {
 // then gives gs = 1), as in the plain amax kernel; one atomic per block.
 constexpr int kRmsChunks = 4;  // uint4 chunks (8 columns each) per thread held in registers
 
-__global__ void __launch_bounds__(kThreads) rms_stats_kernel(
+__global__ void __launch_bounds__(kThreads, 4) rms_stats_kernel(
     const __nv_bfloat16* __restrict__ x, int64_t rows, int64_t cols, int64_t ld,
     const __nv_bfloat16* __restrict__ gamma, float eps, float* __restrict__ rstd_out,
     uint32_t* __restrict__ amax_bits) {
@@ -108,14 +109,21 @@ __global__ void __launch_bounds__(kThreads) rms_stats_kernel(
       m = max(m, __float_as_uint(y1) & 0x7FFFFFFFu);
     }
   };
-  for (int64_t row = blockIdx.x; row < rows; row += gridDim.x) {
-    const uint4* xr = reinterpret_cast<const uint4*>(x + row * ld);
-    uint4 q[kRmsChunks];
+  auto load_row = [&](int64_t r, uint4 (&q)[kRmsChunks]) {
+    const uint4* xr = reinterpret_cast<const uint4*>(x + r * ld);
 #pragma unroll
     for (int j = 0; j < kRmsChunks; ++j) {
       const int64_t c = tid + (int64_t)j * kThreads;
-      q[j] = c < n8 ? __ldg(xr + c) : make_uint4(0u, 0u, 0u, 0u);
+      q[j] = (r < rows && c < n8) ? __ldg(xr + c) : make_uint4(0u, 0u, 0u, 0u);
     }
+  };
+  uint4 q[kRmsChunks];
+  load_row(blockIdx.x, q);
+  for (int64_t row = blockIdx.x; row < rows; row += gridDim.x) {
+    const uint4* xr = reinterpret_cast<const uint4*>(x + row * ld);
+    // the block's next row is loaded while this one is reduced
+    uint4 qn[kRmsChunks];
+    load_row(row + gridDim.x, qn);
     double ss = 0.0;
 #pragma unroll
     for (int j = 0; j < kRmsChunks; ++j) ss += sq(q[j]);
@@ -146,6 +154,8 @@ __global__ void __launch_bounds__(kThreads) rms_stats_kernel(
         fold_amax(__ldg(xr + c), __ldg(gr + c), rstd);
     }
     __syncthreads();  // part[] and s_rstd are rewritten for the next row
+#pragma unroll
+    for (int j = 0; j < kRmsChunks; ++j) q[j] = qn[j];
   }
   if (amax_bits == nullptr) return;
 #pragma unroll
