@@ -16,6 +16,9 @@ namespace nvfp4 {
 namespace {
 
 constexpr int kThreads = 256;
+// quantize_kernel's grid: one row per blockIdx.x, at most 65535 column chunks of kThreads blocks
+constexpr int64_t kMaxQuantRows = 0x7FFFFFFF;
+constexpr int64_t kMaxQuantCols = 65535LL * kThreads * 16;
 
 // max|x| over the (rows x cols) bf16 matrix with row stride ld -> atomicMax on the float bits
 // (non-negative floats order like their bit patterns).
@@ -169,10 +172,11 @@ __global__ void __launch_bounds__(kThreads, 4) rms_stats_kernel(
   }
 }
 
-// One thread per 16-element block.  gs comes from the amax word (compute mode, and thread 0
-// publishes it to *gs) or is read from *gs.  Codes and the scale byte go to output row i
-// (dst_row == nullptr) or to the k rows dst_row[i*k + j].  NORM: each element is first
-// normalized with its row's rstd and gamma (rms_apply), exactly as rms_stats_kernel did.
+// One thread per 16-element block, on a 2-D grid: blockIdx.x is the row, blockIdx.y a chunk of
+// blockDim.x blocks of it (no index division).  gs comes from the amax word (compute mode, and
+// the first thread publishes it to *gs) or is read from *gs.  Codes and the scale byte go to
+// output row i (dst_row == nullptr) or to the k rows dst_row[i*k + j].  NORM: each element is
+// first normalized with its row's rstd and gamma (rms_apply), exactly as rms_stats_kernel did.
 template <bool NORM>
 __global__ void __launch_bounds__(kThreads) quantize_kernel(
     const __nv_bfloat16* __restrict__ x, int64_t rows, int64_t cols, int64_t ld,
@@ -181,19 +185,18 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(
     const float* __restrict__ rstd, const __nv_bfloat16* __restrict__ gamma,
     int32_t* __restrict__ dev_status) {
   const int64_t nblk_row = cols / 16;
-  const int64_t nblk = rows * nblk_row;
-  const int64_t gid = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
   float gs;
   if (amax_bits != nullptr) {
     gs = gs_from_amax(__uint_as_float(__ldg(amax_bits)));
-    if (gid == 0) *gs_io = gs;
+    if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *gs_io = gs;
   } else {
     gs = __ldg(gs_io);
   }
   // no early return: the 4 lanes of a 4-block group exchange their scale bytes with shuffles
-  // (blocks 4g..4g+3 of a row are 4 consecutive lanes, since cols % 64 == 0)
-  const bool valid = gid < nblk;
-  const int64_t r = valid ? gid / nblk_row : 0, c = valid ? gid - r * nblk_row : 0;
+  // (blocks 4g..4g+3 of a row are 4 consecutive lanes: blockDim.x is a multiple of 32)
+  const int64_t r = blockIdx.x;
+  const int64_t c = (int64_t)blockIdx.y * blockDim.x + threadIdx.x;
+  const bool valid = r < rows && c < nblk_row;
   uint32_t sbyte = 0;
   uint2 packed = make_uint2(0u, 0u);
   if (valid) {
@@ -253,12 +256,31 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(
   }
 }
 
+// Launch shape of quantize_kernel: one row per block column, each row's cols/16 blocks cut into
+// the fewest chunks of at most kThreads threads, each chunk a whole number of warps (448 blocks
+// of a 7168-column row: 2 chunks of 224).  A grid of one row when there are none, so that the
+// global scale is still published.
+struct QuantGrid {
+  dim3 grid, block;
+};
+
+QuantGrid quant_grid(int64_t rows, int64_t cols) {
+  const int64_t nblk_row = cols / 16;
+  const int64_t chunks = (nblk_row + kThreads - 1) / kThreads;
+  const int64_t per = (nblk_row + chunks - 1) / chunks;
+  QuantGrid q;
+  q.block = dim3(static_cast<unsigned>((per + 31) / 32 * 32));
+  q.grid = dim3(static_cast<unsigned>(rows > 0 ? rows : 1), static_cast<unsigned>(chunks));
+  return q;
+}
+
 }  // namespace
 
 nvfp4_status_t quantize_launch(const void* x, int64_t rows, int64_t cols, int64_t ld,
                                const int32_t* dst_row, int k, int64_t out_rows, uint8_t* codes,
                                uint8_t* sf, float* gs, int compute_gs, void* ws,
                                int32_t* dev_status, cudaStream_t s) {
+  if (rows > kMaxQuantRows || cols > kMaxQuantCols) return NVFP4_ERR_UNSUPPORTED_SHAPE;
   uint32_t* amax = nullptr;
   if (compute_gs) {
     amax = static_cast<uint32_t*>(ws);
@@ -274,9 +296,8 @@ nvfp4_status_t quantize_launch(const void* x, int64_t rows, int64_t cols, int64_
       if (st != NVFP4_OK) return st;
     }
   }
-  const int64_t nblk = rows * (cols / 16);
-  const int64_t grid = nblk > 0 ? (nblk + kThreads - 1) / kThreads : 1;
-  quantize_kernel<false><<<static_cast<unsigned>(grid), kThreads, 0, s>>>(
+  const QuantGrid qg = quant_grid(rows, cols);
+  quantize_kernel<false><<<qg.grid, qg.block, 0, s>>>(
       static_cast<const __nv_bfloat16*>(x), rows, cols, ld, dst_row, k, out_rows, codes, sf, gs,
       amax, nullptr, nullptr, dev_status);
   return check_launch("quantize_kernel");
@@ -290,6 +311,7 @@ nvfp4_status_t rmsnorm_quantize_launch(const void* x, int64_t rows, int64_t cols
                                        int k, int64_t out_rows, uint8_t* codes, uint8_t* sf,
                                        float* gs, int compute_gs, void* ws, int32_t* dev_status,
                                        cudaStream_t s) {
+  if (rows > kMaxQuantRows || cols > kMaxQuantCols) return NVFP4_ERR_UNSUPPORTED_SHAPE;
   uint32_t* amax = compute_gs ? static_cast<uint32_t*>(ws) : nullptr;
   float* rstd = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + kRmsRstdOffset);
   const auto* xb = static_cast<const __nv_bfloat16*>(x);
@@ -303,9 +325,8 @@ nvfp4_status_t rmsnorm_quantize_launch(const void* x, int64_t rows, int64_t cols
     nvfp4_status_t st = check_launch("rms_stats_kernel");
     if (st != NVFP4_OK) return st;
   }
-  const int64_t nblk = rows * (cols / 16);
-  const int64_t grid = nblk > 0 ? (nblk + kThreads - 1) / kThreads : 1;
-  quantize_kernel<true><<<static_cast<unsigned>(grid), kThreads, 0, s>>>(
+  const QuantGrid qg = quant_grid(rows, cols);
+  quantize_kernel<true><<<qg.grid, qg.block, 0, s>>>(
       xb, rows, cols, ld, dst_row, k, out_rows, codes, sf, gs, amax, rstd, gb, dev_status);
   return check_launch("quantize_kernel");
 }
@@ -327,6 +348,7 @@ extern "C" nvfp4_status_t nvfp4_quantize(const void* x, int64_t rows, int64_t co
   using namespace nvfp4;
   if (rows < 0 || out_rows < 0 || cols <= 0 || ld < cols) return NVFP4_ERR_INVALID_ARG;
   if (cols % 64 != 0 || ld % 8 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (rows > kMaxQuantRows || cols > kMaxQuantCols) return NVFP4_ERR_UNSUPPORTED_SHAPE;
   if (gs == nullptr) return NVFP4_ERR_INVALID_ARG;
   if (rows > 0 && (x == nullptr || codes == nullptr || sf == nullptr)) return NVFP4_ERR_INVALID_ARG;
   if (dst_row == nullptr) {
@@ -354,6 +376,7 @@ extern "C" nvfp4_status_t nvfp4_rmsnorm_quantize(const void* x, int64_t rows, in
   using namespace nvfp4;
   if (rows < 0 || out_rows < 0 || cols <= 0 || ld < cols) return NVFP4_ERR_INVALID_ARG;
   if (cols % 64 != 0 || ld % 8 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (rows > kMaxQuantRows || cols > kMaxQuantCols) return NVFP4_ERR_UNSUPPORTED_SHAPE;
   if (gs == nullptr || ws == nullptr || !(eps >= 0.0f)) return NVFP4_ERR_INVALID_ARG;
   if (rows > 0 && (x == nullptr || gamma == nullptr || codes == nullptr || sf == nullptr))
     return NVFP4_ERR_INVALID_ARG;
