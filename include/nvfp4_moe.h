@@ -88,7 +88,8 @@ typedef enum {
  *   codes    uint8 [out_rows][cols/2];  sf: tiled scales for out_rows rows (see top).
  *   gs       device float[1]: written when compute_gs = 1, read when compute_gs = 0.
  *   ws       device scratch of nvfp4_quantize_workspace_size() bytes (the amax word).
- *   Constraints: cols % 64 == 0, rows >= 0, k in [1, 64] when dst_row != NULL.
+ *   Constraints: cols % 64 == 0, 0 <= rows <= 2^31 - 1, cols <= 268,431,360 (65535 chunks of 256
+ *   blocks), k in [1, 64] when dst_row != NULL.
  * ------------------------------------------------------------------------------------------- */
 NVFP4_API size_t nvfp4_quantize_workspace_size(void);
 NVFP4_API nvfp4_status_t nvfp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t ld,
@@ -113,7 +114,7 @@ NVFP4_API nvfp4_status_t nvfp4_quantize(const void* x, int64_t rows, int64_t col
  *   gamma    bf16 [cols] (16-byte aligned);  eps >= 0
  *   ws       device scratch of nvfp4_rmsnorm_quantize_workspace_size(rows) bytes (the amax word
  *            and one float per row)
- *   everything else as nvfp4_quantize.
+ *   everything else, the size limits included, as nvfp4_quantize.
  * ------------------------------------------------------------------------------------------- */
 NVFP4_API size_t nvfp4_rmsnorm_quantize_workspace_size(int64_t rows);
 NVFP4_API nvfp4_status_t nvfp4_rmsnorm_quantize(const void* x, int64_t rows, int64_t cols,
