@@ -31,10 +31,14 @@ Readings where the pages are silent
   whole tensor, block scales and codes by :func:`oracle.quant.quantize`.
 * Linear: out = dequant(quantize(x)) @ dequant(W)^T in float64, W of shape (N, K) with one
   FP32 global scale; the bf16 output is that value rounded once.
+* Shared expert: the expert FFN of the MoE path applied to every token with weight 1 (one
+  expert, top-1): [RMSNorm ->] quantize -> L1 -> SwiGLU -> re-quantize with the static gs_h ->
+  L2.  It is evaluated by :func:`oracle.moe.moe_ffn` with every token routed to expert 0.
 """
 
 import numpy as np
 
+from .moe import moe_ffn
 from .quant import dequantize, global_scale, quantize
 
 
@@ -83,3 +87,17 @@ def linear(x, w_codes, w_sf, gs_w):
     a = dequantize(codes, sf, gs_x)
     b = dequantize(w_codes, w_sf, np.float32(gs_w))
     return a @ b.T, dict(codes=codes, sf=sf, gs=gs_x)
+
+
+def shared_expert(x, w1, w2, gs_h, gamma=None, eps=1e-6):
+    """The shared expert's FFN on every row of x (float32 (M, H)): RMSNorm first when ``gamma``
+    is given, then the expert FFN of :func:`oracle.moe.moe_ffn` with one expert (``w1``, ``w2``
+    QuantWeights with E = 1) and every token routed to it with weight 1.  Returns float64 (M, H).
+    """
+    x32 = np.asarray(x, dtype=np.float32)
+    if gamma is not None:
+        x32, _ = rmsnorm(x32, gamma, eps)
+    M = x32.shape[0]
+    ids = np.zeros((M, 1), dtype=np.int32)
+    w = np.ones((M, 1), dtype=np.float64)
+    return moe_ffn(x32, None, 1, w1, w2, np.float32(gs_h), ids=ids, weights=w)["out"]

@@ -129,3 +129,27 @@ def test_linear_one_hot_row_selects_a_weight_column():
     w = F.e2m1_decode(w_codes)
     assert np.array_equal(out[0], 2688.0 * w[:, 17])
     assert np.array_equal(out[1], -1344.0 * w[:, 40])
+
+
+def test_shared_expert_is_the_per_row_ffn():
+    """The shared expert evaluated row by row from the definitions: normalize, quantize with the
+    batch's global scale, L1, SwiGLU, re-quantize with gs_h, L2 (weight 1, no routing)."""
+    from oracle import moe as M
+    H, I, Mr = 128, 64, 9
+    x = _bf16_values((Mr, H), seed=21)
+    gamma = _bf16_values((H,), seed=22) + np.float32(1.0)
+    w1 = M.QuantWeights.from_float(_bf16_values((1, 2 * I, H), seed=23, scale=0.05))
+    w2 = M.QuantWeights.from_float(_bf16_values((1, H, I), seed=24, scale=0.05))
+    gs_h = np.float32(16.0)
+    out = D.shared_expert(x, w1, w2, gs_h, gamma=gamma, eps=1e-6)
+    y, _ = D.rmsnorm(x, gamma, 1e-6)
+    gs_x = Q.global_scale(y)
+    xd = Q.dequantize(*Q.quantize(y, gs_x), gs_x)
+    for t in range(Mr):
+        c1 = xd[t] @ w1.dequant(0).T
+        h = (c1[:I] / (1 + np.exp(-c1[:I])) * c1[I:]).astype(np.float32)[None]
+        hd = Q.dequantize(*Q.quantize(h, gs_h), gs_h)[0]
+        assert np.allclose(out[t], hd @ w2.dequant(0).T, rtol=1e-13, atol=1e-14)
+    # without gamma the input is used as given
+    plain = D.shared_expert(x, w1, w2, gs_h)
+    assert not np.allclose(plain, out)
