@@ -1,7 +1,8 @@
 """Throughput of the NVFP4 MoE expert-FFN hot path on B200 (one JSON line on rank 0).
 
     python bench.py [--gpus N] [--steps K] [--warmup W]
-                    [--config decode|mid|prefill|tiny|sweep|dense_decode|dense_prefill]
+                    [--config decode|mid|prefill|tiny|sweep|dense_decode|dense_prefill|
+                              shared_decode|shared_prefill]
                     [--impl ours|reference] [--no-cpu-baseline] [--experts E] [--tokens T]
 
 A step is one pass of the whole path over one batch: routing (top-k + expert buckets), amax ->
@@ -23,6 +24,10 @@ K=7168, N=4096, bf16 output): a step is one grouped-GEMM launch over NVFP4 opera
 activation quantizer (the MoE shared expert's gate/up projection: M = 16 or 8192 rows, K = 7168,
 N = 4096): a step is RMSNorm + amax -> quantize -> dense GEMM, bf16 out, with L2 flushed before
 every step (the 16.5 MB weight would otherwise stay in the 126 MB L2).
+
+--config shared_decode | shared_prefill times the whole shared expert (M = 16 or 8192 rows,
+hidden 7168, intermediate 2048): RMSNorm + quantize -> L1 with SwiGLU + FP4 re-quantization ->
+down projection, bf16 out, L2 flushed before every step.
 
 --impl reference times the CPU oracle (numpy, float64) on a bounded sample of the same workload.
 """
@@ -1015,19 +1020,266 @@ def run_reference_dense(args):
                 "d2h_bytes_per_step": 0}}), flush=True)
 
 
+# ----------------------------------------------------------------------------- shared expert
+
+SHARED_METRIC = "MoE shared expert (RMSNorm fused) on 1 B200, % of NVFP4 tensor/HBM roofline"
+
+
+def shared_algorithmic(cfg):
+    """Bytes and FLOPs of one shared-expert step and of its L1 launch: x read as bf16 (and
+    gamma), x codes written and read once, W1 and W2 codes + scales read once, h codes written
+    and read once, bf16 out written."""
+    M, H, I = cfg.M, cfg.H, cfg.I
+    x_q = M * H * FP4_ELEM_BYTES
+    h_q = M * I * FP4_ELEM_BYTES
+    w1 = 2 * I * H * FP4_ELEM_BYTES
+    w2 = H * I * FP4_ELEM_BYTES
+    return dict(flops=cfg.flops(), bytes=M * H * 2 + H * 2 + 2 * x_q + w1 + 2 * h_q + w2 + M * H * 2,
+                l1_flops=2 * M * H * 2 * I, l1_bytes=x_q + w1 + h_q)
+
+
+def run_shared(args):
+    import torch
+    import torch.distributed as dist
+
+    import nvfp4_block_scaled_gsa_b200 as nv
+    from nvfp4_block_scaled_gsa_b200._native import call
+    from synth import CONFIGS, gen_shared
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local = int(os.environ.get("LOCAL_RANK", 0))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    cfg = CONFIGS[args.config]
+    x_cpu, gamma, w1f, w2f = gen_shared(cfg, device=dev)
+    gamma = gamma.to(dev)
+    w1 = nv.quantize_w1(lambda e: w1f, 1, cfg.I, cfg.H, device=dev)
+    w2 = nv.quantize_weights(lambda e: w2f, 1, cfg.H, cfg.I, device=dev)
+    del w1f, w2f
+    gs_h = torch.tensor([cfg.gs_h], dtype=torch.float32, device=dev)
+    x = x_cpu.to(dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    out = torch.empty(cfg.M, cfg.H, dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(nv.shared_expert_workspace_bytes(cfg.M, cfg.H, cfg.I), dtype=torch.uint8,
+                     device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    acc = shared_algorithmic(cfg)
+
+    def step():
+        nv.shared_expert(x, w1, w2, gs_h, gamma=gamma, eps=cfg.eps, out=out, ws=ws, status=status)
+
+    def graph_of(fn):
+        fn()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, capture_error_mode="thread_local"):
+            fn()
+        torch.cuda.synchronize()
+        return g
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    graph = graph_of(step)
+    sampler = ClockSampler(local) if rank == 0 else None
+    t_end = time.time() + args.soak
+    while time.time() < t_end:
+        for _ in range(8):
+            graph.replay()
+        torch.cuda.synchronize()
+    K = args.steps
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    torch.cuda.nvtx.range_push("timed")
+    total_ms = _timed_steps(graph.replay, flush, K)
+    torch.cuda.nvtx.range_pop()
+    clocks = sampler.stop() if sampler else None
+    if world > 1:
+        dist.barrier()
+
+    # the L1 stage alone (the dominant kernel: GEMM + SwiGLU + FP4 re-quantization, one dense
+    # segment given as offsets [0, rows]) on the codes the fused quantizer wrote
+    Mp = (cfg.M + 127) // 128 * 128
+    codes, sf, gs = nv.rmsnorm_quantize(x, gamma, cfg.eps, out_rows=Mp)
+    offs = torch.tensor([0, Mp], dtype=torch.int32, device=dev)
+    hq = torch.empty(Mp, cfg.I // 2, dtype=torch.uint8, device=dev)
+    hsf = torch.empty(nv.sf_bytes(Mp, cfg.I), dtype=torch.uint8, device=dev)
+    s_ = lambda: torch.cuda.current_stream().cuda_stream  # noqa: E731
+
+    def l1_stage():
+        call("moe_grouped_gemm_l1_swiglu_q", codes.data_ptr(), sf.data_ptr(), gs.data_ptr(),
+             w1.codes.data_ptr(), w1.sf.data_ptr(), w1.gs.data_ptr(), offs.data_ptr(), None, 1,
+             cfg.H, cfg.I, Mp, gs_h.data_ptr(), hq.data_ptr(), hsf.data_ptr(), status.data_ptr(),
+             s_())
+
+    kg = max(1, min(K, 50))
+    l1_ms = _timed_steps(graph_of(l1_stage).replay, flush, kg) / kg
+    code, rc = nv.read_status(status)
+    if code != 0:
+        raise RuntimeError(f"device status {code} after the timed region")
+
+    total_ms = slowest_rank_ms(total_ms, world, dev)
+    ms_step = total_ms / K
+    gbs = whole_job_rate(acc["bytes"], K, world, total_ms) / 1e9
+    tflops = whole_job_rate(acc["flops"], K, world, total_ms) / 1e12
+
+    x_h = x_cpu.pin_memory()
+    out_h = torch.empty(cfg.M, cfg.H, dtype=torch.bfloat16).pin_memory()
+    x_d = torch.empty_like(x)
+
+    def e2e_step():
+        x_d.copy_(x_h, non_blocking=True)
+        nv.shared_expert(x_d, w1, w2, gs_h, gamma=gamma, eps=cfg.eps, out=out, ws=ws,
+                         status=status)
+        out_h.copy_(out, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    ke = max(1, min(K, 50))
+    e2e_ms = slowest_rank_ms(_timed_steps(e2e_step, flush, ke), world, dev) / ke
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = shared_cpu_baseline(cfg)
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    peaks = load_peaks()
+    fp4_peak = peaks["bf16"] * FP4_PER_BF16
+    tensor_bound = acc["l1_flops"] / acc["l1_bytes"] > fp4_peak * 1e12 / (peaks["hbm"] * 1e9)
+    l1_tf = acc["l1_flops"] / (l1_ms * 1e-3) / 1e12
+    l1_gb = acc["l1_bytes"] / (l1_ms * 1e-3) / 1e9
+    kname = "grouped_gemm_kernel<L1_SWIGLU>"
+    if tensor_bound:
+        value, unit = tflops, "TFLOP/s"
+        roof = {"bound": "tensor", "kernel": kname, "achieved": round(l1_tf, 1),
+                "peak": round(fp4_peak, 1), "unit": "TFLOP/s", "frac": round(l1_tf / fp4_peak, 4),
+                "traffic": None, "algorithmic_flops_per_launch": int(acc["l1_flops"]),
+                "peak_source": f"{peaks['src']} bf16 burst x {FP4_PER_BF16} (nominal FP4/BF16 "
+                               "dense ratio)",
+                "step_frac": round(tflops / world / fp4_peak, 4)}
+    else:
+        value, unit = gbs, "GB/s"
+        roof = {"bound": "hbm", "kernel": kname, "achieved": round(l1_gb, 1),
+                "peak": peaks["hbm"], "unit": "GB/s", "frac": round(l1_gb / peaks["hbm"], 4),
+                "traffic": None, "algorithmic_bytes_per_launch": int(acc["l1_bytes"]),
+                "peak_source": peaks["src"], "step_frac": round(gbs / world / peaks["hbm"], 4)}
+    e2e_rate = (world * acc["flops"] / (e2e_ms * 1e-3) / 1e12 if tensor_bound
+                else world * acc["bytes"] / (e2e_ms * 1e-3) / 1e9)
+    split = nv.lib().nvfp4_gemm_dense_workspace_size(cfg.M, cfg.H, cfg.I) > 0
+    line = {
+        "metric": SHARED_METRIC, "value": round(value, 2), "unit": unit, "n_gpus": world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "nvfp4 (e2m1 + e4m3/16), fp32 accumulate",
+        "data": "synthetic (seeded N(0,1) bf16 activations, gamma 1 + 0.1 N(0,1), N(0,0.02) "
+                "weights quantized to NVFP4 on the GPU)",
+        "config": {"workload": f"{cfg.name}: RMSNorm + shared expert FFN, M={cfg.M}, "
+                               f"H={cfg.H}, I={cfg.I}, bf16 out",
+                   "parallelism": f"replicas x{world}",
+                   "l2": "flushed before every step (256 MB write, outside the timed events)",
+                   "cuda_graph": True, "down_projection_k_splits": bool(split)},
+        "tflops": round(tflops, 3), "gbs": round(gbs, 2),
+        "algorithmic": {"bytes_per_step": int(acc["bytes"]), "flops_per_step": int(acc["flops"]),
+                        "l1_bytes_per_launch": int(acc["l1_bytes"])},
+        "roofline": roof,
+        "stages_ms": {"l1_gemm_swiglu_q": round(l1_ms, 5)},
+        "e2e": {"value": round(e2e_rate, 2), "unit": unit,
+                "h2d_bytes_per_step": x_h.numel() * 2, "d2h_bytes_per_step": out_h.numel() * 2,
+                "ms_per_step": round(e2e_ms, 5)},
+        "gpu_launches": (5 if split else 4) * K,
+        "clocks": clocks,
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def _shared_oracle_sample(cfg, rows=4):
+    """The oracle's shared expert on the first `rows` rows (their own global scale); weight
+    pre-packing by the oracle, untimed."""
+    from oracle import dense as D
+    from oracle import moe as M
+    from synth import gen_shared
+    x, gamma, w1, w2 = gen_shared(cfg)
+    x = x[:rows].float().numpy()
+    g = gamma.float().numpy()
+    q1 = M.QuantWeights.from_float(w1.float().numpy()[None])
+    q2 = M.QuantWeights.from_float(w2.float().numpy()[None])
+
+    def run():
+        return D.shared_expert(x, q1, q2, cfg.gs_h, gamma=g, eps=cfg.eps)
+
+    n = x.shape[0]
+    flops = 6 * n * cfg.H * cfg.I
+    nbytes = (n * cfg.H * 2 + cfg.H * 2 + 2 * n * cfg.H * FP4_ELEM_BYTES
+              + 3 * cfg.I * cfg.H * FP4_ELEM_BYTES + 2 * n * cfg.I * FP4_ELEM_BYTES
+              + n * cfg.H * 2)
+    return run, flops, nbytes, n
+
+
+def shared_cpu_baseline(cfg):
+    run, flops, nbytes, n = _shared_oracle_sample(cfg)
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        run()
+        reps += 1
+        dt = time.perf_counter() - t0
+        if dt >= 10.0:
+            break
+    unit = "GB/s" if cfg.M <= 128 else "TFLOP/s"
+    val = nbytes * reps / dt / 1e9 if unit == "GB/s" else flops * reps / dt / 1e12
+    return {"value": round(val, 6), "unit": unit, "cores": _threads(), "kind": "oracle",
+            "sample": f"first {n} rows of {cfg.name} through the oracle's RMSNorm + shared expert, "
+                      f"{reps} repetitions in {dt:.1f} s"}
+
+
+def run_reference_shared(args):
+    from synth import CONFIGS
+    cfg = CONFIGS[args.config]
+    run, flops, nbytes, n = _shared_oracle_sample(cfg)
+    for _ in range(args.warmup):
+        run()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        run()
+    dt = time.perf_counter() - t0
+    unit = "GB/s" if cfg.M <= 128 else "TFLOP/s"
+    value = nbytes * args.steps / dt / 1e9 if unit == "GB/s" else flops * args.steps / dt / 1e12
+    sample = f"each step: the first {n} rows of {cfg.name} through the oracle's shared expert"
+    print(json.dumps({
+        "impl": "reference", "metric": SHARED_METRIC, "value": round(value, 6), "unit": unit,
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{cfg.name}: RMSNorm + shared expert FFN, M={cfg.M}, "
+                               f"H={cfg.H}, I={cfg.I}, bf16 out"},
+        "cpu_baseline": {"value": round(value, 6), "unit": unit, "cores": _threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 6), "unit": unit, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0}}), flush=True)
+
+
 def main():
     args = parse()
     dense = args.config.startswith("dense_")
+    shared = args.config.startswith("shared_")
     if args.impl == "reference":
-        if dense:
+        if dense or shared:
             if int(os.environ.get("RANK", 0)) == 0:
-                run_reference_dense(args)
+                (run_reference_dense if dense else run_reference_shared)(args)
         else:
             run_reference(args)
     elif args.config == "sweep":
         run_sweep(args)
     elif dense:
         run_dense(args)
+    elif shared:
+        run_shared(args)
     else:
         run_ours(args)
 

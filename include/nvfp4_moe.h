@@ -227,6 +227,32 @@ NVFP4_API nvfp4_status_t nvfp4_linear(const void* x, int64_t M, int K, int64_t l
                                       nvfp4_stream_t stream);
 
 /* ---------------------------------------------------------------------------------------------
+ * nvfp4_shared_expert — the MoE shared expert: the expert FFN on every token, weight 1.
+ *
+ * The shared expert of the pages' model quantizes with a GPU-side gsa for both its projections
+ * (commit log of dsv4/kernels/cuda, nvfp4-megamoe-kernel, "Updated layers": shared_expert.py).
+ * Steps: [RMSNorm +] amax -> quantize -> L1 GEMM with SwiGLU and FP4 re-quantization in the
+ * epilogue (moe_grouped_gemm_l1_swiglu_q's kernel, one dense segment) -> down projection
+ * (nvfp4_gemm_dense) -> bf16.
+ *
+ *   x          bf16 [M][ld] (ld >= H, ld % 8 == 0); gamma NULL or bf16 [H] (RMSNorm, eps)
+ *   w1, sfw1   NVFP4 [2I][H] in the gate/up interleave of moe_w1_row_map; gs_w1 device float[1]
+ *   w2, sfw2   NVFP4 [H][I]; gs_w2 device float[1]
+ *   gs_h       device float[1]: static global scale of the intermediate
+ *   out        bf16 [M][H]
+ *   ws         device scratch of nvfp4_shared_expert_workspace_size(M, H, I) bytes
+ *   Constraints: H % 256 == 0, I % 128 == 0, M >= 0.
+ * ------------------------------------------------------------------------------------------- */
+NVFP4_API size_t nvfp4_shared_expert_workspace_size(int64_t M, int H, int I);
+NVFP4_API nvfp4_status_t nvfp4_shared_expert(const void* x, int64_t M, int H, int64_t ld,
+                                             const void* gamma, float eps, const uint8_t* w1,
+                                             const uint8_t* sfw1, const float* gs_w1,
+                                             const uint8_t* w2, const uint8_t* sfw2,
+                                             const float* gs_w2, int I, const float* gs_h,
+                                             void* out, void* ws, size_t ws_bytes,
+                                             int32_t* dev_status, nvfp4_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------------
  * moe_grouped_gemm_l1_swiglu_q — L1 grouped GEMM with SwiGLU and NVFP4 re-quantization fused in
  * the epilogue ("May 24, 2026 — Session Start Plan", section 5 "NVFP4-1.1": L1 GEMM -> SwiGLU ->
  * FP4 pack in registers -> FP4 GMEM).

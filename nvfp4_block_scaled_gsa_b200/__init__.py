@@ -24,5 +24,7 @@ from .api import (  # noqa: F401
     read_status,
     rows_max,
     sf_bytes,
+    shared_expert,
+    shared_expert_workspace_bytes,
 )
 from ._native import Nvfp4Error, lib  # noqa: F401

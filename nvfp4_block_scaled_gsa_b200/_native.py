@@ -42,6 +42,10 @@ SIGNATURES = {
     "nvfp4_linear_workspace_size": (c_size, [c_i64, c_int, c_int]),
     "nvfp4_linear": (c_int, [c_void, c_i64, c_int, c_i64, c_void, c_float, c_void, c_void, c_void,
                              c_int, c_void, c_void, c_size, c_void, c_void]),
+    "nvfp4_shared_expert_workspace_size": (c_size, [c_i64, c_int, c_int]),
+    "nvfp4_shared_expert": (c_int, [c_void, c_i64, c_int, c_i64, c_void, c_float, c_void, c_void,
+                                    c_void, c_void, c_void, c_void, c_int, c_void, c_void, c_void,
+                                    c_size, c_void, c_void]),
     "moe_grouped_gemm_l1_swiglu_q": (c_int, [c_void, c_void, c_void, c_void, c_void, c_void,
                                              c_void, c_void, c_int, c_int, c_int, c_i64, c_void,
                                              c_void, c_void, c_void, c_void]),

@@ -114,6 +114,30 @@ def linear(x, w: "NVFP4Weights", gamma=None, eps=1e-6, out=None, ws=None, status
     return out
 
 
+def shared_expert_workspace_bytes(M, H, I):
+    return int(lib().nvfp4_shared_expert_workspace_size(M, H, I))
+
+
+def shared_expert(x, w1: "NVFP4Weights", w2: "NVFP4Weights", gs_h, gamma=None, eps=1e-6,
+                  out=None, ws=None, status=None):
+    """The shared expert's FFN on every row of bf16 x (M, H): w1 from quantize_w1 with E = 1
+    (gate/up interleave), w2 from quantize_weights with E = 1 (H x I); gs_h device float[1].
+    gamma (bf16 (H,)) fuses an RMSNorm into the first quantizer.  Returns bf16 (M, H)."""
+    assert x.dtype == BF16 and x.dim() == 2 and x.stride(1) == 1 and w1.E == 1 and w2.E == 1
+    M, H = x.shape
+    I = w1.N // 2
+    assert w1.K == H and w2.N == H and w2.K == I
+    if out is None:
+        out = torch.empty(M, H, dtype=BF16, device=x.device)
+    if ws is None:
+        ws = torch.empty(max(shared_expert_workspace_bytes(M, H, I), 256), dtype=U8,
+                         device=x.device)
+    call("nvfp4_shared_expert", _p(x), M, H, x.stride(0), _p(gamma), float(eps), _p(w1.codes),
+         _p(w1.sf), _p(w1.gs), _p(w2.codes), _p(w2.sf), _p(w2.gs), I, _p(gs_h), _p(out), _p(ws),
+         ws.numel(), _p(status), _stream())
+    return out
+
+
 def quantize_weights(get_expert, E, N, K, device="cuda", row_map=None):
     """Pre-pack expert weights: get_expert(e) -> bf16 (N, K) on the device; each expert gets its
     own global scale from its amax.  row_map (device int32 [N]): stored row of each row."""

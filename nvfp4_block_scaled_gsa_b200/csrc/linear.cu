@@ -1,5 +1,5 @@
 // linear.cu — dense NVFP4 linear, y = x W^T, with the activation quantized on the fly and an
-// optional RMSNorm fused into that quantizer.
+// optional RMSNorm fused into that quantizer; and the shared expert built from the same pieces.
 //
 // The pages' dense layer (Nvfp4Linear, and the shared expert's two projections) quantizes its
 // bf16 activation with a GPU-computed global scale and runs an NVFP4 GEMM against pre-packed
@@ -24,6 +24,11 @@ nvfp4_status_t gemm_dense(const uint8_t* a, const uint8_t* sfa, const float* gs_
                           int K, void* out_bf16, float* part, int64_t part_floats, int32_t* status,
                           cudaStream_t s);
 int dense_k_splits(int64_t M, int N, int K, int sms, int64_t part_floats);
+nvfp4_status_t gemm_l1(const uint8_t* a, const uint8_t* sfa, const float* gs_a, const uint8_t* w1,
+                       const uint8_t* sfw1, const float* gs_w1, const int32_t* offs,
+                       const int32_t* row_slot, int E, int H, int I, int64_t R_max,
+                       const float* gs_h, uint8_t* h, uint8_t* sfh, int32_t* status,
+                       cudaStream_t s);
 
 namespace {
 
@@ -60,6 +65,44 @@ LinearLayout linear_layout(int64_t M, int N, int K) {
   L.part = take(L.part_floats * 4);
   L.total = o;
   return L;
+}
+
+// Byte offsets of the nvfp4_shared_expert workspace regions (each 256-byte aligned).
+struct SharedLayout {
+  int64_t quant_ws, gs, xq, xsf, hq, hsf, part, total;
+  int64_t part_floats;
+};
+
+SharedLayout shared_layout(int64_t M, int H, int I) {
+  SharedLayout L{};
+  const int64_t Mp = round_up(M, 128);
+  int64_t o = 0;
+  auto take = [&](int64_t bytes) {
+    const int64_t at = o;
+    o += round_up(bytes, 256);
+    return at;
+  };
+  L.quant_ws = take(static_cast<int64_t>(nvfp4_rmsnorm_quantize_workspace_size(M)));
+  L.gs = take(4);
+  L.xq = take(Mp * (H / 2));
+  L.xsf = take(Mp * (H / 16));
+  L.hq = take(Mp * (I / 2));
+  L.hsf = take(Mp * (I / 16));
+  L.part_floats = dense_part_floats(M, H, I);
+  L.part = take(L.part_floats * 4);
+  L.total = o;
+  return L;
+}
+
+// [RMSNorm +] quantize x into the workspace's code rows (rows past M are padding).
+nvfp4_status_t quantize_rows(const void* x, int64_t M, int K, int64_t ld, const void* gamma,
+                             float eps, uint8_t* codes, uint8_t* sf, float* gs, void* qws,
+                             int32_t* dev_status, cudaStream_t s) {
+  const int64_t Mp = round_up(M, 128);
+  return gamma != nullptr
+             ? rmsnorm_quantize_launch(x, M, K, ld, gamma, eps, nullptr, 1, Mp, codes, sf, gs, 1,
+                                       qws, dev_status, s)
+             : quantize_launch(x, M, K, ld, nullptr, 1, Mp, codes, sf, gs, 1, qws, dev_status, s);
 }
 
 }  // namespace
@@ -119,14 +162,51 @@ extern "C" nvfp4_status_t nvfp4_linear(const void* x, int64_t M, int K, int64_t 
   uint8_t* codes = base + L.codes;
   uint8_t* sf = base + L.sf;
   float* gs = reinterpret_cast<float*>(base + L.gs);
-  const int64_t Mp = round_up(M, 128);
   nvfp4_status_t st =
-      gamma != nullptr
-          ? rmsnorm_quantize_launch(x, M, K, ld, gamma, eps, nullptr, 1, Mp, codes, sf, gs, 1,
-                                    base + L.quant_ws, dev_status, s)
-          : quantize_launch(x, M, K, ld, nullptr, 1, Mp, codes, sf, gs, 1, base + L.quant_ws,
-                            dev_status, s);
+      quantize_rows(x, M, K, ld, gamma, eps, codes, sf, gs, base + L.quant_ws, dev_status, s);
   if (st != NVFP4_OK) return st;
   float* part = L.part_floats > 0 ? reinterpret_cast<float*>(base + L.part) : nullptr;
   return gemm_dense(codes, sf, gs, w, sfw, gs_w, M, N, K, out, part, L.part_floats, dev_status, s);
+}
+
+extern "C" size_t nvfp4_shared_expert_workspace_size(int64_t M, int H, int I) {
+  if (M < 0 || H <= 0 || I <= 0) return 0;
+  return static_cast<size_t>(nvfp4::shared_layout(M, H, I).total);
+}
+
+extern "C" nvfp4_status_t nvfp4_shared_expert(const void* x, int64_t M, int H, int64_t ld,
+                                              const void* gamma, float eps, const uint8_t* w1,
+                                              const uint8_t* sfw1, const float* gs_w1,
+                                              const uint8_t* w2, const uint8_t* sfw2,
+                                              const float* gs_w2, int I, const float* gs_h,
+                                              void* out, void* ws, size_t ws_bytes,
+                                              int32_t* dev_status, nvfp4_stream_t stream) {
+  using namespace nvfp4;
+  if (M < 0 || H <= 0 || I <= 0 || ld < H || !(eps >= 0.0f)) return NVFP4_ERR_INVALID_ARG;
+  if (H % 256 || I % 128 || ld % 8) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (M > (int64_t)INT32_MAX - 127) return NVFP4_ERR_UNSUPPORTED_SHAPE;  // rows index as int
+  if (!w1 || !sfw1 || !gs_w1 || !w2 || !sfw2 || !gs_w2 || !gs_h || !ws)
+    return NVFP4_ERR_INVALID_ARG;
+  if (M > 0 && (!x || !out)) return NVFP4_ERR_INVALID_ARG;
+  const SharedLayout L = shared_layout(M, H, I);
+  if ((int64_t)ws_bytes < L.total) return NVFP4_ERR_WORKSPACE_TOO_SMALL;
+  if (!aligned16(x) || !aligned16(gamma) || !aligned16(w1) || !aligned16(sfw1) ||
+      !aligned16(w2) || !aligned16(sfw2) || !aligned16(out) || !aligned16(ws) ||
+      (reinterpret_cast<uintptr_t>(gs_w1) & 3u) || (reinterpret_cast<uintptr_t>(gs_w2) & 3u) ||
+      (reinterpret_cast<uintptr_t>(gs_h) & 3u))
+    return NVFP4_ERR_MISALIGNED;
+  if (M == 0) return NVFP4_OK;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  float* gs_x = reinterpret_cast<float*>(base + L.gs);
+  nvfp4_status_t st = quantize_rows(x, M, H, ld, gamma, eps, base + L.xq, base + L.xsf, gs_x,
+                                    base + L.quant_ws, dev_status, s);
+  if (st != NVFP4_OK) return st;
+  // L1 with SwiGLU + FP4 re-quantization over one dense segment (no offsets, every row written)
+  st = gemm_l1(base + L.xq, base + L.xsf, gs_x, w1, sfw1, gs_w1, nullptr, nullptr, 1, H, I,
+               round_up(M, 128), gs_h, base + L.hq, base + L.hsf, dev_status, s);
+  if (st != NVFP4_OK) return st;
+  float* part = L.part_floats > 0 ? reinterpret_cast<float*>(base + L.part) : nullptr;
+  return gemm_dense(base + L.hq, base + L.hsf, gs_h, w2, sfw2, gs_w2, M, H, I, out, part,
+                    L.part_floats, dev_status, s);
 }

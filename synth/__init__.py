@@ -5,4 +5,4 @@ arithmetic lives here, so both sides of a parity check receive the same inputs w
 sharing any of the method's code.
 """
 
-from .inputs import CONFIGS, DenseConfig, MoEConfig, SweepConfig, gen_dense, gen_logits, gen_x, gen_weight_expert, gen_sweep  # noqa: F401
+from .inputs import CONFIGS, DenseConfig, MoEConfig, SharedConfig, SweepConfig, gen_dense, gen_logits, gen_shared, gen_x, gen_weight_expert, gen_sweep  # noqa: F401

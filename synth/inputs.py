@@ -66,6 +66,21 @@ class DenseConfig:
         return 2 * self.M * self.N * self.K
 
 
+@dataclass(frozen=True)
+class SharedConfig:
+    """The MoE shared expert on every token: RMSNorm(x) -> L1 (2I x H) + SwiGLU -> L2 (H x I)."""
+    name: str
+    M: int
+    H: int
+    I: int
+    eps: float = 1e-6
+    gs_h: float = 1.0
+    seed: int = 0
+
+    def flops(self):
+        return 2 * self.M * self.H * 2 * self.I + 2 * self.M * self.I * self.H
+
+
 CONFIGS = {
     "tiny": MoEConfig("tiny", T=64, H=256, I=128, E=8, k=2, logits="normal", gs_h=64.0),
     "decode": MoEConfig("decode", T=16, H=7168, I=2048, E=256, k=8, logits="uniform"),
@@ -74,6 +89,8 @@ CONFIGS = {
     "sweep": SweepConfig("sweep", E=32, K=7168, N=4096, m_max=4096),
     "dense_decode": DenseConfig("dense_decode", M=16, N=4096, K=7168),
     "dense_prefill": DenseConfig("dense_prefill", M=8192, N=4096, K=7168),
+    "shared_decode": SharedConfig("shared_decode", M=16, H=7168, I=2048),
+    "shared_prefill": SharedConfig("shared_prefill", M=8192, H=7168, I=2048),
 }
 
 
@@ -151,3 +168,18 @@ def gen_dense(cfg, device="cpu"):
     g = torch.Generator(device=device).manual_seed(cfg.seed + 13)
     w = (torch.randn(cfg.N, cfg.K, generator=g, dtype=torch.float32, device=device) * 0.02)
     return x, gamma, w.to(torch.bfloat16)
+
+
+def gen_shared(cfg, device="cpu"):
+    """Inputs of a shared-expert workload: x bf16 (M, H) N(0, 1) (seed + 21), gamma bf16 (H,)
+    1 + 0.1 N(0, 1) (seed + 22); W1 (2I x H, gate rows then up rows) and W2 (H x I) bf16
+    N(0, 0.02) from seeds seed + 23 and seed + 24 (on `device`)."""
+    g = torch.Generator().manual_seed(cfg.seed + 21)
+    x = torch.randn(cfg.M, cfg.H, generator=g, dtype=torch.float32).to(torch.bfloat16)
+    g = torch.Generator().manual_seed(cfg.seed + 22)
+    gamma = (1.0 + 0.1 * torch.randn(cfg.H, generator=g, dtype=torch.float32)).to(torch.bfloat16)
+    g = torch.Generator(device=device).manual_seed(cfg.seed + 23)
+    w1 = torch.randn(2 * cfg.I, cfg.H, generator=g, dtype=torch.float32, device=device) * 0.02
+    g = torch.Generator(device=device).manual_seed(cfg.seed + 24)
+    w2 = torch.randn(cfg.H, cfg.I, generator=g, dtype=torch.float32, device=device) * 0.02
+    return x, gamma, w1.to(torch.bfloat16), w2.to(torch.bfloat16)

@@ -169,3 +169,25 @@ def test_dense_entry_points_reject_bad_arguments(L):
     assert rq(f, 4, 64, 64, f, 0.0, None, 1, 4, f, f, f, 1, f, 256, None, None) == 4   # ws
     assert rq(f, 4, 96, 96, f, 0.0, None, 1, 4, f, f, f, 1, f, big, None, None) == 2   # cols % 64
     assert rq(f, 4, 64, 64, odd, 0.0, None, 1, 4, f, f, f, 1, f, big, None, None) == 3
+
+
+def test_shared_expert_workspace_and_argument_checks(L):
+    # quantizer scratch, gs, x codes + scales, h codes + scales (128 padded rows each) and 5 K
+    # ranges of FP32 partials for the down projection (28 output tiles: 148 // 28 = 5)
+    want = 512 + 256 + 128 * 3584 + 128 * 448 + 128 * 1024 + 128 * 128 + 5 * 16 * 7168 * 4
+    assert L.nvfp4_shared_expert_workspace_size(16, 7168, 2048) == want
+    assert L.nvfp4_shared_expert_workspace_size(-1, 7168, 2048) == 0
+    f = FAKE
+    big = 1 << 40
+    se = L.nvfp4_shared_expert
+    # x, M, H, ld, gamma, eps, w1, sfw1, gs_w1, w2, sfw2, gs_w2, I, gs_h, out, ws, ws_bytes, ...
+    assert se(f, 16, 200, 200, None, 0.0, f, f, f, f, f, f, 128, f, f, f, big, None, None) == 2
+    assert se(f, 16, 256, 256, None, 0.0, f, f, f, f, f, f, 64, f, f, f, big, None, None) == 2
+    assert se(f, 16, 256, 128, None, 0.0, f, f, f, f, f, f, 128, f, f, f, big, None, None) == 1
+    assert se(f, 16, 256, 256, None, 0.0, f, f, f, f, f, f, 128, None, f, f, big, None,
+              None) == 1  # no gs_h
+    assert se(f, 16, 256, 256, None, 0.0, f, f, f, f, f, f, 128, f, f, f, 100, None, None) == 4
+    odd = ctypes.c_void_p((1 << 20) + 8)
+    assert se(f, 16, 256, 256, None, 0.0, f, f, f, odd, f, f, 128, f, f, f, big, None, None) == 3
+    assert se(None, 0, 256, 256, None, 0.0, f, f, f, f, f, f, 128, f, None, f, big, None,
+              None) == 0

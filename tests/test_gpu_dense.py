@@ -171,3 +171,39 @@ def test_linear_prefill_size_sampled_rows():
     c, s = Q.quantize(y[rows], gs)
     ref = Q.dequantize(c, s, gs) @ qw.dequant(0).T
     _assert_close(out[torch.from_numpy(rows)].float().cpu().numpy(), ref)
+
+
+def _expert_weights(H, I, seed, scale=0.02):
+    from tests._gpu_util import upload_weights
+    g = torch.Generator().manual_seed(seed)
+    w1f = (torch.randn(1, 2 * I, H, generator=g) * scale).to(torch.bfloat16).float().numpy()
+    w2f = (torch.randn(1, H, I, generator=g) * scale).to(torch.bfloat16).float().numpy()
+    q1, q2 = M.QuantWeights.from_float(w1f), M.QuantWeights.from_float(w2f)
+    return q1, q2, upload_weights(q1, w1=True), upload_weights(q2)
+
+
+# (M, H, I, gs_h): one tile, ragged rows, pair tiles from 1024 rows, and the decode shape of the
+# model's shared expert (hidden 7168, intermediate 2048; split-K down projection)
+SHARED_CASES = [(1, 256, 128, 64.0), (37, 256, 128, 64.0), (200, 512, 256, 64.0),
+                (1100, 256, 128, 64.0), (16, 7168, 2048, 1.0)]
+
+
+@pytest.mark.parametrize("norm", [False, True])
+@pytest.mark.parametrize("case", SHARED_CASES)
+def test_shared_expert_parity(case, norm):
+    Mr, H, I, gs_h = case
+    x, gamma = _inputs(Mr, H, seed=Mr * 3 + H)
+    q1, q2, w1, w2 = _expert_weights(H, I, seed=H + I)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    gs_h_d = torch.tensor([gs_h], dtype=torch.float32, device=DEV)
+    out = nv.shared_expert(x.to(DEV), w1, w2, gs_h_d, gamma=gamma.to(DEV) if norm else None,
+                           eps=1e-6, status=status)
+    torch.cuda.synchronize()
+    assert nv.read_status(status) == (0, 0)
+    ref = D.shared_expert(x.float().numpy(), q1, q2, np.float32(gs_h),
+                          gamma=gamma.float().numpy() if norm else None, eps=1e-6)
+    got = out.float().cpu().numpy()
+    # the intermediate is re-quantized (a rare one-step E2M1 difference is allowed there), so
+    # the bars are the output-level ones of the MoE FFN
+    assert rel_fro(got, M.bf16_round(ref)) <= 1e-3
+    assert cosine(got, ref) >= 0.9999
