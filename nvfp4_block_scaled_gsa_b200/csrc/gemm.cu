@@ -905,6 +905,22 @@ int dense_k_splits(int64_t M, int N, int K, int sms, int64_t part_floats) {
 
 int device_sms() { return num_sms(); }
 
+// FP32 partial products of a dense C = A B^T over ks K ranges, plane r = range r, M rows of N
+// floats each, for a consumer that finishes the sum itself.  ks comes from dense_k_splits (so
+// ks <= K/256 and the rows stay below the pair-tile threshold).
+nvfp4_status_t gemm_dense_parts(const uint8_t* a, const uint8_t* sfa, const float* gs_a,
+                                const uint8_t* b, const uint8_t* sfb, const float* gs_b,
+                                int64_t M, int N, int K, int ks, float* part, int32_t* status,
+                                cudaStream_t s) {
+  if (M == 0) return NVFP4_OK;
+  GemmArgs g{};
+  g.sfa = sfa; g.sfb = sfb; g.gs_a = gs_a; g.gs_b = gs_b; g.offs = nullptr;
+  g.E = 1; g.N = N; g.K = K; g.n_tiles = N / TileCfg<PLAIN_F32, 1>::BN; g.R_max = round_up(M, 128);
+  g.out_rows = M; g.status = status; g.out = part; g.k_splits = ks;
+  g.split_stride = M * (int64_t)N;
+  return launch<PLAIN_F32>(a, b, N, g, s);
+}
+
 // Dense C = A B^T for A NVFP4 [round_up(M, 128)][K] (rows past M are padding that is never
 // stored) and B NVFP4 [N][K]: one segment, no offsets.  With K splits the ranges' FP32 partial
 // products go to `part` and splitk_reduce_kernel adds them; otherwise the bf16 result is stored

@@ -24,6 +24,11 @@ nvfp4_status_t gemm_dense(const uint8_t* a, const uint8_t* sfa, const float* gs_
                           int K, void* out_bf16, float* part, int64_t part_floats, int32_t* status,
                           cudaStream_t s);
 int dense_k_splits(int64_t M, int N, int K, int sms, int64_t part_floats);
+int device_sms();
+nvfp4_status_t gemm_dense_parts(const uint8_t* a, const uint8_t* sfa, const float* gs_a,
+                                const uint8_t* b, const uint8_t* sfb, const float* gs_b,
+                                int64_t M, int N, int K, int ks, float* part, int32_t* status,
+                                cudaStream_t s);
 nvfp4_status_t gemm_l1(const uint8_t* a, const uint8_t* sfa, const float* gs_a, const uint8_t* w1,
                        const uint8_t* sfw1, const float* gs_w1, const int32_t* offs,
                        const int32_t* row_slot, int E, int H, int I, int64_t R_max,
@@ -67,10 +72,70 @@ LinearLayout linear_layout(int64_t M, int N, int K) {
   return L;
 }
 
+// The shared expert's L1 from split-K partial products (few rows: the fused-epilogue L1 would
+// run one CTA per N tile).  Per 16-feature block: the ks planes of its 16 gate columns and 16 up
+// columns (the W1 interleave: column 32j + i is gate feature 16j + i, column 32j + 16 + i its up
+// partner) are added in plane order, then h = g * u / (1 + e^-g) and the block is quantized
+// with the static gs_h, the fused L1 epilogue's arithmetic.  One thread per block on a
+// (row x chunk) grid; the 4 lanes of a 4-block group assemble their scale bytes into one word.
+__global__ void __launch_bounds__(256) swiglu_quant_kernel(const float* __restrict__ part, int ks,
+                                                           int64_t M, int I,
+                                                           const float* __restrict__ gs_h_p,
+                                                           uint8_t* __restrict__ h,
+                                                           uint8_t* __restrict__ sfh) {
+  const int64_t nblk_row = I / 16;
+  const int64_t r = blockIdx.x;
+  const int64_t c = (int64_t)blockIdx.y * blockDim.x + threadIdx.x;
+  const bool valid = r < M && c < nblk_row;
+  uint32_t sbyte = 0;
+  uint2 packed = make_uint2(0u, 0u);
+  if (valid) {
+    const float gs_h = __ldg(gs_h_p);
+    const int64_t n2 = 2 * (int64_t)I;
+    const float* base = part + r * n2 + 32 * c;
+    float g[16], u[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) g[i] = u[i] = 0.0f;
+    for (int p = 0; p < ks; ++p) {
+      const float4* q = reinterpret_cast<const float4*>(base + p * M * n2);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float4 a = __ldg(q + j), b = __ldg(q + 4 + j);
+        g[4 * j] += a.x; g[4 * j + 1] += a.y; g[4 * j + 2] += a.z; g[4 * j + 3] += a.w;
+        u[4 * j] += b.x; u[4 * j + 1] += b.y; u[4 * j + 2] += b.z; u[4 * j + 3] += b.w;
+      }
+    }
+    float hv[16];
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      hv[i] = __fdividef(g[i] * u[i], 1.0f + __expf(-g[i]));
+      amax = fmaxf(amax, fabsf(hv[i]));
+    }
+    float rcp;
+    sbyte = nvfp4_block_scale(amax, gs_h, rcp);
+    packed.x = nvfp4_pack8(hv, rcp);
+    packed.y = nvfp4_pack8(hv + 8, rcp);
+  }
+  uint32_t sword = sbyte;
+  sword |= __shfl_down_sync(0xffffffffu, sbyte, 1) << 8;
+  sword |= __shfl_down_sync(0xffffffffu, sbyte, 2) << 16;
+  sword |= __shfl_down_sync(0xffffffffu, sbyte, 3) << 24;
+  if (!valid) return;
+  *reinterpret_cast<uint2*>(h + r * (I / 2) + c * 8) = packed;
+  if ((c & 3) == 0) *reinterpret_cast<uint32_t*>(sfh + sf_offset(r, c, nblk_row)) = sword;
+}
+
+// L1 partial products of the shared expert, sized for kSizingSms (0 when the fused L1 is used).
+int64_t shared_l1_part_floats(int64_t M, int H, int I) {
+  const int ks = dense_k_splits(M, 2 * I, H, kSizingSms, INT64_MAX / 4);
+  return ks > 1 ? ks * M * 2 * (int64_t)I : 0;
+}
+
 // Byte offsets of the nvfp4_shared_expert workspace regions (each 256-byte aligned).
 struct SharedLayout {
-  int64_t quant_ws, gs, xq, xsf, hq, hsf, part, total;
-  int64_t part_floats;
+  int64_t quant_ws, gs, xq, xsf, hq, hsf, part, part1, total;
+  int64_t part_floats, part1_floats;
 };
 
 SharedLayout shared_layout(int64_t M, int H, int I) {
@@ -90,6 +155,8 @@ SharedLayout shared_layout(int64_t M, int H, int I) {
   L.hsf = take(Mp * (I / 16));
   L.part_floats = dense_part_floats(M, H, I);
   L.part = take(L.part_floats * 4);
+  L.part1_floats = shared_l1_part_floats(M, H, I);
+  L.part1 = take(L.part1_floats * 4);
   L.total = o;
   return L;
 }
@@ -202,9 +269,26 @@ extern "C" nvfp4_status_t nvfp4_shared_expert(const void* x, int64_t M, int H, i
   nvfp4_status_t st = quantize_rows(x, M, H, ld, gamma, eps, base + L.xq, base + L.xsf, gs_x,
                                     base + L.quant_ws, dev_status, s);
   if (st != NVFP4_OK) return st;
-  // L1 with SwiGLU + FP4 re-quantization over one dense segment (no offsets, every row written)
-  st = gemm_l1(base + L.xq, base + L.xsf, gs_x, w1, sfw1, gs_w1, nullptr, nullptr, 1, H, I,
-               round_up(M, 128), gs_h, base + L.hq, base + L.hsf, dev_status, s);
+  // L1 + SwiGLU + FP4 re-quantization: split along K when the output has too few tiles for the
+  // SMs (partials, then swiglu_quant_kernel); otherwise the fused-epilogue kernel over one dense
+  // segment (no offsets, every row written)
+  const int ks1 = dense_k_splits(M, 2 * I, H, device_sms(), L.part1_floats);
+  if (ks1 > 1) {
+    float* part1 = reinterpret_cast<float*>(base + L.part1);
+    st = gemm_dense_parts(base + L.xq, base + L.xsf, gs_x, w1, sfw1, gs_w1, M, 2 * I, H, ks1,
+                          part1, dev_status, s);
+    if (st != NVFP4_OK) return st;
+    const int64_t nblk_row = I / 16;
+    const int64_t chunks = (nblk_row + 255) / 256;
+    const int64_t per = (nblk_row + chunks - 1) / chunks;
+    swiglu_quant_kernel<<<dim3(static_cast<unsigned>(M), static_cast<unsigned>(chunks)),
+                          dim3(static_cast<unsigned>((per + 31) / 32 * 32)), 0, s>>>(
+        part1, ks1, M, I, gs_h, base + L.hq, base + L.hsf);
+    st = check_launch("swiglu_quant_kernel");
+  } else {
+    st = gemm_l1(base + L.xq, base + L.xsf, gs_x, w1, sfw1, gs_w1, nullptr, nullptr, 1, H, I,
+                 round_up(M, 128), gs_h, base + L.hq, base + L.hsf, dev_status, s);
+  }
   if (st != NVFP4_OK) return st;
   float* part = L.part_floats > 0 ? reinterpret_cast<float*>(base + L.part) : nullptr;
   return gemm_dense(base + L.hq, base + L.hsf, gs_h, w2, sfw2, gs_w2, M, H, I, out, part,

@@ -172,11 +172,16 @@ def test_dense_entry_points_reject_bad_arguments(L):
 
 
 def test_shared_expert_workspace_and_argument_checks(L):
-    # quantizer scratch, gs, x codes + scales, h codes + scales (128 padded rows each) and 5 K
-    # ranges of FP32 partials for the down projection (28 output tiles: 148 // 28 = 5)
-    want = 512 + 256 + 128 * 3584 + 128 * 448 + 128 * 1024 + 128 * 128 + 5 * 16 * 7168 * 4
+    # quantizer scratch, gs, x codes + scales, h codes + scales (128 padded rows each), 5 K
+    # ranges of FP32 partials for the down projection (28 output tiles: 148 // 28 = 5) and 9 for
+    # the L1 (16 output tiles of 2I = 4096 columns: 148 // 16 = 9)
+    want = (512 + 256 + 128 * 3584 + 128 * 448 + 128 * 1024 + 128 * 128 + 5 * 16 * 7168 * 4
+            + 9 * 16 * 4096 * 4)
     assert L.nvfp4_shared_expert_workspace_size(16, 7168, 2048) == want
     assert L.nvfp4_shared_expert_workspace_size(-1, 7168, 2048) == 0
+    # 8192 rows: no split anywhere (fused-epilogue L1, direct bf16 down projection)
+    assert L.nvfp4_shared_expert_workspace_size(8192, 7168, 2048) == (
+        256 + 8192 * 4 + 256 + 8192 * 3584 + 8192 * 448 + 8192 * 1024 + 8192 * 128)
     f = FAKE
     big = 1 << 40
     se = L.nvfp4_shared_expert
