@@ -76,54 +76,66 @@ LinearLayout linear_layout(int64_t M, int N, int K) {
 // run one CTA per N tile).  Per 16-feature block: the ks planes of its 16 gate columns and 16 up
 // columns (the W1 interleave: column 32j + i is gate feature 16j + i, column 32j + 16 + i its up
 // partner) are added in plane order, then h = g * u / (1 + e^-g) and the block is quantized
-// with the static gs_h, the fused L1 epilogue's arithmetic.  One thread per block on a
-// (row x chunk) grid; the 4 lanes of a 4-block group assemble their scale bytes into one word.
+// with the static gs_h, the fused L1 epilogue's arithmetic.  One thread per 4 features on a
+// (row x chunk) grid, loads issued 4 planes at a time; the 4 lanes of a block share its amax by
+// shuffles, and lanes 16g, +4, +8, +12 (blocks 4g..4g+3) assemble one scale word.
 __global__ void __launch_bounds__(256) swiglu_quant_kernel(const float* __restrict__ part, int ks,
                                                            int64_t M, int I,
                                                            const float* __restrict__ gs_h_p,
                                                            uint8_t* __restrict__ h,
                                                            uint8_t* __restrict__ sfh) {
-  const int64_t nblk_row = I / 16;
   const int64_t r = blockIdx.x;
-  const int64_t c = (int64_t)blockIdx.y * blockDim.x + threadIdx.x;
-  const bool valid = r < M && c < nblk_row;
-  uint32_t sbyte = 0;
-  uint2 packed = make_uint2(0u, 0u);
+  const int64_t t = (int64_t)blockIdx.y * blockDim.x + threadIdx.x;  // features 4t .. 4t+3
+  const bool valid = r < M && t < I / 4;
+  const int64_t blk = t >> 2, q = t & 3;
+  float hv[4] = {0.f, 0.f, 0.f, 0.f};
+  float amax = 0.0f;
   if (valid) {
-    const float gs_h = __ldg(gs_h_p);
     const int64_t n2 = 2 * (int64_t)I;
-    const float* base = part + r * n2 + 32 * c;
-    float g[16], u[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) g[i] = u[i] = 0.0f;
-    for (int p = 0; p < ks; ++p) {
-      const float4* q = reinterpret_cast<const float4*>(base + p * M * n2);
+    const float* gate = part + r * n2 + 32 * blk + 4 * q;
+    float g[4] = {0.f, 0.f, 0.f, 0.f}, u[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int p0 = 0; p0 < ks; p0 += 4) {
+      float4 a[4], b[4];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const float4 a = __ldg(q + j), b = __ldg(q + 4 + j);
-        g[4 * j] += a.x; g[4 * j + 1] += a.y; g[4 * j + 2] += a.z; g[4 * j + 3] += a.w;
-        u[4 * j] += b.x; u[4 * j + 1] += b.y; u[4 * j + 2] += b.z; u[4 * j + 3] += b.w;
+        if (p0 + j < ks) {
+          const float* pg = gate + (p0 + j) * M * n2;
+          a[j] = __ldg(reinterpret_cast<const float4*>(pg));
+          b[j] = __ldg(reinterpret_cast<const float4*>(pg + 16));
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        if (p0 + j < ks) {
+          g[0] += a[j].x; g[1] += a[j].y; g[2] += a[j].z; g[3] += a[j].w;
+          u[0] += b[j].x; u[1] += b[j].y; u[2] += b[j].z; u[3] += b[j].w;
+        }
       }
     }
-    float hv[16];
-    float amax = 0.0f;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
+    for (int i = 0; i < 4; ++i) {
       hv[i] = __fdividef(g[i] * u[i], 1.0f + __expf(-g[i]));
       amax = fmaxf(amax, fabsf(hv[i]));
     }
-    float rcp;
-    sbyte = nvfp4_block_scale(amax, gs_h, rcp);
-    packed.x = nvfp4_pack8(hv, rcp);
-    packed.y = nvfp4_pack8(hv + 8, rcp);
   }
-  uint32_t sword = sbyte;
-  sword |= __shfl_down_sync(0xffffffffu, sbyte, 1) << 8;
-  sword |= __shfl_down_sync(0xffffffffu, sbyte, 2) << 16;
-  sword |= __shfl_down_sync(0xffffffffu, sbyte, 3) << 24;
+  // the block's amax over its 4 consecutive lanes (invalid lanes hold 0 and sit in whole
+  // invalid blocks: I / 4 is a multiple of 32)
+  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+  const float gs_h = __ldg(gs_h_p);
+  float rcp;
+  const uint32_t sb = nvfp4_block_scale(amax, gs_h, rcp);
+  uint32_t sword = sb;
+  sword |= __shfl_down_sync(0xffffffffu, sb, 4) << 8;
+  sword |= __shfl_down_sync(0xffffffffu, sb, 8) << 16;
+  sword |= __shfl_down_sync(0xffffffffu, sb, 12) << 24;
   if (!valid) return;
-  *reinterpret_cast<uint2*>(h + r * (I / 2) + c * 8) = packed;
-  if ((c & 3) == 0) *reinterpret_cast<uint32_t*>(sfh + sf_offset(r, c, nblk_row)) = sword;
+  const uint32_t codes =
+      rcp == 0.0f ? 0u
+                  : (cvt_e2m1x2(scaled(hv[0], rcp), scaled(hv[1], rcp)) |
+                     (cvt_e2m1x2(scaled(hv[2], rcp), scaled(hv[3], rcp)) << 8));
+  *reinterpret_cast<uint16_t*>(h + r * (I / 2) + 2 * t) = static_cast<uint16_t>(codes);
+  if ((t & 15) == 0) *reinterpret_cast<uint32_t*>(sfh + sf_offset(r, blk, I / 16)) = sword;
 }
 
 // L1 partial products of the shared expert, sized for kSizingSms (0 when the fused L1 is used).
@@ -278,9 +290,9 @@ extern "C" nvfp4_status_t nvfp4_shared_expert(const void* x, int64_t M, int H, i
     st = gemm_dense_parts(base + L.xq, base + L.xsf, gs_x, w1, sfw1, gs_w1, M, 2 * I, H, ks1,
                           part1, dev_status, s);
     if (st != NVFP4_OK) return st;
-    const int64_t nblk_row = I / 16;
-    const int64_t chunks = (nblk_row + 255) / 256;
-    const int64_t per = (nblk_row + chunks - 1) / chunks;
+    const int64_t quads = I / 4;  // threads per row, a multiple of 32 (I % 128 == 0)
+    const int64_t chunks = (quads + 255) / 256;
+    const int64_t per = (quads + chunks - 1) / chunks;
     swiglu_quant_kernel<<<dim3(static_cast<unsigned>(M), static_cast<unsigned>(chunks)),
                           dim3(static_cast<unsigned>((per + 31) / 32 * 32)), 0, s>>>(
         part1, ks1, M, I, gs_h, base + L.hq, base + L.hsf);
