@@ -1110,20 +1110,31 @@ def run_shared(args):
     if world > 1:
         dist.barrier()
 
-    # the L1 stage alone (the dominant kernel: GEMM + SwiGLU + FP4 re-quantization, one dense
-    # segment given as offsets [0, rows]) on the codes the fused quantizer wrote
+    # the L1 stage alone (the dominant kernel), on the codes the fused quantizer wrote, in the
+    # form the step runs: with few rows the L1 GEMM is split along K (FP32 partials, then an
+    # ordered sum; timed here with the bf16 reduction in place of the SwiGLU kernel), otherwise
+    # the fused GEMM + SwiGLU + FP4 epilogue over one dense segment (offsets [0, rows])
     Mp = (cfg.M + 127) // 128 * 128
     codes, sf, gs = nv.rmsnorm_quantize(x, gamma, cfg.eps, out_rows=Mp)
-    offs = torch.tensor([0, Mp], dtype=torch.int32, device=dev)
-    hq = torch.empty(Mp, cfg.I // 2, dtype=torch.uint8, device=dev)
-    hsf = torch.empty(nv.sf_bytes(Mp, cfg.I), dtype=torch.uint8, device=dev)
-    s_ = lambda: torch.cuda.current_stream().cuda_stream  # noqa: E731
+    l1_split = nv.lib().nvfp4_gemm_dense_workspace_size(cfg.M, 2 * cfg.I, cfg.H) > 0
+    if l1_split:
+        g_ws = torch.empty(int(nv.lib().nvfp4_gemm_dense_workspace_size(cfg.M, 2 * cfg.I, cfg.H)),
+                           dtype=torch.uint8, device=dev)
+        c1 = torch.empty(cfg.M, 2 * cfg.I, dtype=torch.bfloat16, device=dev)
 
-    def l1_stage():
-        call("moe_grouped_gemm_l1_swiglu_q", codes.data_ptr(), sf.data_ptr(), gs.data_ptr(),
-             w1.codes.data_ptr(), w1.sf.data_ptr(), w1.gs.data_ptr(), offs.data_ptr(), None, 1,
-             cfg.H, cfg.I, Mp, gs_h.data_ptr(), hq.data_ptr(), hsf.data_ptr(), status.data_ptr(),
-             s_())
+        def l1_stage():
+            nv.gemm_dense(codes, sf, gs, cfg.M, w1, out=c1, ws=g_ws)
+    else:
+        offs = torch.tensor([0, Mp], dtype=torch.int32, device=dev)
+        hq = torch.empty(Mp, cfg.I // 2, dtype=torch.uint8, device=dev)
+        hsf = torch.empty(nv.sf_bytes(Mp, cfg.I), dtype=torch.uint8, device=dev)
+        s_ = lambda: torch.cuda.current_stream().cuda_stream  # noqa: E731
+
+        def l1_stage():
+            call("moe_grouped_gemm_l1_swiglu_q", codes.data_ptr(), sf.data_ptr(), gs.data_ptr(),
+                 w1.codes.data_ptr(), w1.sf.data_ptr(), w1.gs.data_ptr(), offs.data_ptr(), None,
+                 1, cfg.H, cfg.I, Mp, gs_h.data_ptr(), hq.data_ptr(), hsf.data_ptr(),
+                 status.data_ptr(), s_())
 
     kg = max(1, min(K, 50))
     l1_ms = _timed_steps(graph_of(l1_stage).replay, flush, kg) / kg
@@ -1164,7 +1175,8 @@ def run_shared(args):
     tensor_bound = acc["l1_flops"] / acc["l1_bytes"] > fp4_peak * 1e12 / (peaks["hbm"] * 1e9)
     l1_tf = acc["l1_flops"] / (l1_ms * 1e-3) / 1e12
     l1_gb = acc["l1_bytes"] / (l1_ms * 1e-3) / 1e9
-    kname = "grouped_gemm_kernel<L1_SWIGLU>"
+    kname = ("grouped_gemm_kernel<PLAIN_F32> (L1, split along K) + reduction" if l1_split
+             else "grouped_gemm_kernel<L1_SWIGLU>")
     if tensor_bound:
         value, unit = tflops, "TFLOP/s"
         roof = {"bound": "tensor", "kernel": kname, "achieved": round(l1_tf, 1),
@@ -1193,7 +1205,8 @@ def run_shared(args):
                                f"H={cfg.H}, I={cfg.I}, bf16 out",
                    "parallelism": f"replicas x{world}",
                    "l2": "flushed before every step (256 MB write, outside the timed events)",
-                   "cuda_graph": True, "down_projection_k_splits": bool(split)},
+                   "cuda_graph": True, "l1_k_splits": bool(l1_split),
+                   "down_projection_k_splits": bool(split)},
         "tflops": round(tflops, 3), "gbs": round(gbs, 2),
         "algorithmic": {"bytes_per_step": int(acc["bytes"]), "flops_per_step": int(acc["flops"]),
                         "l1_bytes_per_launch": int(acc["l1_bytes"])},
@@ -1202,7 +1215,7 @@ def run_shared(args):
         "e2e": {"value": round(e2e_rate, 2), "unit": unit,
                 "h2d_bytes_per_step": x_h.numel() * 2, "d2h_bytes_per_step": out_h.numel() * 2,
                 "ms_per_step": round(e2e_ms, 5)},
-        "gpu_launches": (5 if split else 4) * K,
+        "gpu_launches": (4 + (1 if split else 0) + (1 if l1_split else 0)) * K,
         "clocks": clocks,
         "cpu_baseline": cpu,
     }
