@@ -9,10 +9,12 @@ import numpy as np
 import pytest
 
 from oracle import dense as D
+from oracle import formats as F
 from oracle import moe as M
 from oracle import quant as Q
 from oracle import routing as R
 from tests import test_oracle_dense as PD
+from tests import test_oracle_formats as PF
 from tests import test_oracle_quant as PQ
 from tests import test_oracle_routing_moe as PR
 
@@ -68,6 +70,55 @@ def _silu_is_sigmoid(g):
         return 1.0 / (1.0 + np.exp(-np.asarray(g, dtype=np.float64)))
 
 
+def _e2m1_ties_away_from_zero(y):
+    """E2M1 encoder rounding halfway cases away from zero instead of to the even code."""
+    y = np.asarray(y, dtype=np.float64)
+    vals = F.e2m1_decode(np.arange(8, dtype=np.uint8))
+    a = np.minimum(np.abs(y), 6.0)
+    idx = np.searchsorted(vals, a, side="left")
+    idx = np.clip(idx, 0, 7)
+    lo = np.clip(idx - 1, 0, 7)
+    pick = np.where(np.abs(vals[lo] - a) < np.abs(vals[idx] - a), lo, idx)
+    sign = np.where(np.signbit(y), 8, 0)
+    return (pick | sign).astype(np.uint8)
+
+
+def _e4m3_no_saturation(v):
+    """E4M3 encoder that returns the NaN code past 448 instead of saturating."""
+    out = F.__dict__["_orig_e4m3_encode"](v)
+    big = np.abs(np.asarray(v, dtype=np.float64)) > 448
+    return np.where(big, np.uint8(0x7F), out).astype(np.uint8)
+
+
+def _sf_offset_rows_not_interleaved(r, c, n_sf_cols):
+    """Tile map with rows 0..127 of an atom laid out in order (r % 128) * 4 + c % 4."""
+    r = np.asarray(r, dtype=np.int64)
+    c = np.asarray(c, dtype=np.int64)
+    atom = (r // 128) * (n_sf_cols // 4) + (c // 4)
+    return atom * 512 + (r % 128) * 4 + (c % 4)
+
+
+def _grouped_gemm_wrong_expert(a, b_dequant, offs, rows_valid=None):
+    """Grouped GEMM that multiplies every segment by the first expert's weights."""
+    return M.__dict__["_orig_grouped_gemm"](a, lambda e: b_dequant(0), offs, rows_valid)
+
+
+def _pins_formats():
+    return [PF.test_e2m1_encode_bruteforce,
+            lambda: PF.test_e2m1_encode_ties_and_saturation(2.5, 4),
+            PF.test_e4m3_encode_bruteforce_and_saturation,
+            PF.test_e4m3_encode_matches_torch_cast]
+
+
+def _pins_tile_map():
+    return [PQ.test_sf_tile_offsets_hand_worked, PQ.test_sf_tile_is_bijection_and_inverse]
+
+
+def _pins_gemm():
+    return [PR.test_grouped_gemm_vs_triple_loop, PR.test_grouped_gemm_closed_form_all_ones,
+            PR.test_grouped_gemm_one_hot_selects_weight_column]
+
+
 def _pins_dense_rmsnorm():
     return [lambda: PD.test_rmsnorm_matches_the_library_routine_in_float64(1e-6),
             PD.test_rmsnorm_closed_forms,
@@ -115,6 +166,14 @@ MUTANTS = [
     ("permutation: tokens in descending order inside an expert", R, "permute",
      _permute_descending_tokens, _pins_routing),
     ("SwiGLU: sigmoid(g) in place of silu(g)", M, "silu", _silu_is_sigmoid, _pins_ffn),
+    ("E2M1: halfway cases away from zero", F, "e2m1_encode", _e2m1_ties_away_from_zero,
+     _pins_formats),
+    ("E4M3: NaN instead of saturation past 448", F, "e4m3_encode", _e4m3_no_saturation,
+     _pins_formats),
+    ("scale tiles: rows of an atom not interleaved by 32", Q, "sf_tile_offset",
+     _sf_offset_rows_not_interleaved, _pins_tile_map),
+    ("grouped GEMM: every segment against expert 0", M, "grouped_gemm",
+     _grouped_gemm_wrong_expert, _pins_gemm),
 ]
 
 
@@ -134,6 +193,7 @@ def test_a_planted_mistake_fails_a_pin(case, monkeypatch):
 
 
 def test_the_pins_pass_without_a_mistake():
-    for pins in (_pins_dense_rmsnorm, _pins_dense_linear, _pins_quant, _pins_routing, _pins_ffn):
+    for pins in (_pins_dense_rmsnorm, _pins_dense_linear, _pins_quant, _pins_routing, _pins_ffn,
+                 _pins_formats, _pins_tile_map, _pins_gemm):
         for pin in pins():
             pin()
