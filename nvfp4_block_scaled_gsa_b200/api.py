@@ -164,8 +164,9 @@ def w1_row_map(I):
 
 
 def quantize_w1(get_expert, E, I, H, device="cuda"):
-    """Pre-pack W1 (E experts of [2I][H]: gate rows then up rows) into the kernels' 64-row
-    gate/up interleaved layout."""
+    """Pre-pack W1 (E experts of [2I][H]: gate rows then up rows) into the kernels' gate/up
+    interleave of 16-row blocks (stored row 32j + i = gate row 16j + i, 32j + 16 + i = up row
+    16j + i; moe_w1_row_map)."""
     row_map = w1_row_map(I).to(device)
     return quantize_weights(get_expert, E, 2 * I, H, device=device, row_map=row_map)
 

@@ -67,7 +67,7 @@ def compare_requant(c_gpu, s_gpu, c_ref, s_ref, gs):
 
 def upload_weights(qw, w1=False):
     """Oracle QuantWeights -> device NVFP4Weights.  With w1=True the rows are stored in the
-    kernels' 64-row gate/up interleaved layout (moe_w1_row_map)."""
+    kernels' gate/up interleave of 16-row blocks (moe_w1_row_map)."""
     import nvfp4_block_scaled_gsa_b200 as nv
     E, N, K2 = qw.codes.shape
     K = 2 * K2
