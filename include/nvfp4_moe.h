@@ -285,6 +285,9 @@ NVFP4_API nvfp4_status_t moe_grouped_gemm_l1_swiglu_q(const uint8_t* a, const ui
 /* ---------------------------------------------------------------------------------------------
  * moe_w1_row_map — host helper: the stored row of each logical W1 row (gate rows [0, I), up rows
  * [I, 2I)) in the 16-row interleaved layout above.  map: host int32 [2I].  I % 16 == 0.
+ * The pages deinterleave gate and up after the GEMM ("May 24, 2026 — Session Start Plan",
+ * section 5 "NVFP4-1.1"); interleaving the weight rows instead puts each gate row next to its
+ * up partner inside one accumulator tile, so the SwiGLU runs in the L1 epilogue.
  * Pure host computation, no CUDA call.  Pass the map (copied to the device) as dst_row with k = 1
  * to nvfp4_quantize when pre-packing an expert's W1.
  * ------------------------------------------------------------------------------------------- */
@@ -342,7 +345,8 @@ NVFP4_API nvfp4_status_t moe_grouped_gemm_l2_scatter_noalloc(
     void* out_bf16, int32_t* dev_status, nvfp4_stream_t stream);
 
 /* ---------------------------------------------------------------------------------------------
- * moe_ffn_forward — the whole expert FFN in one stream-ordered call:
+ * moe_ffn_forward — the whole expert FFN in one stream-ordered call, the pipeline of "NVFP4
+ * MegaMoE Kernel Rewrite — CuTeDSL", section "Phase 3: Full MoE pipeline":
  *   moe_permute -> nvfp4_quantize (amax -> gs on the GPU, permuted write) ->
  *   moe_grouped_gemm_l1_swiglu_q -> moe_grouped_gemm_l2_scatter (per-slot rows + combine) ->
  *   bf16 out.
