@@ -13,9 +13,10 @@ quant     NVFP4 quantizer (global scale from amax, FP8-round-tripped block scale
 routing   softmax top-k routing and the expert-bucketed row permutation
 moe       grouped GEMM, SwiGLU, re-quantization, weighted scatter, whole FFN
 dense     dense NVFP4 linear, and the RMSNorm fused in front of the quantizer
+mx        MXFP4 (32-element blocks, UE8M0 scales), the format the pages contrast with NVFP4
 
 Every function says which page passage it follows.  Functions with no independent pin say
 "parity unpinned" in their docstring.
 """
 
-from . import formats, quant, routing, moe, dense  # noqa: F401
+from . import formats, quant, routing, moe, dense, mx  # noqa: F401

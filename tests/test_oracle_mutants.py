@@ -11,10 +11,12 @@ import pytest
 from oracle import dense as D
 from oracle import formats as F
 from oracle import moe as M
+from oracle import mx as MX
 from oracle import quant as Q
 from oracle import routing as R
 from tests import test_oracle_dense as PD
 from tests import test_oracle_formats as PF
+from tests import test_oracle_mx as PMX
 from tests import test_oracle_quant as PQ
 from tests import test_oracle_routing_moe as PR
 
@@ -103,6 +105,24 @@ def _grouped_gemm_wrong_expert(a, b_dequant, offs, rows_valid=None):
     return M.__dict__["_orig_grouped_gemm"](a, lambda e: b_dequant(0), offs, rows_valid)
 
 
+def _mx_exponent_rounded_up(amax):
+    """ceil(log2(amax)) - 2 in place of floor: the block's largest element lands in (2, 4]."""
+    a = np.asarray(amax, dtype=np.float64)
+    with np.errstate(divide="ignore"):
+        e = np.ceil(np.log2(np.where(a > 0, a, 1.0))).astype(np.int64) - 2
+    return np.clip(np.where(a > 0, e, -127), -127, 127)
+
+
+def _mx_exponent_emax3(amax):
+    """floor(log2(amax)) - 3: the exponent of E2M1's largest value taken as 3."""
+    return np.clip(MX.__dict__["_orig_block_exponent"](amax) - 1, -127, 127)
+
+
+def _pins_mx():
+    return [PMX.test_block_exponent_closed_forms, PMX.test_block_exponent_defining_inequality,
+            lambda: PMX.test_round_trip_on_grid_blocks(5), PMX.test_saturation_clips_to_six_times_the_scale]
+
+
 def _pins_formats():
     return [PF.test_e2m1_encode_bruteforce,
             lambda: PF.test_e2m1_encode_ties_and_saturation(2.5, 4),
@@ -174,6 +194,9 @@ MUTANTS = [
      _sf_offset_rows_not_interleaved, _pins_tile_map),
     ("grouped GEMM: every segment against expert 0", M, "grouped_gemm",
      _grouped_gemm_wrong_expert, _pins_gemm),
+    ("MXFP4: the scale exponent rounded up", MX, "block_exponent", _mx_exponent_rounded_up,
+     _pins_mx),
+    ("MXFP4: 3 as E2M1's largest exponent", MX, "block_exponent", _mx_exponent_emax3, _pins_mx),
 ]
 
 
@@ -194,6 +217,6 @@ def test_a_planted_mistake_fails_a_pin(case, monkeypatch):
 
 def test_the_pins_pass_without_a_mistake():
     for pins in (_pins_dense_rmsnorm, _pins_dense_linear, _pins_quant, _pins_routing, _pins_ffn,
-                 _pins_formats, _pins_tile_map, _pins_gemm):
+                 _pins_formats, _pins_tile_map, _pins_gemm, _pins_mx):
         for pin in pins():
             pin()
