@@ -7,6 +7,7 @@ import socket
 import subprocess
 import sys
 
+import pytest
 import torch.multiprocessing as mp
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -49,10 +50,11 @@ def test_single_process_is_unchanged():
     assert bench.whole_job_rate(10.0, 2, 1, 4.0) == 10.0 * 2 / 4e-3
 
 
-def test_reference_arm_on_a_non_zero_rank_prints_nothing():
+@pytest.mark.parametrize("config", ["decode", "sweep", "dense_decode", "shared_prefill"])
+def test_reference_arm_on_a_non_zero_rank_prints_nothing(config):
     env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
     p = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
-                        "--steps", "1", "--warmup", "0"], env=env, capture_output=True, text=True,
-                       timeout=300)
-    assert p.returncode == 0
+                        "--config", config, "--steps", "1", "--warmup", "0"], env=env,
+                       capture_output=True, text=True, timeout=300)
+    assert p.returncode == 0, p.stderr
     assert p.stdout.strip() == ""
