@@ -105,6 +105,39 @@ def _grouped_gemm_wrong_expert(a, b_dequant, offs, rows_valid=None):
     return M.__dict__["_orig_grouped_gemm"](a, lambda e: b_dequant(0), offs, rows_valid)
 
 
+def _ffn_weight_omitted(x, logits, k, w1, w2, gs_h, renormalize=True, ids=None, weights=None,
+                        **kw):
+    """The expert FFN with the routing weight left out of the scatter (every slot at weight 1)."""
+    if ids is None:
+        ids, weights = R.route_topk(logits, k, renormalize)
+    return M.__dict__["_orig_moe_ffn"](x, None, k, w1, w2, gs_h, ids=ids,
+                                       weights=np.ones_like(np.asarray(weights, np.float64)), **kw)
+
+
+class _GateUpSwapped:
+    """W1 whose gate rows [0, I) and up rows [I, 2I) trade places: silu(up) * gate."""
+
+    def __init__(self, w):
+        self.w, self.E, self.N = w, w.E, w.N
+
+    def dequant(self, e):
+        d = self.w.dequant(e)
+        half = d.shape[0] // 2
+        return np.concatenate([d[half:], d[:half]])
+
+
+def _ffn_gate_up_swapped(x, logits, k, w1, w2, gs_h, **kw):
+    return M.__dict__["_orig_moe_ffn"](x, logits, k, _GateUpSwapped(w1), w2, gs_h, **kw)
+
+
+def _ffn_requant_with_gs_x(x, logits, k, w1, w2, gs_h, **kw):
+    """The intermediate re-quantized with the activations' global scale in place of gs_h."""
+    gs_x = kw.get("gs_x")
+    if gs_x is None:
+        gs_x = Q.global_scale(np.asarray(x, np.float32))
+    return M.__dict__["_orig_moe_ffn"](x, logits, k, w1, w2, np.float32(gs_x), **kw)
+
+
 def _mx_exponent_rounded_up(amax):
     """ceil(log2(amax)) - 2 in place of floor: the block's largest element lands in (2, 4]."""
     a = np.asarray(amax, dtype=np.float64)
@@ -166,7 +199,10 @@ def _pins_routing():
 
 def _pins_ffn():
     tiny = PR._tiny_inputs()
-    return [PR.test_silu_closed_forms, lambda: PR.test_top1_weight1_is_plain_expert_ffn(tiny)]
+    return [PR.test_silu_closed_forms, lambda: PR.test_top1_weight1_is_plain_expert_ffn(tiny),
+            PR.test_worked_example_by_hand,
+            lambda: PR.test_both_slots_on_one_expert_equal_its_single_slot_ffn(tiny),
+            lambda: PR.test_output_is_linear_in_the_routing_weights(tiny)]
 
 
 MUTANTS = [
@@ -186,6 +222,11 @@ MUTANTS = [
     ("permutation: tokens in descending order inside an expert", R, "permute",
      _permute_descending_tokens, _pins_routing),
     ("SwiGLU: sigmoid(g) in place of silu(g)", M, "silu", _silu_is_sigmoid, _pins_ffn),
+    ("FFN: routing weight left out of the scatter", M, "moe_ffn", _ffn_weight_omitted,
+     _pins_ffn),
+    ("FFN: gate and up projections swapped", M, "moe_ffn", _ffn_gate_up_swapped, _pins_ffn),
+    ("FFN: intermediate re-quantized with gs_x for gs_h", M, "moe_ffn", _ffn_requant_with_gs_x,
+     _pins_ffn),
     ("E2M1: halfway cases away from zero", F, "e2m1_encode", _e2m1_ties_away_from_zero,
      _pins_formats),
     ("E4M3: NaN instead of saturation past 448", F, "e4m3_encode", _e4m3_no_saturation,

@@ -194,3 +194,112 @@ def test_bf16_round_matches_torch():
     v = np.concatenate([v, [0.0, -0.0, 1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8]])
     t = torch.from_numpy(v.astype(np.float32)).to(torch.bfloat16).double().numpy()
     assert np.array_equal(M.bf16_round(v), t)
+
+
+# ------------------------------------------------- routing weight and the FFN composition
+#
+# The pages scatter each expert's output back to its token with the routing weight
+# ("NVFP4 MegaMoE Kernel Rewrite — CuTeDSL", section "Our Adaptation": scatter with routing
+# weights; section "Phase 3: Full MoE pipeline") after L1 -> SwiGLU -> FP4 -> L2.  These pins
+# fix that composition without restating moe_ffn's formula: a worked example whose every
+# intermediate is derived by hand below from the format definitions, and two relations the
+# weighted sum must obey whatever the experts compute.
+
+E2M1_CODE = {0.0: 0, 0.5: 1, 1.0: 2, 1.5: 3, 2.0: 4, 3.0: 5, 4.0: 6, 6.0: 7}
+
+
+def _codes_of(values):
+    """E2M1 codes (sign in bit 3) of values already on the E2M1 grid."""
+    return np.array([E2M1_CODE[abs(v)] | (8 if v < 0 else 0) for v in values], dtype=np.uint8)
+
+
+def _unit_scale_weights(mats):
+    """QuantWeights from float matrices on the E2M1 grid: block scales 1.0 (E4M3 0x38) and
+    global scales 1, so each dequantized element is exactly the given value."""
+    mats = np.asarray(mats, dtype=np.float64)
+    E, N, K = mats.shape
+    codes = np.stack([_codes_of(m.ravel()).reshape(N, K) for m in mats])
+    return M.QuantWeights(F.pack_nibbles(codes), np.full((E, N, K // 16), 0x38, np.uint8),
+                          np.ones(E, np.float32))
+
+
+# W2 column 0 of the two experts (every other W2 entry is 0)
+C0 = [1.0, -2.0, 0.5, 3.0, 0.0, -6.0, 4.0, 1.5, -1.0, 2.0, -0.5, -3.0, 6.0, 0.0, -4.0, 1.0]
+C1 = [-1.0, 0.5, 2.0, -3.0, 6.0, 1.0, -0.5, 0.0, 4.0, -2.0, 1.5, 3.0, -6.0, 1.0, 0.5, -4.0]
+
+
+def _worked_example():
+    """One token, H = I = 16, two experts, both chosen with weights (0.25, 0.75).
+
+    x = (6, 0, ..., 0): gs_x = 2688 / 6 = 448; the block scale (6/6)*448 = 448 is E4M3's largest
+    value, d = 448, so x*gs_x/d = x and the codes hold x exactly: x dequantizes to itself.
+    W1 of expert e has gate row 0 = (a_e, 0, ...), up row 0 = (b_e, 0, ...), all else 0, so
+    gate_0 = 6*a_e, up_0 = 6*b_e and every other h feature is silu(0)*up = 0.
+      expert 0: a = 1,   b = 0.5 -> g = 6, u = 3  -> h_0 = 18 / (1 + e^-6) = 17.9555
+      expert 1: a = 0.5, b = 2   -> g = 3, u = 12 -> h_0 = 36 / (1 + e^-3) = 34.2927
+    Re-quantized with gs_h = 1 (a single nonzero element in the block):
+      expert 0: s = 17.9555/6 = 2.9926 -> nearest E4M3 is 3.0 (byte 0x44); h_0/3 = 5.985 rounds
+                to E2M1 6, so h_0 dequantizes to 6 * 3 = 18
+      expert 1: s = 34.2927/6 = 5.7154 -> below the 5.75 midpoint of 5.5 and 6.0, so 5.5 (0x4B);
+                h_0/5.5 = 6.235 saturates to 6, so h_0 dequantizes to 6 * 5.5 = 33
+    W2 of expert e has column 0 = C_e, all else 0, so Y_e = hq_0 * C_e, and
+      out = 0.25 * 18 * C0 + 0.75 * 33 * C1 = 4.5 * C0 + 24.75 * C1   (exact in float64)."""
+    H = I = 16
+    x = np.zeros((1, H), np.float32)
+    x[0, 0] = 6.0
+    w1 = np.zeros((2, 2 * I, H))
+    w1[0, 0, 0], w1[0, I, 0] = 1.0, 0.5
+    w1[1, 0, 0], w1[1, I, 0] = 0.5, 2.0
+    w2 = np.zeros((2, H, I))
+    w2[0, :, 0], w2[1, :, 0] = C0, C1
+    ids = np.array([[0, 1]], np.int32)
+    weights = np.array([[0.25, 0.75]])
+    return x, _unit_scale_weights(w1), _unit_scale_weights(w2), ids, weights
+
+
+def test_worked_example_by_hand():
+    x, w1, w2, ids, weights = _worked_example()
+    res = M.moe_ffn(x, None, 2, w1, w2, np.float32(1.0), ids=ids, weights=weights, keep=True)
+    assert res["gs_x"] == np.float32(448.0)
+    expected = 4.5 * np.array(C0) + 24.75 * np.array(C1)
+    assert np.array_equal(res["out"][0], expected)
+    # the intermediates derived above: expert 0's row is 0, expert 1's row is 128
+    assert res["h_sf"][0, 0] == 0x44 and res["h_sf"][128, 0] == 0x4B
+    assert res["h_codes"][0, 0] == 7 and res["h_codes"][128, 0] == 7
+    assert np.all(res["h_codes"][[0, 128], 1:] == 0)
+
+
+def test_both_slots_on_one_expert_equal_its_single_slot_ffn(tiny):
+    """Weights 0.25 and 0.75 on the same expert add up to that expert's output once (weight 1),
+    not twice, whatever the expert computes."""
+    x, lg, w1, w2 = tiny
+    T = x.shape[0]
+    e = np.argmax(lg, axis=1).astype(np.int32)
+    two = M.moe_ffn(x, None, 2, w1, w2, np.float32(64.0), ids=np.stack([e, e], 1),
+                    weights=np.tile([0.25, 0.75], (T, 1)))["out"]
+    one = M.moe_ffn(x, None, 1, w1, w2, np.float32(64.0), ids=e[:, None],
+                    weights=np.ones((T, 1)))["out"]
+    assert np.abs(one).max() > 0
+    assert np.allclose(two, one, rtol=1e-14, atol=1e-15 * np.abs(one).max())
+
+
+def test_output_is_linear_in_the_routing_weights(tiny):
+    """Scaling every routing weight by 2 scales the output by exactly 2 (a power of two is exact
+    in float64); by 3, to within float64 rounding.  The experts' outputs do not depend on the
+    weights, so only a weight applied once, linearly, passes."""
+    x, lg, w1, w2 = tiny
+    ids, w = R.route_topk(lg, 2)
+    base = M.moe_ffn(x, None, 2, w1, w2, np.float32(64.0), ids=ids, weights=w)["out"]
+    twice = M.moe_ffn(x, None, 2, w1, w2, np.float32(64.0), ids=ids, weights=2 * w)["out"]
+    thrice = M.moe_ffn(x, None, 2, w1, w2, np.float32(64.0), ids=ids, weights=3 * w)["out"]
+    assert np.abs(base).max() > 0
+    assert np.array_equal(twice, 2 * base)
+    assert np.allclose(thrice, 3 * base, rtol=1e-14, atol=1e-15 * np.abs(base).max())
+    # and a weight of 0 on one slot leaves exactly the other slot's weighted output
+    w0 = w.copy()
+    w0[:, 1] = 0.0
+    only0 = M.moe_ffn(x, None, 2, w1, w2, np.float32(64.0), ids=ids, weights=w0)["out"]
+    ids_1 = ids[:, :1]
+    alone = M.moe_ffn(x, None, 1, w1, w2, np.float32(64.0), ids=ids_1, weights=w[:, :1])["out"]
+    # (the two calls bucket different row counts per expert, so BLAS may sum in another order)
+    assert np.allclose(only0, alone, rtol=1e-14, atol=1e-15 * np.abs(alone).max())
