@@ -332,7 +332,10 @@ NVFP4_API nvfp4_status_t moe_grouped_gemm_l2_scatter(const uint8_t* h, const uin
  *   the process exits.  T*k*H beyond that returns NVFP4_ERR_WORKSPACE_TOO_SMALL (nothing launched;
  *   nvfp4_last_error() says why).
  *   The array's device address is looked up once per device (cudaGetSymbolAddress) by the first
- *   call made with that device current; make that first call before any stream capture.
+ *   call made with that device current; make that first call before any stream capture.  The
+ *   library keeps that address for the life of the process: after cudaDeviceReset (or anything
+ *   else that destroys the device's primary context) it is stale, so do not call this entry point
+ *   on that device again in the same process.
  *   No cudaMalloc / cudaFree or allocating library routine is called.  All calls share the one
  *   array and every call rewrites the rows it reads back; calls that overlap on the GPU (other
  *   streams, other threads) race on it.

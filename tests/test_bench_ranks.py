@@ -50,7 +50,7 @@ def test_single_process_is_unchanged():
     assert bench.whole_job_rate(10.0, 2, 1, 4.0) == 10.0 * 2 / 4e-3
 
 
-@pytest.mark.parametrize("config", ["decode", "sweep", "dense_decode", "shared_prefill"])
+@pytest.mark.parametrize("config", ["prefill", "decode", "sweep", "dense_decode", "shared_prefill"])
 def test_reference_arm_on_a_non_zero_rank_prints_nothing(config):
     env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
     p = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
