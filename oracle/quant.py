@@ -52,6 +52,48 @@ def global_scale(x):
     return np.float32(gs)
 
 
+def scale_from_amax(amax):
+    """FP32 global scale from a GIVEN amax: 2688 / amax, 1.0 when that is not a finite positive
+    float32.  The rule of :func:`global_scale`, with the amax supplied rather than taken from the
+    tensor being quantized.
+
+    Reading for the intermediate h (the pages derive every activation's global scale from its
+    amax on the GPU — commit log of dsv4/kernels/cuda, the "Two-kernel approach" fix — but fuse
+    h's re-quantization into the L1 epilogue, "May 24, 2026 — Session Start Plan", section 5
+    "NVFP4-1.1", where the amax of all of h is not known when a tile is written): delayed
+    scaling.  Call i quantizes h with scale_from_amax(amax of h in call i-1); a first call uses
+    a given scale.
+    """
+    a = np.float32(amax)
+    with np.errstate(divide="ignore", invalid="ignore", over="ignore"):
+        gs = np.float32(GS_NUMERATOR / a)
+    if not (np.isfinite(gs) and gs > 0):
+        gs = np.float32(1.0)
+    return np.float32(gs)
+
+
+def block_scale_clipping(x, gs):
+    """How many 16-element block scales of ``x`` (rows, cols) the E4M3 format could not hold at
+    global scale ``gs``: (saturated, underflowed).
+
+    saturated   s = (a_b / 6) * gs exceeds 448, E4M3's largest value, and was clipped to it
+                (the block's largest elements then saturate at E2M1's 6)
+    underflowed a_b > 0 but s rounds to the E4M3 zero (s <= 2^-10), so every code of the
+                block is 0
+    s is the float32 value the quantizer computes (two roundings, as in :func:`quantize`).
+    Parity note: the pages name no such count; it measures how well a static or delayed gs
+    fits the data, the trade-off a fused epilogue makes.
+    """
+    x32 = np.asarray(x, dtype=np.float32)
+    rows, cols = x32.shape
+    blocks = x32.reshape(rows, cols // BLOCK, BLOCK)
+    a_b = np.max(np.abs(blocks), axis=-1)
+    s = ((a_b / np.float32(6.0)).astype(np.float32) * np.float32(gs)).astype(np.float32)
+    saturated = int(np.count_nonzero(s > np.float32(448.0)))
+    underflowed = int(np.count_nonzero((a_b > 0) & (e4m3_encode(s) & 0x7F == 0)))
+    return saturated, underflowed
+
+
 def quantize(x, gs):
     """Quantize a (rows, cols) array to NVFP4 with global scale ``gs`` (float32).
 

@@ -54,6 +54,22 @@ def _global_scale_wrong_numerator(x):
     return gs if np.isfinite(gs) and gs > 0 else np.float32(1.0)
 
 
+def _scale_from_amax_wrong_numerator(amax):
+    with np.errstate(divide="ignore", invalid="ignore", over="ignore"):
+        gs = np.float32(np.float32(448.0) / np.float32(amax))
+    return gs if np.isfinite(gs) and gs > 0 else np.float32(1.0)
+
+
+def _clipping_at_or_above_448(x, gs):
+    """Counts a block scale of exactly 448 as saturated (the boundary on the wrong side)."""
+    x32 = np.asarray(x, dtype=np.float32)
+    rows, cols = x32.shape
+    a_b = np.max(np.abs(x32.reshape(rows, cols // 16, 16)), axis=-1)
+    s = ((a_b / np.float32(6.0)).astype(np.float32) * np.float32(gs)).astype(np.float32)
+    under = int(np.count_nonzero((a_b > 0) & (F.e4m3_encode(s) & 0x7F == 0)))
+    return int(np.count_nonzero(s >= np.float32(448.0))), under
+
+
 def _route_without_renormalization(logits, k, renormalize=True):
     return R.__dict__["_orig_route_topk"](logits, k, renormalize=False)
 
@@ -191,6 +207,13 @@ def _pins_quant():
             PQ.test_round_tripped_scale_differs_from_raw_scale]
 
 
+def _pins_hscale():
+    return [PQ.test_scale_from_amax_closed_forms,
+            PQ.test_delayed_scale_from_the_same_data_is_the_dynamic_scale,
+            PQ.test_block_scale_clipping_hand_cases,
+            PQ.test_block_scale_clipping_agrees_with_the_quantizer]
+
+
 def _pins_routing():
     return [PR.test_topk_matches_bruteforce_subsets_on_tiny,
             PR.test_topk_ties_go_to_lower_id_and_no_renorm,
@@ -217,6 +240,10 @@ MUTANTS = [
      _global_scale_wrong_numerator, _pins_quant),
     ("quantizer: codes against the raw block scale", Q, "quantize", Q.quantize_raw_scale,
      _pins_quant),
+    ("delayed scale: 448 / amax", Q, "scale_from_amax", _scale_from_amax_wrong_numerator,
+     _pins_hscale),
+    ("clipping count: a scale of exactly 448 counted as saturated", Q, "block_scale_clipping",
+     _clipping_at_or_above_448, _pins_hscale),
     ("routing: weights not renormalized over the k", R, "route_topk",
      _route_without_renormalization, _pins_routing),
     ("permutation: tokens in descending order inside an expert", R, "permute",
@@ -258,6 +285,7 @@ def test_a_planted_mistake_fails_a_pin(case, monkeypatch):
 
 def test_the_pins_pass_without_a_mistake():
     for pins in (_pins_dense_rmsnorm, _pins_dense_linear, _pins_quant, _pins_routing, _pins_ffn,
+                 _pins_hscale,
                  _pins_formats, _pins_tile_map, _pins_gemm, _pins_mx):
         for pin in pins():
             pin()

@@ -137,3 +137,66 @@ def test_pack_roundtrip_quantize_packed():
     c, sf2 = Q.quantize(x, gs)
     assert p.shape == (8, 32) and np.array_equal(sf, sf2)
     assert np.array_equal(Q.dequantize_packed(p, sf, gs), Q.dequantize(c, sf, gs))
+
+
+# --------------------------------------------- delayed scale of the intermediate, clipping counts
+
+def test_scale_from_amax_closed_forms():
+    assert Q.scale_from_amax(2688.0) == 1.0
+    assert Q.scale_from_amax(1.0) == 2688.0
+    assert Q.scale_from_amax(0.5) == 5376.0
+    assert Q.scale_from_amax(3.0) == np.float32(2688.0) / np.float32(3.0)
+    for bad in (0.0, np.inf, np.nan, -1.0):
+        assert Q.scale_from_amax(bad) == 1.0
+
+
+def test_delayed_scale_from_the_same_data_is_the_dynamic_scale():
+    """Quantizing h with the scale derived from its own amax (delayed scaling on an unchanged
+    batch) gives exactly the dynamic quantization."""
+    rng = np.random.default_rng(11)
+    for scale in (1e-4, 0.3, 7.0, 5e3):
+        h = (rng.standard_normal((32, 128)) * scale).astype(np.float32)
+        amax = np.max(np.abs(h))
+        assert Q.scale_from_amax(amax) == Q.global_scale(h)
+        c1, s1 = Q.quantize(h, Q.scale_from_amax(amax))
+        c2, s2 = Q.quantize(h, Q.global_scale(h))
+        assert np.array_equal(c1, c2) and np.array_equal(s1, s2)
+
+
+def test_block_scale_clipping_hand_cases():
+    """gs = 1, one block per row.  The E4M3 largest value is 448 and its smallest subnormal 2^-9;
+    s = a_b / 6, rounded to float32."""
+    rows = np.zeros((6, 16), np.float32)
+    rows[0, 3] = 6 * 448          # s = 448 exactly: held
+    rows[1, 3] = 6 * 449          # s = 449 > 448: saturated
+    rows[2, 5] = 6 * 2.0 ** -10   # s = 2^-10: the tie between 0 and 2^-9 goes to 0: underflowed
+    rows[3, 5] = 6 * 2.0 ** -9    # s = 2^-9, the smallest subnormal: held
+    rows[4, 0] = -6 * 2.0 ** -12  # s = 2^-12: underflowed (the sign does not matter)
+    # row 5: all zero, neither
+    assert Q.block_scale_clipping(rows, np.float32(1.0)) == (1, 2)
+    # the same data at gs = 2^-3 brings row 1 into range and pushes row 3 under (s = 2^-12)
+    assert Q.block_scale_clipping(rows, np.float32(0.125)) == (0, 3)
+
+
+def test_block_scale_clipping_agrees_with_the_quantizer():
+    """An underflowed block is exactly a nonzero block whose codes all come out 0; a saturated
+    block has scale byte 0x7E (448) and its largest element dequantizes to 6 * 448 / gs, below
+    its true magnitude."""
+    rng = np.random.default_rng(12)
+    x = (rng.standard_normal((64, 256)) * np.exp(rng.uniform(-12, 8, (64, 1)))).astype(np.float32)
+    gs = np.float32(64.0)
+    sat, under = Q.block_scale_clipping(x, gs)
+    codes, sf = Q.quantize(x, gs)
+    blocks = x.reshape(64, 16, 16)
+    nz = np.max(np.abs(blocks), axis=-1) > 0
+    zero_codes = np.all((codes.reshape(64, 16, 16) & 7) == 0, axis=-1)
+    assert under == int(np.count_nonzero(nz & zero_codes)) and under > 0
+    s = ((np.max(np.abs(blocks), -1) / np.float32(6)).astype(np.float32) * gs).astype(np.float32)
+    big = s > 448
+    assert sat == int(np.count_nonzero(big)) and sat > 0
+    assert np.all(sf[big] == 0x7E)
+    xh = Q.dequantize(codes, sf, gs).reshape(64, 16, 16)
+    amax_i = np.argmax(np.abs(blocks), axis=-1)
+    top = np.take_along_axis(np.abs(xh), amax_i[..., None], -1)[..., 0]
+    true = np.max(np.abs(blocks), axis=-1)
+    assert np.all(top[big] == 6 * 448 / 64) and np.all(top[big] < true[big])
