@@ -219,9 +219,20 @@ class Plan:
         self.xq, self.xsf = e(self.R * H // 2, u8), e(self.R * H // 16, u8)
         self.gs_x, self.qws = e(1, f32), e(256, u8)
         self.hq, self.hsf = e(self.R * I // 2, u8), e(self.R * I // 16, u8)
-        self.ys = e(T * k * H, f32)
+        # the L2 form moe_ffn_forward uses for this batch: 1 = token-row reductions (an FP32
+        # [T][H] accumulator), 0 = per-slot rows [T*k][H] summed in slot order
+        self.l2_form = nv.l2_form(T, k, E)
+        self.ys = e(T * H if self.l2_form else T * k * H, f32)
         self.out = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
         self.status = torch.zeros(1, dtype=i32, device=dev)
+        self.ffn_ws = e(nv.ffn_workspace_bytes(T, H, I, E, k), torch.uint8)
+        self.ffn_out = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+
+    def forward(self):
+        """One step through the product call, moe_ffn_forward (the kernels step() runs one by
+        one, chained inside the library)."""
+        self.nv.moe_ffn_forward(self.x, self.logits, self.cfg.k, self.w1, self.w2, self.gs_h,
+                                out=self.ffn_out, ws=self.ffn_ws, status=self.status)
 
     def step(self, ev=None):
         from nvfp4_block_scaled_gsa_b200._native import call
@@ -247,16 +258,22 @@ class Plan:
              p(self.gs_h), p(self.hq), p(self.hsf), p(self.status), s)
         if ev:
             ev[3].record()
-        call("moe_grouped_gemm_l2_scatter", p(self.hq), p(self.hsf), p(self.gs_h),
-             p(self.w2.codes), p(self.w2.sf), p(self.w2.gs), p(self.offs), p(self.row_slot),
-             p(self.row_w), p(self.dst), E, H, I, T, k, self.R, p(self.ys), None, p(self.out),
-             p(self.status), s)
+        if self.l2_form:
+            call("moe_grouped_gemm_l2_scatter_add", p(self.hq), p(self.hsf), p(self.gs_h),
+                 p(self.w2.codes), p(self.w2.sf), p(self.w2.gs), p(self.offs), p(self.row_slot),
+                 p(self.row_w), p(self.dst), E, H, I, T, k, self.R, p(self.ys), p(self.out),
+                 p(self.status), s)
+        else:
+            call("moe_grouped_gemm_l2_scatter", p(self.hq), p(self.hsf), p(self.gs_h),
+                 p(self.w2.codes), p(self.w2.sf), p(self.w2.gs), p(self.offs), p(self.row_slot),
+                 p(self.row_w), p(self.dst), E, H, I, T, k, self.R, p(self.ys), None, p(self.out),
+                 p(self.status), s)
         if ev:
             ev[4].record()
 
 
-KERNELS_PER_STEP = 7  # topk, permute, amax, quantize, L1 GEMM, L2 GEMM, combine (+ a count
-#                       kernel before permute from 4096 slots)
+KERNELS_PER_STEP = 7  # topk, permute, amax, quantize, L1 GEMM, L2 GEMM, combine or bf16
+#                       rounding (+ a count kernel before permute from 4096 slots)
 
 
 def make_config(args):
@@ -306,6 +323,7 @@ def run_ours(args):
 
     for _ in range(max(args.warmup, 3)):
         plan.step()
+        plan.forward()
     torch.cuda.synchronize()
     ids = plan.ids[: cfg.T * cfg.k].cpu()  # tokens per expert, for the byte count
     real = torch.bincount(ids[ids >= 0].long(), minlength=cfg.E).tolist()
@@ -316,7 +334,7 @@ def run_ours(args):
     t_end = time.time() + args.soak
     while time.time() < t_end:
         for _ in range(8):
-            plan.step()
+            plan.forward()
         torch.cuda.synchronize()
 
     K = args.steps
@@ -327,7 +345,7 @@ def run_ours(args):
     torch.cuda.nvtx.range_push("timed")
     start.record()
     for i in range(K):
-        plan.step()
+        plan.forward()
     stop.record()
     torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize()
@@ -647,7 +665,7 @@ def run_sweep(args):
     if world > 1:
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
-    cfg = CONFIGS["sweep"]
+    cfg = make_config(args)  # the sweep, or a reduced one with --experts (profiling captures)
     m, offs, a_bf16, w = sweep_operands(cfg, dev)
     R = a_bf16.shape[0]
     codes, sf, gs = nv.quantize(a_bf16)

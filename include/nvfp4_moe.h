@@ -99,6 +99,26 @@ NVFP4_API nvfp4_status_t nvfp4_quantize(const void* x, int64_t rows, int64_t col
                               nvfp4_stream_t stream);
 
 /* ---------------------------------------------------------------------------------------------
+ * mxfp4_quantize — BF16 -> MXFP4: E2M1 elements with one UE8M0 (power-of-two) scale per 32
+ * elements and no global scale: the format the pages contrast with NVFP4 ("May 24, 2026 —
+ * Session Start Plan", section 1 "NVFP4-0": 32-element blocks, UE8M0 scales).  The pages give no
+ * rounding rule; the OCP Microscaling v1.0 one is used:
+ *
+ *   e = floor(log2(max|x_i|)) - 2, clamped to [-127, 127] (-127 for an all-zero block)
+ *   scale byte = e + 127;   code_i = E2M1_rn_satfinite(x_i * 2^-e)   (exact multiply)
+ *   value = E2M1(code) * 2^(byte - 127)
+ *
+ *   x      bf16 [rows][ld] (ld >= cols, ld % 8 == 0)
+ *   codes  uint8 [rows][cols/2] (element 2j in the low nibble of byte j)
+ *   sf     scale bytes in the tiled layout of the NVFP4 scales (atoms of 128 rows x 4 scale
+ *          columns), with cols/32 scale columns per row: ceil(rows/128)*128 * cols/32 bytes
+ *   Constraints: cols % 128 == 0.  dev_status is unused (kept for a uniform signature).
+ * ------------------------------------------------------------------------------------------- */
+NVFP4_API nvfp4_status_t mxfp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t ld,
+                                        uint8_t* codes, uint8_t* sf, int32_t* dev_status,
+                                        nvfp4_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------------
  * nvfp4_rmsnorm_quantize — RMSNorm fused in front of the BF16 -> NVFP4 quantizer.
  *
  * The commit log of dsv4/kernels/cuda (nvfp4-megamoe-kernel) fuses the RMSNorm with the amax and
@@ -173,6 +193,25 @@ NVFP4_API nvfp4_status_t nvfp4_grouped_gemm(const uint8_t* a, const uint8_t* sfa
                                   const int32_t* offs, int E, int N, int K, int64_t R_max,
                                   void* out, int out_dtype, int32_t* dev_status,
                                   nvfp4_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------------
+ * mxfp4_grouped_gemm — the 2D x 3D grouped GEMM on MXFP4 operands (E2M1, one UE8M0 scale per 32
+ * elements, no global scale; mxfp4_quantize's format), C = A_e * B_e^T per expert, FP32
+ * accumulation: the variant of nvfp4_grouped_gemm for the format the pages contrast with NVFP4
+ * ("May 24, 2026 — Session Start Plan", section 1 "NVFP4-0").  Same tiles, scheduler and
+ * roles; the tensor cores read 2 scales per row per 64 of K (tcgen05.mma kind::mxf4,
+ * scale_vec::2X).  C[r][n] = acc (no global scale to divide by).
+ *
+ *   a, sfa    MXFP4 [R_max][K] (codes [R_max][K/2], tiled scales with K/32 columns)
+ *   b, sfb    MXFP4 [E*N][K]
+ *   offs, out, out_dtype, R_max: as nvfp4_grouped_gemm
+ *   Constraints: K % 128 == 0, N % 256 == 0, R_max % 128 == 0, 1 <= E <= 256.
+ * ------------------------------------------------------------------------------------------- */
+NVFP4_API nvfp4_status_t mxfp4_grouped_gemm(const uint8_t* a, const uint8_t* sfa,
+                                            const uint8_t* b, const uint8_t* sfb,
+                                            const int32_t* offs, int E, int N, int K,
+                                            int64_t R_max, void* out, int out_dtype,
+                                            int32_t* dev_status, nvfp4_stream_t stream);
 
 /* ---------------------------------------------------------------------------------------------
  * nvfp4_gemm_dense — dense block-scaled GEMM on NVFP4 activations: out = A W^T, bf16 out.
@@ -283,6 +322,40 @@ NVFP4_API nvfp4_status_t moe_grouped_gemm_l1_swiglu_q(const uint8_t* a, const ui
                                             nvfp4_stream_t stream);
 
 /* ---------------------------------------------------------------------------------------------
+ * moe_grouped_gemm_l1_swiglu_q_stats — moe_grouped_gemm_l1_swiglu_q, plus what its epilogue sees
+ * of the intermediate h before quantizing it.
+ *
+ * The pages take every activation's global scale from its amax on the GPU (commit log of
+ * dsv4/kernels/cuda, nvfp4-megamoe-kernel: the "Two-kernel approach" fix), but fuse h's
+ * re-quantization into the L1 epilogue ("May 24, 2026 — Session Start Plan", section 5
+ * "NVFP4-1.1"), where the amax of all of h is unknown when a tile is written.  This call records
+ * that amax as the tiles are written, so that a later call can quantize with it (delayed
+ * scaling, nvfp4_scale_from_amax), and counts the block scales the static scale could not hold.
+ *
+ *   h32      device float [R_max][I] or NULL: the FP32 h values (g*u/(1+exp(-g))) before
+ *            quantization, for the real rows (row_slot >= 0, or every row when row_slot is NULL);
+ *            other rows are not written.  A diagnostic output: it adds R_max*I*4 bytes of writes.
+ *   h_stats  device uint32 [3] or NULL, ACCUMULATED into (zero it first): [0] = float bits of
+ *            max|h| over the real rows (atomicMax on the bits, valid because |h| >= 0);
+ *            [1] = block scales that saturated (s = (amax_b/6)*gs_h > 448); [2] = block scales
+ *            that underflowed (amax_b > 0 but s rounded to the E4M3 zero: the block is all zeros).
+ *   Everything else as moe_grouped_gemm_l1_swiglu_q.  h32 must be 16-byte aligned, h_stats 4.
+ * ------------------------------------------------------------------------------------------- */
+NVFP4_API nvfp4_status_t moe_grouped_gemm_l1_swiglu_q_stats(
+    const uint8_t* a, const uint8_t* sfa, const float* gs_a, const uint8_t* w1,
+    const uint8_t* sfw1, const float* gs_w1, const int32_t* offs, const int32_t* row_slot, int E,
+    int H, int I, int64_t R_max, const float* gs_h, uint8_t* h, uint8_t* sfh, float* h32,
+    uint32_t* h_stats, int32_t* dev_status, nvfp4_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------------
+ * nvfp4_scale_from_amax — *gs = 2688 / amax (1.0 when that is not finite and positive), amax
+ * given as the float bits in *amax_bits: the global-scale rule of nvfp4_quantize applied to an
+ * amax recorded earlier (h_stats[0] above), on the device, with no host sync.  One thread.
+ * ------------------------------------------------------------------------------------------- */
+NVFP4_API nvfp4_status_t nvfp4_scale_from_amax(const uint32_t* amax_bits, float* gs,
+                                                nvfp4_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------------
  * moe_w1_row_map — host helper: the stored row of each logical W1 row (gate rows [0, I), up rows
  * [I, 2I)) in the 16-row interleaved layout above.  map: host int32 [2I].  I % 16 == 0.
  * The pages deinterleave gate and up after the GEMM ("May 24, 2026 — Session Start Plan",
@@ -320,6 +393,32 @@ NVFP4_API nvfp4_status_t moe_grouped_gemm_l2_scatter(const uint8_t* h, const uin
                                            nvfp4_stream_t stream);
 
 /* ---------------------------------------------------------------------------------------------
+ * moe_grouped_gemm_l2_scatter_add — the L2 grouped GEMM with the routing weight and a true
+ * scatter-ADD in its epilogue ("NVFP4 MegaMoE Kernel Rewrite — CuTeDSL", section "Our
+ * Adaptation": "Scatter with routing weights"; section "Phase 3"): each routed row's weighted
+ * output row_w[r] * (h_r . W2_e^T) / (gs_h*gs_w2[e]) is added into its token's row of an FP32
+ * [T][H] accumulator as the tile is produced (vector reductions performed at L2), the tiles
+ * running N-slice by N-slice so that the accumulator slice being added into stays in L2; then
+ * the accumulator is rounded to bf16.
+ *
+ *   acc        float [T][H]: zeroed by this call (in stream order), holds the FP32 result after
+ *   out_bf16   bf16 [T][H] or NULL
+ *   The k additions into a token's row happen in whatever order the tiles finish, so the last
+ *   bits of the FP32 sum (rarely a bf16 bit) may change from run to run; moe_grouped_gemm_l2_scatter
+ *   is the bitwise-reproducible form.  Tokens whose slots are all dropped get exact zeros.
+ *   Other arguments and constraints as moe_grouped_gemm_l2_scatter.
+ *
+ * moe_ffn_l2_form — which L2 form moe_ffn_forward(_ex) uses for a batch: 0 = per-slot rows summed
+ * in slot order (moe_grouped_gemm_l2_scatter), 1 = token-row reductions (this call).  Host only.
+ * ------------------------------------------------------------------------------------------- */
+NVFP4_API nvfp4_status_t moe_grouped_gemm_l2_scatter_add(
+    const uint8_t* h, const uint8_t* sfh, const float* gs_h, const uint8_t* w2,
+    const uint8_t* sfw2, const float* gs_w2, const int32_t* offs, const int32_t* row_slot,
+    const float* row_w, const int32_t* dst_row, int E, int H, int I, int T, int k, int64_t R_max,
+    float* acc, void* out_bf16, int32_t* dev_status, nvfp4_stream_t stream);
+NVFP4_API int moe_ffn_l2_form(int T, int k, int E, int flags);
+
+/* ---------------------------------------------------------------------------------------------
  * moe_grouped_gemm_l2_scatter_noalloc — moe_grouped_gemm_l2_scatter without a caller-provided
  * FP32 accumulation buffer.  The pages have no counterpart to this call; it exists for callers
  * that cannot allocate device memory for scratch: runtimes that reserve all device memory up front
@@ -351,8 +450,11 @@ NVFP4_API nvfp4_status_t moe_grouped_gemm_l2_scatter_noalloc(
  * moe_ffn_forward — the whole expert FFN in one stream-ordered call, the pipeline of "NVFP4
  * MegaMoE Kernel Rewrite — CuTeDSL", section "Phase 3: Full MoE pipeline":
  *   moe_permute -> nvfp4_quantize (amax -> gs on the GPU, permuted write) ->
- *   moe_grouped_gemm_l1_swiglu_q -> moe_grouped_gemm_l2_scatter (per-slot rows + combine) ->
- *   bf16 out.
+ *   moe_grouped_gemm_l1_swiglu_q -> L2 grouped GEMM + routing weight + scatter-add -> bf16 out.
+ *   The scatter-add: below 32 routed rows per expert on average, per-slot rows summed in slot
+ *   order (moe_grouped_gemm_l2_scatter); from there, FP32 vector reductions into each token's
+ *   row as the L2 tiles are produced, whose order is not fixed (moe_ffn_forward_ex with
+ *   NVFP4_FFN_DETERMINISTIC keeps the slot-ordered sum at every size).
  *
  *   x_bf16   bf16 [T][H];  logits float [T][E] (softmax top-k routing, renormalized)
  *   w1.. / w2..  expert weights as above; gs_h device float[1] (static intermediate scale)
@@ -366,6 +468,37 @@ NVFP4_API nvfp4_status_t moe_ffn_forward(const void* x_bf16, const float* logits
                                const uint8_t* w2, const uint8_t* sfw2, const float* gs_w2,
                                const float* gs_h, void* out_bf16, void* ws, size_t ws_bytes,
                                int32_t* dev_status, nvfp4_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------------
+ * moe_ffn_forward_ex — moe_ffn_forward with options: the intermediate's statistics, an opt-in
+ * delayed global scale for h (see moe_grouped_gemm_l1_swiglu_q_stats for why h's scale is not
+ * dynamic), and the choice of a bitwise-reproducible output sum.
+ *
+ *   gs_h     device float[1], the scale this call quantizes h with
+ *   flags    0, or an OR of:
+ *            NVFP4_FFN_DELAYED_GS_H  after this call's L2 has used it, *gs_h is replaced, in
+ *                stream order, by 2688 / max|h| of this call (1.0 when not finite and positive):
+ *                call i+1 then quantizes h with call i's amax.  The first call uses the scale the
+ *                caller wrote.  Without it *gs_h is only read (a static scale).
+ *            NVFP4_FFN_DETERMINISTIC  every slot's weighted row is stored and a token's k rows
+ *                are added in slot order, so the output is bitwise reproducible.  Without it,
+ *                from 32 routed rows per expert on average, the rows are added into the token's
+ *                FP32 row as the L2 tiles produce them (vector reductions at L2; no per-slot round
+ *                trip through memory): the order of those k additions, and so the last bits of
+ *                the FP32 sum (rarely a bf16 output bit), may change from run to run.
+ *   h_stats  device uint32[3] or NULL: zeroed by the call, then filled as in
+ *            moe_grouped_gemm_l1_swiglu_q_stats (amax bits, saturated, underflowed).
+ *   Everything else as moe_ffn_forward (same workspace size).  moe_ffn_forward is this call
+ *   with flags = 0 and no statistics.
+ * ------------------------------------------------------------------------------------------- */
+#define NVFP4_FFN_DELAYED_GS_H 1
+#define NVFP4_FFN_DETERMINISTIC 2
+NVFP4_API nvfp4_status_t moe_ffn_forward_ex(const void* x_bf16, const float* logits, int T, int H,
+                                  int I, int E, int k, const uint8_t* w1, const uint8_t* sfw1,
+                                  const float* gs_w1, const uint8_t* w2, const uint8_t* sfw2,
+                                  const float* gs_w2, float* gs_h, int flags, uint32_t* h_stats,
+                                  void* out_bf16, void* ws, size_t ws_bytes, int32_t* dev_status,
+                                  nvfp4_stream_t stream);
 
 /* ---------------------------------------------------------------------------------------------
  * Status helpers.

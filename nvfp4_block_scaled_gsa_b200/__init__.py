@@ -11,15 +11,22 @@ from .api import (  # noqa: F401
     gemm_dense,
     grouped_gemm,
     l1_swiglu_q,
+    l1_swiglu_q_stats,
+    l2_form,
     l2_scatter,
+    l2_scatter_add,
     linear,
     linear_workspace_bytes,
     moe_ffn_forward,
+    mxfp4_grouped_gemm,
+    mxfp4_quantize,
+    moe_ffn_forward_ex,
     permute,
     quantize,
     quantize_w1,
     quantize_weights,
     rmsnorm_quantize,
+    scale_from_amax,
     w1_row_map,
     read_status,
     rows_max,

@@ -26,6 +26,7 @@ SIGNATURES = {
     "nvfp4_quantize_workspace_size": (c_size, []),
     "nvfp4_quantize": (c_int, [c_void, c_i64, c_i64, c_i64, c_void, c_int, c_i64, c_void, c_void,
                                c_void, c_int, c_void, c_size, c_void, c_void]),
+    "mxfp4_quantize": (c_int, [c_void, c_i64, c_i64, c_i64, c_void, c_void, c_void, c_void]),
     "nvfp4_rmsnorm_quantize_workspace_size": (c_size, [c_i64]),
     "nvfp4_rmsnorm_quantize": (c_int, [c_void, c_i64, c_i64, c_i64, c_void, c_float, c_void, c_int,
                                        c_i64, c_void, c_void, c_void, c_int, c_void, c_size, c_void,
@@ -36,6 +37,8 @@ SIGNATURES = {
                             c_void, c_void, c_void, c_size, c_void, c_void]),
     "nvfp4_grouped_gemm": (c_int, [c_void, c_void, c_void, c_void, c_void, c_void, c_void, c_int,
                                    c_int, c_int, c_i64, c_void, c_int, c_void, c_void]),
+    "mxfp4_grouped_gemm": (c_int, [c_void, c_void, c_void, c_void, c_void, c_int, c_int, c_int,
+                                   c_i64, c_void, c_int, c_void, c_void]),
     "nvfp4_gemm_dense_workspace_size": (c_size, [c_i64, c_int, c_int]),
     "nvfp4_gemm_dense": (c_int, [c_void, c_void, c_void, c_i64, c_void, c_void, c_void, c_int, c_int,
                                  c_void, c_void, c_size, c_void, c_void]),
@@ -49,9 +52,19 @@ SIGNATURES = {
     "moe_grouped_gemm_l1_swiglu_q": (c_int, [c_void, c_void, c_void, c_void, c_void, c_void,
                                              c_void, c_void, c_int, c_int, c_int, c_i64, c_void,
                                              c_void, c_void, c_void, c_void]),
+    "moe_grouped_gemm_l1_swiglu_q_stats": (c_int, [c_void, c_void, c_void, c_void, c_void, c_void,
+                                                   c_void, c_void, c_int, c_int, c_int, c_i64,
+                                                   c_void, c_void, c_void, c_void, c_void, c_void,
+                                                   c_void]),
+    "nvfp4_scale_from_amax": (c_int, [c_void, c_void, c_void]),
     "moe_grouped_gemm_l2_scatter": (c_int, [c_void, c_void, c_void, c_void, c_void, c_void, c_void,
                                             c_void, c_void, c_void, c_int, c_int, c_int, c_int,
                                             c_int, c_i64, c_void, c_void, c_void, c_void, c_void]),
+    "moe_grouped_gemm_l2_scatter_add": (c_int, [c_void, c_void, c_void, c_void, c_void, c_void,
+                                                c_void, c_void, c_void, c_void, c_int, c_int,
+                                                c_int, c_int, c_int, c_i64, c_void, c_void,
+                                                c_void, c_void]),
+    "moe_ffn_l2_form": (c_int, [c_int, c_int, c_int, c_int]),
     "moe_grouped_gemm_l2_scatter_noalloc": (c_int, [c_void, c_void, c_void, c_void, c_void,
                                                     c_void, c_void, c_void, c_void, c_void, c_int,
                                                     c_int, c_int, c_int, c_int, c_i64, c_void,
@@ -61,6 +74,9 @@ SIGNATURES = {
     "moe_ffn_forward": (c_int, [c_void, c_void, c_int, c_int, c_int, c_int, c_int, c_void, c_void,
                                 c_void, c_void, c_void, c_void, c_void, c_void, c_void, c_size,
                                 c_void, c_void]),
+    "moe_ffn_forward_ex": (c_int, [c_void, c_void, c_int, c_int, c_int, c_int, c_int, c_void,
+                                   c_void, c_void, c_void, c_void, c_void, c_void, c_int, c_void,
+                                   c_void, c_void, c_size, c_void, c_void]),
     "nvfp4_read_status": (c_int, [c_void, c_void, c_void]),
     "nvfp4_wait_selftest": (c_int, [c_i64, c_void, c_void, c_void]),
     "nvfp4_last_error": (c_char_p, []),

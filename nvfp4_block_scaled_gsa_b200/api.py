@@ -60,6 +60,18 @@ def quantize(x, gs=None, dst_row=None, k=1, out_rows=None, status=None):
     return codes, sf, gs
 
 
+def mxfp4_quantize(x, status=None):
+    """MXFP4-quantize bf16 x (rows, cols): returns (codes (rows, cols/2) uint8, tiled UE8M0
+    scales, one per 32 elements).  cols % 128 == 0; no global scale."""
+    assert x.dtype == BF16 and x.dim() == 2 and x.stride(1) == 1
+    rows, cols = x.shape
+    codes = torch.empty(rows, cols // 2, dtype=U8, device=x.device)
+    sf = torch.empty(round_up(rows, 128) * cols // 32, dtype=U8, device=x.device)
+    call("mxfp4_quantize", _p(x), rows, cols, x.stride(0), _p(codes), _p(sf), _p(status),
+         _stream())
+    return codes, sf
+
+
 def rmsnorm_quantize(x, gamma, eps, gs=None, dst_row=None, k=1, out_rows=None, status=None):
     """RMSNorm of bf16 x (rows, cols) with bf16 gamma (cols,), fused into the NVFP4 quantizer.
     Same outputs and options as quantize(); the normalized tensor itself is never written."""
@@ -212,6 +224,20 @@ def grouped_gemm(a_codes, a_sf, gs_a, w: NVFP4Weights, offs, out_dtype=F32, stat
     return out
 
 
+def mxfp4_grouped_gemm(a_codes, a_sf, b_codes, b_sf, E, N, offs, out_dtype=F32, status=None,
+                       out=None):
+    """2D x 3D grouped GEMM on MXFP4 operands (mxfp4_quantize's format, no global scales):
+    out[r] = A[r] . B_e^T for the rows r of expert e; B is [E*N][K]."""
+    R = a_codes.shape[0]
+    K = 2 * a_codes.shape[1]
+    if out is None:
+        out = torch.empty(R, N, dtype=out_dtype, device=a_codes.device)
+    assert out.shape == (R, N) and out.dtype == out_dtype and out.is_contiguous()
+    call("mxfp4_grouped_gemm", _p(a_codes), _p(a_sf), _p(b_codes), _p(b_sf), _p(offs), E, N, K, R,
+         _p(out), 0 if out_dtype == F32 else 1, _p(status), _stream())
+    return out
+
+
 def l1_swiglu_q(a_codes, a_sf, gs_a, w1: NVFP4Weights, offs, gs_h, row_slot=None, status=None):
     """L1 GEMM + SwiGLU + NVFP4 re-quantization -> (h codes (R, I/2), h tiled scales).
     With row_slot, all-padding groups of 32 rows are skipped (left unwritten)."""
@@ -223,6 +249,33 @@ def l1_swiglu_q(a_codes, a_sf, gs_a, w1: NVFP4Weights, offs, gs_h, row_slot=None
          _p(w1.sf), _p(w1.gs), _p(offs), _p(row_slot), w1.E, w1.K, I, R, _p(gs_h), _p(h),
          _p(sfh), _p(status), _stream())
     return h, sfh
+
+
+def l1_swiglu_q_stats(a_codes, a_sf, gs_a, w1: NVFP4Weights, offs, gs_h, row_slot=None,
+                      h_stats=None, want_h32=False, status=None):
+    """l1_swiglu_q, plus the epilogue's view of h: returns (h codes, h tiled scales, h_stats,
+    h32).  h_stats: device uint32 (3,) accumulated into (zeroed here when not given): amax bits
+    of |h| over real rows, saturated block scales, underflowed block scales.  h32 (with
+    want_h32): the FP32 h values before quantization, (R, I), real rows only."""
+    R = a_codes.shape[0]
+    I = w1.N // 2
+    dev = a_codes.device
+    h = torch.empty(R, I // 2, dtype=U8, device=dev)
+    sfh = torch.empty(sf_bytes(R, I), dtype=U8, device=dev)
+    if h_stats is None:
+        h_stats = torch.zeros(3, dtype=I32, device=dev)
+    h32 = torch.zeros(R, I, dtype=F32, device=dev) if want_h32 else None
+    call("moe_grouped_gemm_l1_swiglu_q_stats", _p(a_codes), _p(a_sf), _p(gs_a), _p(w1.codes),
+         _p(w1.sf), _p(w1.gs), _p(offs), _p(row_slot), w1.E, w1.K, I, R, _p(gs_h), _p(h),
+         _p(sfh), _p(h32), _p(h_stats), _p(status), _stream())
+    return h, sfh, h_stats, h32
+
+
+def scale_from_amax(amax_bits, gs):
+    """gs (device float[1]) = 2688 / amax for the float bits in amax_bits (device 4-byte word),
+    1.0 when not finite and positive; on the device, no host sync."""
+    call("nvfp4_scale_from_amax", _p(amax_bits), _p(gs), _stream())
+    return gs
 
 
 def l2_scatter(h, sfh, gs_h, w2: NVFP4Weights, offs, row_slot, row_w, dst_row, T, k, status=None):
@@ -237,6 +290,25 @@ def l2_scatter(h, sfh, gs_h, w2: NVFP4Weights, offs, row_slot, row_w, dst_row, T
          _p(w2.gs), _p(offs), _p(row_slot), _p(row_w), _p(dst_row), w2.E, H, I, T, k, R, _p(ys),
          _p(out32), _p(out16), _p(status), _stream())
     return out32, out16
+
+
+def l2_scatter_add(h, sfh, gs_h, w2: NVFP4Weights, offs, row_slot, row_w, dst_row, T, k,
+                   status=None):
+    """L2 GEMM + routing weight + scatter-ADD into token rows (reductions at L2, order not fixed)
+    -> (out fp32 (T, H), out bf16 (T, H))."""
+    R = h.shape[0]
+    H, I = w2.N, w2.K
+    acc = torch.empty(T, H, dtype=F32, device=h.device)
+    out16 = torch.empty(T, H, dtype=BF16, device=h.device)
+    call("moe_grouped_gemm_l2_scatter_add", _p(h), _p(sfh), _p(gs_h), _p(w2.codes), _p(w2.sf),
+         _p(w2.gs), _p(offs), _p(row_slot), _p(row_w), _p(dst_row), w2.E, H, I, T, k, R,
+         _p(acc), _p(out16), _p(status), _stream())
+    return acc, out16
+
+
+def l2_form(T, k, E, deterministic=False):
+    """1 when moe_ffn_forward adds L2 rows into token rows for this batch, 0 for slot rows."""
+    return int(lib().moe_ffn_l2_form(T, k, E, 2 if deterministic else 0))
 
 
 def ffn_workspace_bytes(T, H, I, E, k):
@@ -257,6 +329,30 @@ def moe_ffn_forward(x, logits, k, w1: NVFP4Weights, w2: NVFP4Weights, gs_h, out=
     call("moe_ffn_forward", _p(x), _p(logits), T, H, I, E, k, _p(w1.codes), _p(w1.sf), _p(w1.gs),
          _p(w2.codes), _p(w2.sf), _p(w2.gs), _p(gs_h), _p(out), _p(ws), ws.numel(), _p(status),
          _stream())
+    return out
+
+
+FFN_DELAYED_GS_H = 1
+FFN_DETERMINISTIC = 2
+
+
+def moe_ffn_forward_ex(x, logits, k, w1: NVFP4Weights, w2: NVFP4Weights, gs_h, delayed=False,
+                       deterministic=False, h_stats=None, out=None, ws=None, status=None):
+    """moe_ffn_forward with options: h_stats (device int32 (3,), filled: amax bits of |h|,
+    saturated and underflowed block scales); delayed=True: gs_h (device float[1]) replaced after
+    use by 2688 / amax(h) for the next call; deterministic=True: the slot-ordered output sum."""
+    T, H = x.shape
+    E = logits.shape[1]
+    I = w1.N // 2
+    if out is None:
+        out = torch.empty(T, H, dtype=BF16, device=x.device)
+    need = ffn_workspace_bytes(T, H, I, E, k)
+    if ws is None:
+        ws = torch.empty(max(need, 256), dtype=U8, device=x.device)
+    call("moe_ffn_forward_ex", _p(x), _p(logits), T, H, I, E, k, _p(w1.codes), _p(w1.sf),
+         _p(w1.gs), _p(w2.codes), _p(w2.sf), _p(w2.gs), _p(gs_h),
+         (FFN_DELAYED_GS_H if delayed else 0) | (FFN_DETERMINISTIC if deterministic else 0),
+         _p(h_stats), _p(out), _p(ws), ws.numel(), _p(status), _stream())
     return out
 
 

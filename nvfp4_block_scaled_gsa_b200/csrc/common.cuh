@@ -137,6 +137,13 @@ __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
+// *p += v, elementwise, as one vector reduction performed at L2 (no return value).
+__device__ __forceinline__ void red_add_v4(float* p, float4 v) {
+  asm volatile("red.relaxed.gpu.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(v.x),
+               "f"(v.y), "f"(v.z), "f"(v.w)
+               : "memory");
+}
+
 // ------------------------------------------------------------------------------ registers
 // Per-warpgroup register budget (setmaxnreg): every thread of a warpgroup executes the same one.
 // An increase waits until other warpgroups have released enough of the registers the block was
@@ -227,6 +234,35 @@ __device__ __forceinline__ void tc_mma_nvf4_pair_warp(uint32_t d_tmem, uint64_t 
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
       : "memory");
 }
+// MXFP4 forms: E2M1 operands with one UE8M0 scale per 32 elements (K = 64: 2 scales per row).
+// The scale operands are tensor-memory addresses whose bits 30-31 select the byte of each
+// 32-bit column where the MMA's 2 scales start (0 or 2); the instruction descriptor repeats
+// that byte index in its A and B scale-factor id fields.
+__device__ __forceinline__ void tc_mma_mxf4_warp(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                                 uint32_t idesc, uint32_t sfa_tmem,
+                                                 uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::mxf4.block_scale.scale_vec::2X"
+      " [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+__device__ __forceinline__ void tc_mma_mxf4_pair_warp(uint32_t d_tmem, uint64_t adesc,
+                                                      uint64_t bdesc, uint32_t idesc,
+                                                      uint32_t sfa_tmem, uint32_t sfb_tmem,
+                                                      uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::2.kind::mxf4.block_scale.scale_vec::2X"
+      " [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
 __device__ __forceinline__ void tc_commit_warp(uint32_t bar) {
   asm volatile(
       "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
@@ -249,6 +285,14 @@ __host__ __device__ constexpr uint32_t idesc_nvf4(int n, int m = 128) {
          | (static_cast<uint32_t>(n >> 3) << 17)  // N / 8
          | (0u << 23)                            // scale format UE4M3
          | (static_cast<uint32_t>(m >> 4) << 24);  // M / 16
+}
+// Instruction descriptor of the MXFP4 form: as above with scale format UE8M0 (bit 23); the
+// per-MMA scale byte index goes to bits 29-30 (A) and 4-5 (B), see idesc_sf_byte.
+__host__ __device__ constexpr uint32_t idesc_mxf4(int n, int m = 128) {
+  return idesc_nvf4(n, m) | (1u << 23);
+}
+__host__ __device__ constexpr uint32_t idesc_sf_byte(uint32_t idesc, uint32_t byte) {
+  return idesc | (byte << 29) | (byte << 4);
 }
 
 // 32 lanes x 32 consecutive 32-bit columns from tensor memory (one value per column per lane).
@@ -277,6 +321,12 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
       "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
       : "memory");
 }
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+      : "memory");
+}
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
@@ -298,33 +348,38 @@ __device__ __forceinline__ void tmem_wait_st() {
 // one) puts, for K step a, the 4 scales of row i + 32*m at lane i of every quadrant, column
 // 4a + m; in the shared-memory atom those 16 bytes (m = 0..3) are line i, bytes 16i..16i+15.
 // So lane i writes, per 128-row atom, one 16-byte line of its own index as 4 columns.
+template <int NA = 4>
 __device__ __forceinline__ void sf_rows128_to_tmem(uint32_t taddr, const uint8_t* atoms, int lane) {
-  uint32_t r[16];
+  uint32_t r[4 * NA];
 #pragma unroll
-  for (int a = 0; a < 4; ++a) {
+  for (int a = 0; a < NA; ++a) {
     const uint4 v = *reinterpret_cast<const uint4*>(atoms + a * 512 + lane * 16);
     r[4 * a] = v.x;
     r[4 * a + 1] = v.y;
     r[4 * a + 2] = v.z;
     r[4 * a + 3] = v.w;
   }
-  tmem_st16(taddr, r);
+  if constexpr (NA == 4) tmem_st16(taddr, r);
+  else tmem_st8(taddr, r);
 }
-// 256-row operand: columns 8a + 4h + m, h = which 128-row half (atoms of half h at +h*2048).
+// 256-row operand: columns 8a + 4h + m, h = which 128-row half (atoms of half h at
+// +h*NA*512).
+template <int NA = 4>
 __device__ __forceinline__ void sf_rows256_to_tmem(uint32_t taddr, const uint8_t* atoms, int lane) {
-  uint32_t r[32];
+  uint32_t r[8 * NA];
 #pragma unroll
-  for (int a = 0; a < 4; ++a) {
+  for (int a = 0; a < NA; ++a) {
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      const uint4 v = *reinterpret_cast<const uint4*>(atoms + h * 2048 + a * 512 + lane * 16);
+      const uint4 v = *reinterpret_cast<const uint4*>(atoms + h * NA * 512 + a * 512 + lane * 16);
       r[8 * a + 4 * h] = v.x;
       r[8 * a + 4 * h + 1] = v.y;
       r[8 * a + 4 * h + 2] = v.z;
       r[8 * a + 4 * h + 3] = v.w;
     }
   }
-  tmem_st32(taddr, r);
+  if constexpr (NA == 4) tmem_st32(taddr, r);
+  else tmem_st16(taddr, r);
 }
 
 // ------------------------------------------------------------------------------ conversions
@@ -355,12 +410,17 @@ __device__ __forceinline__ uint32_t cvt_e2m1x2(float lo, float hi) {
 // NVFP4 scale of one 16-element block given its amax:
 //   s = (amax / 6) * gs ; byte = E4M3(s) ; d = decode(byte) ; r = gs / d (0 when d == 0).
 // Each step is one IEEE float32 operation (no contraction, no fast-math).
-__device__ __forceinline__ uint32_t nvfp4_block_scale(float amax, float gs, float& r) {
-  const float s = __fmul_rn(__fdiv_rn(amax, 6.0f), gs);
+// `s` returns the unrounded scale (for counting scales the E4M3 format clips).
+__device__ __forceinline__ uint32_t nvfp4_block_scale(float amax, float gs, float& r, float& s) {
+  s = __fmul_rn(__fdiv_rn(amax, 6.0f), gs);
   const uint32_t b = cvt_e4m3(s);
   const float d = e4m3_to_float(b);
   r = (d == 0.0f) ? 0.0f : __fdiv_rn(gs, d);
   return b;
+}
+__device__ __forceinline__ uint32_t nvfp4_block_scale(float amax, float gs, float& r) {
+  float s;
+  return nvfp4_block_scale(amax, gs, r, s);
 }
 
 // x * r for the E2M1 converter; a zero element stays (signed) zero even when r overflowed.

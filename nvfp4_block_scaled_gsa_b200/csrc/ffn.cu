@@ -9,6 +9,7 @@
 #include <cstdio>
 
 #include "common.cuh"
+#include "launch.h"
 
 namespace nvfp4 {
 
@@ -25,29 +26,10 @@ nvfp4_status_t check_launch(const char* what) {
   return NVFP4_ERR_CUDA;
 }
 
-nvfp4_status_t quantize_launch(const void* x, int64_t rows, int64_t cols, int64_t ld,
-                               const int32_t* dst_row, int k, int64_t out_rows, uint8_t* codes,
-                               uint8_t* sf, float* gs, int compute_gs, void* ws,
-                               int32_t* dev_status, cudaStream_t s);
-nvfp4_status_t permute_launch(const float* logits, int T, int E, int k, int renorm,
-                              int32_t* topk_ids, float* topk_w, int32_t* offs, int32_t* dst_row,
-                              int32_t* row_slot, float* row_w, int64_t R_max, int32_t* hist_ws,
-                              int32_t* dev_status, cudaStream_t s);
-size_t permute_workspace_bytes(int T, int E, int k);
-nvfp4_status_t gemm_l1(const uint8_t* a, const uint8_t* sfa, const float* gs_a, const uint8_t* w1,
-                       const uint8_t* sfw1, const float* gs_w1, const int32_t* offs,
-                       const int32_t* row_slot, int E, int H, int I, int64_t R_max,
-                       const float* gs_h, uint8_t* h, uint8_t* sfh, int32_t* status,
-                       cudaStream_t s);
-nvfp4_status_t gemm_l2(const uint8_t* h, const uint8_t* sfh, const float* gs_h, const uint8_t* w2,
-                       const uint8_t* sfw2, const float* gs_w2, const int32_t* offs,
-                       const int32_t* row_slot, const float* row_w, const int32_t* dst_row, int E,
-                       int H, int I, int T, int k, int64_t R_max, float* ys, float* out_f32,
-                       void* out_bf16, int32_t* status, cudaStream_t s);
-
 // Byte offsets of the moe_ffn_forward workspace regions (each 256-byte aligned).
 struct FfnLayout {
-  int64_t amax, gs_x, ids, w, offs, dst_row, row_slot, row_w, hist, xq, xsf, hq, hsf, ys, total;
+  int64_t amax, gs_x, ids, w, offs, dst_row, row_slot, row_w, hist, xq, xsf, hq, hsf, ys, hstats;
+  int64_t total;
   int64_t R_max;
 };
 
@@ -75,8 +57,70 @@ FfnLayout ffn_layout(int T, int H, int I, int E, int k) {
   L.hq = take(L.R_max * I / 2);
   L.hsf = take(L.R_max * I / 16);
   L.ys = take(S * H * 4);
+  L.hstats = take(3 * 4);
   L.total = o;
   return L;
+}
+
+// The next call's global scale of h from this call's amax (delayed scaling): 2688 / amax,
+// 1.0 when that is not finite and positive.
+__global__ void scale_from_amax_kernel(const uint32_t* amax_bits, float* gs) {
+  if (threadIdx.x == 0) *gs = gs_from_amax(__uint_as_float(*amax_bits));
+}
+
+nvfp4_status_t ffn_forward(const void* x_bf16, const float* logits, int T, int H, int I, int E,
+                           int k, const uint8_t* w1, const uint8_t* sfw1, const float* gs_w1,
+                           const uint8_t* w2, const uint8_t* sfw2, const float* gs_w2,
+                           float* gs_h, int flags, uint32_t* h_stats, void* out_bf16, void* ws,
+                           size_t ws_bytes, int32_t* dev_status, nvfp4_stream_t stream) {
+  if (T < 0 || E < 1 || E > 256 || k < 1 || k > 32 || k > E || H <= 0 || I <= 0)
+    return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (H % 256 || I % 128) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if ((int64_t)T * k > (int64_t)1 << 30) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (flags & ~(NVFP4_FFN_DELAYED_GS_H | NVFP4_FFN_DETERMINISTIC)) return NVFP4_ERR_INVALID_ARG;
+  const bool delayed = (flags & NVFP4_FFN_DELAYED_GS_H) != 0;
+  if (T == 0) return NVFP4_OK;
+  if (!x_bf16 || !logits || !w1 || !sfw1 || !gs_w1 || !w2 || !sfw2 || !gs_w2 || !gs_h ||
+      !out_bf16 || !ws)
+    return NVFP4_ERR_INVALID_ARG;
+  const FfnLayout L = ffn_layout(T, H, I, E, k);
+  if (ws_bytes < static_cast<size_t>(L.total)) return NVFP4_ERR_WORKSPACE_TOO_SMALL;
+  const void* ptrs16[] = {x_bf16, w1, sfw1, w2, sfw2, out_bf16};
+  for (const void* p : ptrs16)
+    if (!aligned16(p)) return NVFP4_ERR_MISALIGNED;
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) || (reinterpret_cast<uintptr_t>(logits) & 3u) ||
+      (reinterpret_cast<uintptr_t>(h_stats) & 3u))
+    return NVFP4_ERR_MISALIGNED;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  auto i32 = [&](int64_t off) { return reinterpret_cast<int32_t*>(base + off); };
+  auto f32 = [&](int64_t off) { return reinterpret_cast<float*>(base + off); };
+  // statistics of h: the caller's words, or the workspace's when only the delayed scale needs them
+  uint32_t* stats = h_stats != nullptr ? h_stats
+                    : delayed ? reinterpret_cast<uint32_t*>(base + L.hstats) : nullptr;
+
+  nvfp4_status_t st = permute_launch(logits, T, E, k, 1, i32(L.ids), f32(L.w), i32(L.offs),
+                                     i32(L.dst_row), i32(L.row_slot), f32(L.row_w), L.R_max,
+                                     permute_workspace_bytes(T, E, k) ? i32(L.hist) : nullptr,
+                                     dev_status, s);
+  if (st != NVFP4_OK) return st;
+  st = quantize_launch(x_bf16, T, H, H, i32(L.dst_row), k, L.R_max, base + L.xq, base + L.xsf,
+                       f32(L.gs_x), 1, base + L.amax, dev_status, s);
+  if (st != NVFP4_OK) return st;
+  if (stats != nullptr && cudaMemsetAsync(stats, 0, 3 * sizeof(uint32_t), s) != cudaSuccess)
+    return check_launch("cudaMemsetAsync(h_stats)");
+  st = gemm_l1(base + L.xq, base + L.xsf, f32(L.gs_x), w1, sfw1, gs_w1, i32(L.offs),
+               i32(L.row_slot), E, H, I, L.R_max, gs_h, base + L.hq, base + L.hsf, nullptr, stats,
+               dev_status, s);
+  if (st != NVFP4_OK) return st;
+  st = gemm_l2(base + L.hq, base + L.hsf, gs_h, w2, sfw2, gs_w2, i32(L.offs), i32(L.row_slot),
+               f32(L.row_w), i32(L.dst_row), E, H, I, T, k, L.R_max, f32(L.ys), nullptr,
+               out_bf16, l2_use_atomic(T, k, E, (flags & NVFP4_FFN_DETERMINISTIC) != 0),
+               dev_status, s);
+  if (st != NVFP4_OK || !delayed) return st;
+  // stream order: the L2 above has read this call's gs_h before it is replaced
+  scale_from_amax_kernel<<<1, 32, 0, s>>>(stats, gs_h);
+  return check_launch("scale_from_amax_kernel");
 }
 
 }  // namespace nvfp4
@@ -95,40 +139,31 @@ extern "C" nvfp4_status_t moe_ffn_forward(const void* x_bf16, const float* logit
                                           const float* gs_w2, const float* gs_h, void* out_bf16,
                                           void* ws, size_t ws_bytes, int32_t* dev_status,
                                           nvfp4_stream_t stream) {
-  if (T < 0 || E < 1 || E > 256 || k < 1 || k > 32 || k > E || H <= 0 || I <= 0)
-    return NVFP4_ERR_UNSUPPORTED_SHAPE;
-  if (H % 256 || I % 128) return NVFP4_ERR_UNSUPPORTED_SHAPE;
-  if ((int64_t)T * k > (int64_t)1 << 30) return NVFP4_ERR_UNSUPPORTED_SHAPE;
-  if (T == 0) return NVFP4_OK;
-  if (!x_bf16 || !logits || !w1 || !sfw1 || !gs_w1 || !w2 || !sfw2 || !gs_w2 || !gs_h ||
-      !out_bf16 || !ws)
-    return NVFP4_ERR_INVALID_ARG;
-  const FfnLayout L = ffn_layout(T, H, I, E, k);
-  if (ws_bytes < static_cast<size_t>(L.total)) return NVFP4_ERR_WORKSPACE_TOO_SMALL;
-  const void* ptrs16[] = {x_bf16, w1, sfw1, w2, sfw2, out_bf16};
-  for (const void* p : ptrs16)
-    if (!aligned16(p)) return NVFP4_ERR_MISALIGNED;
-  if ((reinterpret_cast<uintptr_t>(ws) & 255u) || (reinterpret_cast<uintptr_t>(logits) & 3u))
-    return NVFP4_ERR_MISALIGNED;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  uint8_t* base = static_cast<uint8_t*>(ws);
-  auto i32 = [&](int64_t off) { return reinterpret_cast<int32_t*>(base + off); };
-  auto f32 = [&](int64_t off) { return reinterpret_cast<float*>(base + off); };
+  // static scale (gs_h is only read), the fastest L2 form for the batch
+  return ffn_forward(x_bf16, logits, T, H, I, E, k, w1, sfw1, gs_w1, w2, sfw2, gs_w2,
+                     const_cast<float*>(gs_h), 0, nullptr, out_bf16, ws, ws_bytes, dev_status,
+                     stream);
+}
 
-  nvfp4_status_t st = permute_launch(logits, T, E, k, 1, i32(L.ids), f32(L.w), i32(L.offs),
-                                     i32(L.dst_row), i32(L.row_slot), f32(L.row_w), L.R_max,
-                                     permute_workspace_bytes(T, E, k) ? i32(L.hist) : nullptr,
-                                     dev_status, s);
-  if (st != NVFP4_OK) return st;
-  st = quantize_launch(x_bf16, T, H, H, i32(L.dst_row), k, L.R_max, base + L.xq, base + L.xsf,
-                       f32(L.gs_x), 1, base + L.amax, dev_status, s);
-  if (st != NVFP4_OK) return st;
-  st = gemm_l1(base + L.xq, base + L.xsf, f32(L.gs_x), w1, sfw1, gs_w1, i32(L.offs),
-               i32(L.row_slot), E, H, I, L.R_max, gs_h, base + L.hq, base + L.hsf, dev_status, s);
-  if (st != NVFP4_OK) return st;
-  return gemm_l2(base + L.hq, base + L.hsf, gs_h, w2, sfw2, gs_w2, i32(L.offs), i32(L.row_slot),
-                 f32(L.row_w), i32(L.dst_row), E, H, I, T, k, L.R_max, f32(L.ys), nullptr,
-                 out_bf16, dev_status, s);
+extern "C" nvfp4_status_t moe_ffn_forward_ex(const void* x_bf16, const float* logits, int T,
+                                             int H, int I, int E, int k, const uint8_t* w1,
+                                             const uint8_t* sfw1, const float* gs_w1,
+                                             const uint8_t* w2, const uint8_t* sfw2,
+                                             const float* gs_w2, float* gs_h, int flags,
+                                             uint32_t* h_stats, void* out_bf16, void* ws,
+                                             size_t ws_bytes, int32_t* dev_status,
+                                             nvfp4_stream_t stream) {
+  return ffn_forward(x_bf16, logits, T, H, I, E, k, w1, sfw1, gs_w1, w2, sfw2, gs_w2, gs_h, flags,
+                     h_stats, out_bf16, ws, ws_bytes, dev_status, stream);
+}
+
+extern "C" nvfp4_status_t nvfp4_scale_from_amax(const uint32_t* amax_bits, float* gs,
+                                                nvfp4_stream_t stream) {
+  if (!amax_bits || !gs) return NVFP4_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(amax_bits) & 3u) || (reinterpret_cast<uintptr_t>(gs) & 3u))
+    return NVFP4_ERR_MISALIGNED;
+  scale_from_amax_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(amax_bits, gs);
+  return check_launch("scale_from_amax_kernel");
 }
 
 extern "C" nvfp4_status_t nvfp4_read_status(const int32_t* dev_status, int32_t* host_code,

@@ -44,6 +44,7 @@
 #include <mutex>
 
 #include "common.cuh"
+#include "launch.h"
 
 namespace nvfp4 {
 namespace {
@@ -51,7 +52,6 @@ namespace {
 constexpr int BM = 128;
 constexpr int BK_BYTES = 128;  // 256 FP4 elements per stage along K
 constexpr int A_BYTES = BM * BK_BYTES;                // 16 KB
-constexpr int SFA_BYTES = 4 * 512;                    // 128 rows x 16 scales
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int NUM_THREADS = 512;  // 4 role warps + 8 epilogue warps + 4 scale-factor warps
 constexpr int EPI_WARP0 = 4;
@@ -66,7 +66,18 @@ constexpr int MAX_E = 256;
 
 // L2_DIRECT: each epilogue lane stores its own row (4 stages; suits a few rows per expert).
 // L2_STAGED: rows pass through shared memory so a warp writes whole lines (3 stages).
-enum Mode { PLAIN_F32 = 0, PLAIN_BF16 = 1, L1_SWIGLU = 2, L2_DIRECT = 3, L2_STAGED = 4 };
+// L2_ATOMIC: staged like L2_STAGED, but each weighted row is added into its token's row of an
+//            FP32 [T][H] accumulator (red.global.add.v4.f32) instead of stored to its slot's
+//            row; tiles run N-slice by N-slice so the accumulator slice being added into
+//            (T x 256 floats) stays in L2.  The sum order of a token's slots is not fixed.
+enum Mode { PLAIN_F32 = 0, PLAIN_BF16 = 1, L1_SWIGLU = 2, L2_DIRECT = 3, L2_STAGED = 4,
+            L2_ATOMIC = 5 };
+template <int MODE>
+__host__ __device__ constexpr bool is_l2() { return MODE == L2_DIRECT || MODE == L2_STAGED || MODE == L2_ATOMIC; }
+// Tiles numbered N-slice by N-slice (all experts' M-tiles of N-slice 0, then of N-slice 1, ...)
+// rather than expert by expert.
+template <int MODE>
+__host__ __device__ constexpr bool slice_major() { return MODE == L2_ATOMIC; }
 
 // Average routed rows per expert from which the L2 epilogue stages its output
 constexpr int kL2StagedMinRowsPerExpert = 32;
@@ -77,7 +88,7 @@ constexpr int kL1TileN = 256;
 constexpr int kL2TileN = 256;
 template <int MODE>
 constexpr int tile_n() {
-  return MODE == L1_SWIGLU ? kL1TileN : (MODE == L2_DIRECT || MODE == L2_STAGED) ? kL2TileN : 256;
+  return MODE == L1_SWIGLU ? kL1TileN : is_l2<MODE>() ? kL2TileN : 256;
 }
 
 // Tile shape: M = 128 rows per CTA, N = 256 columns, K = 256 per stage.  One MMA instruction
@@ -88,34 +99,43 @@ constexpr int tile_n() {
 // holding 128 rows of A and 128 rows (N) of B per stage, so each SM moves 2/3 of the operand
 // bytes of a 128 x 256 tile for the same MMA work.  The even CTA (the leader) issues the MMAs;
 // both CTAs run producer, scale-factor and epilogue warps.
-template <int MODE, int CTAS>
+// SFV: elements per block scale: 16 (NVFP4: E4M3 scales, 4 per row per 64 of K) or 32 (MXFP4:
+// UE8M0 scales, 2 per row per 64 of K).  The scales come in atoms of 128 rows x 4 scale columns
+// (512 bytes), so one atom covers 4 * SFV elements of K and a 256-element stage takes NA atoms.
+template <int MODE, int CTAS, int SFV = 16>
 struct TileCfg {
+  static_assert(SFV == 16 || SFV == 32, "NVFP4 or MXFP4 block scales");
+  static constexpr int NA = 256 / (4 * SFV);               // scale atoms per stage along K
+  static constexpr int SFA_BYTES = NA * 512;               // 128 rows x NA atoms
+  static constexpr int SFA_COLS = 4 * NA;                  // tensor-memory columns of SFA
   static constexpr int BN = tile_n<MODE>();
   static_assert(BN == 128 || BN == 256, "tile width");
   static_assert(CTAS == 1 || BN == 256, "pair tiles are 256 columns wide");
   static constexpr int B_ROWS = BN / CTAS;                 // B rows (N) per CTA per stage
   static constexpr int B_BYTES = B_ROWS * BK_BYTES;
-  static constexpr int SFB_BYTES = (BN / 128) * 4 * 512;   // scales of all BN rows of B
+  static constexpr int SFB_BYTES = (BN / 128) * NA * 512;  // scales of all BN rows of B
   // A/B ring: STAGES slots of AB_BYTES.  Scale atoms have a ring of their own (SF_STAGES slots of
   // SF_BYTES), filled ahead of the A/B ring by a separate producer warp, so a stage's scales are
   // already in shared memory when its tensor-memory columns become free.
   static constexpr int AB_BYTES = A_BYTES + B_BYTES;
   static constexpr int SF_BYTES = SFA_BYTES + SFB_BYTES;
   static constexpr int SF_STAGES = 4;
-  // L2_STAGED: each epilogue warp stages a 32 x 32 FP32 block in shared memory
-  static constexpr int EPI_STAGE_BYTES = MODE == L2_STAGED ? EPI_WARPS * 4096 : 0;
-  static constexpr uint32_t SFB_COLS = (BN / 128) * 16;  // scale columns of B per stage
+  // L2_STAGED / L2_ATOMIC: each epilogue warp stages a 32 x 32 FP32 block in shared memory
+  static constexpr int EPI_STAGE_BYTES =
+      (MODE == L2_STAGED || MODE == L2_ATOMIC) ? EPI_WARPS * 4096 : 0;
+  static constexpr uint32_t SFB_COLS = (BN / 128) * 4 * NA;  // scale columns of B per stage
   static constexpr int STAGES_SMEM =
       (216 * 1024 - EPI_STAGE_BYTES - SF_STAGES * SF_BYTES) / AB_BYTES;
-  static constexpr int STAGES_TMEM = (TMEM_COLS - BN) / (16 + SFB_COLS);
+  static constexpr int STAGES_TMEM = (TMEM_COLS - BN) / (SFA_COLS + SFB_COLS);
   static constexpr int STAGES = STAGES_SMEM < STAGES_TMEM ? STAGES_SMEM : STAGES_TMEM;
   static constexpr int SF_OFFSET = STAGES * AB_BYTES;
   static constexpr int EPI_OFFSET = SF_OFFSET + SF_STAGES * SF_BYTES;
   static constexpr int SMEM_BYTES = EPI_OFFSET + EPI_STAGE_BYTES + 1024;
-  static constexpr int ACC_BUFS = 2 * BN + STAGES * (16 + SFB_COLS) <= TMEM_COLS ? 2 : 1;
-  static constexpr uint32_t TM_SFA = ACC_BUFS * BN;        // 16 columns per stage
-  static constexpr uint32_t TM_SFB = TM_SFA + STAGES * 16;
-  static constexpr uint32_t IDESC = idesc_nvf4(BN, 128 * CTAS);
+  static constexpr int ACC_BUFS = 2 * BN + STAGES * (SFA_COLS + SFB_COLS) <= TMEM_COLS ? 2 : 1;
+  static constexpr uint32_t TM_SFA = ACC_BUFS * BN;        // SFA_COLS columns per stage
+  static constexpr uint32_t TM_SFB = TM_SFA + STAGES * SFA_COLS;
+  static constexpr uint32_t IDESC =
+      SFV == 16 ? idesc_nvf4(BN, 128 * CTAS) : idesc_mxf4(BN, 128 * CTAS);
   static_assert(AB_BYTES % 1024 == 0, "stages must keep 1024-byte alignment (128B swizzle)");
   static_assert(SF_BYTES % 16 == 0, "bulk copies need 16-byte alignment");
   static_assert(TM_SFB + STAGES * SFB_COLS <= TMEM_COLS, "tensor memory budget");
@@ -137,10 +157,13 @@ struct GemmArgs {
   uint8_t* h;         // L1: [R_max][I/2]
   uint8_t* sfh;       // L1
   int I;              // L1
+  float* h32;         // L1 (optional): FP32 h before quantization [R_max][I]
+  uint32_t* h_stats;  // L1 (optional): amax bits of |h|, saturated and underflowed block scales
   const int32_t* row_slot;   // L2 (required), L1 (optional: skip padding rows)
   const float* row_w;        // L2
-  float* ys;                 // L2: weighted expert outputs per slot [S][H]
+  float* ys;                 // L2: weighted expert outputs per slot [S][H]; L2_ATOMIC: [T][H]
   int S;                     // L2: slots (T*k)
+  int k;                     // L2_ATOMIC: slots per token (token = slot / k)
   int32_t* status;
   int64_t out_rows;          // PLAIN: rows of `out`; rows at or past it are not stored
   int k_splits;              // PLAIN_F32: each tile's K is cut into this many ranges
@@ -153,9 +176,25 @@ struct Tile {
 
 // Tile t -> (expert, first row, N-tile).  Each expert's segment gives ceil(rows / (128*CTAS))
 // M-tiles of 128*CTAS rows.
-template <int CTAS>
+template <int CTAS, bool SLICE_MAJOR = false>
 __device__ __forceinline__ Tile decode_tile(int t, const int* tile_start, const int* seg, int E,
                                             int n_tiles) {
+  if constexpr (SLICE_MAJOR) {
+    // tile_start holds the prefix of M-tiles per expert; one N-slice has tile_start[E] tiles
+    const int per_slice = tile_start[E];
+    Tile r;
+    r.nt = t / per_slice;
+    const int u = t - r.nt * per_slice;
+    int lo = 0, hi = E;  // tile_start[lo] <= u < tile_start[hi]
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (tile_start[mid] <= u) lo = mid;
+      else hi = mid;
+    }
+    r.e = lo;
+    r.m0 = seg[lo] + (u - tile_start[lo]) * (BM * CTAS);
+    return r;
+  }
   int lo = 0, hi = E;  // tile_start[lo] <= t < tile_start[hi]
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
@@ -171,11 +210,12 @@ __device__ __forceinline__ Tile decode_tile(int t, const int* tile_start, const 
   return r;
 }
 
-template <int MODE, int CTAS>
+template <int MODE, int CTAS, int SFV>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_a,
                         const __grid_constant__ CUtensorMap tm_b, const GemmArgs args) {
-  using C = TileCfg<MODE, CTAS>;
+  using C = TileCfg<MODE, CTAS, SFV>;
+  constexpr int NA = C::NA;
   constexpr int STAGES = C::STAGES;
   constexpr int BN = C::BN;
   constexpr int ACC_BUFS = C::ACC_BUFS;
@@ -221,7 +261,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (tid < E) {
     const int lo = seg[tid], hi = seg[tid + 1];
     if (lo < 0 || hi < lo || (lo & 127) || (hi & 127) || hi > args.R_max) bad_offsets = 1;
-    else my_tiles = ((((hi - lo) >> 7) + CTAS - 1) / CTAS) * args.n_tiles;
+    else my_tiles = ((((hi - lo) >> 7) + CTAS - 1) / CTAS) * (slice_major<MODE>() ? 1 : args.n_tiles);
   }
   int incl = my_tiles;
 #pragma unroll
@@ -279,12 +319,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   // PLAIN_F32 may cut each tile's K into KS ranges (split-K, for a dense product with fewer
   // tiles than SMs): work item t is K range t % KS of tile t / KS.  KS is 1 in every other mode.
   const int KS = MODE == PLAIN_F32 ? args.k_splits : 1;
-  const int total = bad_offsets ? 0 : tile_start[E] * KS;
+  const int total =
+      bad_offsets ? 0 : tile_start[E] * KS * (slice_major<MODE>() ? args.n_tiles : 1);
   if (tid == 0 && bad_offsets && blockIdx.x == 0) report(args.status, NVFP4_DEVERR_BAD_OFFSETS);
 
   const int K = args.K;
   const int nk = (K + 255) / 256;  // stages along K
-  const int atoms_k = K / 64;      // 64-element scale atoms along K
+  const int atoms_k = K / (4 * SFV);  // scale atoms along K (64 or 128 elements each)
+  const int mma_k = K / 64;           // K = 64 MMA steps
   // stages [lo, hi) of work item t (the host keeps KS <= nk, so no range is empty)
   auto k_range = [&](int t, int& lo, int& hi) {
     const int ks = t % KS;
@@ -305,7 +347,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         uint32_t it = 0;
         bool ok = true;
         for (int t = cluster_id; t < total && ok; t += num_clusters) {
-          const Tile tl = decode_tile<CTAS>(t / KS, tile_start, seg, E, args.n_tiles);
+          const Tile tl = decode_tile<CTAS, slice_major<MODE>()>(t / KS, tile_start, seg, E, args.n_tiles);
           const int m_cta = tl.m0 + BM * rank;  // this CTA's rows
           // B rows of this N-tile: BN consecutive rows (for L1: 16-row gate blocks each followed by
           // the 16 matching up rows); a pair's CTA r loads rows B_ROWS*r .. B_ROWS*r + B_ROWS-1
@@ -359,7 +401,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         uint32_t it = 0;
         bool ok = true;
         for (int t = cluster_id; t < total && ok; t += num_clusters) {
-          const Tile tl = decode_tile<CTAS>(t / KS, tile_start, seg, E, args.n_tiles);
+          const Tile tl = decode_tile<CTAS, slice_major<MODE>()>(t / KS, tile_start, seg, E, args.n_tiles);
           const int m_cta = tl.m0 + BM * rank;
           // a pair's second half past the expert's segment computes rows it never writes; its
           // scale atoms are taken from the first half so that every read stays inside the tensor
@@ -374,17 +416,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               ok = false;
               break;
             }
-            const int natoms = min(4, atoms_k - kb * 4);
+            const int natoms = min(NA, atoms_k - kb * NA);
             const uint32_t sSFA = smem_u32(smem + C::SF_OFFSET + j * C::SF_BYTES);
             const uint32_t sf_bar = smem_u32(&bar_sfin[j]);
             mbar_arrive_expect_tx(sf_bar, natoms * 512 * (1 + BN / 128));
-            bulk_load(sSFA, args.sfa + ((int64_t)a_blk * atoms_k + kb * 4) * 512, natoms * 512,
+            bulk_load(sSFA, args.sfa + ((int64_t)a_blk * atoms_k + kb * NA) * 512, natoms * 512,
                       sf_bar);
 #pragma unroll
             for (int jj = 0; jj < BN / 128; ++jj) {
-              const int64_t b_atom = (int64_t)(b_blk + jj) * atoms_k + kb * 4;
-              bulk_load(sSFA + SFA_BYTES + jj * 4 * 512, args.sfb + b_atom * 512, natoms * 512,
-                        sf_bar);
+              const int64_t b_atom = (int64_t)(b_blk + jj) * atoms_k + kb * NA;
+              bulk_load(sSFA + C::SFA_BYTES + jj * NA * 512, args.sfb + b_atom * 512,
+                        natoms * 512, sf_bar);
             }
           }
         }
@@ -409,10 +451,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const uint64_t b_desc0 = smem_desc(s0 + A_BYTES, 16, 1024, 2);
         uint32_t it = 0, tile_it = 0;
         bool ok = true;
-        auto mma = [&](uint32_t d, uint64_t ad, uint64_t bd, uint32_t sfa, uint32_t sfb,
-                       uint32_t acc) {
-          if constexpr (PAIR) tc_mma_nvf4_pair_warp(d, ad, bd, C::IDESC, sfa, sfb, acc);
-          else tc_mma_nvf4_warp(d, ad, bd, C::IDESC, sfa, sfb, acc);
+        // MMA a (K = 64) of a stage: NVFP4 reads the 4 scales of each row from column
+        // group a; MXFP4 reads 2 scales, from column group a/2 at byte 2*(a%2)
+        auto mma = [&](uint32_t d, uint64_t ad, uint64_t bd, uint32_t t_sfa, uint32_t t_sfb,
+                       int a, uint32_t acc) {
+          if constexpr (SFV == 16) {
+            const uint32_t sfa = t_sfa + a * 4, sfb = t_sfb + a * (BN / 32);
+            if constexpr (PAIR) tc_mma_nvf4_pair_warp(d, ad, bd, C::IDESC, sfa, sfb, acc);
+            else tc_mma_nvf4_warp(d, ad, bd, C::IDESC, sfa, sfb, acc);
+          } else {
+            const uint32_t byte = 2u * static_cast<uint32_t>(a & 1);
+            const uint32_t sfa = (t_sfa + (a >> 1) * 4) | (byte << 30);
+            const uint32_t sfb = (t_sfb + (a >> 1) * (BN / 32)) | (byte << 30);
+            const uint32_t idesc = idesc_sf_byte(C::IDESC, byte);
+            if constexpr (PAIR) tc_mma_mxf4_pair_warp(d, ad, bd, idesc, sfa, sfb, acc);
+            else tc_mma_mxf4_warp(d, ad, bd, idesc, sfa, sfb, acc);
+          }
         };
         auto commit_all = [&](const uint64_t* bar) {  // arrive on `bar` of every CTA
           if constexpr (PAIR) {
@@ -444,20 +498,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             }
             tc_fence_after();
             const uint64_t so = static_cast<uint64_t>(s) * (C::AB_BYTES >> 4);
-            const uint32_t t_sfa = tmem + C::TM_SFA + s * 16;
+            const uint32_t t_sfa = tmem + C::TM_SFA + s * C::SFA_COLS;
             const uint32_t t_sfb = tmem + C::TM_SFB + s * C::SFB_COLS;
             const uint32_t first = kb == kb_lo ? 0u : 1u;
             // scales of this stage are already in tensor memory (scale-factor warps)
-            const int natoms = min(4, atoms_k - kb * 4);
-            if (natoms == 4) {
+            const int n_mma = min(4, mma_k - kb * 4);
+            if (n_mma == 4) {
   #pragma unroll
               for (int a = 0; a < 4; ++a)
-                mma(d_tmem, a_desc0 + so + 2 * a, b_desc0 + so + 2 * a, t_sfa + a * 4,
-                    t_sfb + a * (BN / 32), a == 0 ? first : 1u);
+                mma(d_tmem, a_desc0 + so + 2 * a, b_desc0 + so + 2 * a, t_sfa, t_sfb, a,
+                    a == 0 ? first : 1u);
             } else {
-              for (int a = 0; a < natoms; ++a)
-                mma(d_tmem, a_desc0 + so + 2 * a, b_desc0 + so + 2 * a, t_sfa + a * 4,
-                    t_sfb + a * (BN / 32), a == 0 ? first : 1u);
+              for (int a = 0; a < n_mma; ++a)
+                mma(d_tmem, a_desc0 + so + 2 * a, b_desc0 + so + 2 * a, t_sfa, t_sfb, a,
+                    a == 0 ? first : 1u);
             }
             commit_all(&bar_empty[s]);
           }
@@ -495,11 +549,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         tc_fence_after();
         const uint8_t* st = smem + C::SF_OFFSET + j * C::SF_BYTES;
-        sf_rows128_to_tmem(tmem + lane_base + C::TM_SFA + s * 16, st, lane);
+        sf_rows128_to_tmem<NA>(tmem + lane_base + C::TM_SFA + s * C::SFA_COLS, st, lane);
         if constexpr (BN == 256)
-          sf_rows256_to_tmem(tmem + lane_base + C::TM_SFB + s * C::SFB_COLS, st + SFA_BYTES, lane);
+          sf_rows256_to_tmem<NA>(tmem + lane_base + C::TM_SFB + s * C::SFB_COLS,
+                                 st + C::SFA_BYTES, lane);
         else
-          sf_rows128_to_tmem(tmem + lane_base + C::TM_SFB + s * C::SFB_COLS, st + SFA_BYTES, lane);
+          sf_rows128_to_tmem<NA>(tmem + lane_base + C::TM_SFB + s * C::SFB_COLS,
+                                 st + C::SFA_BYTES, lane);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
@@ -519,7 +575,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int half = (warp - EPI_WARP0) >> 2;
     uint32_t tile_it = 0;
     for (int t = cluster_id; t < total; t += num_clusters, ++tile_it) {
-      const Tile tl = decode_tile<CTAS>(t / KS, tile_start, seg, E, args.n_tiles);
+      const Tile tl = decode_tile<CTAS, slice_major<MODE>()>(t / KS, tile_start, seg, E, args.n_tiles);
       const int b = tile_it % ACC_BUFS;
       if (!mbar_wait_bounded(smem_u32(&bar_acc_full[b]), (tile_it / ACC_BUFS) & 1u, &abort_flag))
         break;
@@ -527,11 +583,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int m_cta = tl.m0 + BM * rank;
       const bool rows_valid = m_cta < seg[tl.e + 1];  // false: a pair's half past the segment
       const uint32_t t_row = tmem + b * BN + (static_cast<uint32_t>(q * 32) << 16);
-      const float alpha = 1.0f / (__ldg(args.gs_a) * __ldg(args.gs_b + tl.e));
+      // MXFP4 has no global scales: its block scales carry the whole range
+      const float alpha =
+          SFV == 32 ? 1.0f : 1.0f / (__ldg(args.gs_a) * __ldg(args.gs_b + tl.e));
       const int64_t row = m_cta + q * 32 + lane;
       // rows of the row map that are padding produce nothing; skip groups of 32 of them
       int slot = rows_valid ? 0 : -1;
-      if (MODE == L1_SWIGLU || MODE == L2_DIRECT || MODE == L2_STAGED) {
+      if (MODE == L1_SWIGLU || is_l2<MODE>()) {
         if (rows_valid && args.row_slot != nullptr) slot = __ldg(args.row_slot + row);
       }
       const bool live = __any_sync(0xffffffffu, slot >= 0);
@@ -563,6 +621,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           tmem_wait_ld();
           release();
           uint32_t sfw = 0u;
+          // what the epilogue learns about h on real rows (padding rows compute garbage)
+          const bool real = slot >= 0;
+          float h_max = 0.0f;
+          uint32_t n_sat = 0u, n_under = 0u;
 #pragma unroll
           for (int cc = 0; cc < n_chunks; ++cc) {
             // h features 32c..32c+31 of the tile live in accumulator columns 64c..64c+63 as two
@@ -585,14 +647,34 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               float amax = 0.0f;
 #pragma unroll
               for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(hv[16 * bb + i]));
-              float rcp;
-              const uint32_t sb = nvfp4_block_scale(amax, gs_h, rcp);
+              float rcp, sc;
+              const uint32_t sb = nvfp4_block_scale(amax, gs_h, rcp, sc);
               packed[2 * bb] = nvfp4_pack8(hv + 16 * bb, rcp);
               packed[2 * bb + 1] = nvfp4_pack8(hv + 16 * bb + 8, rcp);
               sfw |= sb << (8 * (2 * cc + bb));  // this warp's scale columns, in order
+              h_max = fmaxf(h_max, amax);
+              n_sat += sc > 448.0f ? 1u : 0u;
+              n_under += (amax > 0.0f && sb == 0u) ? 1u : 0u;
             }
             *reinterpret_cast<uint4*>(hrow + 16 * c) =
                 make_uint4(packed[0], packed[1], packed[2], packed[3]);
+            if (args.h32 != nullptr && real) {
+              float4* dst = reinterpret_cast<float4*>(args.h32 + row * I + tl.nt * (BN / 2) + 32 * c);
+#pragma unroll
+              for (int q4 = 0; q4 < 8; ++q4)
+                dst[q4] = make_float4(hv[4 * q4], hv[4 * q4 + 1], hv[4 * q4 + 2], hv[4 * q4 + 3]);
+            }
+          }
+          if (args.h_stats != nullptr) {
+            // |h| >= 0, so the float bits order like the values; one atomic per warp and tile
+            const uint32_t hb = __reduce_max_sync(0xffffffffu, real ? __float_as_uint(h_max) : 0u);
+            const uint32_t ns = __reduce_add_sync(0xffffffffu, real ? n_sat : 0u);
+            const uint32_t nu = __reduce_add_sync(0xffffffffu, real ? n_under : 0u);
+            if (lane == 0) {
+              if (hb) atomicMax(args.h_stats, hb);
+              if (ns) atomicAdd(args.h_stats + 1, ns);
+              if (nu) atomicAdd(args.h_stats + 2, nu);
+            }
           }
           // this warp's 2 * n_chunks scale columns are consecutive bytes of one 4-byte group of
           // the tiled layout
@@ -601,7 +683,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if constexpr (n_chunks == 2) *reinterpret_cast<uint32_t*>(sfp) = sfw;
           else *reinterpret_cast<uint16_t*>(sfp) = static_cast<uint16_t>(sfw);
         }
-      } else if (MODE == L2_DIRECT || MODE == L2_STAGED) {
+      } else if (is_l2<MODE>()) {
         // this row's weighted expert output goes to its slot's row of ys; the combine kernel sums
         // a token's k slot rows
         if (live) {
@@ -614,15 +696,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const int c_lo = (BN / 64) * half;
           // the warp's whole slice (BN/2 columns) is read from tensor memory first; then the
           // accumulator goes back to the MMA warp and the stores overlap the next tile's MMAs
-          if constexpr (MODE == L2_STAGED) {
+          if constexpr (MODE == L2_STAGED || MODE == L2_ATOMIC) {
             // each 32-column chunk passes through shared memory (16-byte units XOR-swizzled by
             // row) so that 8 lanes write one row's 128 contiguous bytes
             float4* stg = reinterpret_cast<float4*>(smem + C::EPI_OFFSET +
                                                     (warp - EPI_WARP0) * 4096);
             const int sub = lane >> 3, c4 = lane & 7;
-            int sl[8];  // slot of row 4i + sub of this warp's 32 rows
+            int sl[8];  // slot (L2_ATOMIC: token) of row 4i + sub of this warp's 32 rows
 #pragma unroll
-            for (int i = 0; i < 8; ++i) sl[i] = __shfl_sync(0xffffffffu, slot, 4 * i + sub);
+            for (int i = 0; i < 8; ++i) {
+              sl[i] = __shfl_sync(0xffffffffu, slot, 4 * i + sub);
+              if (MODE == L2_ATOMIC && sl[i] >= 0) sl[i] /= args.k;
+            }
             auto emit = [&](int c, const uint32_t (&v)[32]) {
 #pragma unroll
               for (int j = 0; j < 8; ++j)
@@ -635,7 +720,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               for (int i = 0; i < 8; ++i) {
                 const int r = 4 * i + sub;
                 const float4 val = stg[r * 8 + (c4 ^ (r & 7))];
-                if (sl[i] >= 0) *reinterpret_cast<float4*>(args.ys + (int64_t)sl[i] * H + col) = val;
+                if (sl[i] >= 0) {
+                  float* dst = args.ys + (int64_t)sl[i] * H + col;
+                  if constexpr (MODE == L2_ATOMIC) red_add_v4(dst, val);
+                  else *reinterpret_cast<float4*>(dst) = val;
+                }
               }
               __syncwarp();
             };
@@ -770,11 +859,11 @@ constexpr int kPairMinBlocksPerExpert = 8;
 // At most this many K ranges per tile of a dense product.
 constexpr int kMaxKSplits = 16;
 
-template <int MODE, int CTAS>
+template <int MODE, int CTAS, int SFV>
 nvfp4_status_t launch_cfg(const CUtensorMap& ma, const CUtensorMap& mb, const GemmArgs& args,
                           cudaStream_t s) {
-  constexpr int smem = TileCfg<MODE, CTAS>::SMEM_BYTES;
-  auto kernel = grouped_gemm_kernel<MODE, CTAS>;
+  constexpr int smem = TileCfg<MODE, CTAS, SFV>::SMEM_BYTES;
+  auto kernel = grouped_gemm_kernel<MODE, CTAS, SFV>;
   if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
       cudaSuccess)
     return check_launch("cudaFuncSetAttribute");
@@ -805,7 +894,7 @@ nvfp4_status_t launch_cfg(const CUtensorMap& ma, const CUtensorMap& mb, const Ge
   return check_launch("grouped_gemm_kernel");
 }
 
-template <int MODE>
+template <int MODE, int SFV = 16>
 nvfp4_status_t launch(const uint8_t* a, const uint8_t* b, int64_t b_rows, GemmArgs args,
                       cudaStream_t s) {
   CUtensorMap ma, mb;
@@ -815,9 +904,9 @@ nvfp4_status_t launch(const uint8_t* a, const uint8_t* b, int64_t b_rows, GemmAr
   }
   if constexpr (TileCfg<MODE, 1>::BN == 256) {
     if (args.R_max >= (int64_t)kPairMinBlocksPerExpert * BM * args.E)
-      return launch_cfg<MODE, 2>(ma, mb, args, s);
+      return launch_cfg<MODE, 2, SFV>(ma, mb, args, s);
   }
-  return launch_cfg<MODE, 1>(ma, mb, args, s);
+  return launch_cfg<MODE, 1, SFV>(ma, mb, args, s);
 }
 
 // out[t] = sum over the token's slots j (in order, skipping dropped ones) of ys[t*k + j]; FP32
@@ -854,6 +943,24 @@ __global__ void combine_kernel(const float* __restrict__ ys, const int32_t* __re
       o.w = *reinterpret_cast<const uint32_t*>(&q3);
       *reinterpret_cast<uint4*>(out_bf16 + t * H + c) = o;
     }
+  }
+}
+
+// out[i] = bf16(acc[i]) (round to nearest even), 8 elements per thread.
+__global__ void __launch_bounds__(256) to_bf16_kernel(const float* __restrict__ acc, int64_t n8,
+                                                      __nv_bfloat16* __restrict__ out) {
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n8;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const float4* p = reinterpret_cast<const float4*>(acc + 8 * i);
+    const float4 a = __ldg(p), b = __ldg(p + 1);
+    const __nv_bfloat162 q0 = __floats2bfloat162_rn(a.x, a.y), q1 = __floats2bfloat162_rn(a.z, a.w),
+                         q2 = __floats2bfloat162_rn(b.x, b.y), q3 = __floats2bfloat162_rn(b.z, b.w);
+    uint4 o;
+    o.x = *reinterpret_cast<const uint32_t*>(&q0);
+    o.y = *reinterpret_cast<const uint32_t*>(&q1);
+    o.z = *reinterpret_cast<const uint32_t*>(&q2);
+    o.w = *reinterpret_cast<const uint32_t*>(&q3);
+    reinterpret_cast<uint4*>(out)[i] = o;
   }
 }
 
@@ -968,12 +1075,13 @@ nvfp4_status_t gemm_plain(const uint8_t* a, const uint8_t* sfa, const float* gs_
 nvfp4_status_t gemm_l1(const uint8_t* a, const uint8_t* sfa, const float* gs_a, const uint8_t* w1,
                        const uint8_t* sfw1, const float* gs_w1, const int32_t* offs,
                        const int32_t* row_slot, int E, int H, int I, int64_t R_max,
-                       const float* gs_h, uint8_t* h, uint8_t* sfh, int32_t* status,
-                       cudaStream_t s) {
+                       const float* gs_h, uint8_t* h, uint8_t* sfh, float* h32,
+                       uint32_t* h_stats, int32_t* status, cudaStream_t s) {
   GemmArgs g{};
   g.sfa = sfa; g.sfb = sfw1; g.gs_a = gs_a; g.gs_b = gs_w1; g.offs = offs;
   g.E = E; g.N = 2 * I; g.K = H; g.n_tiles = 2 * I / TileCfg<L1_SWIGLU, 1>::BN; g.R_max = R_max;
   g.gs_h = gs_h; g.h = h; g.sfh = sfh; g.I = I; g.row_slot = row_slot; g.status = status;
+  g.h32 = h32; g.h_stats = h_stats;
   g.out_rows = R_max; g.k_splits = 1;
   return launch<L1_SWIGLU>(a, w1, (int64_t)E * 2 * I, g, s);
 }
@@ -982,13 +1090,27 @@ nvfp4_status_t gemm_l2(const uint8_t* h, const uint8_t* sfh, const float* gs_h, 
                        const uint8_t* sfw2, const float* gs_w2, const int32_t* offs,
                        const int32_t* row_slot, const float* row_w, const int32_t* dst_row, int E,
                        int H, int I, int T, int k, int64_t R_max, float* ys, float* out_f32,
-                       void* out_bf16, int32_t* status, cudaStream_t s) {
+                       void* out_bf16, bool atomic, int32_t* status, cudaStream_t s) {
   if (T == 0) return NVFP4_OK;
   GemmArgs g{};
   g.sfa = sfh; g.sfb = sfw2; g.gs_a = gs_h; g.gs_b = gs_w2; g.offs = offs;
   g.E = E; g.N = H; g.K = I; g.R_max = R_max; g.n_tiles = H / TileCfg<L2_DIRECT, 1>::BN;
-  g.row_slot = row_slot; g.row_w = row_w; g.ys = ys; g.S = T * k; g.status = status;
+  g.row_slot = row_slot; g.row_w = row_w; g.ys = ys; g.S = T * k; g.k = k; g.status = status;
   g.out_rows = R_max; g.k_splits = 1;
+  if (atomic) {
+    // the token rows are summed in place: in out_f32 when the caller wants it, else in ys
+    float* acc = out_f32 != nullptr ? out_f32 : ys;
+    const int64_t n = (int64_t)T * H;
+    if (cudaMemsetAsync(acc, 0, n * sizeof(float), s) != cudaSuccess)
+      return check_launch("cudaMemsetAsync(accumulator)");
+    g.ys = acc;
+    nvfp4_status_t st = launch<L2_ATOMIC>(h, w2, (int64_t)E * H, g, s);
+    if (st != NVFP4_OK || out_bf16 == nullptr) return st;
+    const int64_t want = (n / 8 + 255) / 256;
+    to_bf16_kernel<<<(unsigned)(want < 148 * 16 ? want : 148 * 16), 256, 0, s>>>(
+        acc, n / 8, static_cast<__nv_bfloat16*>(out_bf16));
+    return check_launch("to_bf16_kernel");
+  }
   const bool staged = (int64_t)T * k >= (int64_t)kL2StagedMinRowsPerExpert * E;
   nvfp4_status_t st = staged ? launch<L2_STAGED>(h, w2, (int64_t)E * H, g, s)
                              : launch<L2_DIRECT>(h, w2, (int64_t)E * H, g, s);
@@ -998,6 +1120,12 @@ nvfp4_status_t gemm_l2(const uint8_t* h, const uint8_t* sfh, const float* gs_h, 
   combine_kernel<<<(unsigned)(want < 148 * 16 ? want : 148 * 16), 256, 0, s>>>(
       ys, dst_row, T, k, H, out_f32, static_cast<__nv_bfloat16*>(out_bf16));
   return check_launch("combine_kernel");
+}
+
+// The L2 form for a batch: slot rows summed in slot order (deterministic) for few rows per expert
+// or on request; otherwise added into token rows as they are produced (no per-slot round trip).
+bool l2_use_atomic(int T, int k, int E, bool deterministic) {
+  return !deterministic && (int64_t)T * k >= (int64_t)kL2StagedMinRowsPerExpert * E;
 }
 
 }  // namespace nvfp4
@@ -1021,11 +1149,35 @@ extern "C" nvfp4_status_t nvfp4_grouped_gemm(const uint8_t* a, const uint8_t* sf
                     reinterpret_cast<cudaStream_t>(stream));
 }
 
-extern "C" nvfp4_status_t moe_grouped_gemm_l1_swiglu_q(
-    const uint8_t* a, const uint8_t* sfa, const float* gs_a, const uint8_t* w1,
-    const uint8_t* sfw1, const float* gs_w1, const int32_t* offs, const int32_t* row_slot, int E,
-    int H, int I, int64_t R_max, const float* gs_h, uint8_t* h, uint8_t* sfh, int32_t* dev_status,
-    nvfp4_stream_t stream) {
+extern "C" nvfp4_status_t mxfp4_grouped_gemm(const uint8_t* a, const uint8_t* sfa,
+                                             const uint8_t* b, const uint8_t* sfb,
+                                             const int32_t* offs, int E, int N, int K,
+                                             int64_t R_max, void* out, int out_dtype,
+                                             int32_t* dev_status, nvfp4_stream_t stream) {
+  if (E < 1 || E > MAX_E || N <= 0 || K <= 0 || R_max < 0) return NVFP4_ERR_INVALID_ARG;
+  if (K % 128 || N % TileCfg<PLAIN_F32, 1, 32>::BN || R_max % 128)
+    return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (out_dtype != 0 && out_dtype != 1) return NVFP4_ERR_INVALID_ARG;
+  if (!offs) return NVFP4_ERR_INVALID_ARG;
+  if (R_max == 0) return NVFP4_OK;
+  if (!ok_ptr(a) || !ok_ptr(sfa) || !ok_ptr(b) || !ok_ptr(sfb) || !ok_ptr(out))
+    return (a && sfa && b && sfb && out) ? NVFP4_ERR_MISALIGNED : NVFP4_ERR_INVALID_ARG;
+  GemmArgs g{};
+  g.sfa = sfa; g.sfb = sfb; g.gs_a = nullptr; g.gs_b = nullptr; g.offs = offs;
+  g.E = E; g.N = N; g.K = K; g.n_tiles = N / TileCfg<PLAIN_F32, 1, 32>::BN; g.R_max = R_max;
+  g.out = out; g.status = dev_status; g.out_rows = R_max; g.k_splits = 1;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t b_rows = (int64_t)E * N;
+  return out_dtype == 0 ? launch<PLAIN_F32, 32>(a, b, b_rows, g, s)
+                        : launch<PLAIN_BF16, 32>(a, b, b_rows, g, s);
+}
+
+namespace {
+nvfp4_status_t l1_checked(const uint8_t* a, const uint8_t* sfa, const float* gs_a,
+                          const uint8_t* w1, const uint8_t* sfw1, const float* gs_w1,
+                          const int32_t* offs, const int32_t* row_slot, int E, int H, int I,
+                          int64_t R_max, const float* gs_h, uint8_t* h, uint8_t* sfh, float* h32,
+                          uint32_t* h_stats, int32_t* dev_status, nvfp4_stream_t stream) {
   if (E < 1 || E > MAX_E || H <= 0 || I <= 0 || R_max < 0) return NVFP4_ERR_INVALID_ARG;
   if (H % 64 || I % 64 || (2 * I) % TileCfg<L1_SWIGLU, 1>::BN || R_max % 128)
     return NVFP4_ERR_UNSUPPORTED_SHAPE;
@@ -1034,8 +1186,29 @@ extern "C" nvfp4_status_t moe_grouped_gemm_l1_swiglu_q(
   if (!ok_ptr(a) || !ok_ptr(sfa) || !ok_ptr(w1) || !ok_ptr(sfw1) || !ok_ptr(h) || !ok_ptr(sfh))
     return (a && sfa && w1 && sfw1 && h && sfh) ? NVFP4_ERR_MISALIGNED : NVFP4_ERR_INVALID_ARG;
   if (reinterpret_cast<uintptr_t>(row_slot) & 3u) return NVFP4_ERR_MISALIGNED;
-  return gemm_l1(a, sfa, gs_a, w1, sfw1, gs_w1, offs, row_slot, E, H, I, R_max, gs_h, h, sfh,
-                 dev_status, reinterpret_cast<cudaStream_t>(stream));
+  if ((h32 && !aligned16(h32)) || (reinterpret_cast<uintptr_t>(h_stats) & 3u))
+    return NVFP4_ERR_MISALIGNED;
+  return gemm_l1(a, sfa, gs_a, w1, sfw1, gs_w1, offs, row_slot, E, H, I, R_max, gs_h, h, sfh, h32,
+                 h_stats, dev_status, reinterpret_cast<cudaStream_t>(stream));
+}
+}  // namespace
+
+extern "C" nvfp4_status_t moe_grouped_gemm_l1_swiglu_q(
+    const uint8_t* a, const uint8_t* sfa, const float* gs_a, const uint8_t* w1,
+    const uint8_t* sfw1, const float* gs_w1, const int32_t* offs, const int32_t* row_slot, int E,
+    int H, int I, int64_t R_max, const float* gs_h, uint8_t* h, uint8_t* sfh, int32_t* dev_status,
+    nvfp4_stream_t stream) {
+  return l1_checked(a, sfa, gs_a, w1, sfw1, gs_w1, offs, row_slot, E, H, I, R_max, gs_h, h, sfh,
+                    nullptr, nullptr, dev_status, stream);
+}
+
+extern "C" nvfp4_status_t moe_grouped_gemm_l1_swiglu_q_stats(
+    const uint8_t* a, const uint8_t* sfa, const float* gs_a, const uint8_t* w1,
+    const uint8_t* sfw1, const float* gs_w1, const int32_t* offs, const int32_t* row_slot, int E,
+    int H, int I, int64_t R_max, const float* gs_h, uint8_t* h, uint8_t* sfh, float* h32,
+    uint32_t* h_stats, int32_t* dev_status, nvfp4_stream_t stream) {
+  return l1_checked(a, sfa, gs_a, w1, sfw1, gs_w1, offs, row_slot, E, H, I, R_max, gs_h, h, sfh,
+                    h32, h_stats, dev_status, stream);
 }
 
 extern "C" nvfp4_status_t moe_grouped_gemm_l2_scatter(
@@ -1053,7 +1226,31 @@ extern "C" nvfp4_status_t moe_grouped_gemm_l2_scatter(
       (out_f32 && !aligned16(out_f32)) || (out_bf16 && !aligned16(out_bf16)))
     return (h && sfh && w2 && sfw2 && ys_ws) ? NVFP4_ERR_MISALIGNED : NVFP4_ERR_INVALID_ARG;
   return gemm_l2(h, sfh, gs_h, w2, sfw2, gs_w2, offs, row_slot, row_w, dst_row, E, H, I, T, k,
-                 R_max, ys_ws, out_f32, out_bf16, dev_status, reinterpret_cast<cudaStream_t>(stream));
+                 R_max, ys_ws, out_f32, out_bf16, false, dev_status,
+                 reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" nvfp4_status_t moe_grouped_gemm_l2_scatter_add(
+    const uint8_t* h, const uint8_t* sfh, const float* gs_h, const uint8_t* w2,
+    const uint8_t* sfw2, const float* gs_w2, const int32_t* offs, const int32_t* row_slot,
+    const float* row_w, const int32_t* dst_row, int E, int H, int I, int T, int k, int64_t R_max,
+    float* acc, void* out_bf16, int32_t* dev_status, nvfp4_stream_t stream) {
+  if (E < 1 || E > MAX_E || H <= 0 || I <= 0 || T < 0 || k < 1 || R_max < 0)
+    return NVFP4_ERR_INVALID_ARG;
+  if (H % TileCfg<L2_ATOMIC, 1>::BN || I % 64 || R_max % 128) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (!gs_h || !gs_w2 || !offs || !row_slot || !row_w || !dst_row || !acc)
+    return NVFP4_ERR_INVALID_ARG;
+  if (T == 0 || R_max == 0) return NVFP4_OK;
+  if (!ok_ptr(h) || !ok_ptr(sfh) || !ok_ptr(w2) || !ok_ptr(sfw2) || !aligned16(acc) ||
+      (out_bf16 && !aligned16(out_bf16)))
+    return (h && sfh && w2 && sfw2) ? NVFP4_ERR_MISALIGNED : NVFP4_ERR_INVALID_ARG;
+  return gemm_l2(h, sfh, gs_h, w2, sfw2, gs_w2, offs, row_slot, row_w, dst_row, E, H, I, T, k,
+                 R_max, nullptr, acc, out_bf16, true, dev_status,
+                 reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" int moe_ffn_l2_form(int T, int k, int E, int flags) {
+  return l2_use_atomic(T, k, E, (flags & NVFP4_FFN_DETERMINISTIC) != 0) ? 1 : 0;
 }
 
 // ------------------------------------------------------------------------------ no-alloc variant
@@ -1108,5 +1305,6 @@ extern "C" nvfp4_status_t moe_grouped_gemm_l2_scatter_noalloc(
   float* ys = l2_noalloc_scratch();
   if (ys == nullptr) return NVFP4_ERR_CUDA;
   return gemm_l2(h, sfh, gs_h, w2, sfw2, gs_w2, offs, row_slot, row_w, dst_row, E, H, I, T, k,
-                 R_max, ys, nullptr, out_bf16, dev_status, reinterpret_cast<cudaStream_t>(stream));
+                 R_max, ys, nullptr, out_bf16, false, dev_status,
+                 reinterpret_cast<cudaStream_t>(stream));
 }

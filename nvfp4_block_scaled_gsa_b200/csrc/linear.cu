@@ -7,33 +7,9 @@
 // fused amax + quantize commit).  Here: [RMSNorm +] amax -> quantize -> the grouped GEMM core
 // with one dense segment (split along K when the output has too few tiles to fill the SMs).
 #include "common.cuh"
+#include "launch.h"
 
 namespace nvfp4 {
-
-nvfp4_status_t quantize_launch(const void* x, int64_t rows, int64_t cols, int64_t ld,
-                               const int32_t* dst_row, int k, int64_t out_rows, uint8_t* codes,
-                               uint8_t* sf, float* gs, int compute_gs, void* ws,
-                               int32_t* dev_status, cudaStream_t s);
-nvfp4_status_t rmsnorm_quantize_launch(const void* x, int64_t rows, int64_t cols, int64_t ld,
-                                       const void* gamma, float eps, const int32_t* dst_row,
-                                       int k, int64_t out_rows, uint8_t* codes, uint8_t* sf,
-                                       float* gs, int compute_gs, void* ws, int32_t* dev_status,
-                                       cudaStream_t s);
-nvfp4_status_t gemm_dense(const uint8_t* a, const uint8_t* sfa, const float* gs_a,
-                          const uint8_t* b, const uint8_t* sfb, const float* gs_b, int64_t M, int N,
-                          int K, void* out_bf16, float* part, int64_t part_floats, int32_t* status,
-                          cudaStream_t s);
-int dense_k_splits(int64_t M, int N, int K, int sms, int64_t part_floats);
-int device_sms();
-nvfp4_status_t gemm_dense_parts(const uint8_t* a, const uint8_t* sfa, const float* gs_a,
-                                const uint8_t* b, const uint8_t* sfb, const float* gs_b,
-                                int64_t M, int N, int K, int ks, float* part, int32_t* status,
-                                cudaStream_t s);
-nvfp4_status_t gemm_l1(const uint8_t* a, const uint8_t* sfa, const float* gs_a, const uint8_t* w1,
-                       const uint8_t* sfw1, const float* gs_w1, const int32_t* offs,
-                       const int32_t* row_slot, int E, int H, int I, int64_t R_max,
-                       const float* gs_h, uint8_t* h, uint8_t* sfh, int32_t* status,
-                       cudaStream_t s);
 
 namespace {
 
@@ -299,7 +275,8 @@ extern "C" nvfp4_status_t nvfp4_shared_expert(const void* x, int64_t M, int H, i
     st = check_launch("swiglu_quant_kernel");
   } else {
     st = gemm_l1(base + L.xq, base + L.xsf, gs_x, w1, sfw1, gs_w1, nullptr, nullptr, 1, H, I,
-                 round_up(M, 128), gs_h, base + L.hq, base + L.hsf, dev_status, s);
+                 round_up(M, 128), gs_h, base + L.hq, base + L.hsf, nullptr, nullptr, dev_status,
+                 s);
   }
   if (st != NVFP4_OK) return st;
   float* part = L.part_floats > 0 ? reinterpret_cast<float*>(base + L.part) : nullptr;

@@ -122,3 +122,39 @@ def test_ffn_prefill_sized_batch_end_to_end(T):
     want = M.bf16_round(ref["out"])
     assert rel_fro(got, want) <= 1e-3
     assert cosine(got, want) >= 0.9999
+
+
+@pytest.mark.parametrize("T", [640, 4096])
+def test_ffn_token_row_reductions_against_slot_ordered_sum(T):
+    """From 32 routed rows per expert the FFN adds each slot's weighted row into its token's
+    FP32 row as the L2 tiles are produced (order not fixed); NVFP4_FFN_DETERMINISTIC keeps the
+    per-slot rows and their slot-ordered sum.  The two differ only by FP32 addition order: at most
+    one bf16 step on a small fraction of the outputs.  Fully dropped tokens stay exact zeros in
+    both, and both match the oracle."""
+    from dataclasses import replace
+    cfg = replace(CONFIGS["tiny"], T=T)
+    assert T * cfg.k >= 32 * cfg.E
+    x, lg = gen_x(cfg), gen_logits(cfg)
+    lg[7] = float("-inf")
+    lg[T - 1] = float("-inf")
+    w1d, w1o = _prepack_both(cfg, 1, 2 * cfg.I, cfg.H)
+    w2d, w2o = _prepack_both(cfg, 2, cfg.H, cfg.I)
+    gs_h = torch.tensor([cfg.gs_h], dtype=torch.float32, device=DEV)
+    xd, lgd = x.to(DEV), lg.to(DEV)
+    fast = nv.moe_ffn_forward_ex(xd, lgd, cfg.k, w1d, w2d, gs_h).float().cpu().numpy()
+    det = nv.moe_ffn_forward_ex(xd, lgd, cfg.k, w1d, w2d, gs_h,
+                                deterministic=True).float().cpu().numpy()
+    det2 = nv.moe_ffn_forward_ex(xd, lgd, cfg.k, w1d, w2d, gs_h,
+                                 deterministic=True).float().cpu().numpy()
+    plain = nv.moe_ffn_forward(xd, lgd, cfg.k, w1d, w2d, gs_h).float().cpu().numpy()
+    assert np.array_equal(det, det2)  # the slot-ordered sum is bitwise reproducible
+    for out in (fast, det, plain):
+        assert np.all(out[7] == 0) and np.all(out[T - 1] == 0)
+    diff = fast != det
+    assert diff.mean() <= 0.01
+    step = np.abs(det) * 2.0 ** -7 + 1e-30  # one bf16 step (8 significant bits) or less
+    assert np.all(np.abs(fast - det)[diff] <= step[diff])
+    ref = M.bf16_round(M.moe_ffn(x.float().numpy(), lg.numpy(), cfg.k, w1o, w2o,
+                                 np.float32(cfg.gs_h))["out"])
+    for out in (fast, det, plain):
+        assert rel_fro(out, ref) <= 1e-3 and cosine(out, ref) >= 0.9999

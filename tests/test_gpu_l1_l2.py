@@ -103,6 +103,16 @@ def test_l1_and_l2_match_oracle(T, H, I, E, k):
     assert torch.equal(out.cpu(), acc.cpu().to(torch.bfloat16))
     dropped = np.all(ids < 0, axis=1)
     assert np.all(acc.cpu().numpy()[dropped] == 0)
+    # the scatter-ADD form (rows added into token rows as tiles are produced, N-slice-major):
+    # the same FP32 sum up to addition order
+    acc2, out2 = nv.l2_scatter_add(h_o, sfh_o, gs_h_d, w2d, offs, row_slot, row_w, dst_row, T, k,
+                                   status=status)
+    torch.cuda.synchronize()
+    code, rc = nv.read_status(status)
+    assert code == 0 and rc == 0
+    assert rel_fro(acc2.cpu().numpy(), ref["out"]) <= 1e-5
+    assert torch.equal(out2.cpu(), acc2.cpu().to(torch.bfloat16))
+    assert np.all(acc2.cpu().numpy()[dropped] == 0)
 
 
 def test_l2_bad_row_slot_is_flagged():
@@ -117,5 +127,13 @@ def test_l2_bad_row_slot_is_flagged():
     nv.l2_scatter(h, sfh, torch.ones(1, device=DEV), w2d, to_dev(perm["offs"].astype(np.int32)),
                   to_dev(rs), to_dev(perm["row_w"].astype(np.float32)),
                   to_dev(perm["dst_row"].reshape(-1).astype(np.int32)), 16, 1, status=status)
+    code, rc = nv.read_status(status)
+    assert code & 2 and rc == 7
+    # the scatter-add form flags (and skips) the same bad slot
+    status.zero_()
+    nv.l2_scatter_add(h, sfh, torch.ones(1, device=DEV), w2d,
+                      to_dev(perm["offs"].astype(np.int32)), to_dev(rs),
+                      to_dev(perm["row_w"].astype(np.float32)),
+                      to_dev(perm["dst_row"].reshape(-1).astype(np.int32)), 16, 1, status=status)
     code, rc = nv.read_status(status)
     assert code & 2 and rc == 7
