@@ -66,10 +66,11 @@ constexpr int MAX_E = 256;
 
 // L2_DIRECT: each epilogue lane stores its own row (4 stages; suits a few rows per expert).
 // L2_STAGED: rows pass through shared memory so a warp writes whole lines (3 stages).
-// L2_ATOMIC: staged like L2_STAGED, but each weighted row is added into its token's row of an
-//            FP32 [T][H] accumulator (red.global.add.v4.f32) instead of stored to its slot's
-//            row; tiles run N-slice by N-slice so the accumulator slice being added into
-//            (T x 256 floats) stays in L2.  The sum order of a token's slots is not fixed.
+// L2_ATOMIC: each weighted row is added into its token's row of an FP32 [T][H] accumulator
+//            (red.global.add.v4.f32, 32-byte sectors whole) instead of stored to its slot's row;
+//            tiles run N-slice by N-slice so the accumulator slice being added into (T x 256
+//            floats) stays in L2.  No staging buffer: 4 stages.  The sum order of a token's
+//            slots is not fixed.
 enum Mode { PLAIN_F32 = 0, PLAIN_BF16 = 1, L1_SWIGLU = 2, L2_DIRECT = 3, L2_STAGED = 4,
             L2_ATOMIC = 5 };
 template <int MODE>
@@ -120,9 +121,8 @@ struct TileCfg {
   static constexpr int AB_BYTES = A_BYTES + B_BYTES;
   static constexpr int SF_BYTES = SFA_BYTES + SFB_BYTES;
   static constexpr int SF_STAGES = 4;
-  // L2_STAGED / L2_ATOMIC: each epilogue warp stages a 32 x 32 FP32 block in shared memory
-  static constexpr int EPI_STAGE_BYTES =
-      (MODE == L2_STAGED || MODE == L2_ATOMIC) ? EPI_WARPS * 4096 : 0;
+  // L2_STAGED: each epilogue warp stages a 32 x 32 FP32 block in shared memory
+  static constexpr int EPI_STAGE_BYTES = MODE == L2_STAGED ? EPI_WARPS * 4096 : 0;
   static constexpr uint32_t SFB_COLS = (BN / 128) * 4 * NA;  // scale columns of B per stage
   static constexpr int STAGES_SMEM =
       (216 * 1024 - EPI_STAGE_BYTES - SF_STAGES * SF_BYTES) / AB_BYTES;
@@ -577,12 +577,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     for (int t = cluster_id; t < total; t += num_clusters, ++tile_it) {
       const Tile tl = decode_tile<CTAS, slice_major<MODE>()>(t / KS, tile_start, seg, E, args.n_tiles);
       const int b = tile_it % ACC_BUFS;
-      if (!mbar_wait_bounded(smem_u32(&bar_acc_full[b]), (tile_it / ACC_BUFS) & 1u, &abort_flag))
-        break;
-      tc_fence_after();
+      // Everything the epilogue reads besides the accumulator (row map, routing weight, global
+      // scales) is fetched before waiting for it, so that these loads do not hold up handing
+      // tensor memory back to the MMA warp.
       const int m_cta = tl.m0 + BM * rank;
       const bool rows_valid = m_cta < seg[tl.e + 1];  // false: a pair's half past the segment
-      const uint32_t t_row = tmem + b * BN + (static_cast<uint32_t>(q * 32) << 16);
       // MXFP4 has no global scales: its block scales carry the whole range
       const float alpha =
           SFV == 32 ? 1.0f : 1.0f / (__ldg(args.gs_a) * __ldg(args.gs_b + tl.e));
@@ -592,6 +591,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (MODE == L1_SWIGLU || is_l2<MODE>()) {
         if (rows_valid && args.row_slot != nullptr) slot = __ldg(args.row_slot + row);
       }
+      const float row_weight = (is_l2<MODE>() && slot >= 0) ? __ldg(args.row_w + row) : 0.0f;
+      const float gs_h = MODE == L1_SWIGLU ? __ldg(args.gs_h) : 0.0f;
+      if (!mbar_wait_bounded(smem_u32(&bar_acc_full[b]), (tile_it / ACC_BUFS) & 1u, &abort_flag))
+        break;
+      tc_fence_after();
+      const uint32_t t_row = tmem + b * BN + (static_cast<uint32_t>(q * 32) << 16);
       const bool live = __any_sync(0xffffffffu, slot >= 0);
       bool released = false;  // accumulator buffer b handed back to the MMA warp
       auto release = [&] {
@@ -606,7 +611,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
       if (MODE == L1_SWIGLU) {
         if (live) {
-          const float gs_h = __ldg(args.gs_h);
           const int I = args.I;
           constexpr int n_chunks = BN / 128;  // 64-column chunks per warp
           uint8_t* hrow = args.h + row * (I / 2) + tl.nt * (BN / 4);
@@ -691,23 +695,56 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             report(args.status, NVFP4_DEVERR_BAD_INDEX);
             slot = -1;
           }
-          const float scale = alpha * (slot >= 0 ? __ldg(args.row_w + row) : 0.0f);
+          const float scale = alpha * (slot >= 0 ? row_weight : 0.0f);
           const int H = args.N;
           const int c_lo = (BN / 64) * half;
           // the warp's whole slice (BN/2 columns) is read from tensor memory first; then the
           // accumulator goes back to the MMA warp and the stores overlap the next tile's MMAs
-          if constexpr (MODE == L2_STAGED || MODE == L2_ATOMIC) {
+          if constexpr (MODE == L2_ATOMIC) {
+            // Added into token rows with no shared-memory staging: within each 8-column group,
+            // lanes 2i and 2i+1 swap half their values so that each vector reduction of the warp
+            // covers 16 rows x 32 bytes (both lanes of a pair on the same row's sector).
+            // Instruction A writes the even lane's row, instruction B the odd lane's.
+            const int tok = slot >= 0 ? slot / args.k : -1;
+            const int tok_peer = __shfl_xor_sync(0xffffffffu, tok, 1);
+            const bool odd = (lane & 1) != 0;
+            const int tok_a = odd ? tok_peer : tok, tok_b = odd ? tok : tok_peer;
+            const int half_col = odd ? 4 : 0;
+            uint32_t v[BN / 64][32];
+#pragma unroll
+            for (int j = 0; j < BN / 64; ++j) tmem_ld32(t_row + 32 * (c_lo + j), v[j]);
+            tmem_wait_ld();
+            release();
+#pragma unroll
+            for (int j = 0; j < BN / 64; ++j) {
+              const int64_t col0 = (int64_t)tl.nt * BN + 32 * (c_lo + j);
+#pragma unroll
+              for (int g = 0; g < 4; ++g) {
+                float own[8], recv[4];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) own[i] = __uint_as_float(v[j][8 * g + i]) * scale;
+                // even lanes pass on columns 4..7 of their row, odd lanes columns 0..3
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                  recv[i] = __shfl_xor_sync(0xffffffffu, odd ? own[i] : own[4 + i], 1);
+                const int64_t col = col0 + 8 * g + half_col;
+                const float4 va = odd ? make_float4(recv[0], recv[1], recv[2], recv[3])
+                                      : make_float4(own[0], own[1], own[2], own[3]);
+                const float4 vb = odd ? make_float4(own[4], own[5], own[6], own[7])
+                                      : make_float4(recv[0], recv[1], recv[2], recv[3]);
+                if (tok_a >= 0) red_add_v4(args.ys + (int64_t)tok_a * H + col, va);
+                if (tok_b >= 0) red_add_v4(args.ys + (int64_t)tok_b * H + col, vb);
+              }
+            }
+          } else if constexpr (MODE == L2_STAGED) {
             // each 32-column chunk passes through shared memory (16-byte units XOR-swizzled by
             // row) so that 8 lanes write one row's 128 contiguous bytes
             float4* stg = reinterpret_cast<float4*>(smem + C::EPI_OFFSET +
                                                     (warp - EPI_WARP0) * 4096);
             const int sub = lane >> 3, c4 = lane & 7;
-            int sl[8];  // slot (L2_ATOMIC: token) of row 4i + sub of this warp's 32 rows
+            int sl[8];  // slot of row 4i + sub of this warp's 32 rows
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              sl[i] = __shfl_sync(0xffffffffu, slot, 4 * i + sub);
-              if (MODE == L2_ATOMIC && sl[i] >= 0) sl[i] /= args.k;
-            }
+            for (int i = 0; i < 8; ++i) sl[i] = __shfl_sync(0xffffffffu, slot, 4 * i + sub);
             auto emit = [&](int c, const uint32_t (&v)[32]) {
 #pragma unroll
               for (int j = 0; j < 8; ++j)
@@ -720,11 +757,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               for (int i = 0; i < 8; ++i) {
                 const int r = 4 * i + sub;
                 const float4 val = stg[r * 8 + (c4 ^ (r & 7))];
-                if (sl[i] >= 0) {
-                  float* dst = args.ys + (int64_t)sl[i] * H + col;
-                  if constexpr (MODE == L2_ATOMIC) red_add_v4(dst, val);
-                  else *reinterpret_cast<float4*>(dst) = val;
-                }
+                if (sl[i] >= 0) *reinterpret_cast<float4*>(args.ys + (int64_t)sl[i] * H + col) = val;
               }
               __syncwarp();
             };
