@@ -221,9 +221,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   constexpr int ACC_BUFS = C::ACC_BUFS;
   constexpr bool PAIR = CTAS == 2;
   extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t bar_full[STAGES];   // A/B landed (a pair: both CTAs')
+  // A/B landed (a pair: both CTAs') and the stage's scales in tensor memory (all CTAs'
+  // scale-factor warps): one barrier, so that the MMA warp waits once per stage
+  __shared__ __align__(8) uint64_t bar_full[STAGES];
   __shared__ __align__(8) uint64_t bar_empty[STAGES];  // MMAs done with the stage
-  __shared__ __align__(8) uint64_t bar_sf[STAGES];     // scales in tensor memory (all CTAs)
   __shared__ __align__(8) uint64_t bar_sfin[C::SF_STAGES];     // scale atoms landed in a slot
   __shared__ __align__(8) uint64_t bar_sfempty[C::SF_STAGES];  // scale slot copied out
   __shared__ __align__(8) uint64_t bar_acc_full[ACC_BUFS];
@@ -287,9 +288,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   // ---- barriers and tensor memory
   if (tid == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(smem_u32(&bar_full[s]), 1);
+      mbar_init(smem_u32(&bar_full[s]), 1 + 4 * CTAS);  // producer + scale-factor warps
       mbar_init(smem_u32(&bar_empty[s]), 1);
-      mbar_init(smem_u32(&bar_sf[s]), 4 * CTAS);
     }
     for (int j = 0; j < C::SF_STAGES; ++j) {
       mbar_init(smem_u32(&bar_sfin[j]), 1);
@@ -485,17 +485,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             ok = false;
             break;
           }
-          tc_fence_after();
           const uint32_t d_tmem = tmem + b * BN;
           int kb_lo, kb_hi;
           k_range(t, kb_lo, kb_hi);
+          // The tensor pipe keeps almost no queue ahead of the issuing warp, so a wait between
+          // two stages adds to every stage (measured: 128 cycles per MMA with no waits, ~160 with
+          // one wait per 4 MMAs).  Each stage's one barrier is therefore waited for while the
+          // previous stage's MMAs still run: the first stage of a tile here, every later one
+          // between the last two MMAs of the stage before it.
+          auto stage_ready = [&](uint32_t j) {
+            return wait_all(&bar_full[j % STAGES], (j / STAGES) & 1u);
+          };
+          if (kb_lo < kb_hi && !stage_ready(it)) {
+            ok = false;
+            break;
+          }
           for (int kb = kb_lo; kb < kb_hi; ++kb, ++it) {
             const int s = it % STAGES;
-            const uint32_t ph = (it / STAGES) & 1u;
-            if (!wait_all(&bar_full[s], ph) || !wait_all(&bar_sf[s], ph)) {
-              ok = false;
-              break;
-            }
             tc_fence_after();
             const uint64_t so = static_cast<uint64_t>(s) * (C::AB_BYTES >> 4);
             const uint32_t t_sfa = tmem + C::TM_SFA + s * C::SFA_COLS;
@@ -503,17 +509,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const uint32_t first = kb == kb_lo ? 0u : 1u;
             // scales of this stage are already in tensor memory (scale-factor warps)
             const int n_mma = min(4, mma_k - kb * 4);
+            const bool more = kb + 1 < kb_hi;
             if (n_mma == 4) {
   #pragma unroll
-              for (int a = 0; a < 4; ++a)
+              for (int a = 0; a < 3; ++a)
                 mma(d_tmem, a_desc0 + so + 2 * a, b_desc0 + so + 2 * a, t_sfa, t_sfb, a,
                     a == 0 ? first : 1u);
+              if (more && !stage_ready(it + 1)) ok = false;
+              mma(d_tmem, a_desc0 + so + 6, b_desc0 + so + 6, t_sfa, t_sfb, 3, 1u);
             } else {
               for (int a = 0; a < n_mma; ++a)
                 mma(d_tmem, a_desc0 + so + 2 * a, b_desc0 + so + 2 * a, t_sfa, t_sfb, a,
                     a == 0 ? first : 1u);
+              if (more && !stage_ready(it + 1)) ok = false;
             }
             commit_all(&bar_empty[s]);
+            if (!ok) break;
           }
           if (!ok) break;
           commit_all(&bar_acc_full[b]);
@@ -561,8 +572,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         __syncwarp();
         if (lane == 0) {
           mbar_arrive(smem_u32(&bar_sfempty[j]));
-          if constexpr (PAIR) mbar_arrive_cluster(at_leader(&bar_sf[s]));
-          else mbar_arrive(smem_u32(&bar_sf[s]));
+          if constexpr (PAIR) mbar_arrive_cluster(at_leader(&bar_full[s]));
+          else mbar_arrive(smem_u32(&bar_full[s]));
         }
       }
     }
