@@ -64,8 +64,8 @@ constexpr uint32_t REGS_EPI = 176, REGS_OTHER = 80;
 static_assert(2 * REGS_EPI + 2 * REGS_OTHER == 4 * 128, "register budgets exceed the launch's");
 constexpr int MAX_E = 256;
 
-// L2_DIRECT: each epilogue lane stores its own row (4 stages; suits a few rows per expert).
-// L2_STAGED: rows pass through shared memory so a warp writes whole lines (3 stages).
+// L2_DIRECT: each epilogue lane stores its own row (suits a few rows per expert).
+// L2_STAGED: rows exchanged between lanes by register shuffles so a warp writes whole lines.
 // L2_ATOMIC: each weighted row is added into its token's row of an FP32 [T][H] accumulator
 //            (red.global.add.v4.f32, 4 rows x 128 bytes per warp instruction) instead of stored
 //            to its slot's row;
@@ -75,7 +75,9 @@ constexpr int MAX_E = 256;
 enum Mode { PLAIN_F32 = 0, PLAIN_BF16 = 1, L1_SWIGLU = 2, L2_DIRECT = 3, L2_STAGED = 4,
             L2_ATOMIC = 5 };
 template <int MODE>
-__host__ __device__ constexpr bool is_l2() { return MODE == L2_DIRECT || MODE == L2_STAGED || MODE == L2_ATOMIC; }
+__host__ __device__ constexpr bool is_l2() {
+  return MODE == L2_DIRECT || MODE == L2_STAGED || MODE == L2_ATOMIC;
+}
 // Tiles numbered N-slice by N-slice (all experts' M-tiles of N-slice 0, then of N-slice 1, ...)
 // rather than expert by expert.
 template <int MODE>
@@ -122,8 +124,7 @@ struct TileCfg {
   static constexpr int AB_BYTES = A_BYTES + B_BYTES;
   static constexpr int SF_BYTES = SFA_BYTES + SFB_BYTES;
   static constexpr int SF_STAGES = 4;
-  // L2_STAGED: each epilogue warp stages a 32 x 32 FP32 block in shared memory
-  static constexpr int EPI_STAGE_BYTES = MODE == L2_STAGED ? EPI_WARPS * 4096 : 0;
+  static constexpr int EPI_STAGE_BYTES = 0;  // no epilogue staging buffer
   static constexpr uint32_t SFB_COLS = (BN / 128) * 4 * NA;  // scale columns of B per stage
   static constexpr int STAGES_SMEM =
       (216 * 1024 - EPI_STAGE_BYTES - SF_STAGES * SF_BYTES) / AB_BYTES;
@@ -263,7 +264,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (tid < E) {
     const int lo = seg[tid], hi = seg[tid + 1];
     if (lo < 0 || hi < lo || (lo & 127) || (hi & 127) || hi > args.R_max) bad_offsets = 1;
-    else my_tiles = ((((hi - lo) >> 7) + CTAS - 1) / CTAS) * (slice_major<MODE>() ? 1 : args.n_tiles);
+    else
+      my_tiles = ((((hi - lo) >> 7) + CTAS - 1) / CTAS) * (slice_major<MODE>() ? 1 : args.n_tiles);
   }
   int incl = my_tiles;
 #pragma unroll
@@ -348,7 +350,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         uint32_t it = 0;
         bool ok = true;
         for (int t = cluster_id; t < total && ok; t += num_clusters) {
-          const Tile tl = decode_tile<CTAS, slice_major<MODE>()>(t / KS, tile_start, seg, E, args.n_tiles);
+          const Tile tl = decode_tile<CTAS, slice_major<MODE>()>(t / KS, tile_start, seg, E,
+                                                                args.n_tiles);
           const int m_cta = tl.m0 + BM * rank;  // this CTA's rows
           // B rows of this N-tile: BN consecutive rows (for L1: 16-row gate blocks each followed by
           // the 16 matching up rows); a pair's CTA r loads rows B_ROWS*r .. B_ROWS*r + B_ROWS-1
@@ -402,7 +405,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         uint32_t it = 0;
         bool ok = true;
         for (int t = cluster_id; t < total && ok; t += num_clusters) {
-          const Tile tl = decode_tile<CTAS, slice_major<MODE>()>(t / KS, tile_start, seg, E, args.n_tiles);
+          const Tile tl = decode_tile<CTAS, slice_major<MODE>()>(t / KS, tile_start, seg, E,
+                                                                args.n_tiles);
           const int m_cta = tl.m0 + BM * rank;
           // a pair's second half past the expert's segment computes rows it never writes; its
           // scale atoms are taken from the first half so that every read stays inside the tensor
@@ -587,7 +591,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int half = (warp - EPI_WARP0) >> 2;
     uint32_t tile_it = 0;
     for (int t = cluster_id; t < total; t += num_clusters, ++tile_it) {
-      const Tile tl = decode_tile<CTAS, slice_major<MODE>()>(t / KS, tile_start, seg, E, args.n_tiles);
+      const Tile tl = decode_tile<CTAS, slice_major<MODE>()>(t / KS, tile_start, seg, E,
+                                                                args.n_tiles);
       const int b = tile_it % ACC_BUFS;
       // Everything the epilogue reads besides the accumulator (row map, routing weight, global
       // scales) is fetched before waiting for it, so that these loads do not hold up handing
@@ -675,7 +680,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             *reinterpret_cast<uint4*>(hrow + 16 * c) =
                 make_uint4(packed[0], packed[1], packed[2], packed[3]);
             if (args.h32 != nullptr && real) {
-              float4* dst = reinterpret_cast<float4*>(args.h32 + row * I + tl.nt * (BN / 2) + 32 * c);
+              float4* dst =
+                  reinterpret_cast<float4*>(args.h32 + row * I + tl.nt * (BN / 2) + 32 * c);
 #pragma unroll
               for (int q4 = 0; q4 < 8; ++q4)
                 dst[q4] = make_float4(hv[4 * q4], hv[4 * q4 + 1], hv[4 * q4 + 2], hv[4 * q4 + 3]);
@@ -712,14 +718,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const int c_lo = (BN / 64) * half;
           // the warp's whole slice (BN/2 columns) is read from tensor memory first; then the
           // accumulator goes back to the MMA warp and the stores overlap the next tile's MMAs
-          if constexpr (MODE == L2_ATOMIC) {
-            // Added into token rows with no shared-memory staging.  Each lane holds 32
-            // consecutive values of its own row per 32-column chunk (8 pieces of 4); the 8 lanes
-            // of an octet transpose those pieces among themselves with register shuffles (three
-            // exchange rounds), after which lane c holds piece c of each of the octet's 8 rows.
-            // Every vector reduction of the warp then covers 4 rows x 128 contiguous bytes, the
-            // shape the SM -> L2 path takes fastest (about 1.7x the rate of 16 rows x 32 bytes).
-            const int tok = slot >= 0 ? slot / args.k : -1;
+          if constexpr (MODE == L2_ATOMIC || MODE == L2_STAGED) {
+            // No shared-memory staging.  Each lane holds 32 consecutive values of its own row
+            // per 32-column chunk (8 pieces of 4); the 8 lanes of an octet transpose those pieces
+            // among themselves with register shuffles (three exchange rounds), after which lane c
+            // holds piece c of each of the octet's 8 rows.  Every vector store (L2_STAGED: the
+            // slot's row) or reduction (L2_ATOMIC: the token's row) of the warp then covers
+            // 4 rows x 128 contiguous bytes, the shape the SM -> L2 path takes fastest (about
+            // 1.7x the rate of 16 rows x 32 bytes).
+            const int tok = slot < 0 ? -1 : MODE == L2_ATOMIC ? slot / args.k : slot;
             int tok_r[8];  // the tokens of the octet's 8 rows
 #pragma unroll
             for (int i = 0; i < 8; ++i) tok_r[i] = __shfl_sync(0xffffffffu, tok, (lane & ~7) | i);
@@ -732,7 +739,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
             for (int j = 0; j < BN / 64; ++j) {
 #pragma unroll
-              for (int i = 0; i < 32; ++i) v[j][i] = __float_as_uint(__uint_as_float(v[j][i]) * scale);
+              for (int i = 0; i < 32; ++i)
+                v[j][i] = __float_as_uint(__uint_as_float(v[j][i]) * scale);
               // round m: a lane with lane bit m set keeps the pieces whose index has bit m set
               // and takes its partner's pieces with bit m set in place of its own with bit m clear;
               // the partner does the converse
@@ -756,44 +764,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
               for (int i = 0; i < 8; ++i) {
                 if (tok_r[i] < 0) continue;
-                red_add_v4(args.ys + (int64_t)tok_r[i] * H + col,
-                           make_float4(__uint_as_float(v[j][4 * i]), __uint_as_float(v[j][4 * i + 1]),
-                                       __uint_as_float(v[j][4 * i + 2]),
-                                       __uint_as_float(v[j][4 * i + 3])));
+                const float4 val =
+                    make_float4(__uint_as_float(v[j][4 * i]), __uint_as_float(v[j][4 * i + 1]),
+                                __uint_as_float(v[j][4 * i + 2]), __uint_as_float(v[j][4 * i + 3]));
+                float* dst = args.ys + (int64_t)tok_r[i] * H + col;
+                if constexpr (MODE == L2_ATOMIC) red_add_v4(dst, val);
+                else *reinterpret_cast<float4*>(dst) = val;
               }
             }
-          } else if constexpr (MODE == L2_STAGED) {
-            // each 32-column chunk passes through shared memory (16-byte units XOR-swizzled by
-            // row) so that 8 lanes write one row's 128 contiguous bytes
-            float4* stg = reinterpret_cast<float4*>(smem + C::EPI_OFFSET +
-                                                    (warp - EPI_WARP0) * 4096);
-            const int sub = lane >> 3, c4 = lane & 7;
-            int sl[8];  // slot of row 4i + sub of this warp's 32 rows
-#pragma unroll
-            for (int i = 0; i < 8; ++i) sl[i] = __shfl_sync(0xffffffffu, slot, 4 * i + sub);
-            auto emit = [&](int c, const uint32_t (&v)[32]) {
-#pragma unroll
-              for (int j = 0; j < 8; ++j)
-                stg[lane * 8 + (j ^ (lane & 7))] = make_float4(
-                    __uint_as_float(v[4 * j]) * scale, __uint_as_float(v[4 * j + 1]) * scale,
-                    __uint_as_float(v[4 * j + 2]) * scale, __uint_as_float(v[4 * j + 3]) * scale);
-              __syncwarp();
-              const int64_t col = (int64_t)tl.nt * BN + 32 * c + 4 * c4;
-#pragma unroll
-              for (int i = 0; i < 8; ++i) {
-                const int r = 4 * i + sub;
-                const float4 val = stg[r * 8 + (c4 ^ (r & 7))];
-                if (sl[i] >= 0) *reinterpret_cast<float4*>(args.ys + (int64_t)sl[i] * H + col) = val;
-              }
-              __syncwarp();
-            };
-            uint32_t v[BN / 64][32];
-#pragma unroll
-            for (int j = 0; j < BN / 64; ++j) tmem_ld32(t_row + 32 * (c_lo + j), v[j]);
-            tmem_wait_ld();
-            release();
-#pragma unroll
-            for (int j = 0; j < BN / 64; ++j) emit(c_lo + j, v[j]);
           } else {
             float* dst = args.ys + (int64_t)(slot >= 0 ? slot : 0) * H + tl.nt * BN;
             auto emit = [&](int c, const uint32_t (&v)[32]) {
