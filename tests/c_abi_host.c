@@ -38,6 +38,20 @@ int main(void) {
     check(moe_w1_row_map(32, map) == NVFP4_OK && map[0] == 0 && map[16] == 32 && map[32] == 16,
           "W1 row map");
   }
+  /* the FFN's L2 form: slot rows below 32 routed rows per expert, token-row reductions from
+     there unless the deterministic flag is given */
+  check(moe_ffn_l2_form(16, 8, 256, 0) == 0 && moe_ffn_l2_form(8192, 8, 256, 0) == 1 &&
+            moe_ffn_l2_form(8192, 8, 256, NVFP4_FFN_DETERMINISTIC) == 0,
+        "FFN L2 form");
+  check(moe_ffn_forward_ex(fake, fake, 16, 7168, 2048, 256, 8, fake, fake, fake, fake, fake, fake,
+                           fake, 4, NULL, fake, fake, (size_t)1 << 40, NULL, NULL) ==
+            NVFP4_ERR_INVALID_ARG,
+        "FFN rejects unknown flags");
+  check(mxfp4_quantize(fake, 4, 96, 96, fake, fake, NULL, NULL) == NVFP4_ERR_UNSUPPORTED_SHAPE,
+        "MXFP4 quantize rejects cols % 128");
+  check(mxfp4_grouped_gemm(fake, fake, fake, fake, fake, 2, 256, 192, 128, fake, 0, NULL, NULL) ==
+            NVFP4_ERR_UNSUPPORTED_SHAPE,
+        "MXFP4 GEMM rejects K % 128");
   check(nvfp4_last_error() != NULL, "last error string");
   return failures == 0 ? 0 : 1;
 }

@@ -24,4 +24,4 @@ def test_c99_client_builds_links_and_passes(tmp_path):
     r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
     assert r.returncode == 0, r.stdout + r.stderr
     lines = r.stdout.splitlines()
-    assert len(lines) == 12 and all(line.startswith("ok ") for line in lines), r.stdout
+    assert len(lines) == 16 and all(line.startswith("ok ") for line in lines), r.stdout
