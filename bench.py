@@ -116,8 +116,8 @@ def kernel_sources_sha16():
 # a reduced capture are scaled to the full launch by the units it processes, as noted there.
 CAPTURED_TRAFFIC = {
     # workload: (kernel_sources_sha16 at the capture, bytes per launch)
-    "decode": ("f092bf14fe8372b3", 1673600000),
-    "prefill": ("f092bf14fe8372b3", 4666000000),
+    "decode": ("49adf8f15b32f17f", 1672600000),
+    "prefill": ("49adf8f15b32f17f", 4669000000),
 }
 
 

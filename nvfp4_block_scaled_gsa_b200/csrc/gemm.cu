@@ -64,27 +64,29 @@ constexpr uint32_t REGS_EPI = 176, REGS_OTHER = 80;
 static_assert(2 * REGS_EPI + 2 * REGS_OTHER == 4 * 128, "register budgets exceed the launch's");
 constexpr int MAX_E = 256;
 
-// L2_DIRECT: each epilogue lane stores its own row (suits a few rows per expert).
-// L2_STAGED: rows exchanged between lanes by register shuffles so a warp writes whole lines.
+// L2_ROWS:   each weighted row is stored to its slot's row of an FP32 [S][H] buffer; the rows
+//            are exchanged between the lanes of an octet by register shuffles so that a warp
+//            writes 4 rows x 128 bytes per store instruction.  A combine kernel then sums each
+//            token's k slot rows in slot order (deterministic).
 // L2_ATOMIC: each weighted row is added into its token's row of an FP32 [T][H] accumulator
 //            (red.global.add.v4.f32, 4 rows x 128 bytes per warp instruction) instead of stored
 //            to its slot's row;
 //            tiles run N-slice by N-slice so the accumulator slice being added into (T x 256
 //            floats) stays in L2.  No staging buffer: 4 stages.  The sum order of a token's
 //            slots is not fixed.
-enum Mode { PLAIN_F32 = 0, PLAIN_BF16 = 1, L1_SWIGLU = 2, L2_DIRECT = 3, L2_STAGED = 4,
-            L2_ATOMIC = 5 };
+enum Mode { PLAIN_F32 = 0, PLAIN_BF16 = 1, L1_SWIGLU = 2, L2_ROWS = 3, L2_ATOMIC = 4 };
 template <int MODE>
 __host__ __device__ constexpr bool is_l2() {
-  return MODE == L2_DIRECT || MODE == L2_STAGED || MODE == L2_ATOMIC;
+  return MODE == L2_ROWS || MODE == L2_ATOMIC;
 }
 // Tiles numbered N-slice by N-slice (all experts' M-tiles of N-slice 0, then of N-slice 1, ...)
 // rather than expert by expert.
 template <int MODE>
 __host__ __device__ constexpr bool slice_major() { return MODE == L2_ATOMIC; }
 
-// Average routed rows per expert from which the L2 epilogue stages its output
-constexpr int kL2StagedMinRowsPerExpert = 32;
+// Average routed rows per expert from which the FFN's L2 adds into token rows (scatter-add)
+// instead of writing slot rows and combining them
+constexpr int kL2AtomicMinRowsPerExpert = 32;
 
 // Tile width (N) per epilogue.  256 columns fill tensor memory with one accumulator; 128 leave
 // room for two, so the epilogue of one tile overlaps the MMAs of the next.
@@ -706,8 +708,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           else *reinterpret_cast<uint16_t*>(sfp) = static_cast<uint16_t>(sfw);
         }
       } else if (is_l2<MODE>()) {
-        // this row's weighted expert output goes to its slot's row of ys; the combine kernel sums
-        // a token's k slot rows
+        // this row's weighted expert output goes to its slot's row of ys (L2_ROWS; the combine
+        // kernel then sums a token's k slot rows) or is added into its token's row (L2_ATOMIC)
         if (live) {
           if (slot >= args.S) {
             report(args.status, NVFP4_DEVERR_BAD_INDEX);
@@ -717,80 +719,59 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const int H = args.N;
           const int c_lo = (BN / 64) * half;
           // the warp's whole slice (BN/2 columns) is read from tensor memory first; then the
-          // accumulator goes back to the MMA warp and the stores overlap the next tile's MMAs
-          if constexpr (MODE == L2_ATOMIC || MODE == L2_STAGED) {
-            // No shared-memory staging.  Each lane holds 32 consecutive values of its own row
-            // per 32-column chunk (8 pieces of 4); the 8 lanes of an octet transpose those pieces
-            // among themselves with register shuffles (three exchange rounds), after which lane c
-            // holds piece c of each of the octet's 8 rows.  Every vector store (L2_STAGED: the
-            // slot's row) or reduction (L2_ATOMIC: the token's row) of the warp then covers
-            // 4 rows x 128 contiguous bytes, the shape the SM -> L2 path takes fastest (about
-            // 1.7x the rate of 16 rows x 32 bytes).
-            const int tok = slot < 0 ? -1 : MODE == L2_ATOMIC ? slot / args.k : slot;
-            int tok_r[8];  // the tokens of the octet's 8 rows
+          // accumulator goes back to the MMA warp and the stores overlap the next tile's MMAs.
+          // No shared-memory staging.  Each lane holds 32 consecutive values of its own row
+          // per 32-column chunk (8 pieces of 4); the 8 lanes of an octet transpose those pieces
+          // among themselves with register shuffles (three exchange rounds), after which lane c
+          // holds piece c of each of the octet's 8 rows.  Every vector store (L2_ROWS: the
+          // slot's row) or reduction (L2_ATOMIC: the token's row) of the warp then covers
+          // 4 rows x 128 contiguous bytes, the shape the SM -> L2 path takes fastest (about
+          // 1.7x the rate of 16 rows x 32 bytes).
+          const int tok = slot < 0 ? -1 : MODE == L2_ATOMIC ? slot / args.k : slot;
+          int tok_r[8];  // the tokens of the octet's 8 rows
 #pragma unroll
-            for (int i = 0; i < 8; ++i) tok_r[i] = __shfl_sync(0xffffffffu, tok, (lane & ~7) | i);
-            const int piece = lane & 7;
-            uint32_t v[BN / 64][32];
+          for (int i = 0; i < 8; ++i) tok_r[i] = __shfl_sync(0xffffffffu, tok, (lane & ~7) | i);
+          const int piece = lane & 7;
+          uint32_t v[BN / 64][32];
 #pragma unroll
-            for (int j = 0; j < BN / 64; ++j) tmem_ld32(t_row + 32 * (c_lo + j), v[j]);
-            tmem_wait_ld();
-            release();
+          for (int j = 0; j < BN / 64; ++j) tmem_ld32(t_row + 32 * (c_lo + j), v[j]);
+          tmem_wait_ld();
+          release();
 #pragma unroll
-            for (int j = 0; j < BN / 64; ++j) {
+          for (int j = 0; j < BN / 64; ++j) {
 #pragma unroll
-              for (int i = 0; i < 32; ++i)
-                v[j][i] = __float_as_uint(__uint_as_float(v[j][i]) * scale);
-              // round m: a lane with lane bit m set keeps the pieces whose index has bit m set
-              // and takes its partner's pieces with bit m set in place of its own with bit m clear;
-              // the partner does the converse
+            for (int i = 0; i < 32; ++i)
+              v[j][i] = __float_as_uint(__uint_as_float(v[j][i]) * scale);
+            // round m: a lane with lane bit m set keeps the pieces whose index has bit m set
+            // and takes its partner's pieces with bit m set in place of its own with bit m clear;
+            // the partner does the converse
 #pragma unroll
-              for (int m = 4; m >= 1; m >>= 1) {
-                const bool hi = (lane & m) != 0;
+            for (int m = 4; m >= 1; m >>= 1) {
+              const bool hi = (lane & m) != 0;
 #pragma unroll
-                for (int j0 = 0; j0 < 8; ++j0) {
-                  if (j0 & m) continue;
-                  const int j1 = j0 | m;
+              for (int j0 = 0; j0 < 8; ++j0) {
+                if (j0 & m) continue;
+                const int j1 = j0 | m;
 #pragma unroll
-                  for (int e = 0; e < 4; ++e) {
-                    const uint32_t snd = hi ? v[j][4 * j0 + e] : v[j][4 * j1 + e];
-                    const uint32_t rcv = __shfl_xor_sync(0xffffffffu, snd, m);
-                    if (hi) v[j][4 * j0 + e] = rcv;
-                    else v[j][4 * j1 + e] = rcv;
-                  }
+                for (int e = 0; e < 4; ++e) {
+                  const uint32_t snd = hi ? v[j][4 * j0 + e] : v[j][4 * j1 + e];
+                  const uint32_t rcv = __shfl_xor_sync(0xffffffffu, snd, m);
+                  if (hi) v[j][4 * j0 + e] = rcv;
+                  else v[j][4 * j1 + e] = rcv;
                 }
               }
-              const int64_t col = (int64_t)tl.nt * BN + 32 * (c_lo + j) + 4 * piece;
-#pragma unroll
-              for (int i = 0; i < 8; ++i) {
-                if (tok_r[i] < 0) continue;
-                const float4 val =
-                    make_float4(__uint_as_float(v[j][4 * i]), __uint_as_float(v[j][4 * i + 1]),
-                                __uint_as_float(v[j][4 * i + 2]), __uint_as_float(v[j][4 * i + 3]));
-                float* dst = args.ys + (int64_t)tok_r[i] * H + col;
-                if constexpr (MODE == L2_ATOMIC) red_add_v4(dst, val);
-                else *reinterpret_cast<float4*>(dst) = val;
-              }
             }
-          } else {
-            float* dst = args.ys + (int64_t)(slot >= 0 ? slot : 0) * H + tl.nt * BN;
-            auto emit = [&](int c, const uint32_t (&v)[32]) {
-              if (slot < 0) return;
-              float4* o = reinterpret_cast<float4*>(dst + 32 * c);
+            const int64_t col = (int64_t)tl.nt * BN + 32 * (c_lo + j) + 4 * piece;
 #pragma unroll
-              for (int i = 0; i < 8; ++i)
-                o[i] = make_float4(__uint_as_float(v[4 * i]) * scale,
-                                   __uint_as_float(v[4 * i + 1]) * scale,
-                                   __uint_as_float(v[4 * i + 2]) * scale,
-                                   __uint_as_float(v[4 * i + 3]) * scale);
-            };
-            uint32_t v[BN / 64][32];
-#pragma unroll
-            for (int j = 0; j < BN / 64; ++j) tmem_ld32(t_row + 32 * (c_lo + j), v[j]);
-            tmem_wait_ld();
-            release();
-#pragma unroll
-            for (int j = 0; j < BN / 64; ++j) emit(c_lo + j, v[j]);
+            for (int i = 0; i < 8; ++i) {
+              if (tok_r[i] < 0) continue;
+              const float4 val =
+                  make_float4(__uint_as_float(v[j][4 * i]), __uint_as_float(v[j][4 * i + 1]),
+                              __uint_as_float(v[j][4 * i + 2]), __uint_as_float(v[j][4 * i + 3]));
+              float* dst = args.ys + (int64_t)tok_r[i] * H + col;
+              if constexpr (MODE == L2_ATOMIC) red_add_v4(dst, val);
+              else *reinterpret_cast<float4*>(dst) = val;
+            }
           }
         }
       } else if (rows_valid) {
@@ -1131,7 +1112,7 @@ nvfp4_status_t gemm_l2(const uint8_t* h, const uint8_t* sfh, const float* gs_h, 
   if (T == 0) return NVFP4_OK;
   GemmArgs g{};
   g.sfa = sfh; g.sfb = sfw2; g.gs_a = gs_h; g.gs_b = gs_w2; g.offs = offs;
-  g.E = E; g.N = H; g.K = I; g.R_max = R_max; g.n_tiles = H / TileCfg<L2_DIRECT, 1>::BN;
+  g.E = E; g.N = H; g.K = I; g.R_max = R_max; g.n_tiles = H / TileCfg<L2_ROWS, 1>::BN;
   g.row_slot = row_slot; g.row_w = row_w; g.ys = ys; g.S = T * k; g.k = k; g.status = status;
   g.out_rows = R_max; g.k_splits = 1;
   if (atomic) {
@@ -1148,9 +1129,7 @@ nvfp4_status_t gemm_l2(const uint8_t* h, const uint8_t* sfh, const float* gs_h, 
         acc, n / 8, static_cast<__nv_bfloat16*>(out_bf16));
     return check_launch("to_bf16_kernel");
   }
-  const bool staged = (int64_t)T * k >= (int64_t)kL2StagedMinRowsPerExpert * E;
-  nvfp4_status_t st = staged ? launch<L2_STAGED>(h, w2, (int64_t)E * H, g, s)
-                             : launch<L2_DIRECT>(h, w2, (int64_t)E * H, g, s);
+  nvfp4_status_t st = launch<L2_ROWS>(h, w2, (int64_t)E * H, g, s);
   if (st != NVFP4_OK) return st;
   const int64_t n = (int64_t)T * H / 8;
   const int64_t want = (n + 255) / 256;
@@ -1162,7 +1141,7 @@ nvfp4_status_t gemm_l2(const uint8_t* h, const uint8_t* sfh, const float* gs_h, 
 // The L2 form for a batch: slot rows summed in slot order (deterministic) for few rows per expert
 // or on request; otherwise added into token rows as they are produced (no per-slot round trip).
 bool l2_use_atomic(int T, int k, int E, bool deterministic) {
-  return !deterministic && (int64_t)T * k >= (int64_t)kL2StagedMinRowsPerExpert * E;
+  return !deterministic && (int64_t)T * k >= (int64_t)kL2AtomicMinRowsPerExpert * E;
 }
 
 }  // namespace nvfp4
@@ -1255,7 +1234,7 @@ extern "C" nvfp4_status_t moe_grouped_gemm_l2_scatter(
     float* ys_ws, float* out_f32, void* out_bf16, int32_t* dev_status, nvfp4_stream_t stream) {
   if (E < 1 || E > MAX_E || H <= 0 || I <= 0 || T < 0 || k < 1 || R_max < 0)
     return NVFP4_ERR_INVALID_ARG;
-  if (H % TileCfg<L2_DIRECT, 1>::BN || I % 64 || R_max % 128) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (H % TileCfg<L2_ROWS, 1>::BN || I % 64 || R_max % 128) return NVFP4_ERR_UNSUPPORTED_SHAPE;
   if (!gs_h || !gs_w2 || !offs || !row_slot || !row_w || !dst_row || (!out_f32 && !out_bf16))
     return NVFP4_ERR_INVALID_ARG;
   if (T == 0 || R_max == 0) return NVFP4_OK;
@@ -1328,7 +1307,7 @@ extern "C" nvfp4_status_t moe_grouped_gemm_l2_scatter_noalloc(
     void* out_bf16, int32_t* dev_status, nvfp4_stream_t stream) {
   if (E < 1 || E > MAX_E || H <= 0 || I <= 0 || T < 0 || k < 1 || R_max < 0)
     return NVFP4_ERR_INVALID_ARG;
-  if (H % TileCfg<L2_DIRECT, 1>::BN || I % 64 || R_max % 128) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (H % TileCfg<L2_ROWS, 1>::BN || I % 64 || R_max % 128) return NVFP4_ERR_UNSUPPORTED_SHAPE;
   if (!gs_h || !gs_w2 || !offs || !row_slot || !row_w || !dst_row || !out_bf16)
     return NVFP4_ERR_INVALID_ARG;
   if ((int64_t)T * k * H > NVFP4_L2_NOALLOC_MAX_ELEMS) {
