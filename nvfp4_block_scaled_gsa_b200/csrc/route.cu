@@ -18,14 +18,10 @@ constexpr int kMaxE = 256;
 constexpr int kMaxK = 32;
 constexpr int kPerLane = kMaxE / 32;
 
-// One warp per token.  Lane l holds experts l, l+32, ..., and lane j < k ends up holding the
-// j-th selected expert.
-__global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits, int T, int E,
-                                                   int k, int renorm, int32_t* __restrict__ ids,
-                                                   float* __restrict__ w) {
-  const int lane = threadIdx.x & 31;
-  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (t >= T) return;
+// Top-k of token t by one warp.  Lane l holds experts l, l+32, ..., and lane j < k ends up
+// holding the j-th selected expert.
+__device__ __forceinline__ void topk_token(const float* __restrict__ logits, int t, int E, int k,
+                                           int renorm, int lane, int32_t* ids, float* w) {
   float v[kPerLane];
   float m = -INFINITY;
 #pragma unroll
@@ -84,6 +80,14 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
   }
 }
 
+// One warp per token.
+__global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits, int T, int E,
+                                                   int k, int renorm, int32_t* __restrict__ ids,
+                                                   float* __restrict__ w) {
+  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (t < T) topk_token(logits, t, E, k, renorm, threadIdx.x & 31, ids, w);
+}
+
 // Slots [lo, hi) of one CTA of 32 warps.  Warp w owns a contiguous part of the range, so a
 // per-warp histogram plus an exclusive scan over warps gives every slot a stable rank inside its
 // expert; __match_any_sync ranks the slots of one 32-slot step that share an expert.  Both passes
@@ -94,15 +98,15 @@ constexpr int kUnroll = 8;
 constexpr int kMultiMinSlots = 4096;
 constexpr int kChunkSlots = 2048;  // slots per CTA in the multi-CTA form
 
-__device__ __forceinline__ void warp_histogram(const int32_t* __restrict__ ids, int lo, int hi,
-                                               int E, int lane, int* __restrict__ hist_w,
-                                               bool& bad) {
+// ids is read with plain loads: in the single-CTA form the same kernel has just written it.
+__device__ __forceinline__ void warp_histogram(const int32_t* ids, int lo, int hi, int E, int lane,
+                                               int* __restrict__ hist_w, bool& bad) {
   for (int base = lo; base < hi; base += 32 * kUnroll) {
     int e[kUnroll];
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
       const int s = base + 32 * u + lane;
-      e[u] = s < hi ? __ldg(ids + s) : -1;
+      e[u] = s < hi ? ids[s] : -1;
     }
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
@@ -130,20 +134,24 @@ __global__ void __launch_bounds__(1024) permute_count_kernel(const int32_t* __re
   for (int e = tid; e < E; e += blockDim.x) hist_g[(int64_t)blockIdx.x * E + e] = hist[e];
 }
 
-// kMulti = false: one CTA over all S slots.  kMulti = true: CTA c over chunk c, with the expert
-// totals and the chunk's base per expert taken from hist_g (nch chunks).
+// kMulti = false: one CTA over all S slots; with logits given, it first takes the top-k of the
+// T = S / k tokens itself (one warp per token) and writes ids and w, so that a small batch routes
+// in one launch.  kMulti = true: CTA c over chunk c, with the expert totals and the chunk's base
+// per expert taken from hist_g (nch chunks).
 template <bool kMulti>
 __global__ void __launch_bounds__(1024) permute_kernel(
-    const int32_t* __restrict__ ids, const float* __restrict__ w, int S, int E, int64_t R_max,
-    const int32_t* __restrict__ hist_g, int nch, int32_t* __restrict__ offs_out,
+    const float* __restrict__ logits, int k, int renorm, int32_t* ids, float* w, int S, int E,
+    int64_t R_max, const int32_t* __restrict__ hist_g, int nch, int32_t* __restrict__ offs_out,
     int32_t* __restrict__ dst_row, int32_t* __restrict__ row_slot, float* __restrict__ row_w,
     int32_t* __restrict__ dev_status) {
   __shared__ int hist[32][kMaxE];
   __shared__ int cnt[kMaxE];
   __shared__ int offs[kMaxE + 1];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (!kMulti && logits != nullptr)
+    for (int t = warp; t < S / k; t += 32) topk_token(logits, t, E, k, renorm, lane, ids, w);
   for (int i = tid; i < 32 * kMaxE; i += blockDim.x) (&hist[0][0])[i] = 0;
-  __syncthreads();
+  __syncthreads();  // also: this CTA's ids and w writes are visible to all its threads
   const int c0 = kMulti ? blockIdx.x * kChunkSlots : 0;
   const int c1 = kMulti ? min(S, c0 + kChunkSlots) : S;
   const int per = (c1 - c0 + 31) / 32;
@@ -205,8 +213,8 @@ __global__ void __launch_bounds__(1024) permute_kernel(
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
       const int s = base + 32 * u + lane;
-      e[u] = s < hi ? __ldg(ids + s) : -1;
-      wv[u] = s < hi ? __ldg(w + s) : 0.0f;
+      e[u] = s < hi ? ids[s] : -1;
+      wv[u] = s < hi ? w[s] : 0.0f;
     }
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
@@ -261,23 +269,27 @@ nvfp4_status_t permute_launch(const float* logits, int T, int E, int k, int reno
                               int32_t* topk_ids, float* topk_w, int32_t* offs, int32_t* dst_row,
                               int32_t* row_slot, float* row_w, int64_t R_max, int32_t* hist_ws,
                               int32_t* dev_status, cudaStream_t s) {
-  if (logits != nullptr && T > 0) {
+  const int S = T * k;
+  const int nch = permute_chunks(T, k);
+  const bool multi = nch > 0 && hist_ws != nullptr;
+  if (logits != nullptr && T > 0 && multi) {
     topk_kernel<<<(T + 7) / 8, 256, 0, s>>>(logits, T, E, k, renorm, topk_ids, topk_w);
     nvfp4_status_t st = check_launch("topk_kernel");
     if (st != NVFP4_OK) return st;
   }
-  const int S = T * k;
-  const int nch = permute_chunks(T, k);
-  if (nch > 0 && hist_ws != nullptr) {
+  if (multi) {
     permute_count_kernel<<<nch, 1024, 0, s>>>(topk_ids, S, E, hist_ws, dev_status);
     nvfp4_status_t st = check_launch("permute_count_kernel");
     if (st != NVFP4_OK) return st;
-    permute_kernel<true><<<nch, 1024, 0, s>>>(topk_ids, topk_w, S, E, R_max, hist_ws, nch, offs,
-                                              dst_row, row_slot, row_w, dev_status);
+    permute_kernel<true><<<nch, 1024, 0, s>>>(nullptr, k, renorm, topk_ids, topk_w, S, E, R_max,
+                                              hist_ws, nch, offs, dst_row, row_slot, row_w,
+                                              dev_status);
     return check_launch("permute_kernel");
   }
-  permute_kernel<false><<<1, 1024, 0, s>>>(topk_ids, topk_w, S, E, R_max, nullptr, 0, offs,
-                                           dst_row, row_slot, row_w, dev_status);
+  // a small batch: top-k and the row map in one CTA, one launch
+  permute_kernel<false><<<1, 1024, 0, s>>>(T > 0 ? logits : nullptr, k, renorm, topk_ids,
+                                           topk_w, S, E, R_max, nullptr, 0, offs, dst_row,
+                                           row_slot, row_w, dev_status);
   return check_launch("permute_kernel");
 }
 
