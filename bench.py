@@ -201,7 +201,8 @@ class ClockSampler:
 # ----------------------------------------------------------------------------- our arm
 
 class Plan:
-    """Pre-allocated buffers for the staged path (same kernels as moe_ffn_forward)."""
+    """Pre-allocated buffers for the step run call by call (the kernels moe_ffn_forward chains),
+    with events between the calls for the stage breakdown."""
 
     def __init__(self, nv, cfg, x, logits, w1, w2, gs_h):
         import torch

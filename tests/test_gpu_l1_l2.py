@@ -46,7 +46,8 @@ def _setup(T, H, I, E, k, seed=0, drop=0.0):
     # decode-like batches (few tokens per expert)
     (16, 256, 128, 8, 2), (32, 512, 256, 6, 3), (20, 7168, 2048, 3, 2), (16, 256, 128, 256, 8),
     (1, 256, 128, 4, 1),
-    # 128+ rows per expert (the L2 epilogue staged through shared memory)
+    # 128+ rows per expert (several M-tiles per expert; from 32 rows per expert the FFN adds
+    # into token rows)
     (640, 256, 128, 4, 2), (640, 1024, 512, 2, 1),
     # 1024+ rows per expert: 256-row tiles on CTA pairs (odd block counts: half-empty pair tiles)
     (2304, 256, 128, 2, 1)])
