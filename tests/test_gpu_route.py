@@ -86,5 +86,19 @@ def test_permute_without_workspace_matches_multi_cta():
          dst.data_ptr(), rs.data_ptr(), rw.data_ptr(), None, 0, None,
          torch.cuda.current_stream().cuda_stream)
     torch.cuda.synchronize()
+    # the single CTA also takes the top-k itself
+    assert torch.equal(ids, a["ids"]) and torch.equal(w, a["weights"])
     assert torch.equal(offs, a["offs"]) and torch.equal(dst, a["dst_row"])
     assert torch.equal(rs, a["row_slot"]) and torch.equal(rw, a["row_w"])
+
+
+@pytest.mark.parametrize("T,E,k", [(511, 256, 8), (4095, 64, 1), (100, 7, 7)])
+def test_route_one_launch_below_the_multi_cta_size(T, E, k):
+    """Below 4096 slots one CTA takes the top-k of every token (one warp per token, many tokens
+    per warp here) and then builds the row map."""
+    rng = np.random.default_rng(T + E + k)
+    lg = torch.from_numpy(rng.standard_normal((T, E)).astype(np.float32))
+    lg[rng.random((T, E)) < 0.05] = -np.inf  # some experts masked per token
+    p = nv.permute(lg.to(DEV), k)
+    ids_ref, w_ref = R.route_topk(lg.numpy(), k)
+    _compare(p, ids_ref, w_ref, E, k)
