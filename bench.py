@@ -273,8 +273,12 @@ class Plan:
             ev[4].record()
 
 
-KERNELS_PER_STEP = 7  # topk, permute, amax, quantize, L1 GEMM, L2 GEMM, combine or bf16
-#                       rounding (+ a count kernel before permute from 4096 slots)
+def kernels_per_step(nv, cfg):
+    """Kernels one moe_ffn_forward launches: the routing (one kernel below 4096 slots, the row map
+    taking the top-k itself; from 4096 slots a top-k, a count and a row-map kernel), amax,
+    quantize, the L1 GEMM, the L2 GEMM, and the combine or the bf16 rounding."""
+    multi = nv.lib().moe_permute_workspace_size(cfg.T, cfg.E, cfg.k) > 0
+    return (3 if multi else 1) + 5
 
 
 def make_config(args):
@@ -505,8 +509,7 @@ def run_ours(args):
                             "each step's copies overlap its neighbours' compute",
                 "serialized": {"value": round(serial_value, 2), "unit": "GB/s",
                                "ms_per_step": round(serial_ms / K, 4)}},
-        "gpu_launches": (KERNELS_PER_STEP + (1 if nv.lib().moe_permute_workspace_size(
-            cfg.T, cfg.E, cfg.k) else 0)) * K,
+        "gpu_launches": kernels_per_step(nv, cfg) * K,
         "clocks": clocks,
         "cpu_baseline": cpu,
     }

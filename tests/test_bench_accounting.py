@@ -57,3 +57,13 @@ def test_roofline_bound_choice_follows_the_ridge():
     sp = bench.shared_algorithmic(CONFIGS["shared_prefill"])
     assert dp["flops"] / dp["gemm_bytes"] > ridge
     assert sp["l1_flops"] / sp["l1_bytes"] > ridge
+
+
+def test_moe_step_kernel_count():
+    """The launches the bench line claims per step match the path's kernels: one routing kernel
+    below 4096 slots (decode: 128), three from 4096 (mid, prefill), then amax, quantize, L1, L2
+    and the combine or bf16 rounding."""
+    import nvfp4_block_scaled_gsa_b200 as nv
+    assert bench.kernels_per_step(nv, CONFIGS["decode"]) == 6
+    assert bench.kernels_per_step(nv, CONFIGS["mid"]) == 8
+    assert bench.kernels_per_step(nv, CONFIGS["prefill"]) == 8
