@@ -32,9 +32,10 @@ def _inputs(T, H, E, seed):
     return x, lg
 
 
+@pytest.mark.parametrize("T", [256, 1024])  # 1024 x 4 slots: the multi-CTA routing
 @pytest.mark.parametrize("deterministic", [True, False])
-def test_ffn_alternating_inputs(deterministic):
-    T, H, I, E, k = 256, 1024, 512, 16, 4  # T*k = 1024 >= 32*E: the scatter-add form by default
+def test_ffn_alternating_inputs(deterministic, T):
+    H, I, E, k = 1024, 512, 16, 4  # T*k >= 32*E: the scatter-add form by default
     w1, w2 = _weights(E, H, I, 11)
     gs_h = torch.ones(1, dtype=torch.float32, device=DEV)
     sets = [_inputs(T, H, E, 100 + i) for i in range(2)]
