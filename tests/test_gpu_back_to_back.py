@@ -1,10 +1,9 @@
 """Back-to-back calls on one stream, sharing one workspace, with no host synchronization between
-them.  Each kernel of the library may start while the kernel before it is finishing, so every
-kernel has to see its predecessor's writes complete and must not overwrite a buffer that an
-earlier kernel still reads.  Two input sets alternate over many calls; each output must equal
-the output of the same inputs computed alone (bitwise on the deterministic paths; for the
-scatter-add form, whose summation order is free, within one bf16 ulp per value plus the FP32
-reordering error).
+them: every buffer a call accumulates into (amax word, statistics, the scatter-add accumulator)
+must be reset by that call, and nothing one call leaves in the workspace may leak into the next.
+Two input sets alternate over many calls; each output must equal the output of the same inputs
+computed alone (bitwise on the deterministic paths; for the scatter-add form, whose summation
+order is free, within one bf16 ulp per value plus the FP32 reordering error).
 """
 
 import pytest
