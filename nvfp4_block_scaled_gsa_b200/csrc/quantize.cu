@@ -37,7 +37,11 @@ __global__ void __launch_bounds__(kThreads) amax_kernel(const __nv_bfloat16* __r
       m = max(m, (w[i] >> 16) & 0x7FFFu);
     }
   };
+  // contiguous rows (ld == cols, the usual case): the flat index is the address, with no 64-bit
+  // division per load
+  const bool flat = ld == cols;
   auto load = [&](int64_t v) {
+    if (flat) return __ldg(reinterpret_cast<const uint4*>(x) + v);
     const int64_t r = v / vec_per_row, c = (v - r * vec_per_row) * 8;
     return __ldg(reinterpret_cast<const uint4*>(x + r * ld + c));
   };
